@@ -1,0 +1,435 @@
+/*
+ * nf4_oracle.c -- plain, slow CPU oracle for the QLoRA frozen-base linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: only the tests, the smoke check and the benchmark's cpu_baseline
+ * leg use it. It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes, step by step, with the passage each step follows:
+ *
+ *  - NF4 table: the 16 values printed in "QLoRA paper notes" (tqpw.cn),
+ *    section "Method / NormalFloat Quantization (NF4)". They are typed below as
+ *    printed; each is an exact fp32 value.
+ *  - Blocks of 64 consecutive weights of the row-major flattened W, absmax per
+ *    block, weights normalised into [-1, 1] by that absmax: same section
+ *    ("g64", weights normalised to [-1,1] before quantisation) and "How QLoRA
+ *    works" (aivaro.ru) section 5 (one constant per 64 weights, stored fp32).
+ *  - Nearest code: "QLoRA & PEFT family" (ai-reference-codex) section 3.1
+ *    (remember which of the 16 values each weight is closest to). Ties go to
+ *    the lower index; an all-zero block gets code 7 (the value 0).
+ *  - Double quantisation: "QLoRA paper notes", section "Double Quantization"
+ *    (block constants quantised to FP8 in groups of 256 after subtracting
+ *    their mean, then symmetric quantisation). FP8 is E4M3 (finite variant,
+ *    max 448); the group absmax maps to 448; one fp32 scale per group; one
+ *    fp32 mean per tensor, the exact mean rounded once to fp32.
+ *  - Dequantisation to the compute type and the LoRA sum h = W x + B A x:
+ *    "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), equations
+ *    h = Wx + BAx and h = dequant(W_NF4) x + BAx; shapes W (d x k),
+ *    B (d x r), A (r x k) from "How QLoRA works" section 2; the LoRA branch is
+ *    scaled by alpha/r (lora_alpha is the scaling factor, LoRA/QLoRA talk
+ *    summary, "QLoRA ... practice guide").
+ *  - Input gradient through the frozen, dequantised base: "How QLoRA works"
+ *    section 7 (the 4-bit weights are dequantised on the fly to compute
+ *    gradients and are not updated).
+ *
+ * All sums of the linear layer are taken in fp64 in plain loop order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define OR_BLOCK 64
+#define OR_GROUP 256
+#define OR_E4M3_MAX 448.0f
+
+/* The NF4 code values exactly as printed on the page (ascending). */
+static const double OR_NF4[16] = {
+    -1.0,
+    -0.6961928009986877,
+    -0.5250730514526367,
+    -0.39491748809814453,
+    -0.28444138169288635,
+    -0.18477343022823334,
+    -0.09105003625154495,
+    0.0,
+    0.07958029955625534,
+    0.16093020141124725,
+    0.24611230194568634,
+    0.33791524171829224,
+    0.44070982933044434,
+    0.5626170039176941,
+    0.7229568362236023,
+    1.0,
+};
+
+/* ------------------------------------------------------------------ scalars */
+
+void or_nf4_table(double *out16) {
+    for (int i = 0; i < 16; ++i) out16[i] = OR_NF4[i];
+}
+
+int or_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static float bf16_bits_to_float(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even (finite inputs). */
+uint16_t or_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) return (uint16_t)(u >> 16); /* inf/nan: truncate */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* E4M3 (finite variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits.
+ * 0x7f / 0xff are NaN; the largest finite magnitude is 448 (0x7e). */
+double or_e4m3_decode(uint8_t v) {
+    int s = v >> 7, e = (v >> 3) & 15, m = v & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, -9);
+    else
+        mag = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* fp32 -> E4M3 by exhaustive search over the 127 finite magnitudes: nearest
+ * value, ties to the even code, magnitudes above 448 saturate to 448, the sign
+ * is kept (a negative value that rounds to zero gives 0x80). */
+uint8_t or_e4m3_encode(float f) {
+    if (f != f) return 0x7f;
+    uint8_t sign = (f < 0.0f || (f == 0.0f && signbit(f))) ? 0x80 : 0x00;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7e;
+    int best = 0;
+    double best_err = a; /* code 0 is +0 */
+    for (int c = 1; c <= 0x7e; ++c) {
+        double err = fabs(or_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* ------------------------------------------------------- exact tensor mean */
+
+/* 320-bit unsigned fixed-point accumulator; unit = 2^-133 (the smallest
+ * positive bf16 subnormal), so every bf16 absmax is an integer in it. */
+typedef struct { uint64_t limb[5]; } or_big;
+
+static void big_add_shifted(or_big *acc, uint64_t m, int pos) {
+    /* acc += m << pos, m < 2^9 */
+    int li = pos / 64, sh = pos % 64;
+    unsigned __int128 v = ((unsigned __int128)m) << sh;
+    uint64_t carry = 0;
+    for (int i = li; i < 5; ++i) {
+        unsigned __int128 add = (i == li) ? (uint64_t)v : (i == li + 1 ? (uint64_t)(v >> 64) : 0);
+        unsigned __int128 s = (unsigned __int128)acc->limb[i] + add + carry;
+        acc->limb[i] = (uint64_t)s;
+        carry = (uint64_t)(s >> 64);
+    }
+}
+
+static int big_bitlen(const or_big *a) {
+    for (int i = 4; i >= 0; --i)
+        if (a->limb[i]) return i * 64 + (64 - __builtin_clzll(a->limb[i]));
+    return 0;
+}
+
+static int big_bit(const or_big *a, int pos) {
+    if (pos < 0 || pos >= 320) return 0;
+    return (int)((a->limb[pos / 64] >> (pos % 64)) & 1u);
+}
+
+/* Correctly rounded fp32 of (S * 2^-133) / n, S the big integer. */
+static float big_div_round_f32(const or_big *S, uint64_t n) {
+    const int W = 100;
+    int bl = big_bitlen(S);
+    if (bl == 0 || n == 0) return 0.0f;
+    int sh = bl - W;
+    unsigned __int128 top = 0;
+    int sticky0 = 0;
+    for (int b = W - 1; b >= 0; --b) {
+        top = (top << 1) | (unsigned __int128)big_bit(S, b + sh);
+    }
+    for (int b = 0; b < sh; ++b)
+        if (big_bit(S, b)) { sticky0 = 1; break; }
+    unsigned __int128 Q = top / n, R = top % n;
+    int rem_nz = (R != 0) || sticky0;
+    int e0 = sh - 133; /* value = (Q + frac) * 2^e0 */
+    int qb = 0;
+    for (unsigned __int128 t = Q; t; t >>= 1) ++qb;
+    int e_lead = qb - 1 + e0;
+    int lsb_exp = e_lead - 23;
+    if (lsb_exp < -149) lsb_exp = -149;
+    int s2 = lsb_exp - e0;
+    unsigned __int128 mant = (s2 >= 128) ? 0 : (Q >> s2);
+    int rbit = (s2 - 1 >= 0 && s2 - 1 < 128) ? (int)((Q >> (s2 - 1)) & 1) : 0;
+    int sticky = rem_nz;
+    for (int b = 0; b < s2 - 1 && b < 128; ++b)
+        if ((Q >> b) & 1) { sticky = 1; break; }
+    if (rbit && (sticky || (mant & 1))) mant += 1;
+    return (float)ldexp((double)(uint64_t)mant, lsb_exp);
+}
+
+/* mu = fl32( (sum of the nb fp32 block absmaxes, exactly) / nb ).
+ * Each absmax must be an exactly representable bf16 value (it is the absolute
+ * value of a bf16 weight). */
+float or_exact_mean_f32(const float *c, int64_t nb) {
+    or_big S;
+    memset(&S, 0, sizeof S);
+    for (int64_t b = 0; b < nb; ++b) {
+        uint32_t u;
+        memcpy(&u, &c[b], 4);
+        u &= 0x7fffffffu;
+        uint32_t E = u >> 23, frac7 = (u >> 16) & 0x7f;
+        if (E == 0) {
+            big_add_shifted(&S, frac7, 0);
+        } else {
+            big_add_shifted(&S, 128u + frac7, (int)E - 1);
+        }
+    }
+    return big_div_round_f32(&S, (uint64_t)nb);
+}
+
+/* ------------------------------------------------------------- quantiser */
+
+static int nearest_code(float x) {
+    int best = 0;
+    double best_err = fabs((double)x - OR_NF4[0]);
+    for (int i = 1; i < 16; ++i) {
+        double err = fabs((double)x - OR_NF4[i]);
+        if (err < best_err) { /* strict: ties keep the lower index */
+            best = i;
+            best_err = err;
+        }
+    }
+    return best;
+}
+
+/* Code of one bf16 weight w in a block with absmax c (exposed for tests). */
+int or_nf4_code(float w, float c) {
+    if (c == 0.0f) return 7;
+    float x = w / c;
+    return nearest_code(x);
+}
+
+int64_t or_num_blocks(int64_t n, int64_t k) { return n * k / OR_BLOCK; }
+int64_t or_num_groups(int64_t n, int64_t k) { return (or_num_blocks(n, k) + OR_GROUP - 1) / OR_GROUP; }
+
+/* W: n x k bf16 bits, row-major. Outputs: codes (n*k/2 bytes, element e in the
+ * low nibble of byte e/2 when e is even, high nibble when odd), q (nb bytes
+ * E4M3), sigma (ng floats), mu (1 float), absmax (nb floats, may be NULL).
+ * Returns 0, or -1 when k is not a multiple of 64. */
+int or_nf4_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q,
+                    float *sigma, float *mu, float *absmax) {
+    if (k % OR_BLOCK != 0 || n < 0 || k < 0) return -1;
+    int64_t nb = or_num_blocks(n, k), ng = or_num_groups(n, k);
+    float *c = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    if (!c) return -2;
+
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) {
+        const uint16_t *w = W + b * OR_BLOCK;
+        float m = 0.0f;
+        for (int i = 0; i < OR_BLOCK; ++i) {
+            float a = fabsf(bf16_bits_to_float(w[i]));
+            if (a > m) m = a;
+        }
+        c[b] = m;
+        for (int i = 0; i < OR_BLOCK; i += 2) {
+            int lo = or_nf4_code(bf16_bits_to_float(w[i]), m);
+            int hi = or_nf4_code(bf16_bits_to_float(w[i + 1]), m);
+            codes[(b * OR_BLOCK + i) / 2] = (uint8_t)(lo | (hi << 4));
+        }
+    }
+
+    float m_all = or_exact_mean_f32(c, nb);
+    *mu = m_all;
+
+#pragma omp parallel for schedule(static)
+    for (int64_t g = 0; g < ng; ++g) {
+        int64_t b0 = g * OR_GROUP, b1 = b0 + OR_GROUP < nb ? b0 + OR_GROUP : nb;
+        float S = 0.0f;
+        for (int64_t b = b0; b < b1; ++b) {
+            float d = c[b] - m_all;
+            float a = fabsf(d);
+            if (a > S) S = a;
+        }
+        float sg = S / OR_E4M3_MAX;
+        sigma[g] = sg;
+        for (int64_t b = b0; b < b1; ++b) {
+            float d = c[b] - m_all;
+            q[b] = (sg == 0.0f) ? (uint8_t)0 : or_e4m3_encode(d / sg);
+        }
+    }
+    if (absmax) memcpy(absmax, c, sizeof(float) * (size_t)nb);
+    free(c);
+    return 0;
+}
+
+/* ---------------------------------------------------------- dequantiser */
+
+/* c'_b = fma(decode(q_b), sigma_g, mu), one rounding, fp32. */
+float or_block_constant(uint8_t qb, float sg, float mu) {
+    return fmaf((float)or_e4m3_decode(qb), sg, mu);
+}
+
+static void block_constants(const uint8_t *q, const float *sigma, float mu, int64_t nb, float *cp) {
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) cp[b] = or_block_constant(q[b], sigma[b / OR_GROUP], mu);
+}
+
+static int code_at(const uint8_t *codes, int64_t e) {
+    uint8_t byte = codes[e / 2];
+    return (e & 1) ? (byte >> 4) : (byte & 15);
+}
+
+/* Dequantise into bf16: bf16_rn( fl32( T32[code] * c'_b ) ). */
+void or_nf4_dequant_bf16(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu,
+                         int64_t n, int64_t k, uint16_t *out) {
+    int64_t nb = or_num_blocks(n, k);
+    float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    block_constants(q, sigma, mu, nb, cp);
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n * k; ++e) {
+        float t = (float)OR_NF4[code_at(codes, e)];
+        float v = t * cp[e / OR_BLOCK];
+        out[e] = or_f32_to_bf16(v);
+    }
+    free(cp);
+}
+
+/* Dequantise into fp64 without rounding: T[code] * c'_b. */
+void or_nf4_dequant_f64(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu,
+                        int64_t n, int64_t k, double *out) {
+    int64_t nb = or_num_blocks(n, k);
+    float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    block_constants(q, sigma, mu, nb, cp);
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n * k; ++e) out[e] = OR_NF4[code_at(codes, e)] * (double)cp[e / OR_BLOCK];
+    free(cp);
+}
+
+/* ------------------------------------------------------ linear layer */
+
+/* h[i, j] for the selected token rows rows[i] (i < nsel) of x (m x k):
+ *   h = sum_k W'[j,k] x[row,k] + s * sum_r B[j,r] * (sum_k A[r,k] x[row,k])
+ * with W' = T[code] * c' in fp64, s = fl32(alpha / r). A (r x k) and B (n x r)
+ * may be NULL when r == 0. Output h is nsel x n, fp64. */
+void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
+                  int64_t k, const uint16_t *x, const int64_t *rows, int64_t nsel, const uint16_t *A,
+                  const uint16_t *B, int r, float alpha, double *h) {
+    int64_t nb = or_num_blocks(n, k);
+    float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    block_constants(q, sigma, mu, nb, cp);
+    double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    double *xs = (double *)malloc(sizeof(double) * (size_t)(nsel * k + 1));
+    double *t = (double *)malloc(sizeof(double) * (size_t)(nsel * (r > 0 ? r : 1) + 1));
+    for (int64_t i = 0; i < nsel; ++i)
+        for (int64_t kk = 0; kk < k; ++kk) xs[i * k + kk] = bf16_bits_to_float(x[rows[i] * k + kk]);
+    /* t[i, rr] = sum_k A[rr, k] x[row_i, k] */
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nsel; ++i)
+        for (int rr = 0; rr < r; ++rr) {
+            double acc = 0.0;
+            for (int64_t kk = 0; kk < k; ++kk) acc += bf16_bits_to_float(A[rr * k + kk]) * xs[i * k + kk];
+            t[i * r + rr] = acc;
+        }
+#pragma omp parallel
+    {
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)(k + 1));
+#pragma omp for schedule(static)
+        for (int64_t j = 0; j < n; ++j) {
+            for (int64_t kk = 0; kk < k; ++kk)
+                wrow[kk] = OR_NF4[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
+            for (int64_t i = 0; i < nsel; ++i) {
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < k; ++kk) acc += wrow[kk] * xs[i * k + kk];
+                double lora = 0.0;
+                for (int rr = 0; rr < r; ++rr) lora += bf16_bits_to_float(B[j * r + rr]) * t[i * r + rr];
+                h[i * n + j] = acc + s * lora;
+            }
+        }
+        free(wrow);
+    }
+    free(t);
+    free(xs);
+    free(cp);
+}
+
+/* grad_x[i, kk] for the selected rows of grad_h (m x n):
+ *   grad_x = sum_j grad_h[row,j] W'[j,kk] + s * sum_r A[r,kk] * (sum_j grad_h[row,j] B[j,r])
+ * Output nsel x k, fp64. */
+void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
+                    int64_t k, const uint16_t *gh, const int64_t *rows, int64_t nsel,
+                    const uint16_t *A, const uint16_t *B, int r, float alpha, double *gx) {
+    int64_t nb = or_num_blocks(n, k);
+    float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    block_constants(q, sigma, mu, nb, cp);
+    double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    double *gs = (double *)malloc(sizeof(double) * (size_t)(nsel * n + 1));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(nsel * (r > 0 ? r : 1) + 1));
+    for (int64_t i = 0; i < nsel; ++i)
+        for (int64_t j = 0; j < n; ++j) gs[i * n + j] = bf16_bits_to_float(gh[rows[i] * n + j]);
+    /* u[i, rr] = sum_j grad_h[row_i, j] B[j, rr] */
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nsel; ++i)
+        for (int rr = 0; rr < r; ++rr) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < n; ++j) acc += gs[i * n + j] * bf16_bits_to_float(B[j * r + rr]);
+            u[i * r + rr] = acc;
+        }
+    /* Each thread owns a slice of columns kk and walks all rows j. */
+    const int64_t CH = 256;
+    int64_t nch = (k + CH - 1) / CH;
+#pragma omp parallel
+    {
+        double *acc = (double *)malloc(sizeof(double) * (size_t)(nsel * CH + 1));
+        double *wseg = (double *)malloc(sizeof(double) * (size_t)(CH + 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t ch = 0; ch < nch; ++ch) {
+            int64_t k0 = ch * CH, k1 = k0 + CH < k ? k0 + CH : k;
+            int64_t w = k1 - k0;
+            memset(acc, 0, sizeof(double) * (size_t)(nsel * CH));
+            for (int64_t j = 0; j < n; ++j) {
+                for (int64_t kk = k0; kk < k1; ++kk)
+                    wseg[kk - k0] = OR_NF4[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
+                for (int64_t i = 0; i < nsel; ++i) {
+                    double g = gs[i * n + j];
+                    for (int64_t kk = 0; kk < w; ++kk) acc[i * CH + kk] += g * wseg[kk];
+                }
+            }
+            for (int64_t i = 0; i < nsel; ++i)
+                for (int64_t kk = k0; kk < k1; ++kk) {
+                    double lora = 0.0;
+                    for (int rr = 0; rr < r; ++rr) lora += bf16_bits_to_float(A[rr * k + kk]) * u[i * r + rr];
+                    gx[i * k + kk] = acc[i * CH + (kk - k0)] + s * lora;
+                }
+        }
+        free(wseg);
+        free(acc);
+    }
+    free(u);
+    free(gs);
+    free(cp);
+}

@@ -1,0 +1,198 @@
+"""CPU oracle for the NF4 + double-quant + LoRA linear layer (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
+``bench.py`` may import this module. The product path (the CUDA library and its
+Python binding) never imports, links or executes anything under ``oracle/``.
+
+The arithmetic lives in ``nf4_oracle.c`` (plain C, fp64 sums, OpenMP over
+independent outputs); this module only compiles it with gcc and marshals numpy
+arrays through ctypes. Every function documents the passage it follows in the C
+file's header.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nf4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, OpenMP, strict IEEE)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+           "-fno-fast-math", "-Wall", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.or_nf4_table.argtypes = [P]
+        lib.or_threads.restype = ctypes.c_int
+        lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.or_f32_to_bf16.restype = ctypes.c_uint16
+        lib.or_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.or_e4m3_decode.restype = ctypes.c_double
+        lib.or_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.or_e4m3_encode.restype = ctypes.c_uint8
+        lib.or_exact_mean_f32.argtypes = [P, i64]
+        lib.or_exact_mean_f32.restype = ctypes.c_float
+        lib.or_nf4_code.argtypes = [ctypes.c_float, ctypes.c_float]
+        lib.or_nf4_code.restype = ctypes.c_int
+        lib.or_num_blocks.argtypes = [i64, i64]
+        lib.or_num_blocks.restype = i64
+        lib.or_num_groups.argtypes = [i64, i64]
+        lib.or_num_groups.restype = i64
+        lib.or_nf4_quantize.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.or_nf4_quantize.restype = ctypes.c_int
+        lib.or_block_constant.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
+        lib.or_block_constant.restype = ctypes.c_float
+        lib.or_nf4_dequant_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
+        lib.or_nf4_dequant_f64.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
+        lib.or_qlora_fwd.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, i64, P, P,
+                                     ctypes.c_int, ctypes.c_float, P]
+        lib.or_qlora_bwd_x.argtypes = lib.or_qlora_fwd.argtypes
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits16(a: np.ndarray) -> np.ndarray:
+    """bf16 payload as uint16 bits (accepts uint16 or int16 arrays)."""
+    a = np.ascontiguousarray(a)
+    assert a.dtype in (np.uint16, np.int16), a.dtype
+    return a.view(np.uint16)
+
+
+def threads() -> int:
+    return int(_load().or_threads())
+
+
+def nf4_table() -> np.ndarray:
+    out = np.zeros(16, dtype=np.float64)
+    _load().or_nf4_table(_ptr(out))
+    return out
+
+
+def f32_to_bf16(v: float) -> int:
+    return int(_load().or_f32_to_bf16(float(v)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().or_e4m3_decode(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(_load().or_e4m3_encode(float(v)))
+
+
+def exact_mean_f32(c: np.ndarray) -> np.float32:
+    c = np.ascontiguousarray(c, dtype=np.float32)
+    return np.float32(_load().or_exact_mean_f32(_ptr(c), c.size))
+
+
+def nf4_code(w: float, c: float) -> int:
+    return int(_load().or_nf4_code(float(w), float(c)))
+
+
+def num_blocks(n: int, k: int) -> int:
+    return int(_load().or_num_blocks(n, k))
+
+
+def num_groups(n: int, k: int) -> int:
+    return int(_load().or_num_groups(n, k))
+
+
+def block_constant(qb: int, sigma: float, mu: float) -> np.float32:
+    return np.float32(_load().or_block_constant(int(qb), float(sigma), float(mu)))
+
+
+def nf4_quantize(W_bits: np.ndarray, n: int, k: int):
+    """Quantise a row-major n x k bf16 matrix (given as uint16 bits).
+
+    Returns dict(codes=u8[n*k/2], q=u8[nb], sigma=f32[ng], mu=f32, absmax=f32[nb]).
+    """
+    W = _bits16(W_bits).reshape(-1)
+    assert W.size == n * k
+    nb, ng = num_blocks(n, k), num_groups(n, k)
+    codes = np.zeros(n * k // 2, dtype=np.uint8)
+    q = np.zeros(nb, dtype=np.uint8)
+    sigma = np.zeros(ng, dtype=np.float32)
+    mu = np.zeros(1, dtype=np.float32)
+    absmax = np.zeros(nb, dtype=np.float32)
+    rc = _load().or_nf4_quantize(_ptr(W), n, k, _ptr(codes), _ptr(q), _ptr(sigma), _ptr(mu), _ptr(absmax))
+    if rc != 0:
+        raise ValueError(f"or_nf4_quantize failed: {rc} (k must be a multiple of 64)")
+    return dict(codes=codes, q=q, sigma=sigma, mu=np.float32(mu[0]), absmax=absmax)
+
+
+def nf4_dequant_bf16(qw: dict, n: int, k: int) -> np.ndarray:
+    out = np.zeros(n * k, dtype=np.uint16)
+    _load().or_nf4_dequant_bf16(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]),
+                                n, k, _ptr(out))
+    return out.reshape(n, k)
+
+
+def nf4_dequant_f64(qw: dict, n: int, k: int) -> np.ndarray:
+    out = np.zeros(n * k, dtype=np.float64)
+    _load().or_nf4_dequant_f64(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]),
+                               n, k, _ptr(out))
+    return out.reshape(n, k)
+
+
+def _rows(m: int, rows) -> np.ndarray:
+    if rows is None:
+        return np.arange(m, dtype=np.int64)
+    return np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+
+
+def qlora_fwd(qw: dict, n: int, k: int, x_bits: np.ndarray, m: int, A_bits, B_bits, r: int,
+              alpha: float, rows=None) -> np.ndarray:
+    """h (fp64) for the selected token rows of x (m x k bf16 bits); shape len(rows) x n."""
+    rows = _rows(m, rows)
+    x = _bits16(x_bits).reshape(-1)
+    assert x.size == m * k
+    A = _bits16(A_bits).reshape(-1) if r > 0 else None
+    B = _bits16(B_bits).reshape(-1) if r > 0 else None
+    h = np.zeros(rows.size * n, dtype=np.float64)
+    _load().or_qlora_fwd(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
+                         _ptr(x), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(h))
+    return h.reshape(rows.size, n)
+
+
+def qlora_bwd_x(qw: dict, n: int, k: int, gh_bits: np.ndarray, m: int, A_bits, B_bits, r: int,
+                alpha: float, rows=None) -> np.ndarray:
+    """grad_x (fp64) for the selected token rows of grad_h (m x n bf16 bits); shape len(rows) x k."""
+    rows = _rows(m, rows)
+    g = _bits16(gh_bits).reshape(-1)
+    assert g.size == m * n
+    A = _bits16(A_bits).reshape(-1) if r > 0 else None
+    B = _bits16(B_bits).reshape(-1) if r > 0 else None
+    gx = np.zeros(rows.size * k, dtype=np.float64)
+    _load().or_qlora_bwd_x(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
+                           _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(gx))
+    return gx.reshape(rows.size, k)
