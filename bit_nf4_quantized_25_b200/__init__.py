@@ -1,0 +1,11 @@
+"""NF4 + double-quantisation + LoRA linear layer for B200 (sm_100a).
+
+The computation lives in ``libqlora_nf4.so`` (C ABI: ``include/qlora_nf4.h``); the
+``binding`` module marshals torch tensors into it. Importing the package does not load
+the library; the first call does, and fails loudly if it is missing.
+"""
+from .binding import (NF4Weight, QNError, linear_workspace_size, launch_count, load, nf4_dequantize,
+                      nf4_quantize, qlora_linear_bwd_x, qlora_linear_fwd, quantize_workspace_size, sizes)
+
+__all__ = ["NF4Weight", "QNError", "linear_workspace_size", "launch_count", "load", "nf4_dequantize",
+           "nf4_quantize", "qlora_linear_bwd_x", "qlora_linear_fwd", "quantize_workspace_size", "sizes"]

@@ -1,0 +1,214 @@
+"""Thin Python binding of ``libqlora_nf4.so`` (the C ABI in ``include/qlora_nf4.h``).
+
+Argument marshalling only: torch tensors supply device memory and the current CUDA
+stream; every step of the computation runs in the library's sm_100a kernels. There is
+no fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
+
+QN_OK, QN_EINVAL, QN_ESHAPE, QN_EALIGN, QN_ECUDA, QN_EWORKSPACE = range(6)
+BLOCK, GROUP, MAX_RANK = 64, 256, 256
+
+EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_dequantize",
+            "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x", "qn_status_string",
+            "qn_last_error", "qn_launch_count")
+
+
+class QNError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+class CWeight(ctypes.Structure):
+    _fields_ = [("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
+                ("absmax_mean", ctypes.c_void_p)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load the library (once). Raises if it is missing: there is no other path."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with `python -m bit_nf4_quantized_25_b200.build`")
+        lib = ctypes.CDLL(p)
+        P, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)
+        W = ctypes.POINTER(CWeight)
+        st = ctypes.c_int
+        lib.qn_nf4_sizes.argtypes = [i64, i64, sz, sz, sz, sz]
+        lib.qn_quantize_workspace_size.argtypes = [i64, i64, sz]
+        lib.nf4_quantize.argtypes = [P, W, P, ctypes.c_size_t, P]
+        lib.nf4_dequantize.argtypes = [W, P, P]
+        lib.qlora_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, sz]
+        lib.qlora_linear_fwd.argtypes = [W, P, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, ctypes.c_size_t, P]
+        lib.qlora_linear_bwd_x.argtypes = lib.qlora_linear_fwd.argtypes
+        for f in ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_dequantize",
+                  "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x"):
+            getattr(lib, f).restype = st
+        lib.qn_status_string.argtypes = [st]
+        lib.qn_status_string.restype = ctypes.c_char_p
+        lib.qn_last_error.restype = ctypes.c_char_p
+        lib.qn_launch_count.argtypes = [ctypes.c_int]
+        lib.qn_launch_count.restype = ctypes.c_uint64
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _check(status: int, what: str):
+    if status != QN_OK:
+        lib = load()
+        raise QNError(status, f"{what}: {lib.qn_status_string(status).decode()} ({lib.qn_last_error().decode()})")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_bf16(t: torch.Tensor, name: str):
+    if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+def sizes(n_out: int, k_in: int):
+    """(codes, absmax_q, group_scale, absmax_mean) byte sizes of a quantised weight."""
+    a, b, c, d = (ctypes.c_size_t() for _ in range(4))
+    _check(load().qn_nf4_sizes(n_out, k_in, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(d)),
+           "qn_nf4_sizes")
+    return a.value, b.value, c.value, d.value
+
+
+def quantize_workspace_size(n_out: int, k_in: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().qn_quantize_workspace_size(n_out, k_in, ctypes.byref(v)), "qn_quantize_workspace_size")
+    return v.value
+
+
+def linear_workspace_size(M: int, n_out: int, k_in: int, r: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().qlora_workspace_size(M, n_out, k_in, r, ctypes.byref(v)), "qlora_workspace_size")
+    return v.value
+
+
+def launch_count(reset: bool = False) -> int:
+    return int(load().qn_launch_count(1 if reset else 0))
+
+
+@dataclasses.dataclass
+class NF4Weight:
+    """A quantised weight: four device buffers plus the shape (see include/qlora_nf4.h)."""
+    n_out: int
+    k_in: int
+    codes: torch.Tensor        # uint8 [n_out*k_in/2]
+    absmax_q: torch.Tensor     # uint8 [nb], E4M3 bits
+    group_scale: torch.Tensor  # float32 [ng]
+    absmax_mean: torch.Tensor  # float32 [1]
+
+    @staticmethod
+    def empty(n_out: int, k_in: int, device="cuda") -> "NF4Weight":
+        cb, ab, sb, _ = sizes(n_out, k_in)
+        u8 = dict(dtype=torch.uint8, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        return NF4Weight(n_out, k_in, torch.empty(cb, **u8), torch.empty(ab, **u8),
+                         torch.empty(sb // 4, **f32), torch.empty(1, **f32))
+
+    def c_struct(self) -> CWeight:
+        return CWeight(self.n_out, self.k_in, self.codes.data_ptr(), self.absmax_q.data_ptr(),
+                       self.group_scale.data_ptr(), self.absmax_mean.data_ptr())
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.absmax_q, self.group_scale,
+                                                          self.absmax_mean))
+
+
+def nf4_quantize(W: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
+                 stream=None) -> NF4Weight:
+    """Quantise a bf16 (n_out x k_in) CUDA tensor to NF4 with double quantisation."""
+    _dev_bf16(W, "W")
+    n, k = W.shape
+    out = out or NF4Weight.empty(n, k, W.device)
+    need = quantize_workspace_size(n, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    cw = out.c_struct()
+    _check(load().nf4_quantize(_ptr(W), ctypes.byref(cw), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "nf4_quantize")
+    return out
+
+
+def nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    _dev_bf16(out, "out")
+    cw = w.c_struct()
+    _check(load().nf4_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "nf4_dequantize")
+    return out
+
+
+def _lora(A, B, r):
+    if r == 0:
+        return None, None
+    _dev_bf16(A, "A")
+    _dev_bf16(B, "B")
+    return A, B
+
+
+def qlora_linear_fwd(w: NF4Weight, x: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
+                     alpha: float, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """h = dequant(W) x + (alpha/r) B (A x); x is M x k_in, h is M x n_out (bf16)."""
+    _dev_bf16(x, "x")
+    M = x.shape[0]
+    r = 0 if A is None else A.shape[0]
+    A, B = _lora(A, B, r)
+    out = out if out is not None else torch.empty(M, w.n_out, dtype=torch.bfloat16, device=x.device)
+    _dev_bf16(out, "out")
+    need = linear_workspace_size(M, w.n_out, w.k_in, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    cw = w.c_struct()
+    _check(load().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)), "qlora_linear_fwd")
+    return out
+
+
+def qlora_linear_bwd_x(w: NF4Weight, grad_h: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
+                       alpha: float, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """grad_x = dequant(W)^T grad_h + (alpha/r) A^T (B^T grad_h); grad_h is M x n_out."""
+    _dev_bf16(grad_h, "grad_h")
+    M = grad_h.shape[0]
+    r = 0 if A is None else A.shape[0]
+    A, B = _lora(A, B, r)
+    out = out if out is not None else torch.empty(M, w.k_in, dtype=torch.bfloat16, device=grad_h.device)
+    _dev_bf16(out, "out")
+    need = linear_workspace_size(M, w.n_out, w.k_in, r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=grad_h.device)
+    cw = w.c_struct()
+    _check(load().qlora_linear_bwd_x(ctypes.byref(cw), _ptr(grad_h), M, _ptr(A), _ptr(B), r, float(alpha),
+                                     _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "qlora_linear_bwd_x")
+    return out

@@ -1,0 +1,221 @@
+// api.cu -- the extern "C" boundary declared in include/qlora_nf4.h: argument checks,
+// size queries, path selection (few-token decode kernels or the tcgen05 GEMM) and launches.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "../../include/qlora_nf4.h"
+#include "kernels.h"
+
+namespace qn {
+
+thread_local uint64_t g_launches = 0;
+thread_local std::string g_err;
+
+void count_launch(int n) { g_launches += static_cast<uint64_t>(n); }
+
+namespace {
+
+qn_status fail(qn_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+qn_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) {
+        g_err.clear();
+        return QN_OK;
+    }
+    return fail(QN_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+qn_status check_shape(int64_t n, int64_t k) {
+    if (n < 0 || k < 0) return fail(QN_EINVAL, "negative size n_out=%lld k_in=%lld", (long long)n, (long long)k);
+    if (k % QN_BLOCK != 0) return fail(QN_ESHAPE, "k_in=%lld is not a multiple of %d", (long long)k, QN_BLOCK);
+    if (n > kMaxDim || k > kMaxDim) return fail(QN_ESHAPE, "n_out or k_in above 2^31-1");
+    if (n > 0 && k > 0 && (n * k) / QN_BLOCK >= (int64_t(1) << 40))
+        return fail(QN_ESHAPE, "more than 2^40 blocks");
+    return QN_OK;
+}
+
+qn_status check_weight(const qn_nf4_weight *w) {
+    if (!w) return fail(QN_EINVAL, "null weight struct");
+    qn_status s = check_shape(w->n_out, w->k_in);
+    if (s != QN_OK) return s;
+    if (w->n_out == 0 || w->k_in == 0) return QN_OK;
+    if (!w->codes || !w->absmax_q || !w->group_scale || !w->absmax_mean)
+        return fail(QN_EINVAL, "null pointer in the quantised weight");
+    if (!aligned16(w->codes)) return fail(QN_EALIGN, "codes not 16-byte aligned");
+    return QN_OK;
+}
+
+WeightView view(const qn_nf4_weight *w) {
+    return WeightView{w->n_out, w->k_in, w->codes, w->absmax_q, w->group_scale, w->absmax_mean};
+}
+
+qn_status check_lora(const void *A, const void *B, int r, float alpha) {
+    if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
+    if (r == 0) {
+        if (A || B) return fail(QN_EINVAL, "r == 0 requires A == B == NULL");
+        return QN_OK;
+    }
+    if (!A || !B) return fail(QN_EINVAL, "null adapter pointer with r=%d", r);
+    if (!aligned16(A) || !aligned16(B)) return fail(QN_EALIGN, "A or B not 16-byte aligned");
+    if (!(alpha == alpha) || alpha - alpha != 0.0f) return fail(QN_EINVAL, "alpha is not finite");
+    return QN_OK;
+}
+
+}  // namespace
+}  // namespace qn
+
+using namespace qn;
+
+extern "C" {
+
+const char *qn_status_string(qn_status s) {
+    switch (s) {
+        case QN_OK: return "ok";
+        case QN_EINVAL: return "invalid argument";
+        case QN_ESHAPE: return "unsupported shape";
+        case QN_EALIGN: return "misaligned pointer";
+        case QN_ECUDA: return "CUDA error";
+        case QN_EWORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *qn_last_error(void) { return g_err.c_str(); }
+
+uint64_t qn_launch_count(int reset) {
+    const uint64_t v = g_launches;
+    if (reset) g_launches = 0;
+    return v;
+}
+
+qn_status qn_nf4_sizes(int64_t n_out, int64_t k_in, size_t *codes_bytes, size_t *absmax_bytes, size_t *scale_bytes,
+                       size_t *mean_bytes) {
+    if (!codes_bytes || !absmax_bytes || !scale_bytes || !mean_bytes) return fail(QN_EINVAL, "null output pointer");
+    qn_status s = check_shape(n_out, k_in);
+    if (s != QN_OK) return s;
+    const int64_t nb = n_out * k_in / QN_BLOCK;
+    *codes_bytes = static_cast<size_t>(n_out * k_in / 2);
+    *absmax_bytes = static_cast<size_t>(nb);
+    *scale_bytes = sizeof(float) * static_cast<size_t>((nb + QN_GROUP - 1) / QN_GROUP);
+    *mean_bytes = sizeof(float);
+    g_err.clear();
+    return QN_OK;
+}
+
+qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_bytes) {
+    if (!ws_bytes) return fail(QN_EINVAL, "null output pointer");
+    qn_status s = check_shape(n_out, k_in);
+    if (s != QN_OK) return s;
+    *ws_bytes = quantize_workspace_bytes(n_out, k_in);
+    g_err.clear();
+    return QN_OK;
+}
+
+qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t ws_bytes, void *stream) {
+    qn_status s = check_weight(out);
+    if (s != QN_OK) return s;
+    if (out->n_out == 0 || out->k_in == 0) return QN_OK;
+    if (!W) return fail(QN_EINVAL, "null W");
+    if (!aligned16(W)) return fail(QN_EALIGN, "W not 16-byte aligned");
+    const size_t need = quantize_workspace_bytes(out->n_out, out->k_in);
+    if (!ws || ws_bytes < need) return fail(QN_EWORKSPACE, "quantize workspace needs %zu bytes", need);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
+    return cuda_status(launch_quantize(static_cast<const uint16_t *>(W), out->n_out, out->k_in, out->codes,
+                                       out->absmax_q, out->group_scale, out->absmax_mean, ws,
+                                       static_cast<cudaStream_t>(stream)),
+                       "nf4_quantize");
+}
+
+qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream) {
+    qn_status s = check_weight(w);
+    if (s != QN_OK) return s;
+    if (w->n_out == 0 || w->k_in == 0) return QN_OK;
+    if (!W_out) return fail(QN_EINVAL, "null W_out");
+    if (!aligned16(W_out)) return fail(QN_EALIGN, "W_out not 16-byte aligned");
+    return cuda_status(launch_dequant(view(w), static_cast<uint16_t *>(W_out), static_cast<cudaStream_t>(stream)),
+                       "nf4_dequantize");
+}
+
+qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, size_t *ws_bytes) {
+    if (!ws_bytes) return fail(QN_EINVAL, "null output pointer");
+    qn_status s = check_shape(n_out, k_in);
+    if (s != QN_OK) return s;
+    if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
+    if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
+    (void)M;
+    *ws_bytes = 256;  // the decode kernels need none; kept non-zero so callers can always pass a buffer
+    g_err.clear();
+    return QN_OK;
+}
+
+static qn_status check_linear(const qn_nf4_weight *w, const void *in, int64_t M, const void *A, const void *B, int r,
+                              float alpha, const void *out, void *ws, size_t ws_bytes) {
+    qn_status s = check_weight(w);
+    if (s != QN_OK) return s;
+    if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
+    s = check_lora(A, B, r, alpha);
+    if (s != QN_OK) return s;
+    if (M == 0 || w->n_out == 0 || w->k_in == 0) return QN_OK;
+    if (!in || !out) return fail(QN_EINVAL, "null activation or output pointer");
+    if (!aligned16(in) || !aligned16(out)) return fail(QN_EALIGN, "activation or output not 16-byte aligned");
+    if (in == out) return fail(QN_EINVAL, "output aliases the input");
+    size_t need = 0;
+    qlora_workspace_size(M, w->n_out, w->k_in, r, &need);
+    if (!ws || ws_bytes < need) return fail(QN_EWORKSPACE, "linear workspace needs %zu bytes", need);
+    return QN_OK;
+}
+
+qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B, int r,
+                           float alpha, void *h, void *ws, size_t ws_bytes, void *stream) {
+    qn_status s = check_linear(w, x, M, A, B, r, alpha, h, ws, ws_bytes);
+    if (s != QN_OK) return s;
+    if (M == 0 || w->n_out == 0) return QN_OK;
+    const float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
+    const WeightView wv = view(w);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t *xp = static_cast<const uint16_t *>(x);
+    uint16_t *hp = static_cast<uint16_t *>(h);
+    for (int64_t m0 = 0; m0 < M; m0 += kDecodeMaxM) {
+        const int mc = static_cast<int>(M - m0 < kDecodeMaxM ? M - m0 : kDecodeMaxM);
+        cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, static_cast<const uint16_t *>(A),
+                                          static_cast<const uint16_t *>(B), r, sc, hp + m0 * w->n_out, st);
+        if (e != cudaSuccess) return cuda_status(e, "qlora_linear_fwd");
+    }
+    return cuda_status(cudaSuccess, "");
+}
+
+qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A, const void *B,
+                             int r, float alpha, void *grad_x, void *ws, size_t ws_bytes, void *stream) {
+    qn_status s = check_linear(w, grad_h, M, A, B, r, alpha, grad_x, ws, ws_bytes);
+    if (s != QN_OK) return s;
+    if (M == 0 || w->k_in == 0) return QN_OK;
+    const float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
+    const WeightView wv = view(w);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t *gp = static_cast<const uint16_t *>(grad_h);
+    uint16_t *xp = static_cast<uint16_t *>(grad_x);
+    constexpr int kChunk = 32;
+    for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
+        const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);
+        cudaError_t e = launch_decode_bwd(wv, gp + m0 * w->n_out, mc, static_cast<const uint16_t *>(A),
+                                          static_cast<const uint16_t *>(B), r, sc, xp + m0 * w->k_in, st);
+        if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
+    }
+    return cuda_status(cudaSuccess, "");
+}
+
+}  // extern "C"

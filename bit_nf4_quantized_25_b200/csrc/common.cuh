@@ -1,0 +1,101 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of the NF4 + LoRA linear layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qn {
+
+constexpr int kBlock = 64;   // weights per absmax block
+constexpr int kGroup = 256;  // blocks per double-quantisation group
+
+// The 16 NF4 values, ascending, as printed in "QLoRA paper notes" (tqpw.cn),
+// section "NormalFloat Quantization (NF4)". Each is an exact fp32 value.
+#define QN_NF4_VALUES                                                                       \
+    {-1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,              \
+     -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,            \
+     0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f, \
+     0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f}
+
+static __constant__ float c_nf4_table[16] = QN_NF4_VALUES;
+
+__host__ __device__ inline float nf4_value(int i) {
+#ifdef __CUDA_ARCH__
+    return c_nf4_table[i];
+#else
+    constexpr float T[16] = QN_NF4_VALUES;
+    return T[i];
+#endif
+}
+
+// ---------------------------------------------------------------- loads
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Cached (L1) read-only loads for small operands that many warps re-read.
+__device__ __forceinline__ uint4 ld_ro_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+__device__ __forceinline__ uint2 ld_ro_v2(const void *p) { return __ldg(reinterpret_cast<const uint2 *>(p)); }
+__device__ __forceinline__ uint32_t ld_ro_u32(const void *p) { return __ldg(reinterpret_cast<const unsigned int *>(p)); }
+__device__ __forceinline__ uint16_t ld_ro_u16(const void *p) { return __ldg(reinterpret_cast<const unsigned short *>(p)); }
+
+// ------------------------------------------------------------ numerics
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t v) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(v), __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+__device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float v) {
+    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Block constant c'_b = fma(decode(q_b), sigma_g, mu), single rounding.
+__device__ __forceinline__ float block_constant(uint8_t q, float sigma, float mu) {
+    return __fmaf_rn(e4m3_to_f32(q), sigma, mu);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// D = A(16x16, row) * B(16x8, col) + C, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------- programmatic launch
+// Wait until the preceding grid on the stream has completed (no-op when the
+// kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+}  // namespace qn

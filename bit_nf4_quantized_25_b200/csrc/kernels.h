@@ -1,0 +1,52 @@
+// kernels.h -- internal launchers (host side) of the sm_100a kernels. Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qn {
+
+struct WeightView {
+    int64_t n, k;  // W is n x k, k % 64 == 0
+    const uint8_t *codes;
+    const uint8_t *q;
+    const float *sigma;
+    const float *mu;
+};
+
+// Lookup used by the quantiser: the interval [-1, 1] split into 64 cells of
+// width 1/32 plus the point 1.0; for cell j, `base[j]` is the number of code
+// thresholds below the cell and `thr[j]` the single threshold inside the cell
+// (or 2.0 when there is none).
+struct QuantCells {
+    float thr[65];
+    int base[65];
+};
+
+// Launch counter (per host thread).
+void count_launch(int n = 1);
+
+// nf4_quantize: two kernels plus a memset of the exponent bins.
+cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
+                            float *mu, void *ws, cudaStream_t s);
+size_t quantize_workspace_bytes(int64_t n, int64_t k);
+
+// nf4_dequantize.
+cudaError_t launch_dequant(const WeightView &w, uint16_t *out, cudaStream_t s);
+
+// Token-count bound of the decode kernels (M <= kDecodeMaxM).
+constexpr int kDecodeMaxM = 64;
+
+// h = dequant(W) x + s B (A x) for M <= kDecodeMaxM tokens, one launch.
+cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A,
+                              const uint16_t *B, int r, float s, uint16_t *h, cudaStream_t st);
+// grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h) for M <= kDecodeMaxM tokens.
+cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
+                              const uint16_t *B, int r, float s, uint16_t *gx, cudaStream_t st);
+
+// Adapter down-projection for many tokens: out[m, j] = bf16(s * sum_i act[m,i] S(j,i)),
+// S(j,i) = small[j*ldj + i*ldk]; out is M x RT with zeros for j >= r. Clears *err.
+cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, int *err, cudaStream_t st);
+
+}  // namespace qn

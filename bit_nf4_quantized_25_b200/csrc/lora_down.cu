@@ -1,0 +1,121 @@
+// lora_down.cu -- adapter down-projection for many tokens, the operand of the GEMM's
+// extra up-projection steps:
+//   fwd: t[m, j] = bf16(s * sum_k x[m,k] A[j,k])         (A: r x k)
+//   bwd: u[m, j] = bf16(s * sum_n grad_h[m,n] B[n,j])    (B: n x r)
+// written as a row-major M x RT bf16 matrix, RT = r rounded up to 64, zeros for j >= r.
+// "How does QLoRA work for training?" (aivaro.ru), section 2: B (d x r), A (r x k).
+//
+// HBM-bound on the activations (read once). One CTA = 16 tokens; its 4 warps split the
+// reduction, each running mma.sync m16n8k16 (tokens x adapter rank), and reduce through
+// shared memory. Thread 0 of CTA 0 also clears the GEMM's error word.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qn {
+
+namespace {
+
+constexpr int kLdWarps = 4;
+
+struct LoraDownParams {
+    const uint16_t *act;  // M x red
+    int64_t M, red;
+    const uint16_t *small;  // element (j, kk) at small[j * ldj + kk * ldk]
+    int64_t ldj, ldk;
+    int r;
+    float s;
+    uint16_t *out;  // M x RT
+    int RT;
+    int *err;
+};
+
+template <int NT>  // 8*NT adapter columns per pass
+__global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParams p) {
+    __shared__ float red[kLdWarps][16][8 * NT];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.err) *p.err = 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 16;
+    const int64_t rowA = m0 + g, rowB = m0 + g + 8;
+    const bool vA = rowA < p.M, vB = rowB < p.M;
+    const uint16_t *aA = p.act + (vA ? rowA : 0) * p.red;
+    const uint16_t *aB = p.act + (vB ? rowB : 0) * p.red;
+    const int64_t steps = p.red / 16;  // red is a multiple of 16 on this path
+    const int64_t s_lo = steps * warp / kLdWarps, s_hi = steps * (warp + 1) / kLdWarps;
+
+    for (int j0 = 0; j0 < p.RT; j0 += 8 * NT) {
+        float d[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.0f;
+        if (j0 < p.r) {
+            for (int64_t st = s_lo; st < s_hi; ++st) {
+                const int64_t k0 = st * 16;
+                const uint32_t a0 = vA ? ld_ro_u32(aA + k0 + 2 * t) : 0u;
+                const uint32_t a1 = vB ? ld_ro_u32(aB + k0 + 2 * t) : 0u;
+                const uint32_t a2 = vA ? ld_ro_u32(aA + k0 + 2 * t + 8) : 0u;
+                const uint32_t a3 = vB ? ld_ro_u32(aB + k0 + 2 * t + 8) : 0u;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int j = j0 + nt * 8 + g;
+                    uint32_t b0 = 0u, b1 = 0u;
+                    if (j < p.r) {
+                        const uint16_t *sp = p.small + static_cast<int64_t>(j) * p.ldj;
+                        if (p.ldk == 1) {
+                            b0 = ld_ro_u32(sp + k0 + 2 * t);
+                            b1 = ld_ro_u32(sp + k0 + 2 * t + 8);
+                        } else {
+                            const int64_t L = p.ldk;
+                            b0 = ld_ro_u16(sp + (k0 + 2 * t) * L) | (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 1) * L)) << 16);
+                            b1 = ld_ro_u16(sp + (k0 + 2 * t + 8) * L) |
+                                 (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 9) * L)) << 16);
+                        }
+                    }
+                    mma_16816(d[nt], a0, a1, a2, a3, b0, b1);
+                }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            red[warp][g][nt * 8 + 2 * t] = d[nt][0];
+            red[warp][g][nt * 8 + 2 * t + 1] = d[nt][1];
+            red[warp][g + 8][nt * 8 + 2 * t] = d[nt][2];
+            red[warp][g + 8][nt * 8 + 2 * t + 1] = d[nt][3];
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < 16 * 8 * NT; i += blockDim.x) {
+            const int row = i / (8 * NT), col = i % (8 * NT);
+            const int64_t m = m0 + row;
+            const int j = j0 + col;
+            if (m < p.M && j < p.RT) {
+                float v = 0.0f;
+                if (j < p.r) {
+#pragma unroll
+                    for (int w = 0; w < kLdWarps; ++w) v += red[w][row][col];
+                    v *= p.s;
+                }
+                p.out[m * p.RT + j] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, int *err, cudaStream_t st) {
+    LoraDownParams p{act, M, red, small, ldj, ldk, r, s, out, RT, err};
+    const unsigned grid = static_cast<unsigned>((M + 15) / 16);
+    if (r <= 8)
+        k_lora_down<1><<<grid, kLdWarps * 32, 0, st>>>(p);
+    else if (r <= 16)
+        k_lora_down<2><<<grid, kLdWarps * 32, 0, st>>>(p);
+    else if (r <= 32)
+        k_lora_down<4><<<grid, kLdWarps * 32, 0, st>>>(p);
+    else
+        k_lora_down<8><<<grid, kLdWarps * 32, 0, st>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace qn

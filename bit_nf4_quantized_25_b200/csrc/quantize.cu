@@ -1,0 +1,277 @@
+// quantize.cu -- nf4_quantize on sm_100a: NF4 codes with blockwise absmax (64 weights) and
+// double quantisation of the block absmaxes (tensor mean, FP8 E4M3 in groups of 256).
+//
+// "QLoRA paper notes" (tqpw.cn), sections "NormalFloat Quantization (NF4)" and
+// "Double Quantization"; "How does QLoRA work for training?" (aivaro.ru), section 5.
+//
+// Kernel 1 (HBM-bound, one pass over W): each 8-lane group owns one 64-weight block
+// (16-byte coalesced loads), takes the absmax with three shuffles, divides each weight
+// by it (IEEE division), picks the code through a 65-cell lookup of the 15 decision
+// thresholds, packs 8 codes per 32-bit word, writes the fp32 absmax to the workspace
+// and adds it to 256 exponent bins (integer sums, so the tensor sum is exact and
+// independent of scheduling).
+// Kernel 2 (1/64 of the data): every CTA rebuilds the exact mean from the bins, then
+// each warp double-quantises one group of 256 block absmaxes.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qn {
+
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kDqThreads = 256;
+constexpr size_t kBinsBytes = 256 * sizeof(unsigned long long);
+
+__device__ __forceinline__ uint32_t mag_max2(uint32_t u) {
+    return max(u & 0x7fffu, (u >> 16) & 0x7fffu);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ codes, float *__restrict__ cblk,
+               unsigned long long *__restrict__ bins, QuantCells cells) {
+    __shared__ float s_thr[65];
+    __shared__ int s_base[65];
+    __shared__ unsigned s_bins[256];
+    for (int i = threadIdx.x; i < 65; i += blockDim.x) {
+        s_thr[i] = cells.thr[i];
+        s_base[i] = cells.base[i];
+    }
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0u;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane >> 3;  // which of the warp's 4 blocks
+    const int l8 = lane & 7;    // 8 weights of that block
+    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    uint32_t cached_e = 0u, cached_sum = 0u;
+
+    for (int64_t b0 = warp_global * 4; b0 < nb; b0 += nwarps * 4) {
+        const int64_t b = b0 + sub;
+        const bool valid = b < nb;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) v = ld_nc_v4(W + b * 8 + l8);
+        uint32_t m = max(max(mag_max2(v.x), mag_max2(v.y)), max(mag_max2(v.z), mag_max2(v.w)));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        const float c = __uint_as_float(m << 16);  // block absmax, exact (a bf16 value)
+        uint32_t word = 0x77777777u;               // all-zero block: code 7 everywhere
+        if (c != 0.0f) {
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            word = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bits = (i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16);
+                const float x = __fdiv_rn(__uint_as_float(bits), c);
+                int j = __float2int_rz(__fmaf_rn(x, 32.0f, 32.0f));
+                j = min(max(j, 0), 64);
+                const int code = s_base[j] + (x > s_thr[j] ? 1 : 0);
+                word |= static_cast<uint32_t>(code) << (4 * i);
+            }
+        }
+        if (valid) {
+            codes[b * 8 + l8] = word;
+            if (l8 == 0) {
+                cblk[b] = c;
+                const uint32_t e = m >> 7;
+                const uint32_t sig = (e == 0u) ? (m & 0x7fu) : (0x80u | (m & 0x7fu));
+                if (e == cached_e) {
+                    cached_sum += sig;
+                } else {
+                    if (cached_sum) atomicAdd(&s_bins[cached_e], cached_sum);
+                    cached_e = e;
+                    cached_sum = sig;
+                }
+            }
+        }
+    }
+    if (cached_sum) atomicAdd(&s_bins[cached_e], cached_sum);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (s_bins[i]) atomicAdd(&bins[i], static_cast<unsigned long long>(s_bins[i]));
+}
+
+// Exact mean of the block absmaxes from the exponent bins, rounded once to fp32.
+// bins[e] = sum of the 8-bit significands of the absmaxes with exponent field e;
+// such an absmax equals significand * 2^(p - 133) with p = max(e - 1, 0). Run by
+// one thread.
+__device__ float mean_from_bins(const unsigned long long *bins, int64_t nb) {
+    uint64_t S[6] = {0, 0, 0, 0, 0, 0};  // S * 2^-133 is the exact sum
+    for (int e = 0; e < 256; ++e) {
+        const uint64_t v = bins[e];
+        if (v == 0) continue;
+        const int p = e ? e - 1 : 0;
+        const int li = p >> 6, sh = p & 63;
+        uint64_t add[2] = {v << sh, sh ? (v >> (64 - sh)) : 0ull};
+        uint64_t carry = 0;
+        for (int i = li; i < 6; ++i) {
+            const uint64_t a = (i - li < 2) ? add[i - li] : 0ull;
+            const uint64_t t = S[i] + a;
+            const uint64_t c1 = t < a;
+            const uint64_t t2 = t + carry;
+            const uint64_t c2 = t2 < carry;
+            S[i] = t2;
+            carry = c1 + c2;
+        }
+    }
+    int top = 5;
+    while (top >= 0 && S[top] == 0) --top;
+    if (top < 0 || nb <= 0) return 0.0f;
+    const int L = top * 64 + (64 - __clzll(static_cast<long long>(S[top])));  // bit length
+    // S64 = the top 64 bits of S (left-aligned), e2 = L - 64: S = S64 * 2^e2 + rest.
+    uint64_t S64;
+    bool sticky = false;
+    const int e2 = L - 64;
+    if (e2 <= 0) {
+        S64 = S[0] << (-e2);  // L <= 64: S is limb 0
+    } else {
+        const int li = e2 >> 6, sh = e2 & 63;
+        S64 = (sh == 0) ? S[li] : ((S[li] >> sh) | (S[li + 1] << (64 - sh)));
+        for (int i = 0; i < li && !sticky; ++i) sticky = S[i] != 0;
+        if (sh) sticky = sticky || (S[li] & ((1ull << sh) - 1)) != 0;
+    }
+    // Quotient with >= 40 significant bits: S64 / nb alone when that is wide enough,
+    // else one more 64-bit division step on the remainder (nb < 2^40 keeps r1 << 24
+    // and Q below 2^64). value = (Q + frac) * 2^eb.
+    const uint64_t n = static_cast<uint64_t>(nb);
+    const uint64_t q1 = S64 / n, r1 = S64 % n;
+    uint64_t Q;
+    int eb;  // exponent of Q's least significant bit
+    if (q1 >> 39) {
+        Q = q1;
+        sticky = sticky || (r1 != 0);
+        eb = e2 - 133;
+    } else {
+        const uint64_t q2 = (r1 << 24) / n, r2 = (r1 << 24) % n;
+        Q = (q1 << 24) | q2;
+        sticky = sticky || (r2 != 0);
+        eb = e2 - 24 - 133;
+    }
+    const int lead = 63 - __clzll(static_cast<long long>(Q));
+    const int lsb_exp = max(lead + eb - 23, -149);
+    const int drop = lsb_exp - eb;
+    uint64_t mant;
+    int rbit;
+    if (drop > 64) {
+        mant = 0;
+        rbit = 0;
+        sticky = true;
+    } else if (drop == 64) {
+        mant = 0;
+        rbit = static_cast<int>(Q >> 63);
+        sticky = sticky || (Q & ~(1ull << 63)) != 0;
+    } else {
+        mant = Q >> drop;
+        rbit = static_cast<int>((Q >> (drop - 1)) & 1ull);
+        if (drop > 1) sticky = sticky || (Q & ((1ull << (drop - 1)) - 1)) != 0;
+    }
+    if (rbit && (sticky || (mant & 1ull))) mant += 1;
+    return ldexpf(static_cast<float>(mant), lsb_exp);
+}
+
+__global__ void __launch_bounds__(kDqThreads)
+k_double_quant(const float *__restrict__ cblk, int64_t nb, const unsigned long long *__restrict__ bins,
+               uint8_t *__restrict__ q, float *__restrict__ sigma, float *__restrict__ mu_out) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ float s_mu;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = bins[i];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_mu = mean_from_bins(s_bins, nb);
+        if (blockIdx.x == 0) *mu_out = s_mu;
+    }
+    __syncthreads();
+    const float mu = s_mu;
+    const int lane = threadIdx.x & 31;
+    const int64_t ng = (nb + kGroup - 1) / kGroup;
+    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t g = warp_global; g < ng; g += nwarps) {
+        const int64_t b0 = g * kGroup;
+        float d[8];
+        float S = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t b = b0 + i * 32 + lane;
+            d[i] = (b < nb) ? __fsub_rn(cblk[b], mu) : 0.0f;
+            S = fmaxf(S, fabsf(d[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) S = fmaxf(S, __shfl_xor_sync(0xffffffffu, S, o));
+        const float sg = __fdiv_rn(S, 448.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t b = b0 + i * 32 + lane;
+            if (b < nb) q[b] = (sg == 0.0f) ? static_cast<uint8_t>(0) : f32_to_e4m3_satfinite(__fdiv_rn(d[i], sg));
+        }
+        if (lane == 0) sigma[g] = sg;
+    }
+}
+
+// Decision thresholds t_i = largest fp32 not above the midpoint of table values i and
+// i+1; for an fp32 x, "x > t_i" equals "x is nearer to value i+1 than to value i, or
+// at equal distance goes to the lower index".
+QuantCells make_cells() {
+    QuantCells c;
+    double t[15];
+    for (int i = 0; i < 15; ++i) {
+        const double m = (static_cast<double>(nf4_value(i)) + static_cast<double>(nf4_value(i + 1))) * 0.5;
+        float f = static_cast<float>(m);
+        if (static_cast<double>(f) > m) f = nextafterf(f, -2.0f);
+        t[i] = f;
+    }
+    for (int j = 0; j <= 64; ++j) {
+        const double lo = -1.0 + j / 32.0, hi = (j == 64) ? 1.0 : -1.0 + (j + 1) / 32.0;
+        int base = 0;
+        float thr = 2.0f;
+        for (int i = 0; i < 15; ++i) {
+            if (t[i] < lo) ++base;
+            else if (t[i] < hi || (j == 64 && t[i] <= hi)) thr = static_cast<float>(t[i]);
+        }
+        c.base[j] = base;
+        c.thr[j] = thr;
+    }
+    return c;
+}
+
+}  // namespace
+
+size_t quantize_workspace_bytes(int64_t n, int64_t k) {
+    const int64_t nb = n * k / kBlock;
+    return kBinsBytes + ((static_cast<size_t>(nb) * sizeof(float) + 255) & ~size_t(255));
+}
+
+cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
+                            float *mu, void *ws, cudaStream_t s) {
+    static const QuantCells cells = make_cells();
+    const int64_t nb = n * k / kBlock;
+    if (nb == 0) return cudaSuccess;
+    auto *bins = static_cast<unsigned long long *>(ws);
+    auto *cblk = reinterpret_cast<float *>(static_cast<char *>(ws) + kBinsBytes);
+    cudaError_t e = cudaMemsetAsync(bins, 0, kBinsBytes, s);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // 32 blocks per CTA per pass; enough CTAs for 8 per SM, never more than needed,
+    // and few enough passes per thread that the 32-bit smem bins cannot overflow.
+    int64_t grid = (nb + 31) / 32;
+    grid = grid < static_cast<int64_t>(sms) * 8 ? grid : static_cast<int64_t>(sms) * 8;
+    const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
+    if (grid < min_grid) grid = min_grid;
+    k_quant_blocks<<<static_cast<unsigned>(grid), kQuantThreads, 0, s>>>(
+        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, cells);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t ng = (nb + kGroup - 1) / kGroup;
+    int64_t grid2 = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
+    grid2 = grid2 < static_cast<int64_t>(sms) * 4 ? grid2 : static_cast<int64_t>(sms) * 4;
+    k_double_quant<<<static_cast<unsigned>(grid2), kDqThreads, 0, s>>>(cblk, nb, bins, q, sigma, mu);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace qn

@@ -1,0 +1,171 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) NF4 + double-quant + LoRA linear layer.
+ *
+ * The library quantises a frozen base weight W (n_out x k_in, bf16) to 4-bit
+ * NormalFloat codes with one absmax per 64 consecutive weights, double-quantises
+ * those absmaxes, and evaluates the QLoRA linear layer and its input gradient:
+ *
+ *   h      = dequant(W) x + s * B (A x)                       (forward)
+ *   grad_x = dequant(W)^T grad_h + s * A^T (B^T grad_h)       (input gradient)
+ *   s      = alpha / r
+ *
+ * Sources (page title, section):
+ *   - NF4 table, 64-weight blocks, double quantisation of the block constants to
+ *     FP8 in groups of 256 after subtracting their mean: "QLoRA paper notes"
+ *     (tqpw.cn), sections "NormalFloat Quantization (NF4)" and
+ *     "Double Quantization".
+ *   - h = Wx + BAx and h = dequant(W_NF4) x + BAx, dequantisation to bf16 for the
+ *     matmul: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), the two
+ *     forward equations and the list of the four configuration knobs.
+ *   - Shapes W (d x k), B (d x r), A (r x k); one constant per 64 weights;
+ *     gradients through the dequantised, frozen base: "How does QLoRA work for
+ *     training?" (aivaro.ru), sections 2, 5 and 7.
+ *   - lora_alpha as the adapter's scaling factor: LoRA/QLoRA talk summary
+ *     (spark.aweffr.cn), "practice guide" configuration list.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are row-major and contiguous. bf16 tensors are passed as
+ *     `const void *` / `void *` pointing at 16-bit bf16 values.
+ *   - Every tensor pointer is a DEVICE pointer (memory of the current CUDA
+ *     device), except the `qn_nf4_weight` struct itself, which lives in host
+ *     memory and holds device pointers. Sizes are element counts unless named
+ *     *_bytes.
+ *   - The caller owns and allocates every buffer, workspaces included. The
+ *     library allocates no memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *     enqueues work on it and returns; results are ready when the stream is.
+ *   - Argument errors are returned synchronously, before anything is enqueued.
+ *     QN_ECUDA means a launch failed; faults inside a kernel surface at the
+ *     caller's next synchronisation of the stream.
+ *   - Calls are reentrant. Two calls that run concurrently on the GPU must not
+ *     share an output buffer or a workspace.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QN_OK = 0,
+    QN_EINVAL = 1,     /* null pointer, negative size, bad r or alpha          */
+    QN_ESHAPE = 2,     /* k_in not a multiple of 64, or a size above the limits */
+    QN_EALIGN = 3,     /* a tensor pointer is not 16-byte aligned               */
+    QN_ECUDA = 4,      /* a CUDA launch or attribute call failed                */
+    QN_EWORKSPACE = 5  /* workspace pointer null or smaller than required       */
+} qn_status;
+
+/* Blocking of the format: one absmax per QN_BLOCK consecutive weights of the
+ * row-major flattened W, one fp32 scale per QN_GROUP consecutive blocks. */
+#define QN_BLOCK 64
+#define QN_GROUP 256
+/* Largest supported LoRA rank. */
+#define QN_MAX_RANK 256
+
+/* A quantised weight. The struct is host memory; the four buffers are device
+ * memory owned by the caller, with the sizes qn_nf4_sizes() returns.
+ *   codes        : n_out*k_in/2 bytes. Weight e = n*k_in + k (row-major) is the
+ *                  low nibble of byte e/2 when e is even, the high nibble when e
+ *                  is odd. A nibble is an index 0..15 into the NF4 table
+ *                  (ascending values, index 7 is 0.0).
+ *   absmax_q     : nb = n_out*k_in/64 bytes, the FP8 E4M3 (finite variant,
+ *                  max 448) code of d_b = absmax_b - mean, divided by the
+ *                  group scale.
+ *   group_scale  : ng = ceil(nb/256) floats; group g covers blocks
+ *                  [256 g, 256 g + 256) of the flattened block index (groups may
+ *                  straddle rows).
+ *   absmax_mean  : 1 float, the exact mean of all nb block absmaxes, rounded
+ *                  once to fp32.
+ * Block constant: c'_b = fma(e4m3_decode(absmax_q[b]), group_scale[b/256],
+ * absmax_mean) in fp32; dequantised weight: NF4[code] * c'_b. */
+typedef struct {
+    int64_t n_out;
+    int64_t k_in;
+    uint8_t *codes;
+    uint8_t *absmax_q;
+    float *group_scale;
+    float *absmax_mean;
+} qn_nf4_weight;
+
+/* Byte sizes of the four buffers of a quantised n_out x k_in weight.
+ * Errors: QN_EINVAL (null output pointer, negative size), QN_ESHAPE
+ * (k_in % 64 != 0). Host-only; touches no GPU. */
+qn_status qn_nf4_sizes(int64_t n_out, int64_t k_in, size_t *codes_bytes, size_t *absmax_bytes,
+                       size_t *scale_bytes, size_t *mean_bytes);
+
+/* Workspace bytes nf4_quantize needs for an n_out x k_in weight. Host-only. */
+qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_bytes);
+
+/* nf4_quantize -- W (n_out x k_in bf16, device) -> the quantised weight `out`.
+ * Per block of 64: absmax c_b, code = index of the table value nearest to
+ * fl32(w / c_b) (ties to the lower index; c_b == 0 gives code 7), two codes per
+ * byte. Then mean mu of all c_b (exact, rounded once), d_b = fl32(c_b - mu),
+ * group scale sigma_g = fl32(max_b |d_b| / 448), absmax_q[b] =
+ * e4m3_rn_satfinite(fl32(d_b / sigma_g)) (0 when sigma_g == 0).
+ * Source: "QLoRA paper notes" (tqpw.cn), "NormalFloat Quantization (NF4)" and
+ * "Double Quantization"; "How does QLoRA work for training?" (aivaro.ru) 5.
+ * W must not contain NaN or Inf (the result is then unspecified).
+ * ws: device workspace of at least qn_quantize_workspace_size() bytes, 256-byte
+ * aligned; its contents on entry do not matter.
+ * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (W or codes not 16-byte aligned),
+ * QN_EWORKSPACE, QN_ECUDA. */
+qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t ws_bytes, void *stream);
+
+/* nf4_dequantize -- quantised weight -> W_out (n_out x k_in bf16, device):
+ * W_out[e] = bf16_rn(fl32(NF4[code_e] * c'_b)).
+ * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), the
+ * dequantisation step to bf16 before the matmul.
+ * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (codes or W_out not 16-byte
+ * aligned), QN_ECUDA. */
+qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream);
+
+/* Workspace bytes qlora_linear_fwd / qlora_linear_bwd_x need for M tokens,
+ * an n_out x k_in weight and rank r (0 <= r <= 256). Host-only. */
+qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, size_t *ws_bytes);
+
+/* qlora_linear_fwd -- h = dequant(W) x + (alpha/r) B (A x), per token row:
+ *   h[m, n] = sum_k W'[n,k] x[m,k] + s * sum_j B[n,j] sum_k A[j,k] x[m,k].
+ *   x : M x k_in bf16 (tokens x features); A : r x k_in bf16; B : n_out x r bf16;
+ *   h : M x n_out bf16 (written, must not alias x, A or B).
+ * fp32 accumulation; the block constant is applied in fp32; the adapter
+ * product A x is rounded to bf16 once before the up-projection.
+ * r == 0 means no adapter (A and B must then be NULL; alpha is ignored).
+ * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), forward
+ * equations; "How does QLoRA work for training?" (aivaro.ru) 2.
+ * ws: device workspace of at least qlora_workspace_size() bytes, 256-byte
+ * aligned, contents on entry irrelevant. M may be 0 (nothing is enqueued).
+ * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (x, h, codes, A or B not 16-byte
+ * aligned), QN_EWORKSPACE, QN_ECUDA. */
+qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
+                           int r, float alpha, void *h, void *ws, size_t ws_bytes, void *stream);
+
+/* qlora_linear_bwd_x -- input gradient through the frozen base and the adapter:
+ *   grad_x[m, k] = sum_n grad_h[m,n] W'[n,k] + s * sum_j A[j,k] sum_n grad_h[m,n] B[n,j].
+ *   grad_h : M x n_out bf16; grad_x : M x k_in bf16 (written, no aliasing).
+ * W is frozen: nothing is written to the quantised weight.
+ * Source: "How does QLoRA work for training?" (aivaro.ru) 7 (weights are
+ * dequantised on the fly for the gradient and not updated).
+ * Same workspace, alignment and error rules as qlora_linear_fwd. */
+qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A,
+                             const void *B, int r, float alpha, void *grad_x, void *ws, size_t ws_bytes,
+                             void *stream);
+
+/* Static description of a status code. */
+const char *qn_status_string(qn_status s);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char *qn_last_error(void);
+
+/* Number of this library's kernels enqueued on the calling host thread since
+ * the last reset (a launch counter for benchmarks). */
+uint64_t qn_launch_count(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+function declared in include/*.h, answers size queries, and rejects bad arguments
+before anything is enqueued (no call here reaches the GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_nf4_quantized_25_b200 import binding, build
+    build.build()
+    return binding.load()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                             src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for f in ("nf4_quantize", "qlora_linear_fwd", "qlora_linear_bwd_x", "nf4_dequantize"):
+        assert f in names
+
+
+def test_library_exports_every_declared_function(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def _sizes(lib, n, k):
+    a, b, c, d = (ctypes.c_size_t() for _ in range(4))
+    st = lib.qn_nf4_sizes(n, k, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(d))
+    return st, (a.value, b.value, c.value, d.value)
+
+
+def test_sizes_give_the_double_quant_overhead(lib):
+    # "QLoRA & PEFT family" (ai-reference-codex) 3.3: 0.5 -> 0.127 bit per parameter.
+    st, (cb, ab, sb, mb) = _sizes(lib, 4096, 4096)
+    assert st == 0
+    n = 4096 * 4096
+    assert cb == n // 2 and ab == n // 64 and sb == 4 * (n // 64 // 256) and mb == 4
+    assert (8 * ab + 8 * sb) / n == 0.126953125
+    assert round((8 * ab + 8 * sb) / n, 3) == 0.127
+
+
+def test_7b_stack_is_about_3p5_gb(lib):
+    # "QLoRA & PEFT family" 3.1: a 7B base goes from 14 GB to about 3.5 GB in 4 bits.
+    shapes = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
+    total = 0
+    for n, k in shapes:
+        st, s = _sizes(lib, n, k)
+        assert st == 0
+        total += sum(s)
+    total *= 32
+    assert 3.2e9 < total < 3.5e9
+
+
+def test_size_errors(lib):
+    st, _ = _sizes(lib, 4096, 100)
+    assert st == 2  # QN_ESHAPE
+    st, _ = _sizes(lib, -1, 64)
+    assert st == 1  # QN_EINVAL
+
+
+def _weight(n=128, k=128, base=0x100000):
+    from bit_nf4_quantized_25_b200.binding import CWeight
+    return CWeight(n, k, base, base + 0x10000, base + 0x20000, base + 0x30000)
+
+
+def test_linear_argument_errors_before_launch(lib):
+    from bit_nf4_quantized_25_b200.binding import QN_EALIGN, QN_EINVAL, QN_ESHAPE, QN_EWORKSPACE
+    w = _weight()
+    P = ctypes.c_void_p
+    x, h, A, B, ws = P(0x200000), P(0x300000), P(0x400000), P(0x500000), P(0x600000)
+    f = lib.qlora_linear_fwd
+    assert f(ctypes.byref(w), x, 4, A, B, 300, 1.0, h, ws, 1 << 20, None) == QN_EINVAL  # r > 256
+    assert f(ctypes.byref(w), x, 4, A, None, 4, 1.0, h, ws, 1 << 20, None) == QN_EINVAL  # null B
+    assert f(ctypes.byref(w), x, 4, A, B, 0, 1.0, h, ws, 1 << 20, None) == QN_EINVAL  # r=0 with A, B
+    assert f(ctypes.byref(w), P(0x200008), 4, A, B, 4, 1.0, h, ws, 1 << 20, None) == QN_EALIGN
+    assert f(ctypes.byref(w), x, 4, A, B, 4, 1.0, x, ws, 1 << 20, None) == QN_EINVAL  # aliasing
+    assert f(ctypes.byref(w), x, 4, A, B, 4, 1.0, h, None, 0, None) == QN_EWORKSPACE
+    assert f(ctypes.byref(w), x, -1, A, B, 4, 1.0, h, ws, 1 << 20, None) == QN_EINVAL
+    assert f(ctypes.byref(w), x, 4, A, B, 4, float("nan"), h, ws, 1 << 20, None) == QN_EINVAL
+    bad = _weight(128, 100)
+    assert f(ctypes.byref(bad), x, 4, A, B, 4, 1.0, h, ws, 1 << 20, None) == QN_ESHAPE
+    assert lib.qn_last_error().decode() != ""
+    g = lib.qlora_linear_bwd_x
+    assert g(ctypes.byref(w), x, 4, A, B, 4, 1.0, h, None, 0, None) == QN_EWORKSPACE
+    assert g(None, x, 4, A, B, 4, 1.0, h, ws, 1 << 20, None) == QN_EINVAL
+
+
+def test_quantize_argument_errors_before_launch(lib):
+    from bit_nf4_quantized_25_b200.binding import QN_EALIGN, QN_EINVAL, QN_EWORKSPACE
+    w = _weight()
+    P = ctypes.c_void_p
+    q = lib.nf4_quantize
+    assert q(None, ctypes.byref(w), P(0x700000), 1 << 20, None) == QN_EINVAL
+    assert q(P(0x800004), ctypes.byref(w), P(0x700000), 1 << 20, None) == QN_EALIGN
+    assert q(P(0x800000), ctypes.byref(w), P(0x700000), 16, None) == QN_EWORKSPACE
+    assert q(P(0x800000), ctypes.byref(w), P(0x700010), 1 << 20, None) == QN_EALIGN
+    ws = ctypes.c_size_t()
+    assert lib.qn_quantize_workspace_size(128, 128, ctypes.byref(ws)) == 0 and ws.value >= 4 * 256
+    d = lib.nf4_dequantize
+    assert d(ctypes.byref(w), None, None) == QN_EINVAL
+    assert d(ctypes.byref(w), P(0x900002), None) == QN_EALIGN
+
+
+def test_empty_problems_enqueue_nothing(lib):
+    w = _weight(0, 64)
+    P = ctypes.c_void_p
+    before = lib.qn_launch_count(0)
+    assert lib.nf4_quantize(P(0x800000), ctypes.byref(w), None, 0, None) == 0
+    w2 = _weight()
+    assert lib.qlora_linear_fwd(ctypes.byref(w2), P(0x200000), 0, None, None, 0, 0.0, P(0x300000), None, 0, None) == 0
+    assert lib.qn_launch_count(0) == before
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.qn_status_string(s)

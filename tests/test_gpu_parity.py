@@ -1,0 +1,265 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes, FP8 constants, group scales, the mean and the standalone dequantisation must
+match bit for bit. h and grad_x (bf16, fp32 accumulation) must satisfy, per element,
+|err| <= 1e-2 * |ref| + 1e-2 * rms(ref) against the fp64 oracle.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_25_b200 import binding as qb
+from bit_nf4_quantized_25_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = "cuda"
+RTOL = 1e-2  # relative part of the per-element bound
+STOL = 1e-2  # part relative to the rms of the reference
+
+
+def bits(t):
+    return synth.bf16_bits(t)
+
+
+def bf16_to_f64(u16):
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def assert_close(got_bf16: torch.Tensor, ref: np.ndarray, what: str):
+    g = bf16_to_f64(bits(got_bf16)).reshape(ref.shape)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    err = np.abs(g - ref)
+    bound = RTOL * np.abs(ref) + STOL * rms
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} elements outside tolerance; "
+                           f"worst err/bound = {np.max(err / np.maximum(bound, 1e-300)):.3g}")
+    return float(np.max(err / np.maximum(bound, 1e-300))) if ref.size else 0.0
+
+
+def quantize_both(oracle, W: torch.Tensor):
+    n, k = W.shape
+    w = qb.nf4_quantize(W)
+    torch.cuda.synchronize()
+    ref = oracle.nf4_quantize(bits(W), n, k)
+    return w, ref
+
+
+def assert_quant_equal(w, ref, what=""):
+    codes = w.codes.cpu().numpy()
+    q = w.absmax_q.cpu().numpy()
+    sigma = w.group_scale.cpu().numpy()
+    mu = w.absmax_mean.cpu().numpy()[0]
+    assert mu.view(np.uint32) == np.float32(ref["mu"]).view(np.uint32), (what, mu, ref["mu"])
+    nbad = int(np.sum(codes != ref["codes"]))
+    assert nbad == 0, f"{what}: {nbad} code bytes differ"
+    assert np.array_equal(q, ref["q"]), f"{what}: {int(np.sum(q != ref['q']))} FP8 constants differ"
+    assert np.array_equal(sigma.view(np.uint32), ref["sigma"].view(np.uint32)), f"{what}: group scales differ"
+
+
+def to_host_weight(w):
+    return dict(codes=w.codes.cpu().numpy(), q=w.absmax_q.cpu().numpy(), sigma=w.group_scale.cpu().numpy(),
+                mu=np.float32(w.absmax_mean.cpu().numpy()[0]))
+
+
+# ------------------------------------------------------------------ quantiser
+
+def test_quantize_tiny_bit_exact(oracle):
+    W, *_ = synth.layer_inputs(synth.tiny_case(), DEV)
+    w, ref = quantize_both(oracle, W)
+    assert_quant_equal(w, ref, "tiny")
+
+
+@pytest.mark.parametrize("arrangement", ["shuffled", "sorted", "signed"])
+def test_quantize_every_finite_bf16_pattern(oracle, arrangement):
+    # Every finite bf16 weight, in blocks with absmaxes across the whole range:
+    # exhaustive for the code decision, wide-range for the exact mean.
+    u = np.arange(65536, dtype=np.uint32)
+    finite = ((u >> 7) & 0xFF) != 0xFF
+    pats = u[finite].astype(np.uint16)
+    if arrangement == "shuffled":
+        pats = np.random.default_rng(0).permutation(pats)
+    elif arrangement == "signed":
+        mag = pats[pats < 0x8000]
+        pats = np.stack([mag, mag | 0x8000], 1).reshape(-1)
+        pats = np.random.default_rng(1).permutation(pats.reshape(-1, 64)).reshape(-1)
+    pad = (-pats.size) % (64 * 4)
+    pats = np.concatenate([pats, np.zeros(pad, np.uint16)])
+    n, k = pats.size // 256, 256
+    W = torch.from_numpy(pats.view(np.int16).reshape(n, k).copy()).view(torch.bfloat16).to(DEV)
+    w, ref = quantize_both(oracle, W)
+    assert_quant_equal(w, ref, arrangement)
+
+
+@pytest.mark.parametrize("n,k", [(1, 64), (3, 192), (200, 448), (5, 64 * 172), (4096, 4096), (11008, 4096),
+                                 (4096, 11008), (8192, 8192), (28672, 8192), (8192, 28672)])
+def test_quantize_shapes_bit_exact(oracle, n, k):
+    W = synth.normal_bf16((n, k), 0.015 if max(n, k) > 11008 else 0.02, seed=n * 7 + k, device=DEV)
+    w, ref = quantize_both(oracle, W)
+    assert_quant_equal(w, ref, f"{n}x{k}")
+
+
+def test_quantize_special_blocks(oracle):
+    # all-zero blocks (code 7), blocks with equal absmax (sigma 0), a single non-zero
+    W = torch.zeros(4, 1024, dtype=torch.bfloat16)
+    W[1, ::64] = 0.375
+    W[1, 5::64] = -0.1
+    W[2, 7] = -3.0e-3
+    W[3, :] = 1.0
+    w, ref = quantize_both(oracle, W.to(DEV))
+    assert_quant_equal(w, ref, "special")
+
+
+def test_dequant_bit_exact(oracle):
+    for n, k, seed in [(256, 256, 0), (3, 64 * 172, 5), (4096, 4096, 7)]:
+        W = synth.student_t_bf16((n, k), 0.02, seed, device=DEV)
+        w = qb.nf4_quantize(W)
+        deq = qb.nf4_dequantize(w)
+        torch.cuda.synchronize()
+        ref = oracle.nf4_dequant_bf16(to_host_weight(w), n, k)
+        got = bits(deq).reshape(n, k)
+        assert np.array_equal(got, ref), f"{n}x{k}: {int(np.sum(got != ref))} dequantised weights differ"
+
+
+def _bulk_layers():
+    return int(os.environ.get("QN_BULK_LAYERS", "32"))
+
+
+def test_bulk_quantize_roundtrip(oracle):
+    # 32 layers of the 7B shapes (6.48e9 weights), Student-t(4) * 0.02 with 0.1 % outliers x 20.
+    worst = 0.0
+    for layer in range(_bulk_layers()):
+        for name, (n, k) in synth.SHAPES_7B.items():
+            W = synth.bulk_tensor(layer, name, device=DEV)
+            w = qb.nf4_quantize(W)
+            deq = qb.nf4_dequantize(w)
+            torch.cuda.synchronize()
+            Wh = bits(W)
+            ref = oracle.nf4_quantize(Wh, n, k)
+            assert_quant_equal(w, ref, f"layer {layer} {name}")
+            got = bits(deq).reshape(n, k)
+            rdq = oracle.nf4_dequant_bf16(ref, n, k)
+            assert np.array_equal(got, rdq), f"layer {layer} {name}: dequant differs"
+            # Round-trip error per block: first level within half the widest table gap of
+            # c_b, second level within the FP8 rounding of d_b = c_b - mu (3 mantissa bits,
+            # subnormal step 2^-9 sigma), then one bf16 rounding of the product.
+            wf = bf16_to_f64(Wh).reshape(-1, 64)
+            df = bf16_to_f64(got).reshape(-1, 64)
+            c = ref["absmax"].astype(np.float64)
+            mu = float(ref["mu"])
+            sig = np.repeat(ref["sigma"].astype(np.float64), 256)[: c.size]
+            dq = 2.0 ** -4 * np.abs(c - mu) + 2.0 ** -10 * sig + 2.0 ** -22 * (c + abs(mu))
+            bound = 0.13852 * c + dq + 2.0 ** -8 * (c + dq)
+            err = np.max(np.abs(wf - df), axis=1)
+            assert np.all(err <= bound * (1 + 1e-6)), f"layer {layer} {name}: round-trip bound"
+            worst = max(worst, float(np.max(err / np.maximum(c, 1e-30))))
+            del W, w, deq
+    print(f"worst block round-trip error / absmax: {worst:.4f}")
+
+
+# --------------------------------------------------------------- linear layer
+
+def run_case(oracle, case: synth.LayerCase, rows=None, check_bwd=True):
+    W, A, B, x, gh = synth.layer_inputs(case, DEV, need_grad=check_bwd)
+    w = qb.nf4_quantize(W)
+    r = case.r
+    Ad, Bd = (A, B) if r > 0 else (None, None)
+    h = qb.qlora_linear_fwd(w, x, Ad, Bd, case.alpha)
+    gx = qb.qlora_linear_bwd_x(w, gh, Ad, Bd, case.alpha) if check_bwd else None
+    torch.cuda.synchronize()
+    hw = to_host_weight(w)
+    n, k, M = case.n_out, case.k_in, case.M
+    Ab, Bb = (bits(A), bits(B)) if r > 0 else (None, None)
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    ref_h = oracle.qlora_fwd(hw, n, k, bits(x), M, Ab, Bb, r, case.alpha, rows=sel)
+    worst = assert_close(h[torch.as_tensor(sel, device=DEV)], ref_h, f"{case.name} fwd")
+    if check_bwd:
+        ref_g = oracle.qlora_bwd_x(hw, n, k, bits(gh), M, Ab, Bb, r, case.alpha, rows=sel)
+        worst = max(worst, assert_close(gx[torch.as_tensor(sel, device=DEV)], ref_g, f"{case.name} bwd_x"))
+    return worst
+
+
+def test_tiny_fwd_bwd(oracle):
+    run_case(oracle, synth.tiny_case())
+
+
+@pytest.mark.parametrize("case", synth.decode7b_cases(), ids=lambda c: c.name)
+def test_decode7b_fwd_bwd(oracle, case):
+    run_case(oracle, case, check_bwd=True)
+
+
+@pytest.mark.parametrize("case", [c for c in synth.l70b_cases() if c.M <= 16], ids=lambda c: c.name)
+def test_l70b_decode_fwd_bwd(oracle, case):
+    run_case(oracle, case)
+
+
+def _sample_rows(M, seed, n=128):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(M, size=min(n, M), replace=False).tolist())
+    rows.update([0, M - 1])
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("case", synth.train7b_cases(), ids=lambda c: c.name)
+def test_train7b_sampled_rows(oracle, case):
+    run_case(oracle, case, rows=_sample_rows(case.M, case.seed))
+
+
+@pytest.mark.parametrize("case", [c for c in synth.l70b_cases() if c.M > 16], ids=lambda c: c.name)
+def test_l70b_train_sampled_rows(oracle, case):
+    run_case(oracle, case, rows=_sample_rows(case.M, case.seed, 64))
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 13, 31, 33, 64, 65, 100, 257])
+def test_ragged_token_counts(oracle, M):
+    run_case(oracle, synth.LayerCase(f"ragged_M{M}", 320, 448, M, 16, 32.0, 0.02, 500 + M))
+
+
+@pytest.mark.parametrize("r,alpha", [(0, 0.0), (1, 2.0), (4, 8.0), (64, 16.0), (200, 400.0), (256, 16.0)])
+def test_lora_ranks(oracle, r, alpha):
+    run_case(oracle, synth.LayerCase(f"rank{r}", 192, 512, 12, r, alpha, 0.02, 900 + r))
+
+
+@pytest.mark.parametrize("n,k", [(1, 64), (17, 64), (200, 192), (130, 64 * 19), (4100, 320)])
+def test_ragged_weight_shapes(oracle, n, k):
+    run_case(oracle, synth.LayerCase(f"shape{n}x{k}", n, k, 5, 4, 8.0, 0.02, n + k))
+
+
+def test_zero_adapter_and_zero_base(oracle):
+    case = synth.LayerCase("zeroB", 256, 512, 9, 16, 32.0, 0.02, 77)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV)
+    for Wz, Bz in ((W, torch.zeros_like(B)), (torch.zeros_like(W), B)):
+        w = qb.nf4_quantize(Wz)
+        h = qb.qlora_linear_fwd(w, x, A, Bz, case.alpha)
+        gx = qb.qlora_linear_bwd_x(w, gh, A, Bz, case.alpha)
+        torch.cuda.synchronize()
+        hw = to_host_weight(w)
+        assert_close(h, oracle.qlora_fwd(hw, 256, 512, bits(x), 9, bits(A), bits(Bz), 16, 32.0), "zero fwd")
+        assert_close(gx, oracle.qlora_bwd_x(hw, 256, 512, bits(gh), 9, bits(A), bits(Bz), 16, 32.0), "zero bwd")
+
+
+def test_adjoint_identity_on_gpu(oracle):
+    # <grad_h, fwd(x)> = <bwd_x(grad_h), x> holds for the exact layer; the GPU results
+    # satisfy it to the accuracy of bf16 outputs.
+    case = synth.LayerCase("adjoint", 1024, 2048, 16, 16, 32.0, 0.02, 4242)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV)
+    w = qb.nf4_quantize(W)
+    h = qb.qlora_linear_fwd(w, x, A, B, case.alpha).double()
+    gx = qb.qlora_linear_bwd_x(w, gh, A, B, case.alpha).double()
+    lhs = float((gh.double() * h).sum())
+    rhs = float((gx * x.double()).sum())
+    scale = float(h.norm() * gh.double().norm())
+    assert abs(lhs - rhs) <= 1e-2 * scale
+
+
+def test_empty_token_batch_is_noop():
+    W = synth.normal_bf16((128, 128), 0.02, 1, DEV)
+    w = qb.nf4_quantize(W)
+    x = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
+    h = qb.qlora_linear_fwd(w, x, None, None, 0.0)
+    assert h.shape == (0, 128)
