@@ -1,0 +1,494 @@
+"""Benchmark of the fused NF4 + LoRA linear layer on B200.
+
+Default workload (one GPU): Llama-7B-shaped decode. A step is the forward pass of every
+linear layer of a 32-layer 7B stack (q, k, v, o: 4096x4096; gate, up: 11008x4096;
+down: 4096x11008; LoRA r=16, alpha=32 on each) at M = 1, 4 and 16 tokens: 672 layer
+calls per step through the C ABI, replayed from a CUDA graph. The 3.34 GB of quantised
+weights exceed the 126 MB L2, so every step streams them from HBM.
+
+Printed (rank 0, one JSON line): weight GB/s of the whole job (value), TFLOP/s, the
+roofline of the dominant kernel against MEASURED_PEAKS.json, an end-to-end figure with
+pinned host<->device copies, the CPU oracle baseline, clocks sampled during the timed
+region, and a `detail` object with the other workloads (quantise, dequantise, 7B
+training-shape fwd+bwd at M=4096, 70B layers).
+
+--impl reference times the CPU oracle (the only reference that exists for this method)
+on a bounded sample of the same workload and prints the same line with impl=reference.
+Multi-GPU (torchrun): independent replicas, no data-path collective; value sums all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused NF4+LoRA linear TFLOP/s & weight GB/s at 1 B200; % of roofline"
+SHAPES_7B = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+             ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+DECODE_M = (1, 4, 16)
+RANK_7B, ALPHA_7B = 16, 32.0
+
+
+def weight_bytes(n, k):
+    nb = n * k // 64
+    return n * k // 2 + nb + 4 * ((nb + 255) // 256) + 4
+
+
+def fwd_bytes(n, k, M, r):
+    return weight_bytes(n, k) + 2 * M * k + 2 * r * k + 2 * n * r + 2 * M * n
+
+
+def linear_flops(n, k, M, r):
+    return 2 * M * n * k + 2 * M * r * (k + n)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        loaded = [v for v in sm if v > 0.5 * (max(mx) if mx else 1)] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for nm, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier_max(value, world):
+    import torch
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- ours
+
+def build_stack(layers, device):
+    import torch
+
+    from bit_nf4_quantized_25_b200 import binding as qb
+    from bit_nf4_quantized_25_b200 import synth
+    stack = []
+    for L in range(layers):
+        for j, (name, n, k) in enumerate(SHAPES_7B):
+            seed = 1000 + 100 * L + 10 * j
+            W = synth.normal_bf16((n, k), 0.02, seed, device)
+            w = qb.nf4_quantize(W)
+            del W
+            A = synth.normal_bf16((RANK_7B, k), 0.01, seed + 1, device)
+            B = synth.normal_bf16((n, RANK_7B), 0.01, seed + 2, device)
+            stack.append((name, n, k, w, A, B))
+    torch.cuda.synchronize()
+    return stack
+
+
+def decode_step_fn(stack, xs, outs, ws):
+    from bit_nf4_quantized_25_b200 import binding as qb
+
+    def step():
+        for M in DECODE_M:
+            for (name, n, k, w, A, B) in stack:
+                qb.qlora_linear_fwd(w, xs[(M, k)], A, B, ALPHA_7B, out=outs[(M, n)], workspace=ws)
+    return step
+
+
+def time_graph(graph, steps, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) * 1e-3
+
+
+def time_fn(fn, reps=10, warm=3, flush=None):
+    """Median CUDA-event time of fn() with an optional L2 flush between repetitions."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    s = torch.cuda.current_stream()
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e-3)
+    return statistics.median(ts)
+
+
+def detail_measurements(hbm_peak, tc_peak):
+    """Other workloads of the hot path, each timed with CUDA events (L2 flushed between reps)."""
+    import torch
+
+    from bit_nf4_quantized_25_b200 import binding as qb
+    from bit_nf4_quantized_25_b200 import synth
+    dev = "cuda"
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # 256 MB > L2
+    out = {}
+    # quantise and dequantise (HBM-bound)
+    for (n, k) in [(4096, 4096), (11008, 4096), (28672, 8192)]:
+        W = synth.normal_bf16((n, k), 0.02, 7, dev)
+        w = qb.nf4_quantize(W)
+        ws = torch.empty(qb.quantize_workspace_size(n, k), dtype=torch.uint8, device=dev)
+        deq = torch.empty_like(W)
+        tq = time_fn(lambda: qb.nf4_quantize(W, w, ws), flush=flush)
+        td = time_fn(lambda: qb.nf4_dequantize(w, deq), flush=flush)
+        by = 2 * n * k + weight_bytes(n, k)
+        out[f"quantize_{n}x{k}"] = {"us": round(tq * 1e6, 2), "GB/s": round(by / tq / 1e9, 1),
+                                    "hbm_frac": round(by / tq / 1e9 / hbm_peak, 3)}
+        out[f"dequant_{n}x{k}"] = {"us": round(td * 1e6, 2), "GB/s": round(by / td / 1e9, 1),
+                                   "hbm_frac": round(by / td / 1e9 / hbm_peak, 3)}
+        del W, w, ws, deq
+    # many-token fwd + bwd_x (tensor-core path) and 70B decode
+    cases = [("train7b", n, k, 4096, 16, 32.0, 0.02) for (_, n, k) in SHAPES_7B[3:]] + \
+            [("l70b", n, k, M, 64, 16.0, 0.015) for (n, k) in [(8192, 8192), (28672, 8192), (8192, 28672)]
+             for M in (1, 16, 4096)]
+    for (tag, n, k, M, r, alpha, std) in cases:
+        W = synth.normal_bf16((n, k), std, 11, dev)
+        w = qb.nf4_quantize(W)
+        del W
+        A = synth.normal_bf16((r, k), 0.01, 12, dev)
+        B = synth.normal_bf16((n, r), 0.01, 13, dev)
+        x = synth.normal_bf16((M, k), 1.0, 14, dev)
+        g = synth.normal_bf16((M, n), 1.0, 15, dev)
+        h = torch.empty(M, n, dtype=torch.bfloat16, device=dev)
+        gx = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(qb.linear_workspace_size(M, n, k, r), 256), dtype=torch.uint8, device=dev)
+        tf = time_fn(lambda: qb.qlora_linear_fwd(w, x, A, B, alpha, out=h, workspace=ws), reps=5, flush=flush)
+        tb = time_fn(lambda: qb.qlora_linear_bwd_x(w, g, A, B, alpha, out=gx, workspace=ws), reps=5, flush=flush)
+        fl = linear_flops(n, k, M, r)
+        by = fwd_bytes(n, k, M, r)
+        rec = {"fwd_us": round(tf * 1e6, 2), "bwd_us": round(tb * 1e6, 2),
+               "fwd_TFLOP/s": round(fl / tf / 1e12, 2), "bwd_TFLOP/s": round(fl / tb / 1e12, 2),
+               "fwd_GB/s": round(by / tf / 1e9, 1), "bwd_GB/s": round(by / tb / 1e9, 1)}
+        if M >= 1024:
+            rec["fwd_tensor_frac"] = round(fl / tf / 1e12 / tc_peak, 3)
+            rec["bwd_tensor_frac"] = round(fl / tb / 1e12 / tc_peak, 3)
+        else:
+            rec["fwd_hbm_frac"] = round(by / tf / 1e9 / hbm_peak, 3)
+            rec["bwd_hbm_frac"] = round(by / tb / 1e9 / hbm_peak, 3)
+        out[f"{tag}_{n}x{k}_M{M}"] = rec
+        del w, A, B, x, g, h, gx, ws
+        torch.cuda.empty_cache()
+    del flush
+    return out
+
+
+class CpuSample:
+    """The CPU oracle (fp64, all host cores) on a bounded sample of the decode workload:
+    the three 7B shapes at M = 1, 4, 16, repeated until a time budget is spent."""
+
+    def __init__(self):
+        from bit_nf4_quantized_25_b200 import synth
+        from oracle import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.prepared = []
+        for j, (n, k) in enumerate([(4096, 4096), (11008, 4096), (4096, 11008)]):
+            W = synth.normal_bf16((n, k), 0.02, 5000 + j)
+            qw = oracle.nf4_quantize(synth.bf16_bits(W), n, k)
+            A = synth.bf16_bits(synth.normal_bf16((RANK_7B, k), 0.01, 5100 + j))
+            B = synth.bf16_bits(synth.normal_bf16((n, RANK_7B), 0.01, 5200 + j))
+            xs = {M: synth.bf16_bits(synth.normal_bf16((M, k), 1.0, 5300 + M)) for M in DECODE_M}
+            self.prepared.append((n, k, qw, A, B, xs))
+
+    def run(self, budget_s):
+        done_bytes, done_flops, calls, t0 = 0, 0, 0, time.perf_counter()
+        while True:
+            for (n, k, qw, A, B, xs) in self.prepared:
+                for M in DECODE_M:
+                    self.oracle.qlora_fwd(qw, n, k, xs[M], M, A, B, RANK_7B, ALPHA_7B)
+                    done_bytes += fwd_bytes(n, k, M, RANK_7B)
+                    done_flops += linear_flops(n, k, M, RANK_7B)
+                    calls += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": self.oracle.threads(),
+                "kind": "oracle", "tflops": round(done_flops / dt / 1e12, 6),
+                "sample": f"{calls} forward calls of the 7B decode shapes (4096x4096, 11008x4096, 4096x11008 "
+                          f"at M=1,4,16; r=16) in fp64 on the host, {dt:.1f} s"}
+
+
+def cpu_baseline_sample(budget_s=15.0):
+    return CpuSample().run(budget_s)
+
+
+def run_ours(args):
+    import torch
+
+    from bit_nf4_quantized_25_b200 import binding as qb
+    from bit_nf4_quantized_25_b200 import build as qbuild
+    qbuild.build()
+    world, rank, local = dist_setup(args.gpus)
+    dev = "cuda"
+    hbm_peak, tc_burst, tc_sust, peak_kind = load_peaks()
+    from bit_nf4_quantized_25_b200 import synth
+
+    stack = build_stack(args.layers, dev)
+    xs = {(M, k): synth.normal_bf16((M, k), 1.0, 7000 + M + k, dev) for M in DECODE_M for k in (4096, 11008)}
+    outs = {(M, n): torch.empty(M, n, dtype=torch.bfloat16, device=dev) for M in DECODE_M for n in (4096, 11008)}
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    step = decode_step_fn(stack, xs, outs, ws)
+
+    per_step_bytes = sum(fwd_bytes(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)
+    per_step_flops = sum(linear_flops(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)
+    per_step_calls = len(stack) * len(DECODE_M)
+
+    # warm-up (eager), then capture one step into a CUDA graph
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        qb.launch_count(reset=True)
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        launches_per_step = qb.launch_count(reset=True)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t = time_graph(graph, args.steps, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    barrier(world)
+    t = barrier_max(t, world)
+    clocks = clk.summary()
+
+    ms_per_step = t / args.steps * 1e3
+    value = per_step_bytes * args.steps * world / t / 1e9
+    tflops = per_step_flops * args.steps * world / t / 1e12
+    avg_launch_s = t / (args.steps * launches_per_step)
+    bytes_per_launch = per_step_bytes / launches_per_step
+    achieved = bytes_per_launch / avg_launch_s / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "decode_fwd_traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                traffic = json.load(f).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # end to end through the public API: pinned H2D of the step's inputs, the step, D2H of outputs
+    pinned_in = {key: v.cpu().pin_memory() for key, v in xs.items()}
+    pinned_out = {key: torch.empty(v.shape, dtype=v.dtype).pin_memory() for key, v in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in pinned_out.values())
+
+    def e2e_step():
+        for key, v in pinned_in.items():
+            xs[key].copy_(v, non_blocking=True)
+        graph.replay()
+        for key, v in pinned_out.items():
+            v.copy_(outs[key], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    te = barrier_max(a.elapsed_time(b) * 1e-3, world)
+    e2e_value = per_step_bytes * args.steps * world / te / 1e9
+
+    detail = None
+    cpu = None
+    if rank == 0 and not args.no_detail:
+        del graph
+        detail = detail_measurements(hbm_peak, tc_burst)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_sample(args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nf4/bf16 in, fp32 accumulate, bf16 out",
+            "data": "synthetic (seeded random Llama-7B-shaped weights, no checkpoint)",
+            "config": {"workload": f"llama7b-decode: {args.layers} layers x 7 linears (4096x4096 x4, 11008x4096 x2, "
+                                   f"4096x11008), LoRA r=16 alpha=32, M in {{1,4,16}} per step, forward",
+                       "global_batch": sum(DECODE_M), "layer_calls_per_step": per_step_calls,
+                       "l2": f"inputs larger than L2: {per_step_bytes / len(DECODE_M) / 1e9:.2f} GB of weights "
+                             f"streamed per M", "parallelism": f"replicas x{world}",
+                       "quantised_weight_bytes": int(sum(weight_bytes(n, k) for (_, n, k, *_r) in stack))},
+            "tflops": round(tflops, 3),
+            "gpu_launches": int(launches_per_step * args.steps),
+            "roofline": {"bound": "hbm", "kernel": "k_decode_fwd (few-token NF4+LoRA forward)",
+                         "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind, "traffic": traffic,
+                         "bytes_per_launch": round(bytes_per_launch), "avg_launch_us": round(avg_launch_s * 1e6, 3)},
+            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "detail": detail,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # the oracle, as it stands, on the host cores; each step is a bounded sample
+    steps, warm = max(args.steps, 1), max(args.warmup, 0)
+    budget = max(1.0, min(20.0, 150.0 / (steps + warm)))
+    sampler = CpuSample()
+    for _ in range(warm):
+        sampler.run(budget)
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(steps):
+        last = sampler.run(budget)
+        vals.append(last["value"])
+    dt = time.perf_counter() - t0
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": round(dt / steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama7b-decode (bounded sample on the host CPU: oracle)",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-detail", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

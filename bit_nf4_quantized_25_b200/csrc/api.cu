@@ -156,8 +156,9 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
     if (s != QN_OK) return s;
     if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
     if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
-    (void)M;
-    *ws_bytes = 256;  // the decode kernels need none; kept non-zero so callers can always pass a buffer
+    // The few-token kernels need no workspace (256 bytes keep the pointer non-null); the
+    // tensor-core path stores its error word and the adapter operand there.
+    *ws_bytes = M > kDecodeMaxM ? gemm_workspace_bytes(M, r) : 256;
     g_err.clear();
     return QN_OK;
 }
@@ -189,10 +190,14 @@ qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, con
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *xp = static_cast<const uint16_t *>(x);
     uint16_t *hp = static_cast<uint16_t *>(h);
+    const uint16_t *Ap = static_cast<const uint16_t *>(A), *Bp = static_cast<const uint16_t *>(B);
+    if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, false)) {
+        if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
+        return cuda_status(launch_gemm_fwd(wv, xp, M, Ap, Bp, r, sc, hp, ws, st), "qlora_linear_fwd");
+    }
     for (int64_t m0 = 0; m0 < M; m0 += kDecodeMaxM) {
         const int mc = static_cast<int>(M - m0 < kDecodeMaxM ? M - m0 : kDecodeMaxM);
-        cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, static_cast<const uint16_t *>(A),
-                                          static_cast<const uint16_t *>(B), r, sc, hp + m0 * w->n_out, st);
+        cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, Ap, Bp, r, sc, hp + m0 * w->n_out, st);
         if (e != cudaSuccess) return cuda_status(e, "qlora_linear_fwd");
     }
     return cuda_status(cudaSuccess, "");
@@ -208,11 +213,15 @@ qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *gp = static_cast<const uint16_t *>(grad_h);
     uint16_t *xp = static_cast<uint16_t *>(grad_x);
+    const uint16_t *Ap = static_cast<const uint16_t *>(A), *Bp = static_cast<const uint16_t *>(B);
+    if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, true)) {
+        if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
+        return cuda_status(launch_gemm_bwd(wv, gp, M, Ap, Bp, r, sc, xp, ws, st), "qlora_linear_bwd_x");
+    }
     constexpr int kChunk = 32;
     for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
         const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);
-        cudaError_t e = launch_decode_bwd(wv, gp + m0 * w->n_out, mc, static_cast<const uint16_t *>(A),
-                                          static_cast<const uint16_t *>(B), r, sc, xp + m0 * w->k_in, st);
+        cudaError_t e = launch_decode_bwd(wv, gp + m0 * w->n_out, mc, Ap, Bp, r, sc, xp + m0 * w->k_in, st);
         if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
     }
     return cuda_status(cudaSuccess, "");

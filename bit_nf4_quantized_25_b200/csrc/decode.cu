@@ -34,6 +34,8 @@ constexpr int kDecWarps = 4;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kLutBytes = 256 * 32 * 4;  // 256 code bytes x 32 lane copies x bf16 pair
 constexpr int kMaxCluster = 8;
+constexpr int kBatch = 8;      // 64-weight blocks per batch of loads (forward)
+constexpr int kStepBatch = 4;  // 16-row steps per batch of loads (input gradient)
 
 struct DecodeParams {
     const uint8_t *codes;
@@ -93,6 +95,9 @@ k_decode_fwd(const DecodeParams p) {
     build_pair_lut(lut);
     for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) tpart[i] = 0.0f;
     __syncthreads();
+    // Launched as a programmatic dependent: everything above overlaps the preceding
+    // kernel; no global memory is read before this point.
+    grid_dependency_wait();
 
     const int64_t N = p.n, K = p.k, nbr = K / kBlock;
     const int64_t b_lo = nbr * crank / C, b_hi = nbr * (crank + 1) / C;
@@ -121,37 +126,67 @@ k_decode_fwd(const DecodeParams p) {
 #pragma unroll
         for (int tg = 0; tg < NG; ++tg) acc[tg][0] = acc[tg][1] = acc[tg][2] = acc[tg][3] = 0.0f;
 
-        for (int64_t b = b_lo; b < b_hi; ++b) {
-            const uint2 ca = vA ? __ldcs(reinterpret_cast<const uint2 *>(cA + b * 32)) : make_uint2(0u, 0u);
-            const uint2 cb = vB ? __ldcs(reinterpret_cast<const uint2 *>(cB + b * 32)) : make_uint2(0u, 0u);
-            const float cpA = vA ? block_constant(__ldg(p.q + qA + b), __ldg(p.sigma + (qA + b) / kGroup), mu) : 0.0f;
-            const float cpB = vB ? block_constant(__ldg(p.q + qB + b), __ldg(p.sigma + (qB + b) / kGroup), mu) : 0.0f;
-            uint32_t af[4][4];
+        // Batches of kBatch blocks: every load of a batch is issued before any use, so a
+        // warp keeps 2 x kBatch x 8 bytes of codes per lane in flight.
+        for (int64_t bb = b_lo; bb < b_hi; bb += kBatch) {
+            const int nbk = static_cast<int>(b_hi - bb < kBatch ? b_hi - bb : kBatch);
+            uint2 ca[kBatch], cb[kBatch];
+            uint32_t qa[kBatch], qbv[kBatch];
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t wa = kk < 2 ? ca.x : ca.y, wb = kk < 2 ? cb.x : cb.y;
-                const int i0 = (2 * kk) & 3;
-                af[kk][0] = lut_get(lut, byte_of(wa, i0), lane);
-                af[kk][2] = lut_get(lut, byte_of(wa, i0 + 1), lane);
-                af[kk][1] = lut_get(lut, byte_of(wb, i0), lane);
-                af[kk][3] = lut_get(lut, byte_of(wb, i0 + 1), lane);
-            }
-#pragma unroll
-            for (int tg = 0; tg < NG; ++tg) {
-                uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                if (xv[tg]) {
-                    x0 = ld_ro_v4(xrow[tg] + b * 64);
-                    x1 = ld_ro_v4(xrow[tg] + b * 64 + 8);
+            for (int j = 0; j < kBatch; ++j) {
+                ca[j] = cb[j] = make_uint2(0u, 0u);
+                qa[j] = qbv[j] = 0u;
+                if (j < nbk) {
+                    if (vA) {
+                        ca[j] = __ldcs(reinterpret_cast<const uint2 *>(cA + (bb + j) * 32));
+                        qa[j] = __ldg(p.q + qA + bb + j);
+                    }
+                    if (vB) {
+                        cb[j] = __ldcs(reinterpret_cast<const uint2 *>(cB + (bb + j) * 32));
+                        qbv[j] = __ldg(p.q + qB + bb + j);
+                    }
                 }
-                const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            }
+            // a batch of <= 8 consecutive blocks touches at most two groups
+            const int64_t gA0 = (qA + bb) / kGroup, gB0 = (qB + bb) / kGroup;
+            const int64_t ng_all = (N * nbr + kGroup - 1) / kGroup;
+            const float sA0 = __ldg(p.sigma + gA0), sA1 = __ldg(p.sigma + (gA0 + 1 < ng_all ? gA0 + 1 : gA0));
+            const float sB0 = __ldg(p.sigma + gB0), sB1 = __ldg(p.sigma + (gB0 + 1 < ng_all ? gB0 + 1 : gB0));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_16816(d, af[kk][0], af[kk][1], af[kk][2], af[kk][3], xw[2 * kk], xw[2 * kk + 1]);
-                acc[tg][0] = __fmaf_rn(cpA, d[0], acc[tg][0]);
-                acc[tg][1] = __fmaf_rn(cpA, d[1], acc[tg][1]);
-                acc[tg][2] = __fmaf_rn(cpB, d[2], acc[tg][2]);
-                acc[tg][3] = __fmaf_rn(cpB, d[3], acc[tg][3]);
+            for (int j = 0; j < kBatch; ++j) {
+                if (j >= nbk) break;
+                const int64_t b = bb + j;
+                const float cpA = vA ? block_constant(static_cast<uint8_t>(qa[j]),
+                                                      (qA + b) / kGroup == gA0 ? sA0 : sA1, mu) : 0.0f;
+                const float cpB = vB ? block_constant(static_cast<uint8_t>(qbv[j]),
+                                                      (qB + b) / kGroup == gB0 ? sB0 : sB1, mu) : 0.0f;
+                uint32_t af[4][4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t wa = kk < 2 ? ca[j].x : ca[j].y, wb = kk < 2 ? cb[j].x : cb[j].y;
+                    const int i0 = (2 * kk) & 3;
+                    af[kk][0] = lut_get(lut, byte_of(wa, i0), lane);
+                    af[kk][2] = lut_get(lut, byte_of(wa, i0 + 1), lane);
+                    af[kk][1] = lut_get(lut, byte_of(wb, i0), lane);
+                    af[kk][3] = lut_get(lut, byte_of(wb, i0 + 1), lane);
+                }
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) {
+                    uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+                    if (xv[tg]) {
+                        x0 = ld_ro_v4(xrow[tg] + b * 64);
+                        x1 = ld_ro_v4(xrow[tg] + b * 64 + 8);
+                    }
+                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_16816(d, af[kk][0], af[kk][1], af[kk][2], af[kk][3], xw[2 * kk], xw[2 * kk + 1]);
+                    acc[tg][0] = __fmaf_rn(cpA, d[0], acc[tg][0]);
+                    acc[tg][1] = __fmaf_rn(cpA, d[1], acc[tg][1]);
+                    acc[tg][2] = __fmaf_rn(cpB, d[2], acc[tg][2]);
+                    acc[tg][3] = __fmaf_rn(cpB, d[3], acc[tg][3]);
+                }
             }
         }
         const int rl = warp * 16 + g;
@@ -217,6 +252,7 @@ k_decode_fwd(const DecodeParams p) {
 
     __syncthreads();
     cluster.sync();  // every CTA's partials are complete and visible in the cluster
+    grid_dependents_launch();
 
     if (p.r > 0) {
         for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) {
@@ -291,6 +327,7 @@ k_decode_bwd(const DecodeParams p) {
     build_pair_lut(lut);
     for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) upart[i] = 0.0f;
     __syncthreads();
+    grid_dependency_wait();
 
     const int64_t N = p.n, K = p.k, nbr = K / kBlock;
     const int64_t n16 = (N + 15) / 16;
@@ -310,42 +347,55 @@ k_decode_bwd(const DecodeParams p) {
             for (int tg = 0; tg < NG; ++tg) acc[i][tg][0] = acc[i][tg][1] = acc[i][tg][2] = acc[i][tg][3] = 0.0f;
 
         if (vk) {
-            for (int64_t st = s_lo; st < s_hi; ++st) {
-                const int64_t n0 = st * 16 + 4 * t;  // this lane's 4 reduction rows
-                uint32_t w[4];
-                float cp[4];
+            // Batches of kStepBatch 16-row steps, all loads issued before use.
+            for (int64_t sb = s_lo; sb < s_hi; sb += kStepBatch) {
+                const int nst = static_cast<int>(s_hi - sb < kStepBatch ? s_hi - sb : kStepBatch);
+                uint32_t w[kStepBatch][4], qv[kStepBatch][4];
+                float sg[kStepBatch][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int64_t n = n0 + i;
-                    if (n < N) {
-                        w[i] = ld_nc_u32(p.codes + n * (K / 2) + kbc * 32 + 4 * gq);
-                        const int64_t bi = n * nbr + kbc;
-                        cp[i] = block_constant(__ldg(p.q + bi), __ldg(p.sigma + bi / kGroup), mu);
-                    } else {
-                        w[i] = 0x77777777u;  // value 0
-                        cp[i] = 0.0f;
+                for (int j = 0; j < kStepBatch; ++j)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int64_t n = (sb + j) * 16 + 4 * t + i;
+                        w[j][i] = 0x77777777u;  // value 0
+                        qv[j][i] = 0u;
+                        sg[j][i] = 0.0f;
+                        if (j < nst && n < N) {
+                            const int64_t bi = n * nbr + kbc;
+                            w[j][i] = ld_nc_u32(p.codes + n * (K / 2) + kbc * 32 + 4 * gq);
+                            qv[j][i] = __ldg(p.q + bi);
+                            sg[j][i] = __ldg(p.sigma + bi / kGroup);
+                        }
                     }
-                }
-                uint32_t e01, o01, e23, o23;
-                interleave_rows(w[0], w[1], e01, o01);
-                interleave_rows(w[2], w[3], e23, o23);
-                uint32_t af[4][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    af[i][0] = lut_get(lut, byte_of(e01, i), lane);
-                    af[i][1] = lut_get(lut, byte_of(o01, i), lane);
-                    af[i][2] = lut_get(lut, byte_of(e23, i), lane);
-                    af[i][3] = lut_get(lut, byte_of(o23, i), lane);
-                }
+                for (int j = 0; j < kStepBatch; ++j) {
+                    if (j >= nst) break;
+                    const int64_t n0 = (sb + j) * 16 + 4 * t;  // this lane's 4 reduction rows
+                    float cp[4];
 #pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    const int tok = tg * 8 + gq;
-                    float gv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    if (tok < M) load_g4(p.act, N, tok, n0, gv);
-                    const uint32_t b0 = pack_bf16x2(cp[0] * gv[0], cp[1] * gv[1]);
-                    const uint32_t b1 = pack_bf16x2(cp[2] * gv[2], cp[3] * gv[3]);
+                    for (int i = 0; i < 4; ++i) cp[i] = block_constant(static_cast<uint8_t>(qv[j][i]), sg[j][i], mu);
+                    uint32_t e01, o01, e23, o23;
+                    interleave_rows(w[j][0], w[j][1], e01, o01);
+                    interleave_rows(w[j][2], w[j][3], e23, o23);
+                    uint32_t af[4][4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) mma_16816(acc[i][tg], af[i][0], af[i][1], af[i][2], af[i][3], b0, b1);
+                    for (int i = 0; i < 4; ++i) {
+                        af[i][0] = lut_get(lut, byte_of(e01, i), lane);
+                        af[i][1] = lut_get(lut, byte_of(o01, i), lane);
+                        af[i][2] = lut_get(lut, byte_of(e23, i), lane);
+                        af[i][3] = lut_get(lut, byte_of(o23, i), lane);
+                    }
+#pragma unroll
+                    for (int tg = 0; tg < NG; ++tg) {
+                        const int tok = tg * 8 + gq;
+                        float gv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        if (tok < M) load_g4(p.act, N, tok, n0, gv);
+                        const uint32_t b0 = pack_bf16x2(cp[0] * gv[0], cp[1] * gv[1]);
+                        const uint32_t b1 = pack_bf16x2(cp[2] * gv[2], cp[3] * gv[3]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mma_16816(acc[i][tg], af[i][0], af[i][1], af[i][2], af[i][3], b0, b1);
+                    }
                 }
             }
         }
@@ -410,6 +460,7 @@ k_decode_bwd(const DecodeParams p) {
 
     __syncthreads();
     cluster.sync();
+    grid_dependents_launch();
 
     if (p.r > 0) {
         for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) {
@@ -442,20 +493,40 @@ k_decode_bwd(const DecodeParams p) {
 
 template <typename Kern>
 cudaError_t launch_cluster(Kern kern, dim3 grid, int cluster_x, size_t smem, cudaStream_t st, const DecodeParams &p) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+    // Raise the kernel's dynamic shared-memory limit only when a launch needs more than
+    // any earlier one (the attribute call is skipped on the steady-state path).
+    static thread_local const void *kerns[16];
+    static thread_local size_t limits[16];
+    static thread_local int nk = 0;
+    int slot = -1;
+    for (int i = 0; i < nk; ++i)
+        if (kerns[i] == reinterpret_cast<const void *>(kern)) slot = i;
+    if (slot < 0 || limits[slot] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        if (slot < 0 && nk < 16) {
+            slot = nk++;
+            kerns[slot] = reinterpret_cast<const void *>(kern);
+        }
+        if (slot >= 0) limits[slot] = smem;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cluster_x;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Programmatic dependent launch: the grid may start while the preceding kernel
+    // finishes; the kernel reads no global memory before griddepcontrol.wait.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
+    cudaError_t e;
     e = cudaLaunchKernelEx(&cfg, kern, p);
     count_launch();
     return e;

@@ -1,0 +1,472 @@
+// gemm_sm100.cu -- fused NF4 dequant-GEMM on the 5th-generation tensor cores (tcgen05 + TMEM)
+// for many tokens, forward and input gradient, with the LoRA up-projection accumulated into
+// the same tile.
+//
+//   fwd : h^T[n, m]      = sum_k W'[n,k] x[m,k]       + sum_j B[n,j] t[m,j]    (t = s A x)
+//   bwd : grad_x^T[k, m] = sum_n W'[n,k] grad_h[m,n]  + sum_j A[j,k] u[m,j]    (u = s B^T grad_h)
+// "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com): the 4-bit weights are
+// dequantised to bf16 for the matmul and the adapter output is added; "How does QLoRA work
+// for training?" (aivaro.ru), section 7: the same dequantisation feeds the gradient.
+//
+// One CTA computes a 128 x 256 tile: 128 weight rows (fwd) or 128 input features (bwd) as
+// the MMA M dimension, 256 tokens as the MMA N dimension, fp32 accumulator in TMEM.
+//   warp 0      : TMA producer of the token operand (x / grad_h, then t / u), 64-wide K slabs
+//                 in the 128-byte swizzled K-major layout, 4-stage mbarrier ring.
+//   warp 1      : TMEM allocator and the single MMA-issuing thread (tcgen05.mma kind::f16).
+//   warps 2..9  : two groups of four dequant warps taking alternate stages. A thread owns one
+//                 64-weight block per stage (fwd: one row; bwd: half of a reduction row),
+//                 builds the 16 scaled bf16 values NF4[i] * c'_b in registers, expands the
+//                 nibbles with byte permutes and writes the swizzled A tile (K-major for fwd,
+//                 MN-major for bwd, so W is always read in its stored row-major order).
+//                 The extra LoRA stages copy rows of B (fwd) / A (bwd) into the A tile.
+//   epilogue    : the eight dequant warps read TMEM (tcgen05.ld) and store bf16.
+// Every mbarrier wait is bounded; on a timeout the CTA records an error code, stops issuing
+// work, drains what it issued and frees its TMEM.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace qn {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;  // MMA M: weight rows / input features
+constexpr int kTileN = 256;  // MMA N: tokens
+constexpr int kTileK = 64;   // reduction per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 4;
+constexpr int kDqWarps = 8;
+constexpr int kGemmThreads = (2 + kDqWarps) * 32;
+constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB
+constexpr uint32_t kBBytes = kTileN * kTileK * 2;  // 32 KB
+constexpr uint32_t kTmemCols = 256;
+constexpr size_t kGemmSmem = 1024 + kStages * (kABytes + kBBytes) + 256;
+
+constexpr int kErrTimeout = 1;
+
+struct GemmParams {
+    const uint8_t *codes;
+    const uint8_t *q;
+    const float *sigma;
+    const float *mu;
+    int64_t n, k;           // W is n x k
+    int64_t M;              // tokens
+    const uint16_t *lora;   // fwd: B (n x r); bwd: A (r x k)
+    int r;
+    uint16_t *out;          // fwd: h (M x n); bwd: grad_x (M x k)
+    int *err;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// 16 scaled table values bf16(NF4[i] * cp), split into low-byte planes L0..L3 and
+// high-byte planes H0..H3 (4 entries per register) for byte-permute lookups.
+struct Planes {
+    uint32_t L0, L1, L2, L3, H0, H1, H2, H3;
+};
+
+__device__ __forceinline__ Planes make_planes(float cp) {
+    uint32_t E[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) E[i] = pack_bf16x2(__fmul_rn(nf4_value(2 * i), cp), __fmul_rn(nf4_value(2 * i + 1), cp));
+    Planes P;
+    P.L0 = prmt(E[0], E[1], 0x6420);
+    P.H0 = prmt(E[0], E[1], 0x7531);
+    P.L1 = prmt(E[2], E[3], 0x6420);
+    P.H1 = prmt(E[2], E[3], 0x7531);
+    P.L2 = prmt(E[4], E[5], 0x6420);
+    P.H2 = prmt(E[4], E[5], 0x7531);
+    P.L3 = prmt(E[6], E[7], 0x6420);
+    P.H3 = prmt(E[6], E[7], 0x7531);
+    return P;
+}
+
+// Four codes (nibbles of the low 16 bits of s) -> two bf16x2 words (codes 0,1 and 2,3).
+__device__ __forceinline__ void lookup4(const Planes &P, uint32_t s, uint32_t &o0, uint32_t &o1) {
+    const uint32_t s7 = s & 0x7777u;
+    const uint32_t la = prmt(P.L0, P.L1, s7), lb = prmt(P.L2, P.L3, s7);
+    const uint32_t ha = prmt(P.H0, P.H1, s7), hb = prmt(P.H2, P.H3, s7);
+    // byte j = 0xff where code j >= 8 (bit 3 selects an odd byte of 0xff00ff00)
+    const uint32_t m = prmt(0xff00ff00u, 0xff00ff00u, s >> 3);
+    const uint32_t lo = (la & ~m) | (lb & m), hi = (ha & ~m) | (hb & m);
+    o0 = prmt(lo, hi, 0x5140);
+    o1 = prmt(lo, hi, 0x7362);
+}
+
+// 8 codes (one 32-bit word, element 0 in the low nibble) -> 8 bf16 (16 bytes).
+__device__ __forceinline__ uint4 expand8(const Planes &P, uint32_t w) {
+    uint4 o;
+    lookup4(P, w, o.x, o.y);
+    lookup4(P, w >> 16, o.z, o.w);
+    return o;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Byte offset of 16-byte chunk j (elements 8j..8j+7) of the 64-element row `row` of a
+// 128-byte-swizzled tile whose rows are 128 bytes apart (K-major) -- also the layout of one
+// 64-element MN chunk of an MN-major tile whose K rows are 128 bytes apart.
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t j) { return row * 128u + ((j ^ (row & 7u)) << 4); }
+
+template <bool kBwd>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lora,
+           const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;                        // kStages x 16 KB
+    uint8_t *sB = smem + kStages * kABytes;    // kStages x 32 KB
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBBytes);
+    uint64_t *full_a = bars, *full_b = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t N = p.n, K = p.k, nbr = K / kBlock;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileM;  // fwd: weight row; bwd: feature
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTileN;
+    const int nred = kBwd ? static_cast<int>((N + kTileK - 1) / kTileK) : static_cast<int>(nbr);
+    const int nlora = (p.r + kTileK - 1) / kTileK;
+    const int T = nred + nlora;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_a[s], 4);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_act);
+        tma_prefetch_desc(&tm_lora);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+    grid_dependency_wait();  // activations and adapters may come from the preceding kernel
+
+    auto fail = [&]() {
+        if (atomicExch(const_cast<uint32_t *>(abort_flag), 1u) == 0u && p.err) atomicExch(p.err, kErrTimeout);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t issued_phase[kStages];
+            bool issued[kStages];
+            for (int s = 0; s < kStages; ++s) issued[s] = false;
+            for (int i = 0; i < T && !*abort_flag; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1u;
+                if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_b[s], kBBytes);
+                if (i < nred)
+                    tma_load_2d(sB + s * kBBytes, &tm_act, &full_b[s], i * kTileK, static_cast<int32_t>(tok0));
+                else
+                    tma_load_2d(sB + s * kBBytes, &tm_lora, &full_b[s], (i - nred) * kTileK, static_cast<int32_t>(tok0));
+                issued[s] = true;
+                issued_phase[s] = ph;
+            }
+            // drain: every load this thread issued has landed before the CTA can exit
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s]) mbar_wait(&full_b[s], issued_phase[s]);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(kTileM, kTileN, kBwd ? 1 : 0, 0);
+            for (int i = 0; i < T && !*abort_flag; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1u;
+                if (!mbar_wait(&full_a[s], ph) || !mbar_wait(&full_b[s], ph)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                int nk = 4;
+                if (i >= nred) {
+                    const int rem = p.r - (i - nred) * kTileK;
+                    nk = rem >= kTileK ? 4 : (rem + 15) / 16;
+                }
+                const uint32_t a_base = smem_u32(sA + s * kABytes), b_base = smem_u32(sB + s * kBBytes);
+                for (int kk = 0; kk < nk; ++kk) {
+                    // fwd A: K-major, 16 elements = 32 bytes along the swizzled row.
+                    // bwd A: MN-major, 16 reduction rows = two 8-row groups of 1024 bytes;
+                    //        the two 64-feature chunks are 8192 bytes apart.
+                    const uint64_t ad = kBwd ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                             : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                    mma_bf16_ss(tmem_d, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+            }
+            mma_commit(acc_full);  // arrives when every issued MMA has completed
+        }
+    } else {
+        // ----------------------------------------------------------- dequant groups
+        const int dw = warp - 2;
+        const int grp = dw >> 2;                  // stages i with i % 2 == grp
+        const int tid = (dw & 3) * 32 + lane;     // 0..127 within the group
+        const float mu = __ldg(p.mu);
+        // fwd: thread = A row (weight row row0 + tid), 64 k per stage.
+        // bwd: thread = (reduction row tid/2 of the stage, feature half tid%2).
+        const uint32_t arow = kBwd ? static_cast<uint32_t>(tid >> 1) : static_cast<uint32_t>(tid);
+        const uint32_t half = kBwd ? static_cast<uint32_t>(tid & 1) : 0u;
+        const int64_t kf = row0 + 64 * half;  // bwd: first feature of this thread's block
+        const bool bwd_kvalid = !kBwd || kf < K;
+
+        auto load_codes = [&](int i, uint4 &c0, uint4 &c1, uint32_t &qb, float &sg, bool &valid) {
+            valid = false;
+            c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+            qb = 0u;
+            sg = 0.0f;
+            if (i >= nred) return;
+            int64_t wrow, blk;
+            if (kBwd) {
+                wrow = static_cast<int64_t>(i) * kTileK + arow;
+                if (wrow >= N || !bwd_kvalid) return;
+                blk = wrow * nbr + kf / kBlock;
+            } else {
+                wrow = row0 + arow;
+                if (wrow >= N) return;
+                blk = wrow * nbr + i;
+            }
+            const uint8_t *cp = p.codes + blk * 32;
+            c0 = __ldg(reinterpret_cast<const uint4 *>(cp));
+            c1 = __ldg(reinterpret_cast<const uint4 *>(cp + 16));
+            qb = __ldg(p.q + blk);
+            sg = __ldg(p.sigma + blk / kGroup);
+            valid = true;
+        };
+
+        uint4 n0, n1;
+        uint32_t nq;
+        float ns;
+        bool nv;
+        load_codes(grp, n0, n1, nq, ns, nv);
+        for (int i = grp; i < T; i += 2) {
+            if (*abort_flag) break;
+            const int s = i % kStages;
+            const uint32_t ph = (i / kStages) & 1u;
+            const uint4 c0 = n0, c1 = n1;
+            const uint32_t cq = nq;
+            const float cs = ns;
+            const bool cv = nv;
+            load_codes(i + 2, n0, n1, nq, ns, nv);  // prefetch this group's next stage
+            if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
+                fail();
+                break;
+            }
+            const uint32_t a_base = smem_u32(sA + s * kABytes);
+            // destination of chunk j (8 elements) of this thread's 64-element run
+            auto dst = [&](uint32_t j) -> uint32_t {
+                return kBwd ? a_base + half * 8192u + (arow >> 3) * 1024u + swz(arow & 7u, j)
+                            : a_base + swz(arow, j);
+            };
+            if (i < nred) {
+                if (cv) {
+                    const Planes P = make_planes(block_constant(static_cast<uint8_t>(cq), cs, mu));
+                    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sts128(dst(j), expand8(P, w[j]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sts128(dst(j), make_uint4(0u, 0u, 0u, 0u));
+                }
+            } else {
+                // adapter stage: fwd copies row (row0 + arow) of B (n x r), columns
+                // [64c, 64c + 64); bwd copies row (64c + arow) of A (r x k), features [kf, kf + 64).
+                const int c = i - nred;
+                const uint16_t *src = nullptr;
+                int count = 0;
+                if (kBwd) {
+                    const int j = c * kTileK + static_cast<int>(arow);
+                    if (j < p.r && bwd_kvalid) {
+                        src = p.lora + static_cast<int64_t>(j) * K + kf;
+                        count = 64;
+                    }
+                } else {
+                    const int64_t wrow = row0 + arow;
+                    if (wrow < N) {
+                        src = p.lora + wrow * p.r + c * kTileK;
+                        const int rem = p.r - c * kTileK;
+                        count = rem < 64 ? rem : 64;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (src && 8 * j < count) {
+                        if (8 * j + 8 <= count && ((reinterpret_cast<uintptr_t>(src + 8 * j) & 15u) == 0)) {
+                            v = __ldg(reinterpret_cast<const uint4 *>(src + 8 * j));
+                        } else {
+                            uint32_t e[8];
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) e[x] = (8 * j + x < count) ? ld_ro_u16(src + 8 * j + x) : 0u;
+                            v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16),
+                                           e[6] | (e[7] << 16));
+                        }
+                    }
+                    sts128(dst(j), v);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[s]);
+        }
+
+        // --------------------------------------------------------------- epilogue
+        grid_dependents_launch();
+        const bool ok = mbar_wait(acc_full, 0) && !*abort_flag;
+        if (!ok) fail();
+        tc_fence_after();
+        const uint32_t quarter = static_cast<uint32_t>(warp & 3);  // TMEM lanes this warp may access
+        const int64_t orow = row0 + quarter * 32 + lane;           // fwd: n; bwd: feature k
+        const int64_t ldo = kBwd ? K : N;
+        const bool rvalid = orow < (kBwd ? K : N);
+        for (int cb = grp * 4; cb < grp * 4 + 4; ++cb) {  // 32-column chunks of this group
+            uint32_t v[32];
+            tmem_ld32(tmem_d + ((quarter * 32u) << 16) + static_cast<uint32_t>(cb * 32), v);
+            tmem_ld_wait();
+            if (ok && rvalid) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int64_t m = tok0 + cb * 32 + c;
+                    if (m < p.M) p.out[m * ldo + orow] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem_d, kTmemCols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult qres;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major rows x cols matrix, box 64 (cols) x 256 (rows),
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(kTileN)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kBwd>
+cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M, const uint16_t *lora_rows, int r,
+                             const uint16_t *lora_act, int RT, uint16_t *out, int *err, cudaStream_t st) {
+    CUtensorMap tm_act, tm_lora;
+    const int64_t act_cols = kBwd ? w.n : w.k;
+    if (!make_map(&tm_act, act, M, act_cols)) return cudaErrorInvalidValue;
+    if (r > 0) {
+        if (!make_map(&tm_lora, lora_act, M, RT)) return cudaErrorInvalidValue;
+    } else {
+        tm_lora = tm_act;  // never read
+    }
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_nf4<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kGemmSmem));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    GemmParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, M, lora_rows, r, out, err};
+    const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileM - 1) / kTileM;
+    const int64_t tiles_n = (M + kTileN - 1) / kTileN;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_m), static_cast<unsigned>(tiles_n), 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kGemmSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_nf4<kBwd>, tm_act, tm_lora, p);
+    count_launch();
+    return e;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int64_t M, int r) {
+    const int64_t RT = (r + 63) / 64 * 64;
+    return 256 + ((static_cast<size_t>(M * RT) * 2 + 255) & ~size_t(255));
+}
+
+bool gemm_supported(int64_t n, int64_t k, int64_t M, bool bwd) {
+    // The token operand is read by TMA, whose row stride must be a multiple of 16 bytes:
+    // x (M x k) always is (k % 64 == 0); grad_h (M x n) needs n % 8 == 0.
+    return (k % 64 == 0) && M > 0 && (!bwd || n % 8 == 0);
+}
+
+cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, const uint16_t *A, const uint16_t *B,
+                            int r, float s, uint16_t *h, void *ws, cudaStream_t st) {
+    int *err = static_cast<int *>(ws);
+    uint16_t *t = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
+    const int RT = (r + 63) / 64 * 64;
+    cudaError_t e;
+    if (r > 0) {
+        e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, err, st);
+    } else {
+        e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    }
+    if (e != cudaSuccess) return e;
+    return launch_gemm_impl<false>(w, x, M, B, r, t, RT, h, err, st);
+}
+
+cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, const uint16_t *A, const uint16_t *B,
+                            int r, float s, uint16_t *gx, void *ws, cudaStream_t st) {
+    int *err = static_cast<int *>(ws);
+    uint16_t *u = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
+    const int RT = (r + 63) / 64 * 64;
+    cudaError_t e;
+    if (r > 0) {
+        e = launch_lora_down(gh, M, w.n, B, 1, r, r, s, u, RT, err, st);
+    } else {
+        e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    }
+    if (e != cudaSuccess) return e;
+    return launch_gemm_impl<true>(w, gh, M, A, r, u, RT, gx, err, st);
+}
+
+}  // namespace qn

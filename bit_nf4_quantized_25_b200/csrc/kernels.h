@@ -49,4 +49,13 @@ cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, co
 cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
                              int64_t ldk, int r, float s, uint16_t *out, int RT, int *err, cudaStream_t st);
 
+// tcgen05 fused dequant-GEMM for many tokens (the LoRA down-projection runs first, into
+// the workspace). Workspace: a 256-byte header (error word) then the M x RT adapter operand.
+size_t gemm_workspace_bytes(int64_t M, int r);
+bool gemm_supported(int64_t n, int64_t k, int64_t M, bool bwd);
+cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, const uint16_t *A, const uint16_t *B,
+                            int r, float s, uint16_t *h, void *ws, cudaStream_t st);
+cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, const uint16_t *A, const uint16_t *B,
+                            int r, float s, uint16_t *gx, void *ws, cudaStream_t st);
+
 }  // namespace qn

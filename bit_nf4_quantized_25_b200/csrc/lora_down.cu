@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
     const bool vA = rowA < p.M, vB = rowB < p.M;
     const uint16_t *aA = p.act + (vA ? rowA : 0) * p.red;
     const uint16_t *aB = p.act + (vB ? rowB : 0) * p.red;
-    const int64_t steps = p.red / 16;  // red is a multiple of 16 on this path
+    const int64_t steps = (p.red + 15) / 16;  // red is even; a partial last step reads zeros
     const int64_t s_lo = steps * warp / kLdWarps, s_hi = steps * (warp + 1) / kLdWarps;
 
     for (int j0 = 0; j0 < p.RT; j0 += 8 * NT) {
@@ -50,10 +50,11 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
         if (j0 < p.r) {
             for (int64_t st = s_lo; st < s_hi; ++st) {
                 const int64_t k0 = st * 16;
-                const uint32_t a0 = vA ? ld_ro_u32(aA + k0 + 2 * t) : 0u;
-                const uint32_t a1 = vB ? ld_ro_u32(aB + k0 + 2 * t) : 0u;
-                const uint32_t a2 = vA ? ld_ro_u32(aA + k0 + 2 * t + 8) : 0u;
-                const uint32_t a3 = vB ? ld_ro_u32(aB + k0 + 2 * t + 8) : 0u;
+                const bool lo_ok = k0 + 2 * t < p.red, hi_ok = k0 + 2 * t + 8 < p.red;
+                const uint32_t a0 = (vA && lo_ok) ? ld_ro_u32(aA + k0 + 2 * t) : 0u;
+                const uint32_t a1 = (vB && lo_ok) ? ld_ro_u32(aB + k0 + 2 * t) : 0u;
+                const uint32_t a2 = (vA && hi_ok) ? ld_ro_u32(aA + k0 + 2 * t + 8) : 0u;
+                const uint32_t a3 = (vB && hi_ok) ? ld_ro_u32(aB + k0 + 2 * t + 8) : 0u;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int j = j0 + nt * 8 + g;
@@ -61,13 +62,16 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
                     if (j < p.r) {
                         const uint16_t *sp = p.small + static_cast<int64_t>(j) * p.ldj;
                         if (p.ldk == 1) {
-                            b0 = ld_ro_u32(sp + k0 + 2 * t);
-                            b1 = ld_ro_u32(sp + k0 + 2 * t + 8);
+                            if (lo_ok) b0 = ld_ro_u32(sp + k0 + 2 * t);
+                            if (hi_ok) b1 = ld_ro_u32(sp + k0 + 2 * t + 8);
                         } else {
                             const int64_t L = p.ldk;
-                            b0 = ld_ro_u16(sp + (k0 + 2 * t) * L) | (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 1) * L)) << 16);
-                            b1 = ld_ro_u16(sp + (k0 + 2 * t + 8) * L) |
-                                 (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 9) * L)) << 16);
+                            if (lo_ok)
+                                b0 = ld_ro_u16(sp + (k0 + 2 * t) * L) |
+                                     (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 1) * L)) << 16);
+                            if (hi_ok)
+                                b1 = ld_ro_u16(sp + (k0 + 2 * t + 8) * L) |
+                                     (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 9) * L)) << 16);
                         }
                     }
                     mma_16816(d[nt], a0, a1, a2, a3, b0, b1);

@@ -154,7 +154,8 @@ def test_bulk_quantize_roundtrip(oracle):
             mu = float(ref["mu"])
             sig = np.repeat(ref["sigma"].astype(np.float64), 256)[: c.size]
             dq = 2.0 ** -4 * np.abs(c - mu) + 2.0 ** -10 * sig + 2.0 ** -22 * (c + abs(mu))
-            bound = 0.13852 * c + dq + 2.0 ** -8 * (c + dq)
+            half_gap = float(np.max(np.diff(oracle.nf4_table()))) / 2  # (T[1] - T[0]) / 2
+            bound = half_gap * c + dq + 2.0 ** -8 * (c + dq)
             err = np.max(np.abs(wf - df), axis=1)
             assert np.all(err <= bound * (1 + 1e-6)), f"layer {layer} {name}: round-trip bound"
             worst = max(worst, float(np.max(err / np.maximum(c, 1e-30))))
@@ -182,6 +183,26 @@ def run_case(oracle, case: synth.LayerCase, rows=None, check_bwd=True):
         ref_g = oracle.qlora_bwd_x(hw, n, k, bits(gh), M, Ab, Bb, r, case.alpha, rows=sel)
         worst = max(worst, assert_close(gx[torch.as_tensor(sel, device=DEV)], ref_g, f"{case.name} bwd_x"))
     return worst
+
+
+@pytest.mark.parametrize("n,k,M,r", [(128, 64, 65, 0), (128, 128, 256, 16), (256, 256, 300, 4), (200, 448, 129, 64),
+                                     (384, 192, 513, 200), (136, 1024, 1000, 16)])
+def test_gemm_small(oracle, n, k, M, r):
+    # tensor-core path (M > 64): ragged rows, features, tokens and adapter ranks
+    run_case(oracle, synth.LayerCase(f"gemm{n}x{k}M{M}r{r}", n, k, M, r, 2.0 * max(r, 1), 0.02, n * 3 + k + M))
+
+
+def test_gemm_error_word_stays_clear(oracle):
+    case = synth.LayerCase("gemm_err", 256, 512, 300, 16, 32.0, 0.02, 99)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV)
+    w = qb.nf4_quantize(W)
+    ws = torch.full((qb.linear_workspace_size(300, 256, 512, 16),), 0xAB, dtype=torch.uint8, device=DEV)
+    qb.qlora_linear_fwd(w, x, A, B, 32.0, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    qb.qlora_linear_bwd_x(w, gh, A, B, 32.0, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
 
 
 def test_tiny_fwd_bwd(oracle):
