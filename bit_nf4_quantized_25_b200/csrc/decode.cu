@@ -1,24 +1,30 @@
 // decode.cu -- QLoRA linear forward and input gradient for few tokens (M <= 64) on sm_100a.
 //
-//   fwd : h[m,n]      = sum_k W'[n,k] x[m,k]      + s * sum_j B[n,j] t[m,j],  t = A x
-//   bwd : grad_x[m,k] = sum_n grad_h[m,n] W'[n,k] + s * sum_j A[j,k] u[m,j],  u = B^T grad_h
+//   fwd : h[m,n]      = sum_k W'[n,k] x[m,k]      + sum_j B[n,j] t[m,j],  t = s A x
+//   bwd : grad_x[m,k] = sum_n grad_h[m,n] W'[n,k] + sum_j A[j,k] u[m,j],  u = s B^T grad_h
 // with W'[n,k] = NF4[code] * c'_b ("Quantized LoRA (QLoRA) and 4-bit training", apxml.com,
 // forward equations; "How does QLoRA work for training?", aivaro.ru, sections 2 and 7).
 //
-// Few tokens make this HBM-bound: every packed weight is read once and used M times.
-// B200 streams weights faster than CUDA cores can expand and multiply 4-bit codes, so
-// the multiply-accumulate runs on the tensor cores (mma.sync m16n8k16, A = weights,
-// B = tokens) and the per-weight work is one byte-indexed load from a shared-memory
-// table that maps a code byte (two nibbles) straight to a bf16 pair:
-//   - fwd: the table holds the unscaled NF4 values; each 64-weight block is reduced
-//     into its own fp32 fragment and scaled by its constant c'_b in fp32 (the
-//     block constant is applied after the dot product, which is the same sum).
-//   - bwd: the reduction runs over rows, whose constants differ, so the constants are
-//     folded into the bf16 token operand instead (c'_b * grad_h), and code nibbles of
-//     neighbouring rows are interleaved so that a byte again indexes a bf16 pair.
-// The contraction is split across a thread-block cluster (up to 8 CTAs); partial sums
-// and the LoRA down-projection are exchanged through distributed shared memory, so the
-// whole layer is one launch with no workspace.
+// Few tokens make this HBM-bound: each packed weight is read once and used M times. B200
+// streams about 13e12 weights/s but its SMs issue only ~3.6e13 lane-instructions/s, so the
+// whole per-weight budget is under three instructions. The multiply-accumulate therefore
+// runs on the tensor cores (mma.sync m16n8k16: A = 16 weight rows, B = 8 tokens) and the
+// dequantisation is one byte permute plus one shared-memory load per TWO weights: a
+// 256-entry table maps a code byte (two nibbles) to a bf16 pair. The table is stored once
+// per lane in 256-byte rows, so the permute that extracts the byte also forms the
+// conflict-free address (byte << 8 | lane << 2).
+//   - fwd: the table holds the unscaled NF4 values; every 64-weight block is reduced in its
+//     own fp32 fragment and scaled by its constant c'_b (the same sum, constant applied after
+//     the dot product). A lane computes the constants of one block per group of four and the
+//     quad shares them with shuffles.
+//   - bwd: the reduction runs over rows, whose constants differ, so the constants scale the
+//     bf16 token operand (c'_b * grad_h), and the nibbles of neighbouring rows are
+//     interleaved so that a byte again indexes a pair.
+// The reduction is split across a thread-block cluster (<= 8 CTAs); partial sums and the
+// LoRA down-projection are exchanged through distributed shared memory, so a layer is one
+// launch with no workspace. Codes stream through a two-group register ring; before the
+// programmatic-launch wait each warp asks L2 to prefetch its whole code slice (an L2
+// prefetch cannot return stale data), so the DRAM latency overlaps the preceding kernel.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -30,12 +36,13 @@ namespace qn {
 
 namespace {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kLutBytes = 256 * 32 * 4;  // 256 code bytes x 32 lane copies x bf16 pair
+constexpr int kLutBytes = 256 * 256;  // 256 code bytes x 256-byte rows (32 lane copies used)
 constexpr int kMaxCluster = 8;
-constexpr int kBatch = 8;      // 64-weight blocks per batch of loads (forward)
-constexpr int kStepBatch = 4;  // 16-row steps per batch of loads (input gradient)
+constexpr int kFwdRows = 16 * kDecWarps;  // weight rows per forward CTA
+constexpr int kBwdCols = 2;               // 64-feature block columns per input-gradient CTA
+constexpr int kBwdSub = kDecWarps / kBwdCols;  // reduction sub-slices inside a CTA
 
 struct DecodeParams {
     const uint8_t *codes;
@@ -52,59 +59,147 @@ struct DecodeParams {
     uint16_t *out;  // fwd: h (M x n); bwd: grad_x (M x k)
 };
 
-// Pair table: entry e (a code byte) = bf16x2(NF4[e & 15], NF4[e >> 4]); each entry is
-// stored once per lane so a warp's 32 random lookups hit 32 different banks.
-__device__ __forceinline__ void build_pair_lut(uint32_t *lut) {
-    __shared__ uint32_t s_t16[16];
-    if (threadIdx.x < 16) s_t16[threadIdx.x] = __float_as_uint(nf4_value(threadIdx.x));
-    __syncthreads();
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Pair table: row e (a code byte) holds bf16x2(NF4[e & 15], NF4[e >> 4]) in its first 32
+// words, one copy per lane.
+__device__ __forceinline__ void build_pair_lut(uint8_t *lut) {
     uint4 *l4 = reinterpret_cast<uint4 *>(lut);
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
-        const int e = i >> 3;
-        const uint32_t v = pack_bf16x2(__uint_as_float(s_t16[e & 15]), __uint_as_float(s_t16[e >> 4]));
-        l4[i] = make_uint4(v, v, v, v);
+        const int e = i >> 3, c = i & 7;
+        const uint32_t v = pack_bf16x2(nf4_value(e & 15), nf4_value(e >> 4));
+        l4[e * 16 + c] = make_uint4(v, v, v, v);
     }
 }
 
-__device__ __forceinline__ uint32_t lut_get(const uint32_t *lut, uint32_t byte, int lane) {
-    return lut[(byte << 5) | lane];
+// Pair for byte i (0..3) of word w: the permute builds (byte << 8) | (lane << 2).
+__device__ __forceinline__ uint32_t lut_pair(const uint8_t *lut, uint32_t w, uint32_t lane4, int i) {
+    const uint32_t off = prmt(w, lane4, 0x5504u | (static_cast<uint32_t>(i) << 4));
+    return *reinterpret_cast<const uint32_t *>(lut + off);
 }
-
-__device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return (w >> (8 * i)) & 0xffu; }
 
 __device__ __forceinline__ float round_bf16(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-// --------------------------------------------------------------------------- forward
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_line(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
+// L2 prefetch of an arbitrary byte range [p, p + bytes): 16-byte-aligned bulk part plus the
+// cache lines at the ragged ends.
+__device__ __forceinline__ void prefetch_range(const void *p, int64_t bytes) {
+    if (bytes <= 0) return;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), e = a + static_cast<uintptr_t>(bytes);
+    const uintptr_t a16 = (a + 15) & ~uintptr_t(15), e16 = e & ~uintptr_t(15);
+    if (e16 > a16) prefetch_l2(reinterpret_cast<const void *>(a16), static_cast<uint32_t>(e16 - a16));
+    prefetch_line(p);
+    prefetch_line(reinterpret_cast<const void *>(e - 1));
+}
+
+// Split cluster barrier: arrive once this CTA has finished reading remote shared memory,
+// wait (before exiting) until every CTA has.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// L2 prefetch (before the dependency wait) of the activation slice, the adapter slice and the
+// adapter rows the finalising CTA will read: with every operand already on its way to L2 the
+// kernel pays one DRAM round trip instead of a chain of them.
+__device__ __forceinline__ void prefetch_operands(const DecodeParams &p, int b_lo, int b_hi, int64_t row0, int rows,
+                                                  int crank, int C) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t K = p.k;
+    const int64_t kbytes = static_cast<int64_t>(b_hi - b_lo) * 128;  // 64 bf16 per block
+    if (warp == 0 && lane < p.M && kbytes > 0)
+        prefetch_l2(p.act + lane * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
+    if (warp == 1 && p.r > 0) {
+        for (int j = lane; j < p.r; j += 32)
+            if (kbytes > 0) prefetch_l2(p.A + j * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
+        const int r_lo = rows * crank / C, r_hi = rows * (crank + 1) / C;
+        const int64_t n_lo = row0 + r_lo, n_hi = row0 + r_hi < p.n ? row0 + r_hi : p.n;
+        if (lane == 0 && n_hi > n_lo) prefetch_range(p.B + n_lo * p.r, (n_hi - n_lo) * p.r * 2);
+    }
+}
+
+// ------------------------------------------------------------------------- forward
+// Registers of one group of four 64-weight blocks for rows A (g) and B (g + 8) of a lane.
+struct FwdGroup {
+    uint2 ca[4], cb[4];
+    uint32_t qa, qb;  // this lane's block (t) of the group
+    float sa, sb;
+};
+
 template <int NG>
 __global__ void __launch_bounds__(kDecThreads)
 k_decode_fwd(const DecodeParams p) {
     constexpr int MP = 8 * NG;  // padded token count
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-    float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [64 rows][MP]
+    uint8_t *lut = smem;
+    float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [kFwdRows][MP]
     const int rpad = (p.r + 15) & ~15;
-    float *tpart = part + 64 * MP;     // [rpad][MP] partial A x of this CTA's k-slice
-    float *tfull = tpart + rpad * MP;  // [rpad][MP] s * A x, rounded to bf16
+    float *tpart = part + kFwdRows * MP;  // [rpad][MP] partial A x of this CTA's k-slice
+    float *tfull = tpart + rpad * MP;     // [rpad][MP] s * A x, rounded to bf16
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = static_cast<int>(cluster.num_blocks());
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
 
+    const int64_t N = p.n, K = p.k;
+    const int nbr = static_cast<int>(K / kBlock);
+    const int b_lo = static_cast<int>(static_cast<int64_t>(nbr) * crank / C);
+    const int b_hi = static_cast<int>(static_cast<int64_t>(nbr) * (crank + 1) / C);
+    const int64_t row_base = static_cast<int64_t>(blockIdx.y) * kFwdRows + warp * 16;
+
+    // Before the dependency wait: on-chip setup and an L2 prefetch of the weight codes.
     build_pair_lut(lut);
     for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) tpart[i] = 0.0f;
+    if (lane < 16 && row_base + lane < N && b_hi > b_lo) {
+        const int64_t row = row_base + lane;
+        prefetch_l2(p.codes + row * (K / 2) + static_cast<int64_t>(b_lo) * 32, static_cast<uint32_t>(b_hi - b_lo) * 32u);
+        prefetch_range(p.q + row * nbr + b_lo, b_hi - b_lo);
+        prefetch_line(p.sigma + (row * nbr + b_lo) / kGroup);
+    }
+    prefetch_operands(p, b_lo, b_hi, static_cast<int64_t>(blockIdx.y) * kFwdRows, kFwdRows, crank, C);
     __syncthreads();
-    // Launched as a programmatic dependent: everything above overlaps the preceding
-    // kernel; no global memory is read before this point.
     grid_dependency_wait();
 
-    const int64_t N = p.n, K = p.k, nbr = K / kBlock;
-    const int64_t b_lo = nbr * crank / C, b_hi = nbr * (crank + 1) / C;
     const float mu = __ldg(p.mu);
     const int M = p.M;
+    const int64_t rowA = row_base + g, rowB = rowA + 8;
+    const bool vA = rowA < N, vB = rowB < N;
+    const uint8_t *cA = p.codes + (vA ? rowA : 0) * (K / 2) + 8 * t;
+    const uint8_t *cB = p.codes + (vB ? rowB : 0) * (K / 2) + 8 * t;
+    const int64_t qA = (vA ? rowA : 0) * nbr, qB = (vB ? rowB : 0) * nbr;
 
-    // x fragments: lane (g, t) of token group tg holds x[tg*8+g][64b + 16t .. +16].
+    auto load_group = [&](int b0, FwdGroup &G) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int b = b0 + j;
+            G.ca[j] = (vA && b < b_hi) ? __ldcs(reinterpret_cast<const uint2 *>(cA + static_cast<int64_t>(b) * 32))
+                                       : make_uint2(0u, 0u);
+            G.cb[j] = (vB && b < b_hi) ? __ldcs(reinterpret_cast<const uint2 *>(cB + static_cast<int64_t>(b) * 32))
+                                       : make_uint2(0u, 0u);
+        }
+        const int bt = b0 + t;
+        const bool ok = bt < b_hi;
+        G.qa = (vA && ok) ? __ldg(p.q + qA + bt) : 0u;
+        G.qb = (vB && ok) ? __ldg(p.q + qB + bt) : 0u;
+        G.sa = (vA && ok) ? __ldg(p.sigma + (qA + bt) / kGroup) : 0.0f;
+        G.sb = (vB && ok) ? __ldg(p.sigma + (qB + bt) / kGroup) : 0.0f;
+    };
+
+    // x rows of this lane's tokens: x[tg*8 + g][64b + 16t .. +16]
     const uint16_t *xrow[NG];
     bool xv[NG];
 #pragma unroll
@@ -114,114 +209,37 @@ k_decode_fwd(const DecodeParams p) {
         xrow[tg] = p.act + static_cast<int64_t>(xv[tg] ? tok : 0) * K + 16 * t;
     }
 
-    // ---- base: rows n0+g and n0+g+8 of this warp's 16-row tile, blocks [b_lo, b_hi)
-    {
-        const int64_t rowA = static_cast<int64_t>(blockIdx.y) * 64 + warp * 16 + g;
-        const int64_t rowB = rowA + 8;
-        const bool vA = rowA < N, vB = rowB < N;
-        const uint8_t *cA = p.codes + (vA ? rowA : 0) * (K / 2) + 8 * t;
-        const uint8_t *cB = p.codes + (vB ? rowB : 0) * (K / 2) + 8 * t;
-        const int64_t qA = (vA ? rowA : 0) * nbr, qB = (vB ? rowB : 0) * nbr;
-        float acc[NG][4];
+    float acc[NG][4];
 #pragma unroll
-        for (int tg = 0; tg < NG; ++tg) acc[tg][0] = acc[tg][1] = acc[tg][2] = acc[tg][3] = 0.0f;
+    for (int tg = 0; tg < NG; ++tg) acc[tg][0] = acc[tg][1] = acc[tg][2] = acc[tg][3] = 0.0f;
 
-        // Batches of kBatch blocks: every load of a batch is issued before any use, so a
-        // warp keeps 2 x kBatch x 8 bytes of codes per lane in flight.
-        for (int64_t bb = b_lo; bb < b_hi; bb += kBatch) {
-            const int nbk = static_cast<int>(b_hi - bb < kBatch ? b_hi - bb : kBatch);
-            uint2 ca[kBatch], cb[kBatch];
-            uint32_t qa[kBatch], qbv[kBatch];
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                ca[j] = cb[j] = make_uint2(0u, 0u);
-                qa[j] = qbv[j] = 0u;
-                if (j < nbk) {
-                    if (vA) {
-                        ca[j] = __ldcs(reinterpret_cast<const uint2 *>(cA + (bb + j) * 32));
-                        qa[j] = __ldg(p.q + qA + bb + j);
-                    }
-                    if (vB) {
-                        cb[j] = __ldcs(reinterpret_cast<const uint2 *>(cB + (bb + j) * 32));
-                        qbv[j] = __ldg(p.q + qB + bb + j);
-                    }
-                }
-            }
-            // a batch of <= 8 consecutive blocks touches at most two groups
-            const int64_t gA0 = (qA + bb) / kGroup, gB0 = (qB + bb) / kGroup;
-            const int64_t ng_all = (N * nbr + kGroup - 1) / kGroup;
-            const float sA0 = __ldg(p.sigma + gA0), sA1 = __ldg(p.sigma + (gA0 + 1 < ng_all ? gA0 + 1 : gA0));
-            const float sB0 = __ldg(p.sigma + gB0), sB1 = __ldg(p.sigma + (gB0 + 1 < ng_all ? gB0 + 1 : gB0));
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                if (j >= nbk) break;
-                const int64_t b = bb + j;
-                const float cpA = vA ? block_constant(static_cast<uint8_t>(qa[j]),
-                                                      (qA + b) / kGroup == gA0 ? sA0 : sA1, mu) : 0.0f;
-                const float cpB = vB ? block_constant(static_cast<uint8_t>(qbv[j]),
-                                                      (qB + b) / kGroup == gB0 ? sB0 : sB1, mu) : 0.0f;
-                uint32_t af[4][4];
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t wa = kk < 2 ? ca[j].x : ca[j].y, wb = kk < 2 ? cb[j].x : cb[j].y;
-                    const int i0 = (2 * kk) & 3;
-                    af[kk][0] = lut_get(lut, byte_of(wa, i0), lane);
-                    af[kk][2] = lut_get(lut, byte_of(wa, i0 + 1), lane);
-                    af[kk][1] = lut_get(lut, byte_of(wb, i0), lane);
-                    af[kk][3] = lut_get(lut, byte_of(wb, i0 + 1), lane);
-                }
-#pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                    if (xv[tg]) {
-                        x0 = ld_ro_v4(xrow[tg] + b * 64);
-                        x1 = ld_ro_v4(xrow[tg] + b * 64 + 8);
-                    }
-                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_16816(d, af[kk][0], af[kk][1], af[kk][2], af[kk][3], xw[2 * kk], xw[2 * kk + 1]);
-                    acc[tg][0] = __fmaf_rn(cpA, d[0], acc[tg][0]);
-                    acc[tg][1] = __fmaf_rn(cpA, d[1], acc[tg][1]);
-                    acc[tg][2] = __fmaf_rn(cpB, d[2], acc[tg][2]);
-                    acc[tg][3] = __fmaf_rn(cpB, d[3], acc[tg][3]);
-                }
-            }
-        }
-        const int rl = warp * 16 + g;
-#pragma unroll
-        for (int tg = 0; tg < NG; ++tg) {
-            part[rl * MP + tg * 8 + 2 * t] = acc[tg][0];
-            part[rl * MP + tg * 8 + 2 * t + 1] = acc[tg][1];
-            part[(rl + 8) * MP + tg * 8 + 2 * t] = acc[tg][2];
-            part[(rl + 8) * MP + tg * 8 + 2 * t + 1] = acc[tg][3];
-        }
-    }
+    FwdGroup cur, nxt;
+    if (b_lo < b_hi) load_group(b_lo, cur);
 
-    // ---- LoRA down-projection over this CTA's k-slice: partial t = A x (fp32).
-    // Work item (j-tile, quarter of the slice); warp w takes quarter w of every tile.
+    // ---- LoRA down-projection over this CTA's k-slice (partial t = A x, fp32), while the
+    // first codes are in flight. Item (j-tile, eighth of the slice) per warp.
     if (p.r > 0) {
         const int rt = rpad / 16;
-        const int64_t nb_sl = b_hi - b_lo;
-        const int64_t s_lo = b_lo + nb_sl * warp / kDecWarps, s_hi = b_lo + nb_sl * (warp + 1) / kDecWarps;
+        const int nsl = b_hi - b_lo;
+        const int s_lo = b_lo + nsl * warp / kDecWarps, s_hi = b_lo + nsl * (warp + 1) / kDecWarps;
         for (int jt = 0; jt < rt; ++jt) {
             const int jA = jt * 16 + g, jB = jA + 8;
-            const bool vA = jA < p.r, vB = jB < p.r;
-            const uint16_t *aA = p.A + static_cast<int64_t>(vA ? jA : 0) * K + 16 * t;
-            const uint16_t *aB = p.A + static_cast<int64_t>(vB ? jB : 0) * K + 16 * t;
+            const bool aA = jA < p.r, aB = jB < p.r;
+            const uint16_t *pa = p.A + static_cast<int64_t>(aA ? jA : 0) * K + 16 * t;
+            const uint16_t *pb = p.A + static_cast<int64_t>(aB ? jB : 0) * K + 16 * t;
             float d[NG][4];
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) d[tg][0] = d[tg][1] = d[tg][2] = d[tg][3] = 0.0f;
-            for (int64_t b = s_lo; b < s_hi; ++b) {
+            for (int b = s_lo; b < s_hi; ++b) {
+                const int64_t o = static_cast<int64_t>(b) * 64;
                 uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0, b0 = a0, b1 = a0;
-                if (vA) {
-                    a0 = ld_ro_v4(aA + b * 64);
-                    a1 = ld_ro_v4(aA + b * 64 + 8);
+                if (aA) {
+                    a0 = ld_ro_v4(pa + o);
+                    a1 = ld_ro_v4(pa + o + 8);
                 }
-                if (vB) {
-                    b0 = ld_ro_v4(aB + b * 64);
-                    b1 = ld_ro_v4(aB + b * 64 + 8);
+                if (aB) {
+                    b0 = ld_ro_v4(pb + o);
+                    b1 = ld_ro_v4(pb + o + 8);
                 }
                 const uint32_t ra[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
@@ -229,8 +247,8 @@ k_decode_fwd(const DecodeParams p) {
                 for (int tg = 0; tg < NG; ++tg) {
                     uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
                     if (xv[tg]) {
-                        x0 = ld_ro_v4(xrow[tg] + b * 64);
-                        x1 = ld_ro_v4(xrow[tg] + b * 64 + 8);
+                        x0 = ld_ro_v4(xrow[tg] + o);
+                        x1 = ld_ro_v4(xrow[tg] + o + 8);
                     }
                     const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
@@ -250,6 +268,59 @@ k_decode_fwd(const DecodeParams p) {
         }
     }
 
+    // ---- base: blocks [b_lo, b_hi) of rows A and B, groups of four, double-buffered.
+    for (int b0 = b_lo; b0 < b_hi; b0 += 4) {
+        if (b0 + 4 < b_hi) load_group(b0 + 4, nxt);
+        const float cA4 = vA ? block_constant(static_cast<uint8_t>(cur.qa), cur.sa, mu) : 0.0f;
+        const float cB4 = vB ? block_constant(static_cast<uint8_t>(cur.qb), cur.sb, mu) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int b = b0 + j;
+            if (b >= b_hi) break;
+            const float cpA = __shfl_sync(0xffffffffu, cA4, (lane & ~3) | j);
+            const float cpB = __shfl_sync(0xffffffffu, cB4, (lane & ~3) | j);
+            uint32_t af[4][4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t wa = kk < 2 ? cur.ca[j].x : cur.ca[j].y, wb = kk < 2 ? cur.cb[j].x : cur.cb[j].y;
+                const int i0 = (2 * kk) & 3;
+                af[kk][0] = lut_pair(lut, wa, lane4, i0);
+                af[kk][2] = lut_pair(lut, wa, lane4, i0 + 1);
+                af[kk][1] = lut_pair(lut, wb, lane4, i0);
+                af[kk][3] = lut_pair(lut, wb, lane4, i0 + 1);
+            }
+            const int64_t o = static_cast<int64_t>(b) * 64;
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+                if (xv[tg]) {
+                    x0 = ld_ro_v4(xrow[tg] + o);
+                    x1 = ld_ro_v4(xrow[tg] + o + 8);
+                }
+                const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_16816(d, af[kk][0], af[kk][1], af[kk][2], af[kk][3], xw[2 * kk], xw[2 * kk + 1]);
+                acc[tg][0] = __fmaf_rn(cpA, d[0], acc[tg][0]);
+                acc[tg][1] = __fmaf_rn(cpA, d[1], acc[tg][1]);
+                acc[tg][2] = __fmaf_rn(cpB, d[2], acc[tg][2]);
+                acc[tg][3] = __fmaf_rn(cpB, d[3], acc[tg][3]);
+            }
+        }
+        cur = nxt;
+    }
+    {
+        const int rl = warp * 16 + g;
+#pragma unroll
+        for (int tg = 0; tg < NG; ++tg) {
+            part[rl * MP + tg * 8 + 2 * t] = acc[tg][0];
+            part[rl * MP + tg * 8 + 2 * t + 1] = acc[tg][1];
+            part[(rl + 8) * MP + tg * 8 + 2 * t] = acc[tg][2];
+            part[(rl + 8) * MP + tg * 8 + 2 * t + 1] = acc[tg][3];
+        }
+    }
+
     __syncthreads();
     cluster.sync();  // every CTA's partials are complete and visible in the cluster
     grid_dependents_launch();
@@ -263,11 +334,11 @@ k_decode_fwd(const DecodeParams p) {
     }
     __syncthreads();
 
-    // ---- this CTA finalises rows [64*crank/C, 64*(crank+1)/C) of the 64-row group
-    const int r_lo = 64 * crank / C, r_hi = 64 * (crank + 1) / C, nr = r_hi - r_lo;
+    // ---- this CTA finalises rows [kFwdRows*crank/C, kFwdRows*(crank+1)/C) of the row group
+    const int r_lo = kFwdRows * crank / C, r_hi = kFwdRows * (crank + 1) / C, nr = r_hi - r_lo;
     for (int i = threadIdx.x; i < nr * M; i += blockDim.x) {
         const int rl = r_lo + i % nr, tok = i / nr;
-        const int64_t n = static_cast<int64_t>(blockIdx.y) * 64 + rl;
+        const int64_t n = static_cast<int64_t>(blockIdx.y) * kFwdRows + rl;
         if (n >= N) continue;
         float sum = 0.0f;
         for (int cc = 0; cc < C; ++cc) sum += cluster.map_shared_rank(part, cc)[rl * MP + tok];
@@ -307,117 +378,102 @@ __device__ __forceinline__ void load_g4(const uint16_t *gh, int64_t N, int tok, 
     }
 }
 
+// Registers of one group of two 16-row steps: 4 rows (4t .. 4t+3) x 8 features per step,
+// plus the constant inputs of row (4t + gq % 4) of each step.
+struct BwdGroup {
+    uint32_t w[2][4];
+    uint32_t q[2];
+    float s[2];
+};
+
 template <int NG>
 __global__ void __launch_bounds__(kDecThreads)
 k_decode_bwd(const DecodeParams p) {
     constexpr int MP = 8 * NG;
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-    float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [4 warps x 64 cols][MP]
+    uint8_t *lut = smem;
+    float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [warps][64 features][MP]
     const int rpad = (p.r + 15) & ~15;
-    float *upart = part + 256 * MP;    // [rpad][MP] partial B^T grad_h over this n-slice
-    float *ufull = upart + rpad * MP;  // [rpad][MP] s * B^T grad_h, rounded to bf16
+    float *upart = part + kDecWarps * 64 * MP;  // [rpad][MP] partial B^T grad_h of this CTA
+    float *ufull = upart + rpad * MP;           // [rpad][MP] s * B^T grad_h, rounded to bf16
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = static_cast<int>(cluster.num_blocks());
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, t = lane & 3;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+
+    const int64_t N = p.n, K = p.k;
+    const int64_t nbr = K / kBlock;
+    const int col = warp % kBwdCols, sub = warp / kBwdCols;
+    const int64_t kb = static_cast<int64_t>(blockIdx.y) * kBwdCols + col;  // output block column
+    const bool vk = kb < nbr;
+    const int64_t kbc = vk ? kb : 0;
+    // reduction rows in 16-row steps: cluster slice, then this warp's sub-slice
+    const int64_t n16 = (N + 15) / 16;
+    const int64_t c_lo = n16 * crank / C, c_hi = n16 * (crank + 1) / C;
+    const int64_t s_lo = c_lo + (c_hi - c_lo) * sub / kBwdSub, s_hi = c_lo + (c_hi - c_lo) * (sub + 1) / kBwdSub;
 
     build_pair_lut(lut);
     for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) upart[i] = 0.0f;
+    // L2 prefetch of everything this CTA reads: the warp's codes (rows [16 s_lo, 16 s_hi) x
+    // 32 bytes of column kb) and their constants, the grad_h slice, the adapter rows.
+    if (vk) {
+        for (int64_t rr = s_lo * 16 + lane; rr < s_hi * 16 && rr < N; rr += 32) {
+            prefetch_l2(p.codes + rr * (K / 2) + kbc * 32, 32u);
+            prefetch_line(p.q + rr * nbr + kbc);
+            prefetch_line(p.sigma + (rr * nbr + kbc) / kGroup);
+        }
+    }
+    if (warp == 0 && lane < p.M) {
+        const int64_t n_lo = c_lo * 16, n_hi = c_hi * 16 < N ? c_hi * 16 : N;
+        prefetch_range(p.act + lane * N + n_lo, (n_hi - n_lo) * 2);
+    }
+    if (warp == 1 && p.r > 0) {
+        const int64_t n_lo = c_lo * 16, n_hi = c_hi * 16 < N ? c_hi * 16 : N;
+        if (lane == 0) prefetch_range(p.B + n_lo * p.r, (n_hi - n_lo) * p.r * 2);
+        const int64_t k0 = static_cast<int64_t>(blockIdx.y) * 64 * kBwdCols;
+        const int64_t k1 = k0 + 64 * kBwdCols < K ? k0 + 64 * kBwdCols : K;
+        for (int j = lane; j < p.r; j += 32) prefetch_range(p.A + j * K + k0, (k1 - k0) * 2);
+    }
     __syncthreads();
     grid_dependency_wait();
 
-    const int64_t N = p.n, K = p.k, nbr = K / kBlock;
-    const int64_t n16 = (N + 15) / 16;
-    const int64_t s_lo = n16 * crank / C, s_hi = n16 * (crank + 1) / C;  // 16-row steps of this slice
     const float mu = __ldg(p.mu);
     const int M = p.M;
 
-    // ---- base: output block column kb (64 features), reduction over this slice's rows.
-    {
-        const int64_t kb = static_cast<int64_t>(blockIdx.y) * kDecWarps + warp;
-        const bool vk = kb < nbr;
-        const int64_t kbc = vk ? kb : 0;
-        float acc[4][NG][4];
+    auto load_group = [&](int64_t st0, BwdGroup &G) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 2; ++j) {
+            const int64_t st = st0 + j;
 #pragma unroll
-            for (int tg = 0; tg < NG; ++tg) acc[i][tg][0] = acc[i][tg][1] = acc[i][tg][2] = acc[i][tg][3] = 0.0f;
-
-        if (vk) {
-            // Batches of kStepBatch 16-row steps, all loads issued before use.
-            for (int64_t sb = s_lo; sb < s_hi; sb += kStepBatch) {
-                const int nst = static_cast<int>(s_hi - sb < kStepBatch ? s_hi - sb : kStepBatch);
-                uint32_t w[kStepBatch][4], qv[kStepBatch][4];
-                float sg[kStepBatch][4];
-#pragma unroll
-                for (int j = 0; j < kStepBatch; ++j)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int64_t n = (sb + j) * 16 + 4 * t + i;
-                        w[j][i] = 0x77777777u;  // value 0
-                        qv[j][i] = 0u;
-                        sg[j][i] = 0.0f;
-                        if (j < nst && n < N) {
-                            const int64_t bi = n * nbr + kbc;
-                            w[j][i] = ld_nc_u32(p.codes + n * (K / 2) + kbc * 32 + 4 * gq);
-                            qv[j][i] = __ldg(p.q + bi);
-                            sg[j][i] = __ldg(p.sigma + bi / kGroup);
-                        }
-                    }
-#pragma unroll
-                for (int j = 0; j < kStepBatch; ++j) {
-                    if (j >= nst) break;
-                    const int64_t n0 = (sb + j) * 16 + 4 * t;  // this lane's 4 reduction rows
-                    float cp[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) cp[i] = block_constant(static_cast<uint8_t>(qv[j][i]), sg[j][i], mu);
-                    uint32_t e01, o01, e23, o23;
-                    interleave_rows(w[j][0], w[j][1], e01, o01);
-                    interleave_rows(w[j][2], w[j][3], e23, o23);
-                    uint32_t af[4][4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        af[i][0] = lut_get(lut, byte_of(e01, i), lane);
-                        af[i][1] = lut_get(lut, byte_of(o01, i), lane);
-                        af[i][2] = lut_get(lut, byte_of(e23, i), lane);
-                        af[i][3] = lut_get(lut, byte_of(o23, i), lane);
-                    }
-#pragma unroll
-                    for (int tg = 0; tg < NG; ++tg) {
-                        const int tok = tg * 8 + gq;
-                        float gv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                        if (tok < M) load_g4(p.act, N, tok, n0, gv);
-                        const uint32_t b0 = pack_bf16x2(cp[0] * gv[0], cp[1] * gv[1]);
-                        const uint32_t b1 = pack_bf16x2(cp[2] * gv[2], cp[3] * gv[3]);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            mma_16816(acc[i][tg], af[i][0], af[i][1], af[i][2], af[i][3], b0, b1);
-                    }
-                }
+            for (int i = 0; i < 4; ++i) {
+                const int64_t n = st * 16 + 4 * t + i;
+                G.w[j][i] = (st < s_hi && n < N) ? ld_nc_u32(p.codes + n * (K / 2) + kbc * 32 + 4 * gq) : 0x77777777u;
             }
+            const int64_t n = st * 16 + 4 * t + (gq & 3);
+            const bool ok = st < s_hi && n < N;
+            const int64_t bi = n * nbr + kbc;
+            G.q[j] = ok ? __ldg(p.q + bi) : 0u;
+            G.s[j] = ok ? __ldg(p.sigma + bi / kGroup) : 0.0f;
         }
-        // D row gq of tile i is feature 8*gq + 2i, row gq+8 is feature 8*gq + 2i + 1.
-        float *wp = part + warp * 64 * MP;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int tg = 0; tg < NG; ++tg) {
-                const int f = 8 * gq + 2 * i, tok = tg * 8 + 2 * t;
-                wp[f * MP + tok] = acc[i][tg][0];
-                wp[f * MP + tok + 1] = acc[i][tg][1];
-                wp[(f + 1) * MP + tok] = acc[i][tg][2];
-                wp[(f + 1) * MP + tok + 1] = acc[i][tg][3];
-            }
-    }
+    };
 
-    // ---- LoRA: partial u[j][tok] = sum_n B[n][j] grad_h[tok][n] over this slice.
+    float acc[4][NG][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int tg = 0; tg < NG; ++tg) acc[i][tg][0] = acc[i][tg][1] = acc[i][tg][2] = acc[i][tg][3] = 0.0f;
+
+    BwdGroup cur, nxt;
+    if (vk && s_lo < s_hi) load_group(s_lo, cur);
+
+    // ---- LoRA: partial u[j][tok] = sum_n B[n][j] grad_h[tok][n] over this CTA's slice.
     if (p.r > 0) {
         const int rt = rpad / 16;
-        const int64_t ns = s_hi - s_lo;
-        const int64_t q_lo = s_lo + ns * warp / kDecWarps, q_hi = s_lo + ns * (warp + 1) / kDecWarps;
+        const int64_t ns = c_hi - c_lo;
+        const int64_t q_lo = c_lo + ns * warp / kDecWarps, q_hi = c_lo + ns * (warp + 1) / kDecWarps;
         for (int jt = 0; jt < rt; ++jt) {
             const int jA = jt * 16 + gq, jB = jA + 8;
             float d[NG][4];
@@ -458,6 +514,64 @@ k_decode_bwd(const DecodeParams p) {
         }
     }
 
+    // ---- base: block column kb, reduction over steps [s_lo, s_hi), groups of two steps
+    if (vk) {
+        for (int64_t st0 = s_lo; st0 < s_hi; st0 += 2) {
+            if (st0 + 2 < s_hi) load_group(st0 + 2, nxt);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int64_t st = st0 + j;
+                if (st >= s_hi) break;
+                const int64_t n0 = st * 16 + 4 * t;  // this lane's 4 reduction rows
+                // constant of row n0 + (gq & 3), shared with the lanes of the same t
+                const float mine = block_constant(static_cast<uint8_t>(cur.q[j]), cur.s[j], mu);
+                float cp[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    cp[i] = __shfl_sync(0xffffffffu, mine, (i << 2) | t);
+                    if (n0 + i >= N) cp[i] = 0.0f;
+                }
+                uint32_t e01, o01, e23, o23;
+                interleave_rows(cur.w[j][0], cur.w[j][1], e01, o01);
+                interleave_rows(cur.w[j][2], cur.w[j][3], e23, o23);
+                uint32_t af[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    af[i][0] = lut_pair(lut, e01, lane4, i);
+                    af[i][1] = lut_pair(lut, o01, lane4, i);
+                    af[i][2] = lut_pair(lut, e23, lane4, i);
+                    af[i][3] = lut_pair(lut, o23, lane4, i);
+                }
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) {
+                    const int tok = tg * 8 + gq;
+                    float gv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    if (tok < M) load_g4(p.act, N, tok, n0, gv);
+                    const uint32_t b0 = pack_bf16x2(cp[0] * gv[0], cp[1] * gv[1]);
+                    const uint32_t b1 = pack_bf16x2(cp[2] * gv[2], cp[3] * gv[3]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        mma_16816(acc[i][tg], af[i][0], af[i][1], af[i][2], af[i][3], b0, b1);
+                }
+            }
+            cur = nxt;
+        }
+    }
+    // D row gq of tile i is feature 8*gq + 2i, row gq+8 is feature 8*gq + 2i + 1.
+    {
+        float *wp = part + warp * 64 * MP;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                const int f = 8 * gq + 2 * i, tok = tg * 8 + 2 * t;
+                wp[f * MP + tok] = acc[i][tg][0];
+                wp[f * MP + tok + 1] = acc[i][tg][1];
+                wp[(f + 1) * MP + tok] = acc[i][tg][2];
+                wp[(f + 1) * MP + tok + 1] = acc[i][tg][3];
+            }
+    }
+
     __syncthreads();
     cluster.sync();
     grid_dependents_launch();
@@ -471,14 +585,20 @@ k_decode_bwd(const DecodeParams p) {
     }
     __syncthreads();
 
-    // ---- this CTA finalises features [256*crank/C, 256*(crank+1)/C) of the 256-feature group
-    const int f_lo = 256 * crank / C, f_hi = 256 * (crank + 1) / C, nf = f_hi - f_lo;
+    // ---- this CTA finalises features [F*crank/C, F*(crank+1)/C) of the CTA group's F features
+    constexpr int F = 64 * kBwdCols;
+    const int f_lo = F * crank / C, f_hi = F * (crank + 1) / C, nf = f_hi - f_lo;
     for (int i = threadIdx.x; i < nf * M; i += blockDim.x) {
         const int fl = f_lo + i % nf, tok = i / nf;
-        const int64_t k = static_cast<int64_t>(blockIdx.y) * 256 + fl;
+        const int64_t k = static_cast<int64_t>(blockIdx.y) * F + fl;
         if (k >= K) continue;
+        const int c = fl / 64, f = fl % 64;
         float sum = 0.0f;
-        for (int cc = 0; cc < C; ++cc) sum += cluster.map_shared_rank(part, cc)[fl * MP + tok];
+        for (int cc = 0; cc < C; ++cc) {
+            const float *rp = cluster.map_shared_rank(part, cc);
+#pragma unroll
+            for (int sb = 0; sb < kBwdSub; ++sb) sum += rp[((sb * kBwdCols + c) * 64 + f) * MP + tok];
+        }
         if (p.r > 0) {
             float lora = 0.0f;
             for (int j = 0; j < p.r; ++j)
@@ -521,30 +641,44 @@ cudaError_t launch_cluster(Kern kern, dim3 grid, int cluster_x, size_t smem, cud
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     // Programmatic dependent launch: the grid may start while the preceding kernel
-    // finishes; the kernel reads no global memory before griddepcontrol.wait.
+    // finishes; the kernel reads no global memory before griddepcontrol.wait (only an L2
+    // prefetch of the frozen weight codes is issued earlier).
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e;
-    e = cudaLaunchKernelEx(&cfg, kern, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     count_launch();
     return e;
 }
 
 int pick_groups(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
-// Cluster size: enough CTAs to fill the GPU, at most 8, at least 16 blocks of work per CTA.
-int pick_cluster(int64_t tiles, int64_t red_units, int sms) {
-    int C = 1;
-    while (C < kMaxCluster && tiles * C < 2 * sms && red_units / (2 * C) >= 8) C *= 2;
-    return C;
+// Cluster size: the power of two (<= 8) that brings the CTA count closest to two per SM,
+// keeping at least `min_units` units of reduction work per CTA.
+int pick_cluster(int64_t tiles, int64_t red_units, int64_t min_units, int sms) {
+    int best = 1;
+    double best_score = 1e30;
+    for (int C = 1; C <= kMaxCluster; C *= 2) {
+        if (C > 1 && red_units / C < min_units) break;
+        const double ratio = static_cast<double>(tiles * C) / (2.0 * sms);
+        const double score = ratio > 1.0 ? ratio : 1.0 / ratio;
+        if (score < best_score) {
+            best_score = score;
+            best = C;
+        }
+    }
+    return best;
 }
 
 int num_sms() {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
     return sms;
 }
 
@@ -556,9 +690,9 @@ cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, con
     DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, x, M, A, B, r, s, h};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
-    const size_t smem = kLutBytes + sizeof(float) * (64 * 8 * NG + 2 * rpad * 8 * NG);
-    const int64_t tiles = (w.n + 63) / 64;
-    const int C = pick_cluster(tiles, w.k / kBlock, num_sms());
+    const size_t smem = kLutBytes + sizeof(float) * (kFwdRows * 8 * NG + 2 * rpad * 8 * NG);
+    const int64_t tiles = (w.n + kFwdRows - 1) / kFwdRows;
+    const int C = pick_cluster(tiles, w.k / kBlock, 4, num_sms());
     const dim3 grid(C, static_cast<unsigned>(tiles), 1);
     switch (NG) {
         case 1: return launch_cluster(k_decode_fwd<1>, grid, C, smem, st, p);
@@ -574,9 +708,9 @@ cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, co
     DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, gh, M, A, B, r, s, gx};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
-    const size_t smem = kLutBytes + sizeof(float) * (256 * 8 * NG + 2 * rpad * 8 * NG);
-    const int64_t tiles = (w.k / kBlock + kDecWarps - 1) / kDecWarps;
-    const int C = pick_cluster(tiles, (w.n + 15) / 16 / 4, num_sms());
+    const size_t smem = kLutBytes + sizeof(float) * (kDecWarps * 64 * 8 * NG + 2 * rpad * 8 * NG);
+    const int64_t tiles = (w.k / kBlock + kBwdCols - 1) / kBwdCols;
+    const int C = pick_cluster(tiles, (w.n + 15) / 16 / kBwdSub, 2, num_sms());
     const dim3 grid(C, static_cast<unsigned>(tiles), 1);
     switch (NG) {
         case 1: return launch_cluster(k_decode_bwd<1>, grid, C, smem, st, p);

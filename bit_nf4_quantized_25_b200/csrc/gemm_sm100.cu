@@ -13,13 +13,13 @@
 //   warp 0      : TMA producer of the token operand (x / grad_h, then t / u), 64-wide K slabs
 //                 in the 128-byte swizzled K-major layout, 4-stage mbarrier ring.
 //   warp 1      : TMEM allocator and the single MMA-issuing thread (tcgen05.mma kind::f16).
-//   warps 2..9  : two groups of four dequant warps taking alternate stages. A thread owns one
+//   warps 2..13 : three groups of four dequant warps taking stages round-robin. A thread owns one
 //                 64-weight block per stage (fwd: one row; bwd: half of a reduction row),
 //                 builds the 16 scaled bf16 values NF4[i] * c'_b in registers, expands the
 //                 nibbles with byte permutes and writes the swizzled A tile (K-major for fwd,
 //                 MN-major for bwd, so W is always read in its stored row-major order).
 //                 The extra LoRA stages copy rows of B (fwd) / A (bwd) into the A tile.
-//   epilogue    : the eight dequant warps read TMEM (tcgen05.ld) and store bf16.
+//   epilogue    : the dequant warps read TMEM (tcgen05.ld) and store bf16.
 // Every mbarrier wait is bounded; on a timeout the CTA records an error code, stops issuing
 // work, drains what it issued and frees its TMEM.
 #include <cudaTypedefs.h>
@@ -38,7 +38,8 @@ constexpr int kTileM = 128;  // MMA M: weight rows / input features
 constexpr int kTileN = 256;  // MMA N: tokens
 constexpr int kTileK = 64;   // reduction per stage: one 128-byte swizzle row of bf16
 constexpr int kStages = 4;
-constexpr int kDqWarps = 8;
+constexpr int kDqGroups = 3;               // dequant groups taking stages round-robin
+constexpr int kDqWarps = 4 * kDqGroups;
 constexpr int kGemmThreads = (2 + kDqWarps) * 32;
 constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK * 2;  // 32 KB
@@ -226,7 +227,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
     } else {
         // ----------------------------------------------------------- dequant groups
         const int dw = warp - 2;
-        const int grp = dw >> 2;                  // stages i with i % 2 == grp
+        const int grp = dw >> 2;                  // stages i with i % kDqGroups == grp
         const int tid = (dw & 3) * 32 + lane;     // 0..127 within the group
         const float mu = __ldg(p.mu);
         // fwd: thread = A row (weight row row0 + tid), 64 k per stage.
@@ -265,7 +266,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         float ns;
         bool nv;
         load_codes(grp, n0, n1, nq, ns, nv);
-        for (int i = grp; i < T; i += 2) {
+        for (int i = grp; i < T; i += kDqGroups) {
             if (*abort_flag) break;
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1u;
@@ -273,7 +274,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
             const uint32_t cq = nq;
             const float cs = ns;
             const bool cv = nv;
-            load_codes(i + 2, n0, n1, nq, ns, nv);  // prefetch this group's next stage
+            load_codes(i + kDqGroups, n0, n1, nq, ns, nv);  // prefetch this group's next stage
             if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
                 fail();
                 break;
@@ -345,7 +346,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int64_t orow = row0 + quarter * 32 + lane;           // fwd: n; bwd: feature k
         const int64_t ldo = kBwd ? K : N;
         const bool rvalid = orow < (kBwd ? K : N);
-        for (int cb = grp * 4; cb < grp * 4 + 4; ++cb) {  // 32-column chunks of this group
+        for (int cb = grp; cb < kTileN / 32; cb += kDqGroups) {  // 32-column chunks of this group
             uint32_t v[32];
             tmem_ld32(tmem_d + ((quarter * 32u) << 16) + static_cast<uint32_t>(cb * 32), v);
             tmem_ld_wait();

@@ -10,8 +10,8 @@
 // thresholds, packs 8 codes per 32-bit word, writes the fp32 absmax to the workspace
 // and adds it to 256 exponent bins (integer sums, so the tensor sum is exact and
 // independent of scheduling).
-// Kernel 2 (1/64 of the data): every CTA rebuilds the exact mean from the bins, then
-// each warp double-quantises one group of 256 block absmaxes.
+// The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
+// Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,14 +22,20 @@ namespace {
 constexpr int kQuantThreads = 256;
 constexpr int kDqThreads = 256;
 constexpr size_t kBinsBytes = 256 * sizeof(unsigned long long);
+constexpr size_t kHeaderBytes = kBinsBytes + 256;  // bins, then the finished-CTA counter
 
 __device__ __forceinline__ uint32_t mag_max2(uint32_t u) {
     return max(u & 0x7fffu, (u >> 16) & 0x7fffu);
 }
 
+__device__ float mean_from_bins(const unsigned long long *bins, int64_t nb);
+
+// The last CTA to finish (counted with an atomic, no waiting) rebuilds the exact mean from
+// the completed bins and stores it.
 __global__ void __launch_bounds__(kQuantThreads)
 k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ codes, float *__restrict__ cblk,
-               unsigned long long *__restrict__ bins, QuantCells cells) {
+               unsigned long long *__restrict__ bins, unsigned *__restrict__ done, float *__restrict__ mu_out,
+               QuantCells cells) {
     __shared__ float s_thr[65];
     __shared__ int s_base[65];
     __shared__ unsigned s_bins[256];
@@ -91,6 +97,18 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
     __syncthreads();
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
         if (s_bins[i]) atomicAdd(&bins[i], static_cast<unsigned long long>(s_bins[i]));
+    __threadfence();
+    __syncthreads();
+    __shared__ bool s_last;
+    if (threadIdx.x == 0) s_last = atomicAdd(done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        __shared__ unsigned long long s_all[256];
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) s_all[i] = __ldcg(bins + i);
+        __syncthreads();
+        if (threadIdx.x == 0) *mu_out = mean_from_bins(s_all, nb);
+    }
 }
 
 // Exact mean of the block absmaxes from the exponent bins, rounded once to fp32.
@@ -172,18 +190,9 @@ __device__ float mean_from_bins(const unsigned long long *bins, int64_t nb) {
 }
 
 __global__ void __launch_bounds__(kDqThreads)
-k_double_quant(const float *__restrict__ cblk, int64_t nb, const unsigned long long *__restrict__ bins,
-               uint8_t *__restrict__ q, float *__restrict__ sigma, float *__restrict__ mu_out) {
-    __shared__ unsigned long long s_bins[256];
-    __shared__ float s_mu;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = bins[i];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        s_mu = mean_from_bins(s_bins, nb);
-        if (blockIdx.x == 0) *mu_out = s_mu;
-    }
-    __syncthreads();
-    const float mu = s_mu;
+k_double_quant(const float *__restrict__ cblk, int64_t nb, uint8_t *__restrict__ q, float *__restrict__ sigma,
+               const float *__restrict__ mu_in) {
+    const float mu = __ldcg(mu_in);
     const int lane = threadIdx.x & 31;
     const int64_t ng = (nb + kGroup - 1) / kGroup;
     const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -240,7 +249,7 @@ QuantCells make_cells() {
 
 size_t quantize_workspace_bytes(int64_t n, int64_t k) {
     const int64_t nb = n * k / kBlock;
-    return kBinsBytes + ((static_cast<size_t>(nb) * sizeof(float) + 255) & ~size_t(255));
+    return kHeaderBytes + ((static_cast<size_t>(nb) * sizeof(float) + 255) & ~size_t(255));
 }
 
 cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
@@ -249,8 +258,9 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     const int64_t nb = n * k / kBlock;
     if (nb == 0) return cudaSuccess;
     auto *bins = static_cast<unsigned long long *>(ws);
-    auto *cblk = reinterpret_cast<float *>(static_cast<char *>(ws) + kBinsBytes);
-    cudaError_t e = cudaMemsetAsync(bins, 0, kBinsBytes, s);
+    auto *done = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + kBinsBytes);
+    auto *cblk = reinterpret_cast<float *>(static_cast<char *>(ws) + kHeaderBytes);
+    cudaError_t e = cudaMemsetAsync(bins, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -262,14 +272,14 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
     if (grid < min_grid) grid = min_grid;
     k_quant_blocks<<<static_cast<unsigned>(grid), kQuantThreads, 0, s>>>(
-        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, cells);
+        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, done, mu, cells);
     count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t ng = (nb + kGroup - 1) / kGroup;
     int64_t grid2 = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
     grid2 = grid2 < static_cast<int64_t>(sms) * 4 ? grid2 : static_cast<int64_t>(sms) * 4;
-    k_double_quant<<<static_cast<unsigned>(grid2), kDqThreads, 0, s>>>(cblk, nb, bins, q, sigma, mu);
+    k_double_quant<<<static_cast<unsigned>(grid2), kDqThreads, 0, s>>>(cblk, nb, q, sigma, mu);
     count_launch();
     return cudaGetLastError();
 }
