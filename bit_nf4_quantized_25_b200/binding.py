@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 QN_OK, QN_EINVAL, QN_ESHAPE, QN_EALIGN, QN_ECUDA, QN_EWORKSPACE = range(6)
 BLOCK, GROUP, MAX_RANK = 64, 256, 256
 
-EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_dequantize",
+EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
             "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x", "qn_status_string",
             "qn_last_error", "qn_launch_count")
 
@@ -57,10 +57,11 @@ def load(path: str | None = None):
         lib.qn_quantize_workspace_size.argtypes = [i64, i64, sz]
         lib.nf4_quantize.argtypes = [P, W, P, ctypes.c_size_t, P]
         lib.nf4_dequantize.argtypes = [W, P, P]
+        lib.nf4_quantize_static_ws.argtypes = [P, W, P]
         lib.qlora_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, sz]
         lib.qlora_linear_fwd.argtypes = [W, P, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, ctypes.c_size_t, P]
         lib.qlora_linear_bwd_x.argtypes = lib.qlora_linear_fwd.argtypes
-        for f in ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_dequantize",
+        for f in ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
                   "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x"):
             getattr(lib, f).restype = st
         lib.qn_status_string.argtypes = [st]
@@ -156,6 +157,16 @@ def nf4_quantize(W: torch.Tensor, out: NF4Weight | None = None, workspace: torch
     cw = out.c_struct()
     _check(load().nf4_quantize(_ptr(W), ctypes.byref(cw), _ptr(workspace), workspace.numel(), _stream(stream)),
            "nf4_quantize")
+    return out
+
+
+def nf4_quantize_static_ws(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
+    """nf4_quantize using the library's static device scratch instead of a workspace; the
+    library allocates nothing (the output buffers are the caller's). See the header for the
+    size limit and the rule that overlapping calls race."""
+    _dev_bf16(W, "W")
+    cw = out.c_struct()
+    _check(load().nf4_quantize_static_ws(_ptr(W), ctypes.byref(cw), _stream(stream)), "nf4_quantize_static_ws")
     return out
 
 

@@ -140,6 +140,28 @@ qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t
                        "nf4_quantize");
 }
 
+qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *stream) {
+    qn_status s = check_weight(out);
+    if (s != QN_OK) return s;
+    if (out->n_out == 0 || out->k_in == 0) return QN_OK;
+    const size_t need = quantize_workspace_bytes(out->n_out, out->k_in);
+    if (need > static_scratch_bytes())
+        return fail(QN_EWORKSPACE,
+                    "nf4_quantize_static_ws: a %lld x %lld weight needs %zu bytes of scratch, the static scratch holds "
+                    "%zu (at most %lld weights); use nf4_quantize with a caller workspace",
+                    (long long)out->n_out, (long long)out->k_in, need, static_scratch_bytes(),
+                    (long long)((static_scratch_bytes() - 2304) / 4 * QN_BLOCK));
+    if (!W) return fail(QN_EINVAL, "null W");
+    if (!aligned16(W)) return fail(QN_EALIGN, "W not 16-byte aligned");
+    void *ws = nullptr;
+    cudaError_t e = static_scratch_address(&ws);
+    if (e != cudaSuccess) return cuda_status(e, "nf4_quantize_static_ws: cudaGetSymbolAddress");
+    return cuda_status(launch_quantize(static_cast<const uint16_t *>(W), out->n_out, out->k_in, out->codes,
+                                       out->absmax_q, out->group_scale, out->absmax_mean, ws,
+                                       static_cast<cudaStream_t>(stream)),
+                       "nf4_quantize_static_ws");
+}
+
 qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream) {
     qn_status s = check_weight(w);
     if (s != QN_OK) return s;

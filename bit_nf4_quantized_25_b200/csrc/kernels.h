@@ -30,6 +30,10 @@ void count_launch(int n = 1);
 cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
                             float *mu, void *ws, cudaStream_t s);
 size_t quantize_workspace_bytes(int64_t n, int64_t k);
+// Static scratch of the allocation-free quantiser entry point: size, and its device address on
+// the current device (resolved once per device).
+size_t static_scratch_bytes();
+cudaError_t static_scratch_address(void **out);
 
 // nf4_dequantize.
 cudaError_t launch_dequant(const WeightView &w, uint16_t *out, cudaStream_t s);

@@ -12,6 +12,8 @@
 // independent of scheduling).
 // The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -245,7 +247,35 @@ QuantCells make_cells() {
     return c;
 }
 
+// Scratch for callers that cannot allocate device memory (nf4_quantize_static_ws): a
+// file-scope device array that every GPU loading this library holds until exit.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
+
 }  // namespace
+
+size_t static_scratch_bytes() { return kStaticScratchBytes; }
+
+// Device address of g_quant_scratch on the current device. The symbol's host-side name is not
+// a device address, so it is resolved with cudaGetSymbolAddress, once per device (with that
+// device current), and cached.
+cudaError_t static_scratch_address(void **out) {
+    static std::mutex lock;
+    static void *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> guard(lock);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_quant_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
 
 size_t quantize_workspace_bytes(int64_t n, int64_t k) {
     const int64_t nb = n * k / kBlock;

@@ -115,6 +115,24 @@ qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_byt
  * QN_EWORKSPACE, QN_ECUDA. */
 qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t ws_bytes, void *stream);
 
+/* nf4_quantize_static_ws -- nf4_quantize without a caller workspace and without allocating.
+ * No counterpart in the paper: this entry point exists for callers that cannot allocate
+ * device memory when they quantise -- code running inside a global-mode stream capture (where
+ * cudaMalloc is not permitted), runtimes whose device memory is entirely owned by another
+ * allocator, and latency-critical paths that cannot afford cudaMalloc's implicit device
+ * synchronisation. The scratch is a file-scope 16 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits; it fits weights of at most
+ * 4,193,728 blocks of 64 (268,398,592 weights; 28672 x 8192 fits). Larger weights are
+ * rejected with QN_EWORKSPACE before anything is enqueued.
+ * Results are bit-identical to nf4_quantize. The first call on each device looks up the
+ * scratch address (cudaGetSymbolAddress) with that device current, so make it before any
+ * stream capture. Every call shares the one scratch array (the part that must start at zero is
+ * cleared by each call): calls whose work overlaps on the GPU -- on different streams, or from
+ * different host threads -- race and must be serialised by the caller.
+ * No memory is allocated or freed (no cudaMalloc, cudaFree or allocating library call).
+ * Errors: as nf4_quantize, with QN_EWORKSPACE for weights above the limit. */
+qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *stream);
+
 /* nf4_dequantize -- quantised weight -> W_out (n_out x k_in bf16, device):
  * W_out[e] = bf16_rn(fl32(NF4[code_e] * c'_b)).
  * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), the
