@@ -371,9 +371,14 @@ def run_ours(args):
     traffic = None
     prof = os.path.join(ROOT, "profiles", "decode_fwd_traffic.json")
     if os.path.exists(prof):
+        # the ncu counters count only while the kernel source they were taken on is unchanged
         try:
+            import hashlib
             with open(prof) as f:
-                traffic = json.load(f).get("bytes_per_launch")
+                rec = json.load(f)
+            with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+                same = hashlib.sha256(f.read()).hexdigest()[:16] == rec["source_sha256_16"]
+            traffic = rec["bytes_per_launch"] if same else None
         except Exception:
             traffic = None
 
