@@ -60,9 +60,13 @@ __device__ __forceinline__ uint16_t ld_ro_u16(const void *p) { return __ldg(rein
 
 // ------------------------------------------------------------ numerics
 
+// E4M3 (finite variant) -> fp32, exact. Exponent and mantissa bits are moved into the fp32
+// fields, which reads the value scaled by 2^(7 - 127) (e4m3 bias 7, fp32 bias 127; a zero
+// exponent gives an fp32 subnormal, matching the e4m3 subnormal); one exact multiply by 2^120
+// restores the scale. The two NaN codes (0x7f, 0xff) are never produced by the quantiser.
 __device__ __forceinline__ float e4m3_to_f32(uint8_t v) {
-    __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(v), __NV_E4M3);
-    return __half2float(__half(h));
+    const uint32_t u = v;
+    return __uint_as_float(((u & 0x7fu) << 20) | ((u & 0x80u) << 24)) * 0x1p120f;
 }
 
 __device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float v) {

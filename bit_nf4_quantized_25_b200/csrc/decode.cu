@@ -66,20 +66,48 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // Pair table: row e (a code byte) holds bf16x2(NF4[e & 15], NF4[e >> 4]) in its first 32
-// words, one copy per lane.
+// words, one copy per lane. One row per thread; the eight 16-byte stores of a row start at a
+// column rotated by the row so that the lanes of a warp hit different banks.
 __device__ __forceinline__ void build_pair_lut(uint8_t *lut) {
     uint4 *l4 = reinterpret_cast<uint4 *>(lut);
-    for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
-        const int e = i >> 3, c = i & 7;
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
         const uint32_t v = pack_bf16x2(nf4_value(e & 15), nf4_value(e >> 4));
-        l4[e * 16 + c] = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) l4[e * 16 + ((c + e) & 7)] = make_uint4(v, v, v, v);
     }
 }
 
-// Pair for byte i (0..3) of word w: the permute builds (byte << 8) | (lane << 2).
-__device__ __forceinline__ uint32_t lut_pair(const uint8_t *lut, uint32_t w, uint32_t lane4, int i) {
-    const uint32_t off = prmt(w, lane4, 0x5504u | (static_cast<uint32_t>(i) << 4));
-    return *reinterpret_cast<const uint32_t *>(lut + off);
+// Low 24 bits of the shared-window address of dynamic shared memory when the driver reserves
+// 1 KB per block and the kernel has no static shared memory; in a cluster launch the CTA's
+// rank sits above them. The kernels check it at run time and otherwise take the generic path.
+constexpr uint32_t kDynSmemBase = 1024;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Operand of the table permute: lane << 2 in byte 0 and, on the fixed-base path, the high
+// byte (cluster rank) of the table's shared-window address in byte 3.
+template <bool kFixedBase>
+__device__ __forceinline__ uint32_t lut_lane_operand(const uint8_t *lut, int lane) {
+    const uint32_t l4 = static_cast<uint32_t>(lane) << 2;
+    return kFixedBase ? (l4 | (smem_addr(lut) & 0xff000000u)) : l4;
+}
+
+// Pair for byte i (0..3) of word w. The permute builds (byte << 8) | (lane << 2), plus the rank
+// byte on the fixed-base path, where the table starts at the base of dynamic shared memory and
+// its low address bits are an immediate of the load; otherwise the table address is added.
+template <bool kFixedBase>
+__device__ __forceinline__ uint32_t lut_pair(const uint8_t *lut, uint32_t w, uint32_t lane_op, int i) {
+    if constexpr (kFixedBase) {
+        const uint32_t a = prmt(w, lane_op, 0x7604u | (static_cast<uint32_t>(i) << 4));
+        uint32_t v;
+        asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(kDynSmemBase));
+        return v;
+    } else {
+        const uint32_t off = prmt(w, lane_op, 0x5504u | (static_cast<uint32_t>(i) << 4));
+        return *reinterpret_cast<const uint32_t *>(lut + off);
+    }
 }
 
 __device__ __forceinline__ float round_bf16(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
@@ -110,22 +138,61 @@ __device__ __forceinline__ void cluster_arrive_release() {
 }
 __device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-// L2 prefetch (before the dependency wait) of the activation slice, the adapter slice and the
-// adapter rows the finalising CTA will read: with every operand already on its way to L2 the
-// kernel pays one DRAM round trip instead of a chain of them.
-__device__ __forceinline__ void prefetch_operands(const DecodeParams &p, int b_lo, int b_hi, int64_t row0, int rows,
-                                                  int crank, int C) {
+// L2 prefetch (before the dependency wait) of the activation slice and the adapter slice of
+// this CTA's k-range, so that their first reads after the wait are L2 hits.
+__device__ __forceinline__ void prefetch_operands(const DecodeParams &p, int b_lo, int b_hi) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t K = p.k;
     const int64_t kbytes = static_cast<int64_t>(b_hi - b_lo) * 128;  // 64 bf16 per block
-    if (warp == 0 && lane < p.M && kbytes > 0)
+    if (kbytes <= 0) return;
+    if (warp == 0 && lane < p.M)
         prefetch_l2(p.act + lane * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
-    if (warp == 1 && p.r > 0) {
-        for (int j = lane; j < p.r; j += 32)
-            if (kbytes > 0) prefetch_l2(p.A + j * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
-        const int r_lo = rows * crank / C, r_hi = rows * (crank + 1) / C;
-        const int64_t n_lo = row0 + r_lo, n_hi = row0 + r_hi < p.n ? row0 + r_hi : p.n;
-        if (lane == 0 && n_hi > n_lo) prefetch_range(p.B + n_lo * p.r, (n_hi - n_lo) * p.r * 2);
+    if (warp == 1)
+        for (int j = lane; j < p.r; j += 32) prefetch_l2(p.A + j * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// bf16 pair (B[row][j], B[row][j + 1]) of the row-major n x r adapter B, zero outside it.
+__device__ __forceinline__ uint32_t load_b_pair(const DecodeParams &p, int64_t row, bool valid, int j) {
+    if (!valid || j >= p.r) return 0u;
+    const uint16_t *b = p.B + row * p.r + j;
+    if ((p.r & 1) == 0) return ld_ro_u32(b);  // j even: 4-byte aligned
+    const uint32_t lo = ld_ro_u16(b);
+    const uint32_t hi = j + 1 < p.r ? ld_ro_u16(b + 1) : 0u;
+    return lo | (hi << 16);
+}
+
+// MMA A-fragment of B rows (rowA, rowB) and adapter columns [j, j + 2) and [j + 8, j + 10).
+__device__ __forceinline__ void load_b_frag(const DecodeParams &p, int64_t rowA, int64_t rowB, bool vA, bool vB, int j,
+                                            uint32_t &a0, uint32_t &a1, uint32_t &a2, uint32_t &a3) {
+    a0 = load_b_pair(p, rowA, vA, j);
+    a1 = load_b_pair(p, rowB, vB, j);
+    a2 = load_b_pair(p, rowA, vA, j + 8);
+    a3 = load_b_pair(p, rowB, vB, j + 8);
+}
+
+// Copy columns [k0, k0 + nc) of the first `rows` rows of a row-major bf16 matrix with row
+// stride `ld` to dst[row][c] (row stride nc), eight loads in flight per thread.
+__device__ __forceinline__ void stage_cols(uint16_t *dst, const uint16_t *src, int64_t ld, int64_t k0, int rows,
+                                           int nc) {
+    constexpr int U = 8;
+    const int n = rows * nc;
+    for (int base = threadIdx.x; base < n; base += U * blockDim.x) {
+        uint16_t v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < n) v[u] = ld_ro_u16(src + static_cast<int64_t>(i / nc) * ld + k0 + i % nc);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x;
+            if (i < n) dst[i] = v[u];
+        }
     }
 }
 
@@ -137,124 +204,121 @@ struct FwdGroup {
     float sa, sb;
 };
 
-template <int NG>
-__global__ void __launch_bounds__(kDecThreads)
-k_decode_fwd(const DecodeParams p) {
+template <int NG, bool kFixedBase>
+__device__ __forceinline__ void decode_fwd_body(const DecodeParams &p, uint8_t *smem) {
     constexpr int MP = 8 * NG;  // padded token count
-    extern __shared__ __align__(16) uint8_t smem[];
     uint8_t *lut = smem;
-    float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [kFwdRows][MP]
+    // recv[src][row - r_lo][MP]: the partial sums that cluster rank `src` pushes for the rows
+    // this CTA finalises (at most kFwdRows + kMaxCluster rows in all).
+    float *recv = reinterpret_cast<float *>(smem + kLutBytes);
     const int rpad = (p.r + 15) & ~15;
-    float *tpart = part + kFwdRows * MP;  // [rpad][MP] partial A x of this CTA's k-slice
-    float *tfull = tpart + rpad * MP;     // [rpad][MP] s * A x, rounded to bf16
+    float *tpart = recv + (kFwdRows + kMaxCluster) * MP;  // [rpad][MP] partial A x of this CTA's k-slice
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = static_cast<int>(cluster.num_blocks());
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+    const uint32_t lane4 = lut_lane_operand<kFixedBase>(lut, lane);
 
     const int64_t N = p.n, K = p.k;
     const int nbr = static_cast<int>(K / kBlock);
-    const int b_lo = static_cast<int>(static_cast<int64_t>(nbr) * crank / C);
-    const int b_hi = static_cast<int>(static_cast<int64_t>(nbr) * (crank + 1) / C);
+    // nbr < 2^25 (k_in < 2^31), so the products fit 32 bits
+    const int b_lo = static_cast<int>(static_cast<uint32_t>(nbr * crank) / static_cast<uint32_t>(C));
+    const int b_hi = static_cast<int>(static_cast<uint32_t>(nbr * (crank + 1)) / static_cast<uint32_t>(C));
     const int64_t row_base = static_cast<int64_t>(blockIdx.y) * kFwdRows + warp * 16;
 
-    // Before the dependency wait: on-chip setup and an L2 prefetch of the weight codes.
-    build_pair_lut(lut);
-    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) tpart[i] = 0.0f;
-    if (lane < 16 && row_base + lane < N && b_hi > b_lo) {
-        const int64_t row = row_base + lane;
-        prefetch_l2(p.codes + row * (K / 2) + static_cast<int64_t>(b_lo) * 32, static_cast<uint32_t>(b_hi - b_lo) * 32u);
-        prefetch_range(p.q + row * nbr + b_lo, b_hi - b_lo);
-        prefetch_line(p.sigma + (row * nbr + b_lo) / kGroup);
-    }
-    prefetch_operands(p, b_lo, b_hi, static_cast<int64_t>(blockIdx.y) * kFwdRows, kFwdRows, crank, C);
-    __syncthreads();
+    // Before the dependency wait only an L2 prefetch of the operand slices. The weight codes are
+    // not prefetched (per-row prefetches cost more to issue than they saved): the first two
+    // groups of codes are requested right after the wait, and the pair table is built while
+    // they are in flight.
+    prefetch_operands(p, b_lo, b_hi);
+    cluster_arrive_relaxed();  // phase 1: this CTA is running (its shared memory may be written)
     grid_dependency_wait();
 
     const float mu = __ldg(p.mu);
     const int M = p.M;
     const int64_t rowA = row_base + g, rowB = rowA + 8;
     const bool vA = rowA < N, vB = rowB < N;
-    const uint8_t *cA = p.codes + (vA ? rowA : 0) * (K / 2) + 8 * t;
-    const uint8_t *cB = p.codes + (vB ? rowB : 0) * (K / 2) + 8 * t;
-    const int64_t qA = (vA ? rowA : 0) * nbr, qB = (vB ? rowB : 0) * nbr;
+    uint32_t bf[4] = {0u, 0u, 0u, 0u};  // B fragment of the first 16 adapter columns, loaded early
+    if (p.r > 0) load_b_frag(p, rowA, rowB, vA, vB, 2 * t, bf[0], bf[1], bf[2], bf[3]);
+    // Rows past N read row 0 (valid memory) and get a zero block constant; tokens past M read
+    // token 0 and fill MMA columns that are never stored. The hot loop therefore only needs
+    // the block count of the last (partial) group.
+    const int nblk = b_hi - b_lo, ngrp = (nblk + 3) / 4;
+    const uint2 *pa = reinterpret_cast<const uint2 *>(p.codes + (vA ? rowA : 0) * (K / 2) +
+                                                      static_cast<int64_t>(b_lo) * 32 + 8 * t);
+    const uint2 *pb = reinterpret_cast<const uint2 *>(p.codes + (vB ? rowB : 0) * (K / 2) +
+                                                      static_cast<int64_t>(b_lo) * 32 + 8 * t);
+    // flattened index of lane t's block in group 0 (the lane loads that block's constants)
+    const int64_t eA = (vA ? rowA : 0) * nbr + b_lo + t, eB = (vB ? rowB : 0) * nbr + b_lo + t;
 
-    auto load_group = [&](int b0, FwdGroup &G) {
+    auto load_group = [&](int gi, FwdGroup &G) {
+        const int cnt = nblk - 4 * gi;  // blocks in this group (at least 1)
+        const uint2 *ga = pa + 16 * gi, *gb = pb + 16 * gi;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int b = b0 + j;
-            G.ca[j] = (vA && b < b_hi) ? __ldcs(reinterpret_cast<const uint2 *>(cA + static_cast<int64_t>(b) * 32))
-                                       : make_uint2(0u, 0u);
-            G.cb[j] = (vB && b < b_hi) ? __ldcs(reinterpret_cast<const uint2 *>(cB + static_cast<int64_t>(b) * 32))
-                                       : make_uint2(0u, 0u);
+            G.ca[j] = j < cnt ? __ldcs(ga + 4 * j) : make_uint2(0u, 0u);
+            G.cb[j] = j < cnt ? __ldcs(gb + 4 * j) : make_uint2(0u, 0u);
         }
-        const int bt = b0 + t;
-        const bool ok = bt < b_hi;
-        G.qa = (vA && ok) ? __ldg(p.q + qA + bt) : 0u;
-        G.qb = (vB && ok) ? __ldg(p.q + qB + bt) : 0u;
-        G.sa = (vA && ok) ? __ldg(p.sigma + (qA + bt) / kGroup) : 0.0f;
-        G.sb = (vB && ok) ? __ldg(p.sigma + (qB + bt) / kGroup) : 0.0f;
+        const bool ok = t < cnt;
+        const uint64_t ea = static_cast<uint64_t>(eA + 4 * gi), eb = static_cast<uint64_t>(eB + 4 * gi);
+        G.qa = ok ? __ldg(p.q + ea) : 0u;
+        G.qb = ok ? __ldg(p.q + eb) : 0u;
+        G.sa = ok ? __ldg(p.sigma + ea / kGroup) : 0.0f;
+        G.sb = ok ? __ldg(p.sigma + eb / kGroup) : 0.0f;
     };
 
-    // x rows of this lane's tokens: x[tg*8 + g][64b + 16t .. +16]
-    const uint16_t *xrow[NG];
-    bool xv[NG];
+    // x of this lane's tokens: x[tg*8 + g][64 b + 16 t .. + 16] is xq[tg][8 (b - b_lo)], [.. + 1]
+    const uint4 *xq[NG];
 #pragma unroll
     for (int tg = 0; tg < NG; ++tg) {
         const int tok = tg * 8 + g;
-        xv[tg] = tok < M;
-        xrow[tg] = p.act + static_cast<int64_t>(xv[tg] ? tok : 0) * K + 16 * t;
+        xq[tg] = reinterpret_cast<const uint4 *>(p.act + static_cast<int64_t>(tok < M ? tok : 0) * K +
+                                                 static_cast<int64_t>(b_lo) * 64 + 16 * t);
     }
 
     float acc[NG][4];
 #pragma unroll
     for (int tg = 0; tg < NG; ++tg) acc[tg][0] = acc[tg][1] = acc[tg][2] = acc[tg][3] = 0.0f;
 
-    FwdGroup cur, nxt;
-    if (b_lo < b_hi) load_group(b_lo, cur);
+    FwdGroup G0, G1;  // ping-pong: two groups of codes in flight while one is consumed
+    if (ngrp > 0) load_group(0, G0);
+    if (ngrp > 1) load_group(1, G1);
 
-    // ---- LoRA down-projection over this CTA's k-slice (partial t = A x, fp32), while the
-    // first codes are in flight. Item (j-tile, eighth of the slice) per warp.
-    if (p.r > 0) {
+    // ---- LoRA down-projection over this CTA's k-slice (partial t = A x, fp32), run after the
+    // first group of codes has been consumed (its operands are L2 hits that would otherwise
+    // queue behind the code loads). Item (j-tile, eighth of the slice) per warp.
+    auto lora_down = [&]() {
         const int rt = rpad / 16;
-        const int nsl = b_hi - b_lo;
-        const int s_lo = b_lo + nsl * warp / kDecWarps, s_hi = b_lo + nsl * (warp + 1) / kDecWarps;
+        const int s_lo = nblk * warp / kDecWarps, s_hi = nblk * (warp + 1) / kDecWarps;  // relative to b_lo
         for (int jt = 0; jt < rt; ++jt) {
             const int jA = jt * 16 + g, jB = jA + 8;
             const bool aA = jA < p.r, aB = jB < p.r;
-            const uint16_t *pa = p.A + static_cast<int64_t>(aA ? jA : 0) * K + 16 * t;
-            const uint16_t *pb = p.A + static_cast<int64_t>(aB ? jB : 0) * K + 16 * t;
+            const uint4 *ra = reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(aA ? jA : 0) * K +
+                                                             static_cast<int64_t>(b_lo) * 64 + 16 * t);
+            const uint4 *rb = reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(aB ? jB : 0) * K +
+                                                             static_cast<int64_t>(b_lo) * 64 + 16 * t);
             float d[NG][4];
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) d[tg][0] = d[tg][1] = d[tg][2] = d[tg][3] = 0.0f;
             for (int b = s_lo; b < s_hi; ++b) {
-                const int64_t o = static_cast<int64_t>(b) * 64;
                 uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0, b0 = a0, b1 = a0;
                 if (aA) {
-                    a0 = ld_ro_v4(pa + o);
-                    a1 = ld_ro_v4(pa + o + 8);
+                    a0 = __ldg(ra + 8 * b);
+                    a1 = __ldg(ra + 8 * b + 1);
                 }
                 if (aB) {
-                    b0 = ld_ro_v4(pb + o);
-                    b1 = ld_ro_v4(pb + o + 8);
+                    b0 = __ldg(rb + 8 * b);
+                    b1 = __ldg(rb + 8 * b + 1);
                 }
-                const uint32_t ra[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                 for (int tg = 0; tg < NG; ++tg) {
-                    uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                    if (xv[tg]) {
-                        x0 = ld_ro_v4(xrow[tg] + o);
-                        x1 = ld_ro_v4(xrow[tg] + o + 8);
-                    }
-                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_16816(d[tg], ra[2 * kk], rb[2 * kk], ra[2 * kk + 1], rb[2 * kk + 1], xw[2 * kk],
-                                  xw[2 * kk + 1]);
+                    const uint4 x0 = __ldg(xq[tg] + 8 * b), x1 = __ldg(xq[tg] + 8 * b + 1);
+                    mma_16816(d[tg], a0.x, b0.x, a0.y, b0.y, x0.x, x0.y);
+                    mma_16816(d[tg], a0.z, b0.z, a0.w, b0.w, x0.z, x0.w);
+                    mma_16816(d[tg], a1.x, b1.x, a1.y, b1.y, x1.x, x1.y);
+                    mma_16816(d[tg], a1.z, b1.z, a1.w, b1.w, x1.z, x1.w);
                 }
             }
 #pragma unroll
@@ -266,92 +330,113 @@ k_decode_fwd(const DecodeParams p) {
                 atomicAdd(&tpart[(jl + 8) * MP + tg * 8 + 2 * t + 1], d[tg][3]);
             }
         }
-    }
+    };
 
-    // ---- base: blocks [b_lo, b_hi) of rows A and B, groups of four, double-buffered.
-    for (int b0 = b_lo; b0 < b_hi; b0 += 4) {
-        if (b0 + 4 < b_hi) load_group(b0 + 4, nxt);
-        const float cA4 = vA ? block_constant(static_cast<uint8_t>(cur.qa), cur.sa, mu) : 0.0f;
-        const float cB4 = vB ? block_constant(static_cast<uint8_t>(cur.qb), cur.sb, mu) : 0.0f;
+    // The pair table is built while the first codes are in flight.
+    build_pair_lut(lut);
+    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) tpart[i] = 0.0f;
+    __syncthreads();
+
+    // ---- base: group gi holds blocks b_lo + 4 gi .. + 4 of rows A and B.
+    auto compute_group = [&](const FwdGroup &G, int gi) {
+        const int cnt = nblk - 4 * gi;
+        const bool ok = t < cnt;
+        const float cA4 = (vA && ok) ? block_constant(static_cast<uint8_t>(G.qa), G.sa, mu) : 0.0f;
+        const float cB4 = (vB && ok) ? block_constant(static_cast<uint8_t>(G.qb), G.sb, mu) : 0.0f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int b = b0 + j;
-            if (b >= b_hi) break;
+            if (j >= cnt) break;
             const float cpA = __shfl_sync(0xffffffffu, cA4, (lane & ~3) | j);
             const float cpB = __shfl_sync(0xffffffffu, cB4, (lane & ~3) | j);
             uint32_t af[4][4];
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t wa = kk < 2 ? cur.ca[j].x : cur.ca[j].y, wb = kk < 2 ? cur.cb[j].x : cur.cb[j].y;
+                const uint32_t wa = kk < 2 ? G.ca[j].x : G.ca[j].y, wb = kk < 2 ? G.cb[j].x : G.cb[j].y;
                 const int i0 = (2 * kk) & 3;
-                af[kk][0] = lut_pair(lut, wa, lane4, i0);
-                af[kk][2] = lut_pair(lut, wa, lane4, i0 + 1);
-                af[kk][1] = lut_pair(lut, wb, lane4, i0);
-                af[kk][3] = lut_pair(lut, wb, lane4, i0 + 1);
+                af[kk][0] = lut_pair<kFixedBase>(lut, wa, lane4, i0);
+                af[kk][2] = lut_pair<kFixedBase>(lut, wa, lane4, i0 + 1);
+                af[kk][1] = lut_pair<kFixedBase>(lut, wb, lane4, i0);
+                af[kk][3] = lut_pair<kFixedBase>(lut, wb, lane4, i0 + 1);
             }
-            const int64_t o = static_cast<int64_t>(b) * 64;
+            const int xo = 8 * (4 * gi + j);
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) {
-                uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                if (xv[tg]) {
-                    x0 = ld_ro_v4(xrow[tg] + o);
-                    x1 = ld_ro_v4(xrow[tg] + o + 8);
-                }
-                const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                const uint4 x0 = __ldg(xq[tg] + xo), x1 = __ldg(xq[tg] + xo + 1);
                 float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_16816(d, af[kk][0], af[kk][1], af[kk][2], af[kk][3], xw[2 * kk], xw[2 * kk + 1]);
+                mma_16816(d, af[0][0], af[0][1], af[0][2], af[0][3], x0.x, x0.y);
+                mma_16816(d, af[1][0], af[1][1], af[1][2], af[1][3], x0.z, x0.w);
+                mma_16816(d, af[2][0], af[2][1], af[2][2], af[2][3], x1.x, x1.y);
+                mma_16816(d, af[3][0], af[3][1], af[3][2], af[3][3], x1.z, x1.w);
                 acc[tg][0] = __fmaf_rn(cpA, d[0], acc[tg][0]);
                 acc[tg][1] = __fmaf_rn(cpA, d[1], acc[tg][1]);
                 acc[tg][2] = __fmaf_rn(cpB, d[2], acc[tg][2]);
                 acc[tg][3] = __fmaf_rn(cpB, d[3], acc[tg][3]);
             }
         }
-        cur = nxt;
+    };
+    for (int gi = 0; gi < ngrp; gi += 2) {
+        compute_group(G0, gi);
+        if (gi == 0 && p.r > 0) lora_down();
+        if (gi + 2 < ngrp) load_group(gi + 2, G0);
+        if (gi + 1 < ngrp) {
+            compute_group(G1, gi + 1);
+            if (gi + 3 < ngrp) load_group(gi + 3, G1);
+        }
     }
-    {
-        const int rl = warp * 16 + g;
+    if (ngrp == 0 && p.r > 0) lora_down();
+    __syncthreads();  // tpart holds A x over this CTA's k-slice
+
+    // ---- adapter up-projection of this CTA's k-slice, folded into the partial sums:
+    // acc += B[rows, :] (s * t_c), with t_c = A x over the slice rounded to bf16 as the MMA operand.
+    for (int jt = 0; jt < rpad / 16; ++jt) {
+        uint32_t a0 = bf[0], a1 = bf[1], a2 = bf[2], a3 = bf[3];
+        if (jt > 0) load_b_frag(p, rowA, rowB, vA, vB, jt * 16 + 2 * t, a0, a1, a2, a3);
+        const int j0 = jt * 16 + 2 * t;
 #pragma unroll
         for (int tg = 0; tg < NG; ++tg) {
-            part[rl * MP + tg * 8 + 2 * t] = acc[tg][0];
-            part[rl * MP + tg * 8 + 2 * t + 1] = acc[tg][1];
-            part[(rl + 8) * MP + tg * 8 + 2 * t] = acc[tg][2];
-            part[(rl + 8) * MP + tg * 8 + 2 * t + 1] = acc[tg][3];
+            const int tok = tg * 8 + g;
+            const uint32_t b0 = pack_bf16x2(p.s * tpart[j0 * MP + tok], p.s * tpart[(j0 + 1) * MP + tok]);
+            const uint32_t b1 = pack_bf16x2(p.s * tpart[(j0 + 8) * MP + tok], p.s * tpart[(j0 + 9) * MP + tok]);
+            mma_16816(acc[tg], a0, a1, a2, a3, b0, b1);
         }
     }
 
-    __syncthreads();
-    cluster.sync();  // every CTA's partials are complete and visible in the cluster
+    // ---- push the partials of rows g and g + 8 of this warp to the CTAs that finalise them.
+    const int nrmax = (kFwdRows + C - 1) / C;
+    cluster_wait();  // phase 1: every CTA of the cluster is running
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rl = warp * 16 + g + 8 * h;
+        const int owner = (rl * C + C - 1) / kFwdRows;  // largest c with kFwdRows*c/C <= rl
+        const int rr = rl - kFwdRows * owner / C;
+        float *dst = cluster.map_shared_rank(recv, owner) + (crank * nrmax + rr) * MP + 2 * t;
+#pragma unroll
+        for (int tg = 0; tg < NG; ++tg)
+            *reinterpret_cast<float2 *>(dst + tg * 8) = make_float2(acc[tg][2 * h], acc[tg][2 * h + 1]);
+    }
+    cluster_arrive_release();
+    cluster_wait_acquire();  // phase 2: every partial has landed
     grid_dependents_launch();
 
-    if (p.r > 0) {
-        for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) {
-            float sum = 0.0f;
-            for (int cc = 0; cc < C; ++cc) sum += cluster.map_shared_rank(tpart, cc)[i];
-            tfull[i] = round_bf16(sum * p.s);
-        }
-    }
-    __syncthreads();
-
-    // ---- this CTA finalises rows [kFwdRows*crank/C, kFwdRows*(crank+1)/C) of the row group
+    // ---- this CTA finalises rows [kFwdRows*crank/C, kFwdRows*(crank+1)/C) of the row group.
     const int r_lo = kFwdRows * crank / C, r_hi = kFwdRows * (crank + 1) / C, nr = r_hi - r_lo;
-    for (int i = threadIdx.x; i < nr * M; i += blockDim.x) {
-        const int rl = r_lo + i % nr, tok = i / nr;
-        const int64_t n = static_cast<int64_t>(blockIdx.y) * kFwdRows + rl;
-        if (n >= N) continue;
+    const int64_t n_lo = static_cast<int64_t>(blockIdx.y) * kFwdRows + r_lo;
+    const int nv = static_cast<int>(N - n_lo < nr ? (N - n_lo > 0 ? N - n_lo : 0) : nr);  // rows inside W
+    for (int i = threadIdx.x; i < nv * M; i += blockDim.x) {
+        const int rr = i % nv, tok = i / nv;
         float sum = 0.0f;
-        for (int cc = 0; cc < C; ++cc) sum += cluster.map_shared_rank(part, cc)[rl * MP + tok];
-        if (p.r > 0) {
-            const uint16_t *brow = p.B + n * p.r;
-            float lora = 0.0f;
-            for (int j = 0; j < p.r; ++j)
-                lora = __fmaf_rn(__uint_as_float(static_cast<uint32_t>(ld_ro_u16(brow + j)) << 16), tfull[j * MP + tok], lora);
-            sum += lora;
-        }
-        p.out[static_cast<int64_t>(tok) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+        for (int src = 0; src < C; ++src) sum += recv[(src * nrmax + rr) * MP + tok];
+        p.out[static_cast<int64_t>(tok) * N + n_lo + rr] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
     }
-    cluster.sync();  // keep this CTA's shared memory alive until the cluster is done reading it
+}
+
+template <int NG>
+__global__ void __launch_bounds__(kDecThreads, NG <= 2 ? 2 : 1) k_decode_fwd(const DecodeParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    if ((smem_addr(smem) & 0x00ffffffu) == kDynSmemBase)
+        decode_fwd_body<NG, true>(p, smem);
+    else
+        decode_fwd_body<NG, false>(p, smem);
 }
 
 // ------------------------------------------------------------------- input gradient
@@ -386,11 +471,9 @@ struct BwdGroup {
     float s[2];
 };
 
-template <int NG>
-__global__ void __launch_bounds__(kDecThreads)
-k_decode_bwd(const DecodeParams p) {
+template <int NG, bool kFixedBase>
+__device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *smem) {
     constexpr int MP = 8 * NG;
-    extern __shared__ __align__(16) uint8_t smem[];
     uint8_t *lut = smem;
     float *part = reinterpret_cast<float *>(smem + kLutBytes);  // [warps][64 features][MP]
     const int rpad = (p.r + 15) & ~15;
@@ -402,7 +485,7 @@ k_decode_bwd(const DecodeParams p) {
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, t = lane & 3;
-    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+    const uint32_t lane4 = lut_lane_operand<kFixedBase>(lut, lane);
 
     const int64_t N = p.n, K = p.k;
     const int64_t nbr = K / kBlock;
@@ -415,10 +498,9 @@ k_decode_bwd(const DecodeParams p) {
     const int64_t c_lo = n16 * crank / C, c_hi = n16 * (crank + 1) / C;
     const int64_t s_lo = c_lo + (c_hi - c_lo) * sub / kBwdSub, s_hi = c_lo + (c_hi - c_lo) * (sub + 1) / kBwdSub;
 
-    build_pair_lut(lut);
-    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) upart[i] = 0.0f;
-    // L2 prefetch of everything this CTA reads: the warp's codes (rows [16 s_lo, 16 s_hi) x
-    // 32 bytes of column kb) and their constants, the grad_h slice, the adapter rows.
+    // L2 prefetch of everything this CTA reads (first, so that DRAM streams while the CTA sets
+    // up): the warp's codes (rows [16 s_lo, 16 s_hi) x 32 bytes of column kb) and their
+    // constants, the grad_h slice, the adapter rows.
     if (vk) {
         for (int64_t rr = s_lo * 16 + lane; rr < s_hi * 16 && rr < N; rr += 32) {
             prefetch_l2(p.codes + rr * (K / 2) + kbc * 32, 32u);
@@ -437,6 +519,8 @@ k_decode_bwd(const DecodeParams p) {
         const int64_t k1 = k0 + 64 * kBwdCols < K ? k0 + 64 * kBwdCols : K;
         for (int j = lane; j < p.r; j += 32) prefetch_range(p.A + j * K + k0, (k1 - k0) * 2);
     }
+    build_pair_lut(lut);
+    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) upart[i] = 0.0f;
     __syncthreads();
     grid_dependency_wait();
 
@@ -537,10 +621,10 @@ k_decode_bwd(const DecodeParams p) {
                 uint32_t af[4][4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    af[i][0] = lut_pair(lut, e01, lane4, i);
-                    af[i][1] = lut_pair(lut, o01, lane4, i);
-                    af[i][2] = lut_pair(lut, e23, lane4, i);
-                    af[i][3] = lut_pair(lut, o23, lane4, i);
+                    af[i][0] = lut_pair<kFixedBase>(lut, e01, lane4, i);
+                    af[i][1] = lut_pair<kFixedBase>(lut, o01, lane4, i);
+                    af[i][2] = lut_pair<kFixedBase>(lut, e23, lane4, i);
+                    af[i][3] = lut_pair<kFixedBase>(lut, o23, lane4, i);
                 }
 #pragma unroll
                 for (int tg = 0; tg < NG; ++tg) {
@@ -572,70 +656,109 @@ k_decode_bwd(const DecodeParams p) {
             }
     }
 
-    __syncthreads();
-    cluster.sync();
-    grid_dependents_launch();
-
-    if (p.r > 0) {
-        for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) {
-            float sum = 0.0f;
-            for (int cc = 0; cc < C; ++cc) sum += cluster.map_shared_rank(upart, cc)[i];
-            ufull[i] = round_bf16(sum * p.s);
-        }
-    }
-    __syncthreads();
+    __syncthreads();           // partials written; every warp is done with the pair table
+    cluster_arrive_release();  // this CTA's partials (base and adapter) are ready for the cluster
 
     // ---- this CTA finalises features [F*crank/C, F*(crank+1)/C) of the CTA group's F features
     constexpr int F = 64 * kBwdCols;
     const int f_lo = F * crank / C, f_hi = F * (crank + 1) / C, nf = f_hi - f_lo;
-    for (int i = threadIdx.x; i < nf * M; i += blockDim.x) {
-        const int fl = f_lo + i % nf, tok = i / nf;
-        const int64_t k = static_cast<int64_t>(blockIdx.y) * F + fl;
-        if (k >= K) continue;
-        const int c = fl / 64, f = fl % 64;
-        float sum = 0.0f;
-        for (int cc = 0; cc < C; ++cc) {
-            const float *rp = cluster.map_shared_rank(part, cc);
+    const int64_t k_lo = static_cast<int64_t>(blockIdx.y) * F + f_lo;
+    const int nvf = static_cast<int>(K - k_lo < nf ? (K - k_lo > 0 ? K - k_lo : 0) : nf);  // features inside W
+    // While the cluster barrier completes: stage the adapter columns A[:, k_lo, k_lo + nvf) as
+    // as[j][f] in the (now unused) pair-table region, at most 256 x 128 bf16 = 64 KB.
+    uint16_t *as = reinterpret_cast<uint16_t *>(lut);
+    if (p.r > 0 && nvf > 0) stage_cols(as, p.A, K, k_lo, p.r, nvf);
+    cluster_wait_acquire();  // every CTA's partials are visible in the cluster
+    grid_dependents_launch();
+
+    // Remote reads: adapter sums (ufull[j][tok] = bf16(s * B^T grad_h)) and, with more than one
+    // CTA per cluster, the base sums of the owned features into red[f - f_lo][tok] (at most
+    // 64 x 64 floats) behind the staged A columns.
+    if (p.r > 0) {
+        for (int i = threadIdx.x; i < p.r * M; i += blockDim.x) {
+            const int j = i / M, tok = i % M;
+            float sum = 0.0f;
 #pragma unroll
-            for (int sb = 0; sb < kBwdSub; ++sb) sum += rp[((sb * kBwdCols + c) * 64 + f) * MP + tok];
+            for (int cc = 0; cc < kMaxCluster; ++cc)
+                if (cc < C) sum += cluster.map_shared_rank(upart, cc)[j * MP + tok];
+            ufull[j * MP + tok] = round_bf16(sum * p.s);
         }
+    }
+    auto base_sum = [&](const float *rp, int fl, int tok) {
+        const int c = fl / 64, f = fl % 64;
+        float v = 0.0f;
+#pragma unroll
+        for (int sb = 0; sb < kBwdSub; ++sb) v += rp[((sb * kBwdCols + c) * 64 + f) * MP + tok];
+        return v;
+    };
+    float *red = reinterpret_cast<float *>(lut + kLutBytes / 2);
+    if (C > 1) {
+        for (int i = threadIdx.x; i < nvf * M; i += blockDim.x) {
+            const int ff = i % nvf, tok = i / nvf;
+            float v[kMaxCluster];
+#pragma unroll
+            for (int cc = 0; cc < kMaxCluster; ++cc)
+                v[cc] = cc < C ? base_sum(cluster.map_shared_rank(part, cc), f_lo + ff, tok) : 0.0f;
+            float sum = 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < kMaxCluster; ++cc)
+                if (cc < C) sum += v[cc];
+            red[ff * MP + tok] = sum;
+        }
+    }
+    cluster_arrive_release();  // done reading other CTAs' shared memory
+    __syncthreads();
+
+    for (int i = threadIdx.x; i < nvf * M; i += blockDim.x) {
+        const int ff = i % nvf, tok = i / nvf;
+        float sum = C > 1 ? red[ff * MP + tok] : base_sum(part, f_lo + ff, tok);
         if (p.r > 0) {
             float lora = 0.0f;
             for (int j = 0; j < p.r; ++j)
-                lora = __fmaf_rn(__uint_as_float(static_cast<uint32_t>(ld_ro_u16(p.A + static_cast<int64_t>(j) * K + k)) << 16),
-                                 ufull[j * MP + tok], lora);
+                lora = __fmaf_rn(__uint_as_float(static_cast<uint32_t>(as[j * nvf + ff]) << 16), ufull[j * MP + tok], lora);
             sum += lora;
         }
-        p.out[static_cast<int64_t>(tok) * K + k] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+        p.out[static_cast<int64_t>(tok) * K + k_lo + ff] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
     }
-    cluster.sync();
+    cluster_wait_acquire();  // every CTA is done reading this CTA's shared memory
 }
 
-template <typename Kern>
-cudaError_t launch_cluster(Kern kern, dim3 grid, int cluster_x, size_t smem, cudaStream_t st, const DecodeParams &p) {
-    // Raise the kernel's dynamic shared-memory limit only when a launch needs more than
-    // any earlier one (the attribute call is skipped on the steady-state path).
+template <int NG>
+__global__ void __launch_bounds__(kDecThreads) k_decode_bwd(const DecodeParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    if ((smem_addr(smem) & 0x00ffffffu) == kDynSmemBase)
+        decode_bwd_body<NG, true>(p, smem);
+    else
+        decode_bwd_body<NG, false>(p, smem);
+}
+
+// Raise a kernel's dynamic shared-memory limit only when a launch needs more than any
+// earlier one (the attribute call is skipped on the steady-state path).
+cudaError_t ensure_smem(const void *kern, size_t smem) {
     static thread_local const void *kerns[16];
     static thread_local size_t limits[16];
     static thread_local int nk = 0;
     int slot = -1;
     for (int i = 0; i < nk; ++i)
-        if (kerns[i] == reinterpret_cast<const void *>(kern)) slot = i;
-    if (slot < 0 || limits[slot] < smem) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        if (slot < 0 && nk < 16) {
-            slot = nk++;
-            kerns[slot] = reinterpret_cast<const void *>(kern);
-        }
-        if (slot >= 0) limits[slot] = smem;
+        if (kerns[i] == kern) slot = i;
+    if (slot >= 0 && limits[slot] >= smem) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (slot < 0 && nk < 16) {
+        slot = nk++;
+        kerns[slot] = kern;
     }
+    if (slot >= 0) limits[slot] = smem;
+    return cudaSuccess;
+}
+
+cudaLaunchConfig_t cluster_config(dim3 grid, int cluster_x, size_t smem, cudaStream_t st, cudaLaunchAttribute *attr,
+                                  bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cluster_x;
     attr[0].val.clusterDim.y = 1;
@@ -646,40 +769,67 @@ cudaError_t launch_cluster(Kern kern, dim3 grid, int cluster_x, size_t smem, cud
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cfg;
+}
+
+// Clusters of `C` CTAs with `smem` bytes each that are resident at once on this device
+// (the occupancy query accounts for GPC boundaries), cached per (device, kernel, C, smem).
+int max_active_clusters(const void *kern, int C, size_t smem) {
+    struct Entry {
+        int dev;
+        const void *kern;
+        int C;
+        size_t smem;
+        int n;
+    };
+    static thread_local Entry cache[64];
+    static thread_local int nc = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    for (int i = 0; i < nc; ++i)
+        if (cache[i].dev == dev && cache[i].kern == kern && cache[i].C == C && cache[i].smem == smem) return cache[i].n;
+    int n = 0;
+    if (ensure_smem(kern, smem) == cudaSuccess) {
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = cluster_config(dim3(C, 1, 1), C, smem, nullptr, attr, false);
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+        }
+    }
+    if (nc < 64) cache[nc++] = Entry{dev, kern, C, smem, n};
+    return n;
+}
+
+// Cluster size: the largest C <= 8 whose grid (tiles x C CTAs) is resident in one wave,
+// keeping at least `min_units` units of reduction work per CTA; 1 when none fits.
+int pick_cluster(const void *kern, size_t smem, int64_t tiles, int64_t red_units, int64_t min_units) {
+    for (int C = kMaxCluster; C > 1; --C) {
+        if (red_units / C < min_units) continue;
+        if (tiles <= max_active_clusters(kern, C, smem)) return C;
+    }
+    return 1;
+}
+
+template <typename Kern>
+cudaError_t launch_cluster(Kern kern, dim3 grid, int cluster_x, size_t smem, cudaStream_t st, const DecodeParams &p) {
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = cluster_config(grid, cluster_x, smem, st, attr, true);
+    e = cudaLaunchKernelEx(&cfg, kern, p);
     count_launch();
     return e;
 }
 
 int pick_groups(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
-// Cluster size: the power of two (<= 8) that brings the CTA count closest to two per SM,
-// keeping at least `min_units` units of reduction work per CTA.
-int pick_cluster(int64_t tiles, int64_t red_units, int64_t min_units, int sms) {
-    int best = 1;
-    double best_score = 1e30;
-    for (int C = 1; C <= kMaxCluster; C *= 2) {
-        if (C > 1 && red_units / C < min_units) break;
-        const double ratio = static_cast<double>(tiles * C) / (2.0 * sms);
-        const double score = ratio > 1.0 ? ratio : 1.0 / ratio;
-        if (score < best_score) {
-            best_score = score;
-            best = C;
-        }
-    }
-    return best;
-}
-
-int num_sms() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
+template <typename Kern>
+cudaError_t launch_picked(Kern kern, size_t smem, int64_t tiles, int64_t red_units, int64_t min_units, cudaStream_t st,
+                          const DecodeParams &p) {
+    const int C = pick_cluster(reinterpret_cast<const void *>(kern), smem, tiles, red_units, min_units);
+    return launch_cluster(kern, dim3(C, static_cast<unsigned>(tiles), 1), C, smem, st, p);
 }
 
 }  // namespace
@@ -690,15 +840,14 @@ cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, con
     DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, x, M, A, B, r, s, h};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
-    const size_t smem = kLutBytes + sizeof(float) * (kFwdRows * 8 * NG + 2 * rpad * 8 * NG);
+    const size_t smem = kLutBytes + sizeof(float) * ((kFwdRows + kMaxCluster) * 8 * NG + rpad * 8 * NG);
     const int64_t tiles = (w.n + kFwdRows - 1) / kFwdRows;
-    const int C = pick_cluster(tiles, w.k / kBlock, 4, num_sms());
-    const dim3 grid(C, static_cast<unsigned>(tiles), 1);
+    const int64_t red = w.k / kBlock;
     switch (NG) {
-        case 1: return launch_cluster(k_decode_fwd<1>, grid, C, smem, st, p);
-        case 2: return launch_cluster(k_decode_fwd<2>, grid, C, smem, st, p);
-        case 4: return launch_cluster(k_decode_fwd<4>, grid, C, smem, st, p);
-        default: return launch_cluster(k_decode_fwd<8>, grid, C, smem, st, p);
+        case 1: return launch_picked(k_decode_fwd<1>, smem, tiles, red, 4, st, p);
+        case 2: return launch_picked(k_decode_fwd<2>, smem, tiles, red, 4, st, p);
+        case 4: return launch_picked(k_decode_fwd<4>, smem, tiles, red, 4, st, p);
+        default: return launch_picked(k_decode_fwd<8>, smem, tiles, red, 4, st, p);
     }
 }
 
@@ -710,12 +859,11 @@ cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, co
     const int rpad = (r + 15) & ~15;
     const size_t smem = kLutBytes + sizeof(float) * (kDecWarps * 64 * 8 * NG + 2 * rpad * 8 * NG);
     const int64_t tiles = (w.k / kBlock + kBwdCols - 1) / kBwdCols;
-    const int C = pick_cluster(tiles, (w.n + 15) / 16 / kBwdSub, 2, num_sms());
-    const dim3 grid(C, static_cast<unsigned>(tiles), 1);
+    const int64_t red = (w.n + 15) / 16 / kBwdSub;
     switch (NG) {
-        case 1: return launch_cluster(k_decode_bwd<1>, grid, C, smem, st, p);
-        case 2: return launch_cluster(k_decode_bwd<2>, grid, C, smem, st, p);
-        case 4: return launch_cluster(k_decode_bwd<4>, grid, C, smem, st, p);
+        case 1: return launch_picked(k_decode_bwd<1>, smem, tiles, red, 2, st, p);
+        case 2: return launch_picked(k_decode_bwd<2>, smem, tiles, red, 2, st, p);
+        case 4: return launch_picked(k_decode_bwd<4>, smem, tiles, red, 2, st, p);
         default: return cudaErrorInvalidValue;  // callers split tokens into chunks of 32
     }
 }
