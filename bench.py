@@ -376,9 +376,11 @@ def run_ours(args):
             import hashlib
             with open(prof) as f:
                 rec = json.load(f)
-            with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-                same = hashlib.sha256(f.read()).hexdigest()[:16] == rec["source_sha256_16"]
-            traffic = rec["bytes_per_launch"] if same else None
+            h = hashlib.sha256()
+            for src in rec["sources"]:
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    h.update(f.read())
+            traffic = rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
         except Exception:
             traffic = None
 
