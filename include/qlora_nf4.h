@@ -150,7 +150,9 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
  *   x : M x k_in bf16 (tokens x features); A : r x k_in bf16; B : n_out x r bf16;
  *   h : M x n_out bf16 (written, must not alias x, A or B).
  * fp32 accumulation; the block constant is applied in fp32; the adapter
- * product A x is rounded to bf16 once before the up-projection.
+ * product s (A x) is rounded to bf16 as the operand of the up-projection (for
+ * M <= 64 per K-slice of the split reduction, whose partial up-projections are
+ * then summed in fp32).
  * r == 0 means no adapter (A and B must then be NULL; alpha is ignored).
  * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), forward
  * equations; "How does QLoRA work for training?" (aivaro.ru) 2.
@@ -164,7 +166,9 @@ qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, con
 /* qlora_linear_bwd_x -- input gradient through the frozen base and the adapter:
  *   grad_x[m, k] = sum_n grad_h[m,n] W'[n,k] + s * sum_j A[j,k] sum_n grad_h[m,n] B[n,j].
  *   grad_h : M x n_out bf16; grad_x : M x k_in bf16 (written, no aliasing).
- * W is frozen: nothing is written to the quantised weight.
+ * W is frozen: nothing is written to the quantised weight. fp32 accumulation;
+ * u = s (B^T grad_h) is rounded to bf16 as the up-projection's MMA operand for
+ * M > 64 and kept in fp32 for M <= 64.
  * Source: "How does QLoRA work for training?" (aivaro.ru) 7 (weights are
  * dequantised on the fly for the gradient and not updated).
  * Same workspace, alignment and error rules as qlora_linear_fwd. */
