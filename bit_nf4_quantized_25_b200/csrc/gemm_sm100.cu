@@ -11,7 +11,8 @@
 // One CTA computes a 128 x 256 tile: 128 weight rows (fwd) or 128 input features (bwd) as
 // the MMA M dimension, 256 tokens as the MMA N dimension, fp32 accumulator in TMEM.
 //   warp 0      : TMA producer of the token operand (x / grad_h, then t / u), 64-wide K slabs
-//                 in the 128-byte swizzled K-major layout, 4-stage mbarrier ring.
+//                 in the 128-byte swizzled K-major layout, and of the packed codes of the
+//                 stage's weight tile (4 KB), in a 4-stage mbarrier ring.
 //   warp 1      : TMEM allocator and the single MMA-issuing thread (tcgen05.mma kind::f16).
 //   warps 2..13 : three groups of four dequant warps taking stages round-robin. A thread owns one
 //                 64-weight block per stage (fwd: one row; bwd: half of a reduction row),
@@ -43,8 +44,9 @@ constexpr int kDqWarps = 4 * kDqGroups;
 constexpr int kGemmThreads = (2 + kDqWarps) * 32;
 constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK * 2;  // 32 KB
+constexpr uint32_t kCBytes = kTileM * kTileK / 2;  // 4 KB of packed codes per stage
 constexpr uint32_t kTmemCols = 256;
-constexpr size_t kGemmSmem = 1024 + kStages * (kABytes + kBBytes) + 256;
+constexpr size_t kGemmSmem = 1024 + kStages * (kABytes + kBBytes + kCBytes) + 256;
 
 constexpr int kErrTimeout = 1;
 
@@ -122,14 +124,18 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t j) { return row *
 template <bool kBwd>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lora,
-           const GemmParams p) {
+           const __grid_constant__ CUtensorMap tm_codes, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;                        // kStages x 16 KB
     uint8_t *sB = smem + kStages * kABytes;    // kStages x 32 KB
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBBytes);
+    // packed codes of each stage: fwd 128 weight rows x 32 bytes (one block); bwd 64 reduction
+    // rows x 64 bytes (the two blocks of the tile's 128 features)
+    uint8_t *sC = sB + kStages * kBBytes;      // kStages x 4 KB
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sC + kStages * kCBytes);
     uint64_t *full_a = bars, *full_b = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    uint64_t *full_c = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full_c + kStages);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,6 +151,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
             mbar_init(&full_a[s], 4);
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&full_c[s], 1);
         }
         mbar_init(acc_full, 1);
         *abort_flag = 0u;
@@ -157,6 +164,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_act);
         tma_prefetch_desc(&tm_lora);
+        tma_prefetch_desc(&tm_codes);
     }
     tc_fence_before();
     __syncthreads();
@@ -172,8 +180,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t issued_phase[kStages];
-            bool issued[kStages];
-            for (int s = 0; s < kStages; ++s) issued[s] = false;
+            bool issued[kStages], issued_c[kStages];
+            for (int s = 0; s < kStages; ++s) issued[s] = issued_c[s] = false;
             for (int i = 0; i < T && !*abort_flag; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1u;
@@ -182,16 +190,27 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                     break;
                 }
                 mbar_arrive_expect_tx(&full_b[s], kBBytes);
-                if (i < nred)
+                if (i < nred) {
                     tma_load_2d(sB + s * kBBytes, &tm_act, &full_b[s], i * kTileK, static_cast<int32_t>(tok0));
-                else
+                    // codes: fwd rows [row0, row0 + 128) x bytes [32 i, 32 i + 32);
+                    //        bwd rows [64 i, 64 i + 64) x bytes [row0 / 2, row0 / 2 + 64)
+                    mbar_arrive_expect_tx(&full_c[s], kCBytes);
+                    if (kBwd)
+                        tma_load_2d(sC + s * kCBytes, &tm_codes, &full_c[s], static_cast<int32_t>(row0 / 2), i * kTileK);
+                    else
+                        tma_load_2d(sC + s * kCBytes, &tm_codes, &full_c[s], i * (kBlock / 2), static_cast<int32_t>(row0));
+                } else {
                     tma_load_2d(sB + s * kBBytes, &tm_lora, &full_b[s], (i - nred) * kTileK, static_cast<int32_t>(tok0));
+                }
                 issued[s] = true;
                 issued_phase[s] = ph;
+                issued_c[s] = i < nred;
             }
             // drain: every load this thread issued has landed before the CTA can exit
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < kStages; ++s) {
                 if (issued[s]) mbar_wait(&full_b[s], issued_phase[s]);
+                if (issued[s] && issued_c[s]) mbar_wait(&full_c[s], issued_phase[s]);
+            }
         }
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA issuer
@@ -237,9 +256,10 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int64_t kf = row0 + 64 * half;  // bwd: first feature of this thread's block
         const bool bwd_kvalid = !kBwd || kf < K;
 
-        auto load_codes = [&](int i, uint4 &c0, uint4 &c1, uint32_t &qb, float &sg, bool &valid) {
+        // The block's codes arrive by TMA into sC; its constant inputs (one byte and one float)
+        // are loaded one of this group's stages ahead.
+        auto load_const = [&](int i, uint32_t &qb, float &sg, bool &valid) {
             valid = false;
-            c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
             qb = 0u;
             sg = 0.0f;
             if (i >= nred) return;
@@ -253,31 +273,39 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                 if (wrow >= N) return;
                 blk = wrow * nbr + i;
             }
-            const uint8_t *cp = p.codes + blk * 32;
-            c0 = __ldg(reinterpret_cast<const uint4 *>(cp));
-            c1 = __ldg(reinterpret_cast<const uint4 *>(cp + 16));
             qb = __ldg(p.q + blk);
             sg = __ldg(p.sigma + blk / kGroup);
             valid = true;
         };
+        const uint32_t c_off = kBwd ? arow * 64u + half * 32u : arow * 32u;  // this thread's block in sC
 
-        uint4 n0, n1;
         uint32_t nq;
         float ns;
         bool nv;
-        load_codes(grp, n0, n1, nq, ns, nv);
+        load_const(grp, nq, ns, nv);
         for (int i = grp; i < T; i += kDqGroups) {
             if (*abort_flag) break;
             const int s = i % kStages;
             const uint32_t ph = (i / kStages) & 1u;
-            const uint4 c0 = n0, c1 = n1;
             const uint32_t cq = nq;
             const float cs = ns;
             const bool cv = nv;
-            load_codes(i + kDqGroups, n0, n1, nq, ns, nv);  // prefetch this group's next stage
+            load_const(i + kDqGroups, nq, ns, nv);  // prefetch this group's next stage
             if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
                 fail();
                 break;
+            }
+            // every thread waits for the stage's codes, so the slot is never refilled while a
+            // load into it is still in flight
+            if (i < nred && !mbar_wait(&full_c[s], ph)) {
+                fail();
+                break;
+            }
+            uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0;
+            if (i < nred && cv) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCBytes + c_off);
+                c0 = src[0];
+                c1 = src[1];
             }
             const uint32_t a_base = smem_u32(sA + s * kABytes);
             // destination of chunk j (8 elements) of this thread's 64-element run
@@ -391,12 +419,27 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D uint8 tensor map over the packed codes (n rows of k/2 bytes), no swizzle, zero fill out
+// of bounds. Box: fwd 32 bytes (one block) x 128 rows; bwd 64 bytes (two blocks) x 64 rows.
+bool make_codes_map(CUtensorMap *m, const void *codes, int64_t n, int64_t k, bool bwd) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(n)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+    cuuint32_t box[2] = {bwd ? 64u : 32u, bwd ? 64u : 128u};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool kBwd>
 cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M, const uint16_t *lora_rows, int r,
                              const uint16_t *lora_act, int RT, uint16_t *out, int *err, cudaStream_t st) {
-    CUtensorMap tm_act, tm_lora;
+    CUtensorMap tm_act, tm_lora, tm_codes;
     const int64_t act_cols = kBwd ? w.n : w.k;
     if (!make_map(&tm_act, act, M, act_cols)) return cudaErrorInvalidValue;
+    if (!make_codes_map(&tm_codes, w.codes, w.n, w.k, kBwd)) return cudaErrorInvalidValue;
     if (r > 0) {
         if (!make_map(&tm_lora, lora_act, M, RT)) return cudaErrorInvalidValue;
     } else {
@@ -422,7 +465,7 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_nf4<kBwd>, tm_act, tm_lora, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_nf4<kBwd>, tm_act, tm_lora, tm_codes, p);
     count_launch();
     return e;
 }
