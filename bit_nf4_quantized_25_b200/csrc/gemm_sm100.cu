@@ -8,13 +8,16 @@
 // dequantised to bf16 for the matmul and the adapter output is added; "How does QLoRA work
 // for training?" (aivaro.ru), section 7: the same dequantisation feeds the gradient.
 //
-// One CTA computes a 128 x 256 tile: 128 weight rows (fwd) or 128 input features (bwd) as
-// the MMA M dimension, 256 tokens as the MMA N dimension, fp32 accumulator in TMEM.
+// One CTA computes a 128 x 512 tile: 128 weight rows (fwd) or 128 input features (bwd) as
+// the MMA M dimension and two halves of 256 tokens as the MMA N dimension, each with its own
+// fp32 accumulator in TMEM (512 columns). Each dequantised A tile feeds both halves, which
+// halves the dequantisation work per flop.
 //   warp 0      : TMA producer of the token operand (x / grad_h, then t / u), 64-wide K slabs
-//                 in the 128-byte swizzled K-major layout, and of the packed codes of the
-//                 stage's weight tile (4 KB), in a 4-stage mbarrier ring.
+//                 in the 128-byte swizzled K-major layout (4-slot ring, one slot per k-slab and
+//                 token half), and of the packed codes of each k-slab's weight tile (4 KB, one
+//                 slot per dequant group).
 //   warp 1      : TMEM allocator and the single MMA-issuing thread (tcgen05.mma kind::f16).
-//   warps 2..13 : three groups of four dequant warps taking stages round-robin. A thread owns one
+//   warps 2..13 : three groups of four dequant warps taking k-slabs round-robin. A thread owns one
 //                 64-weight block per stage (fwd: one row; bwd: half of a reduction row),
 //                 builds the 16 scaled bf16 values NF4[i] * c'_b in registers, expands the
 //                 nibbles with byte permutes and writes the swizzled A tile (K-major for fwd,
@@ -36,17 +39,20 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileM = 128;  // MMA M: weight rows / input features
-constexpr int kTileN = 256;  // MMA N: tokens
+constexpr int kTileN = 256;  // MMA N: tokens per accumulator
+constexpr int kHalves = 2;   // accumulators per CTA: a CTA covers kHalves x 256 tokens
 constexpr int kTileK = 64;   // reduction per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
+constexpr int kAStages = 3;  // dequantised A tiles and their code slots (one per dequant group)
+constexpr int kBStages = 4;  // token-operand tiles (one per k-slab and half)
 constexpr int kDqGroups = 3;               // dequant groups taking stages round-robin
 constexpr int kDqWarps = 4 * kDqGroups;
 constexpr int kGemmThreads = (2 + kDqWarps) * 32;
+static_assert(kDqGroups == kAStages, "each dequant group owns one A slot");
 constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK * 2;  // 32 KB
 constexpr uint32_t kCBytes = kTileM * kTileK / 2;  // 4 KB of packed codes per stage
-constexpr uint32_t kTmemCols = 256;
-constexpr size_t kGemmSmem = 1024 + kStages * (kABytes + kBBytes + kCBytes) + 256;
+constexpr uint32_t kTmemCols = kTileN * kHalves;  // 512: the whole TMEM of the SM
+constexpr size_t kGemmSmem = 1024 + kAStages * (kABytes + kCBytes) + kBStages * kBBytes + 256;
 
 constexpr int kErrTimeout = 1;
 
@@ -127,31 +133,35 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
            const __grid_constant__ CUtensorMap tm_codes, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;                        // kStages x 16 KB
-    uint8_t *sB = smem + kStages * kABytes;    // kStages x 32 KB
-    // packed codes of each stage: fwd 128 weight rows x 32 bytes (one block); bwd 64 reduction
+    uint8_t *sA = smem;                         // kAStages x 16 KB
+    uint8_t *sB = smem + kAStages * kABytes;    // kBStages x 32 KB
+    // packed codes of each k-slab: fwd 128 weight rows x 32 bytes (one block); bwd 64 reduction
     // rows x 64 bytes (the two blocks of the tile's 128 features)
-    uint8_t *sC = sB + kStages * kBBytes;      // kStages x 4 KB
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sC + kStages * kCBytes);
-    uint64_t *full_a = bars, *full_b = bars + kStages, *empty = bars + 2 * kStages, *acc_full = bars + 3 * kStages;
-    uint64_t *full_c = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full_c + kStages);
+    uint8_t *sC = sB + kBStages * kBBytes;      // kAStages x 4 KB
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sC + kAStages * kCBytes);
+    uint64_t *full_a = bars, *empty_a = full_a + kAStages, *full_c = empty_a + kAStages;
+    uint64_t *full_b = full_c + kAStages, *empty_b = full_b + kBStages, *acc_full = empty_b + kBStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = p.n, K = p.k, nbr = K / kBlock;
     const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileM;  // fwd: weight row; bwd: feature
-    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTileN;
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTileN * kHalves;
+    const int nh = tok0 + kTileN < p.M ? kHalves : 1;  // token halves with any token in range
     const int nred = kBwd ? static_cast<int>((N + kTileK - 1) / kTileK) : static_cast<int>(nbr);
     const int nlora = (p.r + kTileK - 1) / kTileK;
     const int T = nred + nlora;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kAStages; ++s) {
             mbar_init(&full_a[s], 4);
-            mbar_init(&full_b[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty_a[s], 1);
             mbar_init(&full_c[s], 1);
+        }
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], 1);
         }
         mbar_init(acc_full, 1);
         *abort_flag = 0u;
@@ -179,67 +189,99 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t issued_phase[kStages];
-            bool issued[kStages], issued_c[kStages];
-            for (int s = 0; s < kStages; ++s) issued[s] = issued_c[s] = false;
-            for (int i = 0; i < T && !*abort_flag; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1u;
-                if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
-                    fail();
-                    break;
-                }
-                mbar_arrive_expect_tx(&full_b[s], kBBytes);
+            // k-slab i: its codes (slot i % kAStages, refilled once the MMA has consumed that
+            // slot's A tile), then one token-operand tile per half (B sequence j = i nh + h).
+            uint32_t c_phase[kAStages], b_phase[kBStages];
+            bool c_issued[kAStages], b_issued[kBStages];
+            for (int s = 0; s < kAStages; ++s) c_issued[s] = false;
+            for (int s = 0; s < kBStages; ++s) b_issued[s] = false;
+            bool stop = false;
+            for (int i = 0; i < T && !stop && !*abort_flag; ++i) {
                 if (i < nred) {
-                    tma_load_2d(sB + s * kBBytes, &tm_act, &full_b[s], i * kTileK, static_cast<int32_t>(tok0));
+                    const int sa = i % kAStages;
+                    const uint32_t pa = (i / kAStages) & 1u;
+                    if (i >= kAStages && !mbar_wait(&empty_a[sa], pa ^ 1u)) {
+                        fail();
+                        break;
+                    }
                     // codes: fwd rows [row0, row0 + 128) x bytes [32 i, 32 i + 32);
                     //        bwd rows [64 i, 64 i + 64) x bytes [row0 / 2, row0 / 2 + 64)
-                    mbar_arrive_expect_tx(&full_c[s], kCBytes);
+                    mbar_arrive_expect_tx(&full_c[sa], kCBytes);
                     if (kBwd)
-                        tma_load_2d(sC + s * kCBytes, &tm_codes, &full_c[s], static_cast<int32_t>(row0 / 2), i * kTileK);
+                        tma_load_2d(sC + sa * kCBytes, &tm_codes, &full_c[sa], static_cast<int32_t>(row0 / 2), i * kTileK);
                     else
-                        tma_load_2d(sC + s * kCBytes, &tm_codes, &full_c[s], i * (kBlock / 2), static_cast<int32_t>(row0));
-                } else {
-                    tma_load_2d(sB + s * kBBytes, &tm_lora, &full_b[s], (i - nred) * kTileK, static_cast<int32_t>(tok0));
+                        tma_load_2d(sC + sa * kCBytes, &tm_codes, &full_c[sa], i * (kBlock / 2), static_cast<int32_t>(row0));
+                    c_issued[sa] = true;
+                    c_phase[sa] = pa;
                 }
-                issued[s] = true;
-                issued_phase[s] = ph;
-                issued_c[s] = i < nred;
+                for (int h = 0; h < nh; ++h) {
+                    const int j = i * nh + h;
+                    const int sb = j % kBStages;
+                    const uint32_t pb = (j / kBStages) & 1u;
+                    if (j >= kBStages && !mbar_wait(&empty_b[sb], pb ^ 1u)) {
+                        fail();
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full_b[sb], kBBytes);
+                    const int32_t tk = static_cast<int32_t>(tok0 + h * kTileN);
+                    if (i < nred)
+                        tma_load_2d(sB + sb * kBBytes, &tm_act, &full_b[sb], i * kTileK, tk);
+                    else
+                        tma_load_2d(sB + sb * kBBytes, &tm_lora, &full_b[sb], (i - nred) * kTileK, tk);
+                    b_issued[sb] = true;
+                    b_phase[sb] = pb;
+                }
             }
             // drain: every load this thread issued has landed before the CTA can exit
-            for (int s = 0; s < kStages; ++s) {
-                if (issued[s]) mbar_wait(&full_b[s], issued_phase[s]);
-                if (issued[s] && issued_c[s]) mbar_wait(&full_c[s], issued_phase[s]);
-            }
+            for (int s = 0; s < kAStages; ++s)
+                if (c_issued[s]) mbar_wait(&full_c[s], c_phase[s]);
+            for (int s = 0; s < kBStages; ++s)
+                if (b_issued[s]) mbar_wait(&full_b[s], b_phase[s]);
         }
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(kTileM, kTileN, kBwd ? 1 : 0, 0);
-            for (int i = 0; i < T && !*abort_flag; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1u;
-                if (!mbar_wait(&full_a[s], ph) || !mbar_wait(&full_b[s], ph)) {
+            bool stop = false;
+            for (int i = 0; i < T && !stop && !*abort_flag; ++i) {
+                const int sa = i % kAStages;
+                const uint32_t pa = (i / kAStages) & 1u;
+                if (!mbar_wait(&full_a[sa], pa)) {
                     fail();
                     break;
                 }
-                tc_fence_after();
                 int nk = 4;
                 if (i >= nred) {
                     const int rem = p.r - (i - nred) * kTileK;
                     nk = rem >= kTileK ? 4 : (rem + 15) / 16;
                 }
-                const uint32_t a_base = smem_u32(sA + s * kABytes), b_base = smem_u32(sB + s * kBBytes);
-                for (int kk = 0; kk < nk; ++kk) {
-                    // fwd A: K-major, 16 elements = 32 bytes along the swizzled row.
-                    // bwd A: MN-major, 16 reduction rows = two 8-row groups of 1024 bytes;
-                    //        the two 64-feature chunks are 8192 bytes apart.
-                    const uint64_t ad = kBwd ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
-                                             : smem_desc_sw128(a_base + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                    mma_bf16_ss(tmem_d, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t a_base = smem_u32(sA + sa * kABytes);
+                for (int h = 0; h < nh; ++h) {
+                    const int j = i * nh + h;
+                    const int sb = j % kBStages;
+                    const uint32_t pb = (j / kBStages) & 1u;
+                    if (!mbar_wait(&full_b[sb], pb)) {
+                        fail();
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b_base = smem_u32(sB + sb * kBBytes);
+                    for (int kk = 0; kk < nk; ++kk) {
+                        // fwd A: K-major, 16 elements = 32 bytes along the swizzled row.
+                        // bwd A: MN-major, 16 reduction rows = two 8-row groups of 1024 bytes;
+                        //        the two 64-feature chunks are 8192 bytes apart.
+                        const uint64_t ad = kBwd ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                                 : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                        mma_bf16_ss(tmem_d + static_cast<uint32_t>(h * kTileN), ad, bd, idesc,
+                                    (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty_b[sb]);
                 }
-                mma_commit(&empty[s]);
+                if (stop) break;
+                mma_commit(&empty_a[sa]);
             }
             mma_commit(acc_full);  // arrives when every issued MMA has completed
         }
@@ -285,13 +327,13 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         load_const(grp, nq, ns, nv);
         for (int i = grp; i < T; i += kDqGroups) {
             if (*abort_flag) break;
-            const int s = i % kStages;
-            const uint32_t ph = (i / kStages) & 1u;
+            const int s = i % kAStages;  // == grp: each group owns one A slot
+            const uint32_t ph = (i / kAStages) & 1u;
             const uint32_t cq = nq;
             const float cs = ns;
             const bool cv = nv;
             load_const(i + kDqGroups, nq, ns, nv);  // prefetch this group's next stage
-            if (i >= kStages && !mbar_wait(&empty[s], ph ^ 1u)) {
+            if (i >= kAStages && !mbar_wait(&empty_a[s], ph ^ 1u)) {
                 fail();
                 break;
             }
@@ -374,7 +416,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int64_t orow = row0 + quarter * 32 + lane;           // fwd: n; bwd: feature k
         const int64_t ldo = kBwd ? K : N;
         const bool rvalid = orow < (kBwd ? K : N);
-        for (int cb = grp; cb < kTileN / 32; cb += kDqGroups) {  // 32-column chunks of this group
+        for (int cb = grp; cb < nh * kTileN / 32; cb += kDqGroups) {  // 32-column chunks of this group
             uint32_t v[32];
             tmem_ld32(tmem_d + ((quarter * 32u) << 16) + static_cast<uint32_t>(cb * 32), v);
             tmem_ld_wait();
@@ -454,7 +496,7 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
     }
     GemmParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, M, lora_rows, r, out, err};
     const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileM - 1) / kTileM;
-    const int64_t tiles_n = (M + kTileN - 1) / kTileN;
+    const int64_t tiles_n = (M + kTileN * kHalves - 1) / (kTileN * kHalves);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles_m), static_cast<unsigned>(tiles_n), 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
