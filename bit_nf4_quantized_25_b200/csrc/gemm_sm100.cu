@@ -43,7 +43,7 @@ constexpr int kTileN = 256;  // MMA N: tokens per accumulator
 constexpr int kHalves = 2;   // accumulators per CTA: a CTA covers kHalves x 256 tokens
 constexpr int kTileK = 64;   // reduction per stage: one 128-byte swizzle row of bf16
 constexpr int kAStages = 3;  // dequantised A tiles and their code slots (one per dequant group)
-constexpr int kBStages = 4;  // token-operand tiles (one per k-slab and half)
+constexpr int kBStages = 5;  // token-operand tiles (one per k-slab and half)
 constexpr int kDqGroups = 3;               // dequant groups taking stages round-robin
 constexpr int kDqWarps = 4 * kDqGroups;
 constexpr int kGemmThreads = (2 + kDqWarps) * 32;
@@ -140,7 +140,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
     uint8_t *sC = sB + kBStages * kBBytes;      // kAStages x 4 KB
     uint64_t *bars = reinterpret_cast<uint64_t *>(sC + kAStages * kCBytes);
     uint64_t *full_a = bars, *empty_a = full_a + kAStages, *full_c = empty_a + kAStages;
-    uint64_t *full_b = full_c + kAStages, *empty_b = full_b + kBStages, *acc_full = empty_b + kBStages;
+    uint64_t *empty_c = full_c + kAStages;  // the dequant group has read the slot's codes
+    uint64_t *full_b = empty_c + kAStages, *empty_b = full_b + kBStages, *acc_full = empty_b + kBStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
 
@@ -158,6 +159,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
             mbar_init(&full_a[s], 4);
             mbar_init(&empty_a[s], 1);
             mbar_init(&full_c[s], 1);
+            mbar_init(&empty_c[s], 4);
         }
         for (int s = 0; s < kBStages; ++s) {
             mbar_init(&full_b[s], 1);
@@ -189,8 +191,9 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // k-slab i: its codes (slot i % kAStages, refilled once the MMA has consumed that
-            // slot's A tile), then one token-operand tile per half (B sequence j = i nh + h).
+            // k-slab i: its codes (slot i % kAStages, refilled once the dequant group has read
+            // the slot's previous codes), then one token-operand tile per half (B sequence
+            // j = i nh + h).
             uint32_t c_phase[kAStages], b_phase[kBStages];
             bool c_issued[kAStages], b_issued[kBStages];
             for (int s = 0; s < kAStages; ++s) c_issued[s] = false;
@@ -200,7 +203,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                 if (i < nred) {
                     const int sa = i % kAStages;
                     const uint32_t pa = (i / kAStages) & 1u;
-                    if (i >= kAStages && !mbar_wait(&empty_a[sa], pa ^ 1u)) {
+                    if (i >= kAStages && !mbar_wait(&empty_c[sa], pa ^ 1u)) {
                         fail();
                         break;
                     }
@@ -344,10 +347,14 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                 break;
             }
             uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0;
-            if (i < nred && cv) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCBytes + c_off);
-                c0 = src[0];
-                c1 = src[1];
+            if (i < nred) {
+                if (cv) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCBytes + c_off);
+                    c0 = src[0];
+                    c1 = src[1];
+                }
+                __syncwarp();  // the whole warp has read its codes: the slot may be refilled
+                if (lane == 0) mbar_arrive(&empty_c[s]);
             }
             const uint32_t a_base = smem_u32(sA + s * kABytes);
             // destination of chunk j (8 elements) of this thread's 64-element run
