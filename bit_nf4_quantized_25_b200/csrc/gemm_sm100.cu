@@ -8,10 +8,10 @@
 // dequantised to bf16 for the matmul and the adapter output is added; "How does QLoRA work
 // for training?" (aivaro.ru), section 7: the same dequantisation feeds the gradient.
 //
-// One CTA computes a 256 x 256 tile: two row tiles of 128 weight rows (fwd) or 128 input
-// features (bwd) as the MMA M dimension, each with its own fp32 accumulator in TMEM (512
-// columns), and 256 tokens as the MMA N dimension. Both row tiles share each token tile, which
-// halves the token-operand traffic from L2 per flop (the limit of a 128 x 256 tile).
+// One CTA computes a 128 x 512 tile: 128 weight rows (fwd) or 128 input features (bwd) as
+// the MMA M dimension and two halves of 256 tokens as the MMA N dimension, each with its own
+// fp32 accumulator in TMEM (512 columns). Each dequantised A tile feeds both halves, which
+// halves the dequantisation work per flop.
 //   warp 0      : TMA producer of the token operand (x / grad_h, then t / u), 64-wide K slabs
 //                 in the 128-byte swizzled K-major layout (4-slot ring, one slot per k-slab and
 //                 token half), and of the packed codes of each k-slab's weight tile (4 KB, one
@@ -39,21 +39,20 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileM = 128;  // MMA M: weight rows / input features
-constexpr int kTileN = 256;    // MMA N: tokens
-constexpr int kRowTiles = 2;   // accumulators per CTA: a CTA covers kRowTiles x 128 rows
-constexpr int kTileRows = kTileM * kRowTiles;
-constexpr int kTileK = 64;     // reduction per stage: one 128-byte swizzle row of bf16
-constexpr int kAStages = 3;    // dequantised A tiles and their code slots (one per dequant group)
-constexpr int kBStages = 3;    // token-operand tiles
+constexpr int kTileN = 256;  // MMA N: tokens per accumulator
+constexpr int kHalves = 2;   // accumulators per CTA: a CTA covers kHalves x 256 tokens
+constexpr int kTileK = 64;   // reduction per stage: one 128-byte swizzle row of bf16
+constexpr int kAStages = 3;  // dequantised A tiles and their code slots (one per dequant group)
+constexpr int kBStages = 5;  // token-operand tiles (one per k-slab and half)
 constexpr int kDqGroups = 3;               // dequant groups taking stages round-robin
 constexpr int kDqWarps = 4 * kDqGroups;
 constexpr int kGemmThreads = (2 + kDqWarps) * 32;
 static_assert(kDqGroups == kAStages, "each dequant group owns one A slot");
-constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB per row tile
+constexpr uint32_t kABytes = kTileM * kTileK * 2;  // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK * 2;  // 32 KB
-constexpr uint32_t kCBytes = kTileRows * kTileK / 2;  // 8 KB of packed codes per stage
-constexpr uint32_t kTmemCols = kTileN * kRowTiles;    // 512: the whole TMEM of the SM
-constexpr size_t kGemmSmem = 1024 + kAStages * (kRowTiles * kABytes + kCBytes) + kBStages * kBBytes + 256;
+constexpr uint32_t kCBytes = kTileM * kTileK / 2;  // 4 KB of packed codes per stage
+constexpr uint32_t kTmemCols = kTileN * kHalves;  // 512: the whole TMEM of the SM
+constexpr size_t kGemmSmem = 1024 + kAStages * (kABytes + kCBytes) + kBStages * kBBytes + 256;
 
 constexpr int kErrTimeout = 1;
 
@@ -134,10 +133,10 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
            const __grid_constant__ CUtensorMap tm_codes, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;                                    // kAStages x (2 row tiles x 16 KB)
-    uint8_t *sB = smem + kAStages * kRowTiles * kABytes;   // kBStages x 32 KB
-    // packed codes of each k-slab: fwd 256 weight rows x 32 bytes (one block); bwd 64 reduction
-    // rows x 128 bytes (the four blocks of the tile's 256 features)
+    uint8_t *sA = smem;                         // kAStages x 16 KB
+    uint8_t *sB = smem + kAStages * kABytes;    // kBStages x 32 KB
+    // packed codes of each k-slab: fwd 128 weight rows x 32 bytes (one block); bwd 64 reduction
+    // rows x 64 bytes (the two blocks of the tile's 128 features)
     uint8_t *sC = sB + kBStages * kBBytes;      // kAStages x 4 KB
     uint64_t *bars = reinterpret_cast<uint64_t *>(sC + kAStages * kCBytes);
     uint64_t *full_a = bars, *empty_a = full_a + kAStages, *full_c = empty_a + kAStages;
@@ -148,9 +147,9 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = p.n, K = p.k, nbr = K / kBlock;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;  // fwd: weight row; bwd: feature
-    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTileN;
-    const int nrt = row0 + kTileM < (kBwd ? K : N) ? kRowTiles : 1;  // row tiles with any row in range
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileM;  // fwd: weight row; bwd: feature
+    const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTileN * kHalves;
+    const int nh = tok0 + kTileN < p.M ? kHalves : 1;  // token halves with any token in range
     const int nred = kBwd ? static_cast<int>((N + kTileK - 1) / kTileK) : static_cast<int>(nbr);
     const int nlora = (p.r + kTileK - 1) / kTileK;
     const int T = nred + nlora;
@@ -193,7 +192,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             // k-slab i: its codes (slot i % kAStages, refilled once the dequant group has read
-            // the slot's previous codes), then its token-operand tile (slot i % kBStages).
+            // the slot's previous codes), then one token-operand tile per half (B sequence
+            // j = i nh + h).
             uint32_t c_phase[kAStages], b_phase[kBStages];
             bool c_issued[kAStages], b_issued[kBStages];
             for (int s = 0; s < kAStages; ++s) c_issued[s] = false;
@@ -207,8 +207,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                         fail();
                         break;
                     }
-                    // codes: fwd rows [row0, row0 + 256) x bytes [32 i, 32 i + 32);
-                    //        bwd rows [64 i, 64 i + 64) x bytes [row0 / 2, row0 / 2 + 128)
+                    // codes: fwd rows [row0, row0 + 128) x bytes [32 i, 32 i + 32);
+                    //        bwd rows [64 i, 64 i + 64) x bytes [row0 / 2, row0 / 2 + 64)
                     mbar_arrive_expect_tx(&full_c[sa], kCBytes);
                     if (kBwd)
                         tma_load_2d(sC + sa * kCBytes, &tm_codes, &full_c[sa], static_cast<int32_t>(row0 / 2), i * kTileK);
@@ -217,16 +217,17 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                     c_issued[sa] = true;
                     c_phase[sa] = pa;
                 }
-                {
-                    const int sb = i % kBStages;
-                    const uint32_t pb = (i / kBStages) & 1u;
-                    if (i >= kBStages && !mbar_wait(&empty_b[sb], pb ^ 1u)) {
+                for (int h = 0; h < nh; ++h) {
+                    const int j = i * nh + h;
+                    const int sb = j % kBStages;
+                    const uint32_t pb = (j / kBStages) & 1u;
+                    if (j >= kBStages && !mbar_wait(&empty_b[sb], pb ^ 1u)) {
                         fail();
                         stop = true;
                         break;
                     }
                     mbar_arrive_expect_tx(&full_b[sb], kBBytes);
-                    const int32_t tk = static_cast<int32_t>(tok0);
+                    const int32_t tk = static_cast<int32_t>(tok0 + h * kTileN);
                     if (i < nred)
                         tma_load_2d(sB + sb * kBBytes, &tm_act, &full_b[sb], i * kTileK, tk);
                     else
@@ -246,6 +247,10 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(kTileM, kTileN, kBwd ? 1 : 0, 0);
             bool stop = false;
+            // phase of the last commit to each slot's release barrier (-1: none)
+            int last_a[kAStages], last_b[kBStages];
+            for (int s = 0; s < kAStages; ++s) last_a[s] = -1;
+            for (int s = 0; s < kBStages; ++s) last_b[s] = -1;
             for (int i = 0; i < T && !stop && !*abort_flag; ++i) {
                 const int sa = i % kAStages;
                 const uint32_t pa = (i / kAStages) & 1u;
@@ -258,16 +263,18 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                     const int rem = p.r - (i - nred) * kTileK;
                     nk = rem >= kTileK ? 4 : (rem + 15) / 16;
                 }
-                const int sb = i % kBStages;
-                const uint32_t pb = (i / kBStages) & 1u;
-                if (!mbar_wait(&full_b[sb], pb)) {
-                    fail();
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t b_base = smem_u32(sB + sb * kBBytes);
-                for (int t = 0; t < nrt; ++t) {
-                    const uint32_t a_base = smem_u32(sA + (sa * kRowTiles + t) * kABytes);
+                const uint32_t a_base = smem_u32(sA + sa * kABytes);
+                for (int h = 0; h < nh; ++h) {
+                    const int j = i * nh + h;
+                    const int sb = j % kBStages;
+                    const uint32_t pb = (j / kBStages) & 1u;
+                    if (!mbar_wait(&full_b[sb], pb)) {
+                        fail();
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b_base = smem_u32(sB + sb * kBBytes);
                     for (int kk = 0; kk < nk; ++kk) {
                         // fwd A: K-major, 16 elements = 32 bytes along the swizzled row.
                         // bwd A: MN-major, 16 reduction rows = two 8-row groups of 1024 bytes;
@@ -275,153 +282,144 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                         const uint64_t ad = kBwd ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
                                                  : smem_desc_sw128(a_base + kk * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                        mma_bf16_ss(tmem_d + static_cast<uint32_t>(t * kTileN), ad, bd, idesc,
+                        mma_bf16_ss(tmem_d + static_cast<uint32_t>(h * kTileN), ad, bd, idesc,
                                     (i > 0 || kk > 0) ? 1u : 0u);
                     }
+                    mma_commit(&empty_b[sb]);
+                    last_b[sb] = static_cast<int>(pb);
                 }
-                mma_commit(&empty_b[sb]);
+                if (stop) break;
                 mma_commit(&empty_a[sa]);
+                last_a[sa] = static_cast<int>(pa);
             }
             mma_commit(acc_full);  // arrives when every issued MMA has completed
+            // The commits arrive asynchronously when the MMAs complete. Wait for the last one of
+            // every slot: an arrival still in flight when the CTA exits could land on the
+            // barriers of the next CTA that this SM runs.
+            for (int s = 0; s < kAStages; ++s)
+                if (last_a[s] >= 0) mbar_wait(&empty_a[s], static_cast<uint32_t>(last_a[s]));
+            for (int s = 0; s < kBStages; ++s)
+                if (last_b[s] >= 0) mbar_wait(&empty_b[s], static_cast<uint32_t>(last_b[s]));
         }
     } else {
         // ----------------------------------------------------------- dequant groups
         const int dw = warp - 2;
-        const int grp = dw >> 2;                  // k-slabs i with i % kDqGroups == grp
+        const int grp = dw >> 2;                  // stages i with i % kDqGroups == grp
         const int tid = (dw & 3) * 32 + lane;     // 0..127 within the group
         const float mu = __ldg(p.mu);
-        // A thread owns one 64-weight block of each row tile t per k-slab.
-        // fwd: row tid of tile t (weight row row0 + 128 t + tid), 64 k.
-        // bwd: reduction row tid/2 of the k-slab, feature half tid%2 of tile t
-        //      (features row0 + 128 t + 64 half .. + 64).
+        // fwd: thread = A row (weight row row0 + tid), 64 k per stage.
+        // bwd: thread = (reduction row tid/2 of the stage, feature half tid%2).
         const uint32_t arow = kBwd ? static_cast<uint32_t>(tid >> 1) : static_cast<uint32_t>(tid);
         const uint32_t half = kBwd ? static_cast<uint32_t>(tid & 1) : 0u;
+        const int64_t kf = row0 + 64 * half;  // bwd: first feature of this thread's block
+        const bool bwd_kvalid = !kBwd || kf < K;
 
         // The block's codes arrive by TMA into sC; its constant inputs (one byte and one float)
-        // are loaded one of this group's k-slabs ahead.
-        struct Const {
-            uint32_t q[kRowTiles];
-            float s[kRowTiles];
-            bool v[kRowTiles];
-        };
-        auto load_const = [&](int i, Const &c) {
-#pragma unroll
-            for (int t = 0; t < kRowTiles; ++t) {
-                c.v[t] = false;
-                c.q[t] = 0u;
-                c.s[t] = 0.0f;
-                if (i >= nred) continue;
-                int64_t wrow, blk;
-                if (kBwd) {
-                    const int64_t kf = row0 + kTileM * t + 64 * half;
-                    wrow = static_cast<int64_t>(i) * kTileK + arow;
-                    if (wrow >= N || kf >= K) continue;
-                    blk = wrow * nbr + kf / kBlock;
-                } else {
-                    wrow = row0 + kTileM * t + arow;
-                    if (wrow >= N) continue;
-                    blk = wrow * nbr + i;
-                }
-                c.q[t] = __ldg(p.q + blk);
-                c.s[t] = __ldg(p.sigma + blk / kGroup);
-                c.v[t] = true;
+        // are loaded one of this group's stages ahead.
+        auto load_const = [&](int i, uint32_t &qb, float &sg, bool &valid) {
+            valid = false;
+            qb = 0u;
+            sg = 0.0f;
+            if (i >= nred) return;
+            int64_t wrow, blk;
+            if (kBwd) {
+                wrow = static_cast<int64_t>(i) * kTileK + arow;
+                if (wrow >= N || !bwd_kvalid) return;
+                blk = wrow * nbr + kf / kBlock;
+            } else {
+                wrow = row0 + arow;
+                if (wrow >= N) return;
+                blk = wrow * nbr + i;
             }
+            qb = __ldg(p.q + blk);
+            sg = __ldg(p.sigma + blk / kGroup);
+            valid = true;
         };
-        // this thread's block of tile t in sC
-        auto c_off = [&](int t) -> uint32_t {
-            return kBwd ? arow * 128u + static_cast<uint32_t>(t) * 64u + half * 32u
-                        : (static_cast<uint32_t>(t) * kTileM + arow) * 32u;
-        };
+        const uint32_t c_off = kBwd ? arow * 64u + half * 32u : arow * 32u;  // this thread's block in sC
 
-        Const nc;
-        load_const(grp, nc);
+        uint32_t nq;
+        float ns;
+        bool nv;
+        load_const(grp, nq, ns, nv);
         for (int i = grp; i < T; i += kDqGroups) {
             if (*abort_flag) break;
             const int s = i % kAStages;  // == grp: each group owns one A slot
             const uint32_t ph = (i / kAStages) & 1u;
-            const Const cc = nc;
-            load_const(i + kDqGroups, nc);  // prefetch this group's next k-slab
+            const uint32_t cq = nq;
+            const float cs = ns;
+            const bool cv = nv;
+            load_const(i + kDqGroups, nq, ns, nv);  // prefetch this group's next stage
             if (i >= kAStages && !mbar_wait(&empty_a[s], ph ^ 1u)) {
                 fail();
                 break;
             }
-            // every thread waits for the k-slab's codes, so the slot is never refilled while a
+            // every thread waits for the stage's codes, so the slot is never refilled while a
             // load into it is still in flight
             if (i < nred && !mbar_wait(&full_c[s], ph)) {
                 fail();
                 break;
             }
-            uint4 cw[kRowTiles][2];
+            uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0;
             if (i < nred) {
-#pragma unroll
-                for (int t = 0; t < kRowTiles; ++t) {
-                    cw[t][0] = cw[t][1] = make_uint4(0u, 0u, 0u, 0u);
-                    if (cc.v[t]) {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCBytes + c_off(t));
-                        cw[t][0] = src[0];
-                        cw[t][1] = src[1];
-                    }
+                if (cv) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(sC + s * kCBytes + c_off);
+                    c0 = src[0];
+                    c1 = src[1];
                 }
                 __syncwarp();  // the whole warp has read its codes: the slot may be refilled
                 if (lane == 0) mbar_arrive(&empty_c[s]);
             }
+            const uint32_t a_base = smem_u32(sA + s * kABytes);
+            // destination of chunk j (8 elements) of this thread's 64-element run
+            auto dst = [&](uint32_t j) -> uint32_t {
+                return kBwd ? a_base + half * 8192u + (arow >> 3) * 1024u + swz(arow & 7u, j)
+                            : a_base + swz(arow, j);
+            };
+            if (i < nred) {
+                if (cv) {
+                    const Planes P = make_planes(block_constant(static_cast<uint8_t>(cq), cs, mu));
+                    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int t = 0; t < kRowTiles; ++t) {
-                const uint32_t a_base = smem_u32(sA + (s * kRowTiles + t) * kABytes);
-                // destination of chunk j (8 elements) of this thread's 64-element run in tile t
-                auto dst = [&](uint32_t j) -> uint32_t {
-                    return kBwd ? a_base + half * 8192u + (arow >> 3) * 1024u + swz(arow & 7u, j)
-                                : a_base + swz(arow, j);
-                };
-                if (i < nred) {
-                    if (cc.v[t]) {
-                        const Planes P = make_planes(block_constant(static_cast<uint8_t>(cc.q[t]), cc.s[t], mu));
-                        const uint32_t w[8] = {cw[t][0].x, cw[t][0].y, cw[t][0].z, cw[t][0].w,
-                                               cw[t][1].x, cw[t][1].y, cw[t][1].z, cw[t][1].w};
+                    for (int j = 0; j < 8; ++j) sts128(dst(j), expand8(P, w[j]));
+                } else {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) sts128(dst(j), expand8(P, w[j]));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) sts128(dst(j), make_uint4(0u, 0u, 0u, 0u));
+                    for (int j = 0; j < 8; ++j) sts128(dst(j), make_uint4(0u, 0u, 0u, 0u));
+                }
+            } else {
+                // adapter stage: fwd copies row (row0 + arow) of B (n x r), columns
+                // [64c, 64c + 64); bwd copies row (64c + arow) of A (r x k), features [kf, kf + 64).
+                const int c = i - nred;
+                const uint16_t *src = nullptr;
+                int count = 0;
+                if (kBwd) {
+                    const int j = c * kTileK + static_cast<int>(arow);
+                    if (j < p.r && bwd_kvalid) {
+                        src = p.lora + static_cast<int64_t>(j) * K + kf;
+                        count = 64;
                     }
                 } else {
-                    // adapter stage: fwd copies row (row0 + 128 t + arow) of B (n x r), columns
-                    // [64c, 64c + 64); bwd copies row (64c + arow) of A (r x k), features
-                    // [kf, kf + 64) of tile t.
-                    const int c = i - nred;
-                    const uint16_t *src = nullptr;
-                    int count = 0;
-                    if (kBwd) {
-                        const int64_t kf = row0 + kTileM * t + 64 * half;
-                        const int j = c * kTileK + static_cast<int>(arow);
-                        if (j < p.r && kf < K) {
-                            src = p.lora + static_cast<int64_t>(j) * K + kf;
-                            count = 64;
-                        }
-                    } else {
-                        const int64_t wrow = row0 + kTileM * t + arow;
-                        if (wrow < N) {
-                            src = p.lora + wrow * p.r + c * kTileK;
-                            const int rem = p.r - c * kTileK;
-                            count = rem < 64 ? rem : 64;
+                    const int64_t wrow = row0 + arow;
+                    if (wrow < N) {
+                        src = p.lora + wrow * p.r + c * kTileK;
+                        const int rem = p.r - c * kTileK;
+                        count = rem < 64 ? rem : 64;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (src && 8 * j < count) {
+                        if (8 * j + 8 <= count && ((reinterpret_cast<uintptr_t>(src + 8 * j) & 15u) == 0)) {
+                            v = __ldg(reinterpret_cast<const uint4 *>(src + 8 * j));
+                        } else {
+                            uint32_t e[8];
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) e[x] = (8 * j + x < count) ? ld_ro_u16(src + 8 * j + x) : 0u;
+                            v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16),
+                                           e[6] | (e[7] << 16));
                         }
                     }
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (src && 8 * j < count) {
-                            if (8 * j + 8 <= count && ((reinterpret_cast<uintptr_t>(src + 8 * j) & 15u) == 0)) {
-                                v = __ldg(reinterpret_cast<const uint4 *>(src + 8 * j));
-                            } else {
-                                uint32_t e[8];
-#pragma unroll
-                                for (int x = 0; x < 8; ++x) e[x] = (8 * j + x < count) ? ld_ro_u16(src + 8 * j + x) : 0u;
-                                v = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16),
-                                               e[6] | (e[7] << 16));
-                            }
-                        }
-                        sts128(dst(j), v);
-                    }
+                    sts128(dst(j), v);
                 }
             }
             fence_proxy_async_smem();
@@ -435,20 +433,17 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         if (!ok) fail();
         tc_fence_after();
         const uint32_t quarter = static_cast<uint32_t>(warp & 3);  // TMEM lanes this warp may access
+        const int64_t orow = row0 + quarter * 32 + lane;           // fwd: n; bwd: feature k
         const int64_t ldo = kBwd ? K : N;
-        // 32-column chunks of this group; chunk cb is columns [32 cb, 32 cb + 32) of the
-        // accumulator of row tile cb / 8
-        for (int cb = grp; cb < nrt * kTileN / 32; cb += kDqGroups) {
-            const int t = cb / (kTileN / 32);
-            const int64_t orow = row0 + kTileM * t + quarter * 32 + lane;  // fwd: n; bwd: feature k
-            const bool rvalid = orow < (kBwd ? K : N);
+        const bool rvalid = orow < (kBwd ? K : N);
+        for (int cb = grp; cb < nh * kTileN / 32; cb += kDqGroups) {  // 32-column chunks of this group
             uint32_t v[32];
             tmem_ld32(tmem_d + ((quarter * 32u) << 16) + static_cast<uint32_t>(cb * 32), v);
             tmem_ld_wait();
             if (ok && rvalid) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const int64_t m = tok0 + (cb % (kTileN / 32)) * 32 + c;
+                    const int64_t m = tok0 + cb * 32 + c;
                     if (m < p.M) p.out[m * ldo + orow] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
                 }
             }
@@ -487,13 +482,13 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
 }
 
 // 2-D uint8 tensor map over the packed codes (n rows of k/2 bytes), no swizzle, zero fill out
-// of bounds. Box: fwd 32 bytes (one block) x 256 rows; bwd 128 bytes (four blocks) x 64 rows.
+// of bounds. Box: fwd 32 bytes (one block) x 128 rows; bwd 64 bytes (two blocks) x 64 rows.
 bool make_codes_map(CUtensorMap *m, const void *codes, int64_t n, int64_t k, bool bwd) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(n)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
-    cuuint32_t box[2] = {bwd ? 128u : 32u, bwd ? 64u : 256u};
+    cuuint32_t box[2] = {bwd ? 64u : 32u, bwd ? 64u : 128u};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -520,8 +515,8 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
         configured = true;
     }
     GemmParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, M, lora_rows, r, out, err};
-    const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileRows - 1) / kTileRows;
-    const int64_t tiles_n = (M + kTileN - 1) / kTileN;
+    const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileM - 1) / kTileM;
+    const int64_t tiles_n = (M + kTileN * kHalves - 1) / (kTileN * kHalves);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles_m), static_cast<unsigned>(tiles_n), 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);

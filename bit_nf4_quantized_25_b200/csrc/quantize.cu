@@ -55,11 +55,16 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     uint32_t cached_e = 0u, cached_sum = 0u;
 
+    // software-pipelined: the next pass's 16 bytes are requested before this pass is processed
+    auto load = [&](int64_t bb) {
+        return bb < nb ? ld_nc_v4(W + bb * 8 + l8) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    uint4 v_next = load(warp_global * 4 + sub);
     for (int64_t b0 = warp_global * 4; b0 < nb; b0 += nwarps * 4) {
         const int64_t b = b0 + sub;
         const bool valid = b < nb;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) v = ld_nc_v4(W + b * 8 + l8);
+        const uint4 v = v_next;
+        v_next = load(b + nwarps * 4);
         uint32_t m = max(max(mag_max2(v.x), mag_max2(v.y)), max(mag_max2(v.z), mag_max2(v.w)));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
@@ -295,10 +300,16 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // 32 blocks per CTA per pass; enough CTAs for 8 per SM, never more than needed,
+    static int occ = 0;  // resident CTAs per SM
+    if (occ == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_blocks, kQuantThreads, 0) != cudaSuccess ||
+                     occ <= 0)) {
+        (void)cudaGetLastError();
+        occ = 4;
+    }
+    // 32 blocks per CTA per pass; exactly one wave of resident CTAs, never more than needed,
     // and few enough passes per thread that the 32-bit smem bins cannot overflow.
     int64_t grid = (nb + 31) / 32;
-    grid = grid < static_cast<int64_t>(sms) * 8 ? grid : static_cast<int64_t>(sms) * 8;
+    grid = grid < static_cast<int64_t>(sms) * occ ? grid : static_cast<int64_t>(sms) * occ;
     const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
     if (grid < min_grid) grid = min_grid;
     k_quant_blocks<<<static_cast<unsigned>(grid), kQuantThreads, 0, s>>>(
