@@ -57,6 +57,7 @@ __device__ __forceinline__ void decode_fwd_body(const DecodeParams &p, uint8_t *
     float *recv = reinterpret_cast<float *>(smem + kLutBytes);
     const int rpad = (p.r + 15) & ~15;
     float *tpart = recv + (kFwdRows + kMaxCluster) * MP;  // [rpad][MP] partial A x of this CTA's k-slice
+    float *scratch = tpart + rpad * MP;                   // [kDecWarps / 2][16][MP] warp-sum tree
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = static_cast<int>(cluster.num_blocks());
@@ -167,20 +168,12 @@ __device__ __forceinline__ void decode_fwd_body(const DecodeParams &p, uint8_t *
                     mma_16816(d[tg], a1.z, b1.z, a1.w, b1.w, x1.z, x1.w);
                 }
             }
-#pragma unroll
-            for (int tg = 0; tg < NG; ++tg) {
-                const int jl = jt * 16 + g;
-                atomicAdd(&tpart[jl * MP + tg * 8 + 2 * t], d[tg][0]);
-                atomicAdd(&tpart[jl * MP + tg * 8 + 2 * t + 1], d[tg][1]);
-                atomicAdd(&tpart[(jl + 8) * MP + tg * 8 + 2 * t], d[tg][2]);
-                atomicAdd(&tpart[(jl + 8) * MP + tg * 8 + 2 * t + 1], d[tg][3]);
-            }
+            warp_tree_sum<NG>(d, scratch, tpart + jt * 16 * MP);  // fixed order: bit-reproducible
         }
     };
 
     // The pair table is built while the first codes are in flight.
     build_pair_lut(lut);
-    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) tpart[i] = 0.0f;
     __syncthreads();
 
     // ---- base: group gi holds blocks b_lo + GB gi .. + GB of rows A and B.
@@ -296,7 +289,9 @@ cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, con
     DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, x, M, A, B, r, s, h};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
-    const size_t smem = kLutBytes + sizeof(float) * ((kFwdRows + kMaxCluster) * 8 * NG + rpad * 8 * NG);
+    // table | recv | tpart | warp-sum scratch
+    const size_t smem =
+        kLutBytes + sizeof(float) * ((kFwdRows + kMaxCluster) * 8 * NG + rpad * 8 * NG + kDecWarps / 2 * 16 * 8 * NG);
     const int64_t tiles = (w.n + kFwdRows - 1) / kFwdRows;
     const int64_t red = w.k / kBlock;
     switch (NG) {

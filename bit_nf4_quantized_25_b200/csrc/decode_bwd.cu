@@ -68,7 +68,8 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
     float *recv = reinterpret_cast<float *>(smem + kLutBytes);
     const int rpad = (p.r + 15) & ~15;
     float *upart = recv + (F + kMaxCluster) * MP;                   // [rpad][MP] partial B^T grad_h
-    uint16_t *as = reinterpret_cast<uint16_t *>(upart + rpad * MP);  // [rpad][F] A[:, k0 .. k0 + F)
+    float *scratch = upart + rpad * MP;                              // [kDecWarps / 2][16][MP] warp-sum tree
+    uint16_t *as = reinterpret_cast<uint16_t *>(scratch + kDecWarps / 2 * 16 * MP);  // [rpad][F] A[:, k0 .. k0 + F)
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = static_cast<int>(cluster.num_blocks());
@@ -180,20 +181,12 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
                     mma_16816(d[tg], a0, a1, a2, a3, b0, b1);
                 }
             }
-#pragma unroll
-            for (int tg = 0; tg < NG; ++tg) {
-                const int jl = jt * 16 + gq;
-                atomicAdd(&upart[jl * MP + tg * 8 + 2 * t], d[tg][0]);
-                atomicAdd(&upart[jl * MP + tg * 8 + 2 * t + 1], d[tg][1]);
-                atomicAdd(&upart[(jl + 8) * MP + tg * 8 + 2 * t], d[tg][2]);
-                atomicAdd(&upart[(jl + 8) * MP + tg * 8 + 2 * t + 1], d[tg][3]);
-            }
+            warp_tree_sum<NG>(d, scratch, upart + jt * 16 * MP);  // fixed order: bit-reproducible
         }
     };
 
     // The pair table is built while the first codes are in flight.
     build_pair_lut(lut);
-    for (int i = threadIdx.x; i < rpad * MP; i += blockDim.x) upart[i] = 0.0f;
     __syncthreads();
 
     // ---- base: block column kb, group gi holds steps s_lo + 2 gi, + 1.
@@ -314,9 +307,11 @@ cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, co
     DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, gh, M, A, B, r, s, gx};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
-    // table (later the warps' sums) | recv | upart | staged adapter columns
-    const size_t smem = kLutBytes + sizeof(float) * ((64 * kBwdCols + kMaxCluster) * 8 * NG + rpad * 8 * NG) +
-                        sizeof(uint16_t) * rpad * 64 * kBwdCols;
+    // table (later the warps' sums) | recv | upart | warp-sum scratch | staged adapter columns
+    const size_t smem =
+        kLutBytes +
+        sizeof(float) * ((64 * kBwdCols + kMaxCluster) * 8 * NG + rpad * 8 * NG + kDecWarps / 2 * 16 * 8 * NG) +
+        sizeof(uint16_t) * rpad * 64 * kBwdCols;
     const int64_t tiles = (w.k / kBlock + kBwdCols - 1) / kBwdCols;
     const int64_t red = (w.n + 15) / 16 / kBwdSub;
     switch (NG) {

@@ -131,6 +131,48 @@ __device__ __forceinline__ void prefetch_operands(const DecodeParams &p, int b_l
         for (int j = lane; j < p.r; j += 32) prefetch_l2(p.A + j * K + static_cast<int64_t>(b_lo) * 64, static_cast<uint32_t>(kbytes));
 }
 
+// Deterministic sum over the CTA's warps of one 16-row MMA accumulator tile d[NG][4] (row g or
+// g + 8, token tg*8 + 2t (+1)): a pairwise tree in a fixed order (w += w + 4, w += w + 2,
+// w += w + 1) through `scratch` (kDecWarps / 2 x 16 x MP floats); warp 0 writes the result to
+// dst[row * MP + token]. Every warp of the CTA must call it (it contains __syncthreads).
+template <int NG>
+__device__ __forceinline__ void warp_tree_sum(float (&d)[NG][4], float *scratch, float *dst) {
+    constexpr int MP = 8 * NG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int half = kDecWarps / 2; half >= 1; half >>= 1) {
+        if (warp >= half && warp < 2 * half) {
+            float *sp = scratch + (warp - half) * 16 * MP;
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                *reinterpret_cast<float2 *>(sp + g * MP + tg * 8 + 2 * t) = make_float2(d[tg][0], d[tg][1]);
+                *reinterpret_cast<float2 *>(sp + (g + 8) * MP + tg * 8 + 2 * t) = make_float2(d[tg][2], d[tg][3]);
+            }
+        }
+        __syncthreads();
+        if (warp < half) {
+            const float *sp = scratch + warp * 16 * MP;
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                const float2 u = *reinterpret_cast<const float2 *>(sp + g * MP + tg * 8 + 2 * t);
+                const float2 v = *reinterpret_cast<const float2 *>(sp + (g + 8) * MP + tg * 8 + 2 * t);
+                d[tg][0] += u.x;
+                d[tg][1] += u.y;
+                d[tg][2] += v.x;
+                d[tg][3] += v.y;
+            }
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+#pragma unroll
+        for (int tg = 0; tg < NG; ++tg) {
+            *reinterpret_cast<float2 *>(dst + g * MP + tg * 8 + 2 * t) = make_float2(d[tg][0], d[tg][1]);
+            *reinterpret_cast<float2 *>(dst + (g + 8) * MP + tg * 8 + 2 * t) = make_float2(d[tg][2], d[tg][3]);
+        }
+    }
+}
+
 __device__ __forceinline__ void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }

@@ -284,3 +284,25 @@ def test_empty_token_batch_is_noop():
     x = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
     h = qb.qlora_linear_fwd(w, x, None, None, 0.0)
     assert h.shape == (0, 128)
+
+
+@pytest.mark.parametrize("n,k,M,bwd", [(11008, 4096, 4096, False), (4096, 11008, 4096, True), (11008, 4096, 16, False),
+                                       (4096, 11008, 16, True)])
+def test_repeat_runs_bit_identical(n, k, M, bwd):
+    # The kernels have a fixed reduction order, so repeated calls on the same inputs must give
+    # the same bits; a difference means a race (the many-token grids span several waves).
+    case = synth.LayerCase(f"repeat{n}x{k}M{M}", n, k, M, 16, 32.0, 0.02, 4242 + M)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV, need_grad=bwd)
+    w = qb.nf4_quantize(W)
+    ws = torch.zeros(qb.linear_workspace_size(M, n, k, 16), dtype=torch.uint8, device=DEV)
+    first = None
+    for _ in range(8):
+        out = (qb.qlora_linear_bwd_x(w, gh, A, B, 32.0, workspace=ws) if bwd
+               else qb.qlora_linear_fwd(w, x, A, B, 32.0, workspace=ws))
+        torch.cuda.synchronize()
+        got = out.view(torch.int16).clone()
+        if first is None:
+            first = got
+        else:
+            assert torch.equal(got, first), f"run-to-run difference in {int((got != first).sum())} elements"
+    assert int(ws[:4].view(torch.int32).item()) == 0
