@@ -5,11 +5,15 @@
 // "Double Quantization"; "How does QLoRA work for training?" (aivaro.ru), section 5.
 //
 // Kernel 1 (HBM-bound, one pass over W): each 8-lane group owns one 64-weight block
-// (16-byte coalesced loads), takes the absmax with three shuffles, divides each weight
-// by it (IEEE division), picks the code through a 65-cell lookup of the 15 decision
-// thresholds, packs 8 codes per 32-bit word, writes the fp32 absmax to the workspace
-// and adds it to 256 exponent bins (integer sums, so the tensor sum is exact and
-// independent of scheduling).
+// (16-byte coalesced loads), takes the absmax with three shuffles, forms x = w / absmax,
+// picks the code through a 65-cell lookup of the 15 decision thresholds, packs 8 codes per
+// 32-bit word, writes the fp32 absmax to the workspace and adds it to 256 exponent bins
+// (integer sums, so the tensor sum is exact and independent of scheduling).
+// The codes are defined by the IEEE quotient fl32(w / c). The kernel multiplies by the
+// correctly rounded reciprocal instead (|w*r - w/c| < 2^-22 for |w| <= c, c normal) and
+// redoes the IEEE division only for a weight whose product lies within 2^-21 of its cell's
+// threshold -- the only case where the two can fall on different sides of it (no threshold
+// lies within 2^-21 of a cell edge; the host checks this when it builds the cells).
 // The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include <mutex>
@@ -37,9 +41,10 @@ __device__ float mean_from_bins(const unsigned long long *bins, int64_t nb);
 __global__ void __launch_bounds__(kQuantThreads)
 k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ codes, float *__restrict__ cblk,
                unsigned long long *__restrict__ bins, unsigned *__restrict__ done, float *__restrict__ mu_out,
-               QuantCells cells) {
+               QuantCells cells, int fast_ok_flag) {
     __shared__ float s_thr[65];
     __shared__ int s_base[65];
+    const bool fast_ok = fast_ok_flag != 0;  // reciprocal path allowed (checked on the host)
     __shared__ unsigned s_bins[256];
     for (int i = threadIdx.x; i < 65; i += blockDim.x) {
         s_thr[i] = cells.thr[i];
@@ -73,15 +78,34 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
         uint32_t word = 0x77777777u;               // all-zero block: code 7 everywhere
         if (c != 0.0f) {
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            word = 0u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bits = (i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16);
-                const float x = __fdiv_rn(__uint_as_float(bits), c);
+            auto weight = [&](int i) {
+                return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+            };
+            auto code_of = [&](float x, float &dist) {
                 int j = __float2int_rz(__fmaf_rn(x, 32.0f, 32.0f));
                 j = min(max(j, 0), 64);
-                const int code = s_base[j] + (x > s_thr[j] ? 1 : 0);
+                dist = x - s_thr[j];
+                return s_base[j] + (dist > 0.0f ? 1 : 0);
+            };
+            // c is a bf16 value, so c >= 2^-126 exactly when its exponent field is non-zero
+            const bool fast = fast_ok && (m >> 7) != 0u;
+            const float r = __frcp_rn(c);
+            word = 0u;
+            uint32_t redo = fast ? 0u : 0xffu;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float dist;
+                const int code = code_of(__fmul_rn(weight(i), r), dist);
                 word |= static_cast<uint32_t>(code) << (4 * i);
+                redo |= (fabsf(dist) <= 0x1p-21f ? 1u : 0u) << i;
+            }
+            if (redo) {
+                for (int i = 0; i < 8; ++i) {
+                    if (!((redo >> i) & 1u)) continue;
+                    float dist;
+                    const int code = code_of(__fdiv_rn(weight(i), c), dist);
+                    word = (word & ~(0xfu << (4 * i))) | (static_cast<uint32_t>(code) << (4 * i));
+                }
             }
         }
         if (valid) {
@@ -229,6 +253,16 @@ k_double_quant(const float *__restrict__ cblk, int64_t nb, uint8_t *__restrict__
 // Decision thresholds t_i = largest fp32 not above the midpoint of table values i and
 // i+1; for an fp32 x, "x > t_i" equals "x is nearer to value i+1 than to value i, or
 // at equal distance goes to the lower index".
+// The reciprocal path needs every decision threshold farther than 2^-20 from every cell edge.
+int reciprocal_path_ok() {
+    for (int i = 0; i < 15; ++i) {
+        const double m = (static_cast<double>(nf4_value(i)) + static_cast<double>(nf4_value(i + 1))) * 0.5;
+        for (int j = 0; j <= 64; ++j)
+            if (fabs(m - (-1.0 + j / 32.0)) <= 0x1p-19) return 0;
+    }
+    return 1;
+}
+
 QuantCells make_cells() {
     QuantCells c;
     double t[15];
@@ -290,6 +324,7 @@ size_t quantize_workspace_bytes(int64_t n, int64_t k) {
 cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
                             float *mu, void *ws, cudaStream_t s) {
     static const QuantCells cells = make_cells();
+    static const int fast_ok = reciprocal_path_ok();
     const int64_t nb = n * k / kBlock;
     if (nb == 0) return cudaSuccess;
     auto *bins = static_cast<unsigned long long *>(ws);
@@ -313,7 +348,8 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
     if (grid < min_grid) grid = min_grid;
     k_quant_blocks<<<static_cast<unsigned>(grid), kQuantThreads, 0, s>>>(
-        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, done, mu, cells);
+        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, done, mu, cells,
+        fast_ok);
     count_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
