@@ -23,7 +23,8 @@
 //                 nibbles with byte permutes and writes the swizzled A tile (K-major for fwd,
 //                 MN-major for bwd, so W is always read in its stored row-major order).
 //                 The extra LoRA stages copy rows of B (fwd) / A (bwd) into the A tile.
-//   epilogue    : the dequant warps read TMEM (tcgen05.ld) and store bf16.
+//   epilogue    : the dequant warps read TMEM (tcgen05.ld) and store bf16, staged through shared
+//                 memory for 16-byte stores when the output rows allow it.
 // Every mbarrier wait is bounded; on a timeout the CTA records an error code, stops issuing
 // work, drains what it issued and frees its TMEM.
 #include <cudaTypedefs.h>
@@ -436,11 +437,37 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int64_t orow = row0 + quarter * 32 + lane;           // fwd: n; bwd: feature k
         const int64_t ldo = kBwd ? K : N;
         const bool rvalid = orow < (kBwd ? K : N);
+        // With 16-byte aligned output rows and a full 128-row tile, each 32-token chunk is staged
+        // through the group's (now idle) A slot as [32 tokens][128 rows] bf16 and written with
+        // 16-byte stores, 256 contiguous bytes per token; otherwise one 2-byte store per value.
+        // (vec is the same for every thread of the CTA, so all four warps of a group reach the
+        // group barrier equally often; `ok` only gates the global stores)
+        const bool vec = (ldo % 8 == 0) && (row0 + kTileM <= (kBwd ? K : N));
+        uint16_t *stage = reinterpret_cast<uint16_t *>(sA + grp * kABytes);  // 2 x [32][128] bf16
+        int buf = 0;
         for (int cb = grp; cb < nh * kTileN / 32; cb += kDqGroups) {  // 32-column chunks of this group
             uint32_t v[32];
             tmem_ld32(tmem_d + ((quarter * 32u) << 16) + static_cast<uint32_t>(cb * 32), v);
             tmem_ld_wait();
-            if (ok && rvalid) {
+            if (vec) {
+                uint16_t *S = stage + buf * (32 * kTileM);
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    S[c * kTileM + quarter * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
+                // the group's four warps (128 threads) hold the chunk's four quarters; double
+                // buffering makes one barrier per chunk enough
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(128) : "memory");
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq) {
+                    const int e = tid + 128 * kq;  // 16-byte piece: token e / 16, rows 8 (e % 16) .. + 8
+                    const int c = e >> 4, pr = (e & 15) * 8;
+                    const int64_t m = tok0 + cb * 32 + c;
+                    if (ok && m < p.M)
+                        *reinterpret_cast<uint4 *>(p.out + m * ldo + row0 + pr) =
+                            *reinterpret_cast<const uint4 *>(S + c * kTileM + pr);
+                }
+                buf ^= 1;
+            } else if (ok && rvalid) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     const int64_t m = tok0 + cb * 32 + c;
