@@ -120,15 +120,23 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
     const int64_t erow = (4 * t + (gq & 3)) * nbr + kbc;  // flattened block index, step 0
     const int nst = vk && s_hi > s_lo ? static_cast<int>(s_hi - s_lo) : 0, ngrp = (nst + 1) / 2;
 
+    const int64_t nfull = N / 16;  // steps below this one have all 16 rows inside W
     auto load_group = [&](int gi, BwdGroup &G) {
+        // both steps of the group complete and inside W: no per-row predicates (the common case)
+        const bool gfull = 2 * gi + 2 <= nst && s_lo + 2 * gi + 2 <= nfull;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int64_t st = s_lo + 2 * gi + j;
             const bool sv = 2 * gi + j < nst;
             const uint8_t *rowp = cw + st * 16 * rstride;
+            if (gfull) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                G.w[j][i] = (sv && st * 16 + 4 * t + i < N) ? ld_nc_u32(rowp + i * rstride) : 0x77777777u;
+                for (int i = 0; i < 4; ++i) G.w[j][i] = ld_nc_u32(rowp + i * rstride);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    G.w[j][i] = (sv && st * 16 + 4 * t + i < N) ? ld_nc_u32(rowp + i * rstride) : 0x77777777u;
+            }
             const bool ok = sv && st * 16 + 4 * t + (gq & 3) < N;
             const uint64_t bi = static_cast<uint64_t>(erow + st * 16 * nbr);
             G.q[j] = ok ? __ldg(p.q + bi) : 0u;
@@ -199,9 +207,11 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
             const float mine = block_constant(static_cast<uint8_t>(G.q[j]), G.s[j], mu);
             float cp[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                cp[i] = __shfl_sync(0xffffffffu, mine, (i << 2) | t);
-                if (n0 + i >= N) cp[i] = 0.0f;
+            for (int i = 0; i < 4; ++i) cp[i] = __shfl_sync(0xffffffffu, mine, (i << 2) | t);
+            if (s_lo + 2 * gi + j >= nfull) {  // the step reaches past row N - 1
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (n0 + i >= N) cp[i] = 0.0f;
             }
             uint32_t e01, o01, e23, o23;
             interleave_rows(G.w[j][0], G.w[j][1], e01, o01);
