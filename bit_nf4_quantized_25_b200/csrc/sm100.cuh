@@ -1,5 +1,5 @@
 // sm100.cuh -- inline-PTX wrappers for the Blackwell (sm_100a) pieces the GEMM uses:
-// mbarriers with bounded waits, 2-D TMA loads (no multicast), tcgen05 MMA / TMEM.
+// mbarriers with bounded waits, 2-D TMA loads into the issuing CTA's own shared memory, tcgen05 MMA / TMEM.
 #pragma once
 
 #include <cuda.h>
