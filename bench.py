@@ -137,13 +137,21 @@ def dist_setup(n_gpus):
 
 
 def barrier_max(value, world):
+    """The maximum of `value` over all ranks (the slowest rank's time); `value` itself at one rank."""
     import torch
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_step, steps, world, seconds):
+    """Whole-job rate: every rank processes `units_per_step` per step (weak scaling), over the
+    slowest rank's time."""
+    return units_per_step * steps * world / seconds
 
 
 def barrier(world):
@@ -363,8 +371,8 @@ def run_ours(args):
     clocks = clk.summary()
 
     ms_per_step = t / args.steps * 1e3
-    value = per_step_bytes * args.steps * world / t / 1e9
-    tflops = per_step_flops * args.steps * world / t / 1e12
+    value = job_rate(per_step_bytes, args.steps, world, t) / 1e9
+    tflops = job_rate(per_step_flops, args.steps, world, t) / 1e12
     avg_launch_s = t / (args.steps * launches_per_step)
     bytes_per_launch = per_step_bytes / launches_per_step
     achieved = bytes_per_launch / avg_launch_s / 1e9
@@ -409,7 +417,7 @@ def run_ours(args):
     b.record()
     torch.cuda.synchronize()
     te = barrier_max(a.elapsed_time(b) * 1e-3, world)
-    e2e_value = per_step_bytes * args.steps * world / te / 1e9
+    e2e_value = job_rate(per_step_bytes, args.steps, world, te) / 1e9
 
     detail = None
     cpu = None
