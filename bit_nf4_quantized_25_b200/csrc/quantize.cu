@@ -6,7 +6,9 @@
 //
 // Kernel 1 (HBM-bound, one pass over W): each 8-lane group owns one 64-weight block
 // (16-byte coalesced loads), takes the absmax with three shuffles, forms x = w / absmax,
-// picks the code through a 65-cell lookup of the 15 decision thresholds, packs 8 codes per
+// picks the code through a 65-cell lookup of the 15 decision thresholds (the cell index
+// floor(32 x + 32) is the low bits of one fma rounded toward -inf against 2^23 + 32, and the
+// cell's threshold and base code are one 8-byte shared load), packs 8 codes per
 // 32-bit word, writes the fp32 absmax to the workspace and adds it to 256 exponent bins
 // (integer sums, so the tensor sum is exact and independent of scheduling).
 // The codes are defined by the IEEE quotient fl32(w / c). The kernel multiplies by the
@@ -42,14 +44,10 @@ __global__ void __launch_bounds__(kQuantThreads)
 k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ codes, float *__restrict__ cblk,
                unsigned long long *__restrict__ bins, unsigned *__restrict__ done, float *__restrict__ mu_out,
                QuantCells cells, int fast_ok_flag) {
-    __shared__ float s_thr[65];
-    __shared__ int s_base[65];
+    __shared__ int2 s_cell[65];  // {threshold bits, base code} of each cell
     const bool fast_ok = fast_ok_flag != 0;  // reciprocal path allowed (checked on the host)
     __shared__ unsigned s_bins[256];
-    for (int i = threadIdx.x; i < 65; i += blockDim.x) {
-        s_thr[i] = cells.thr[i];
-        s_base[i] = cells.base[i];
-    }
+    for (int i = threadIdx.x; i < 65; i += blockDim.x) s_cell[i] = make_int2(__float_as_int(cells.thr[i]), cells.base[i]);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0u;
     __syncthreads();
 
@@ -81,30 +79,35 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
             auto weight = [&](int i) {
                 return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
             };
+            // For x in [-1, 1], 32 x + 32 + 2^23 rounded toward -inf is 2^23 + floor(32 x + 32): the
+            // cell index in the mantissa, exactly. x leaves [-1, 1] only by a hair, when c > 2^126
+            // makes fl(1/c) subnormal (the sum then drops below 2^23 and its bits below 2^23's), so
+            // the index is clamped to [0, 64] as a signed integer; non-finite input lands in range too.
             auto code_of = [&](float x, float &dist) {
-                int j = __float2int_rz(__fmaf_rn(x, 32.0f, 32.0f));
-                j = min(max(j, 0), 64);
-                dist = x - s_thr[j];
-                return s_base[j] + (dist > 0.0f ? 1 : 0);
+                const int j =
+                    min(max(static_cast<int>(__float_as_uint(__fmaf_rd(x, 32.0f, 8388640.0f)) - 0x4B000000u), 0), 64);
+                const int2 cell = s_cell[j];
+                dist = x - __int_as_float(cell.x);
+                return cell.y + (dist > 0.0f ? 1 : 0);
             };
             // c is a bf16 value, so c >= 2^-126 exactly when its exponent field is non-zero
             const bool fast = fast_ok && (m >> 7) != 0u;
             const float r = __frcp_rn(c);
             word = 0u;
-            uint32_t redo = fast ? 0u : 0xffu;
+            bool redo = !fast;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float dist;
                 const int code = code_of(__fmul_rn(weight(i), r), dist);
                 word |= static_cast<uint32_t>(code) << (4 * i);
-                redo |= (fabsf(dist) <= 0x1p-21f ? 1u : 0u) << i;
+                redo |= fabsf(dist) <= 0x1p-21f;
             }
-            if (redo) {
+            if (redo) {  // rare: all eight weights of this lane again, by the IEEE quotient
+                word = 0u;
                 for (int i = 0; i < 8; ++i) {
-                    if (!((redo >> i) & 1u)) continue;
                     float dist;
                     const int code = code_of(__fdiv_rn(weight(i), c), dist);
-                    word = (word & ~(0xfu << (4 * i))) | (static_cast<uint32_t>(code) << (4 * i));
+                    word |= static_cast<uint32_t>(code) << (4 * i);
                 }
             }
         }
