@@ -13,9 +13,10 @@
 // (integer sums, so the tensor sum is exact and independent of scheduling).
 // The codes are defined by the IEEE quotient fl32(w / c). The kernel multiplies by the
 // correctly rounded reciprocal instead (|w*r - w/c| < 2^-22 for |w| <= c, c normal) and
-// redoes the IEEE division only for a weight whose product lies within 2^-21 of its cell's
-// threshold -- the only case where the two can fall on different sides of it (no threshold
-// lies within 2^-21 of a cell edge; the host checks this when it builds the cells).
+// redoes the IEEE division, for the lane's eight weights, only when a product lies within
+// 2^-21 of its cell's threshold -- the only case where the two can fall on different sides
+// of it. Near a cell edge the two may pick neighbouring cells; both give the same code there
+// because no threshold lies within 2^-19 of a cell edge (checked on the host).
 // The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include <mutex>
@@ -256,7 +257,7 @@ k_double_quant(const float *__restrict__ cblk, int64_t nb, uint8_t *__restrict__
 // Decision thresholds t_i = largest fp32 not above the midpoint of table values i and
 // i+1; for an fp32 x, "x > t_i" equals "x is nearer to value i+1 than to value i, or
 // at equal distance goes to the lower index".
-// The reciprocal path needs every decision threshold farther than 2^-20 from every cell edge.
+// The reciprocal path needs every decision threshold farther than 2^-19 from every cell edge.
 int reciprocal_path_ok() {
     for (int i = 0; i < 15; ++i) {
         const double m = (static_cast<double>(nf4_value(i)) + static_cast<double>(nf4_value(i + 1))) * 0.5;
