@@ -61,27 +61,42 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs.
+
+    Samples every `period_ms`. `begin()` and `end()` mark the timed region by the number of
+    complete sample lines written so far; the summary keeps the samples inside the region plus
+    the one on each side (all samples when the marks are missing)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_ms: int = 20):
         self.dev = device_index
+        self.period_ms = period_ms
         self.proc = None
         self.path = None
+        self.marks = [None, None]
+
+    def _start(self, period_ms):
+        try:
+            with open(self.path, "w") as out:
+                return subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", str(period_ms)], stdout=out, stderr=subprocess.DEVNULL)
+        except Exception:
+            return None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        self.proc = self._start(self.period_ms)
         time.sleep(0.3)
+        if self.proc is not None and self.proc.poll() is not None and self.period_ms < 200:
+            # the sampler exited at once (an interval it does not accept): the usual 200 ms
+            self.period_ms = 200
+            self.proc = self._start(self.period_ms)
+            time.sleep(0.3)
         return self
 
     def __exit__(self, *a):
@@ -92,17 +107,36 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def _rows(self):
         rows = []
         try:
             with open(self.path) as f:
                 for line in f:
+                    if not line.endswith("\n"):
+                        break  # the line nvidia-smi is still writing
                     parts = [p.strip() for p in line.split(",")]
                     if len(parts) >= 9:
                         rows.append(parts)
+        except Exception:
+            pass
+        return rows
+
+    def begin(self):
+        self.marks[0] = len(self._rows()) if self.path else None
+
+    def end(self):
+        time.sleep(2.5 * self.period_ms / 1e3)  # let the sample after the region land
+        self.marks[1] = len(self._rows()) if self.path else None
+
+    def summary(self):
+        rows = self._rows()
+        try:
             os.unlink(self.path)
         except Exception:
             pass
+        b, e = self.marks
+        if b is not None and e is not None and e > b:
+            rows = rows[max(b - 1, 0):e + 1]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -364,7 +398,9 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        clk.begin()
         t = time_graph(graph, args.steps, torch.cuda.current_stream())
+        clk.end()
     torch.cuda.synchronize()
     barrier(world)
     t = barrier_max(t, world)

@@ -1,0 +1,114 @@
+"""Host logic of bench.py that needs no GPU: the clock record taken during the timed region.
+
+The bench rejects its own number when the clocks seen during the timed region show a hardware
+or thermal slowdown, so the parsing of the nvidia-smi samples and the choice of the samples
+that fall inside the region are checked here on synthetic sample files.
+"""
+import os
+import sys
+import tempfile
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _row(sm, reasons=()):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    flags = ["Active" if n in reasons else "Not Active" for n in names]
+    active = "0x0000000000000004" if reasons else "0x0000000000000000"
+    return ", ".join(["0", str(sm), "1965", "812.40", active, *flags]) + "\n"
+
+
+def _sampler(lines, marks=(None, None), partial=None):
+    fd, path = tempfile.mkstemp(suffix=".csv")
+    with os.fdopen(fd, "w") as f:
+        f.writelines(lines)
+        if partial:
+            f.write(partial)  # a line nvidia-smi has not finished
+    clk = bench.ClockSampler(0)
+    clk.path = path
+    clk.marks = list(marks)
+    return clk
+
+
+def test_summary_keeps_the_timed_window():
+    # two idle samples, the region (3 samples at 1965 MHz with a power cap), two after it
+    lines = [_row(600), _row(645)] + [_row(1965, ("sw_power_cap",))] * 3 + [_row(1800), _row(700)]
+    s = _sampler(lines, marks=(2, 5)).summary()
+    # rows 1..5: one sample before the region, the region, one after
+    assert s["samples"] == 5
+    assert s["sm_mhz"] == 1965.0
+    assert s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_summary_reports_thermal_slowdown_inside_the_window():
+    lines = [_row(1965)] + [_row(1500, ("hw_thermal_slowdown",))] * 2 + [_row(1965)]
+    s = _sampler(lines, marks=(1, 3)).summary()
+    assert "hw_thermal_slowdown" in s["reasons"]
+
+
+def test_summary_without_marks_uses_every_sample_and_skips_a_partial_line():
+    lines = [_row(1965), _row(1960)]
+    s = _sampler(lines, partial="0, 1965, 19").summary()
+    assert s["samples"] == 2
+    assert s["sm_mhz"] == 1962.5
+    assert s["reasons"] == []
+
+
+def test_summary_falls_back_when_no_sample_landed_in_the_window():
+    lines = [_row(1965), _row(1965)]
+    s = _sampler(lines, marks=(2, 2)).summary()
+    assert s["samples"] == 2
+
+
+def test_summary_without_samples_is_marked_unavailable():
+    s = _sampler([]).summary()
+    assert s == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+
+def test_sampler_without_nvidia_smi_degrades_to_unavailable(monkeypatch):
+    # no nvidia-smi on the PATH: the sampler must not raise, and the summary says so
+    monkeypatch.setenv("PATH", tempfile.gettempdir())
+    clk = bench.ClockSampler(0, period_ms=5)
+    with clk:
+        clk.begin()
+        clk.end()
+    assert clk.summary()["reasons"] == ["unavailable"]
+
+
+def _fake_smi(tmp_path, min_ms):
+    """A stand-in nvidia-smi that refuses intervals below `min_ms` and otherwise prints one
+    sample row per interval."""
+    exe = tmp_path / "nvidia-smi"
+    exe.write_text(
+        "#!/bin/sh\n"
+        "ms=0; prev=''\n"
+        "for a in \"$@\"; do if [ \"$prev\" = '-lms' ]; then ms=$a; fi; prev=$a; done\n"
+        f"if [ \"$ms\" -lt {min_ms} ]; then exit 2; fi\n"
+        "while true; do echo '0, 1965, 1965, 700.00, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active'; "
+        "sleep 0.05; done\n")
+    exe.chmod(0o755)
+    return str(tmp_path)
+
+
+def test_sampler_records_rows_from_nvidia_smi(monkeypatch, tmp_path):
+    monkeypatch.setenv("PATH", _fake_smi(tmp_path, 0) + os.pathsep + os.environ.get("PATH", ""))
+    with bench.ClockSampler(0) as clk:
+        clk.begin()
+        clk.end()
+    s = clk.summary()
+    assert clk.period_ms == 20
+    assert s["samples"] >= 1 and s["sm_mhz"] == 1965.0 and s["reasons"] == []
+
+
+def test_sampler_falls_back_to_200_ms_when_the_interval_is_refused(monkeypatch, tmp_path):
+    monkeypatch.setenv("PATH", _fake_smi(tmp_path, 200) + os.pathsep + os.environ.get("PATH", ""))
+    with bench.ClockSampler(0) as clk:
+        clk.begin()
+        clk.end()
+    s = clk.summary()
+    assert clk.period_ms == 200
+    assert s["samples"] >= 1 and s["sm_mhz"] == 1965.0
