@@ -94,6 +94,51 @@ def _dev_bf16(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
 
 
+def _expect_shape(t: torch.Tensor, shape, name: str):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def check_linear_shapes(n_out: int, k_in: int, act: torch.Tensor, A, B, out, bwd: bool) -> int:
+    """Shapes of a linear call; returns the adapter rank r. The library sees only pointers and
+    M, so a tensor of the wrong shape would be read or written out of bounds: it is refused
+    here. Forward: x (M, k_in) -> h (M, n_out); input gradient: grad_h (M, n_out) ->
+    grad_x (M, k_in); A (r, k_in) and B (n_out, r) together, or neither."""
+    name = "grad_h" if bwd else "x"
+    if act.dim() != 2:
+        raise ValueError(f"{name} must be 2-D (tokens x features)")
+    M = act.shape[0]
+    _expect_shape(act, (M, n_out if bwd else k_in), name)
+    if (A is None) != (B is None):
+        raise ValueError("A and B are given together or not at all")
+    r = 0
+    if A is not None:
+        if A.dim() != 2:
+            raise ValueError("A must be 2-D (r x k_in)")
+        r = A.shape[0]
+        _expect_shape(A, (r, k_in), "A")
+        _expect_shape(B, (n_out, r), "B")
+    if out is not None:
+        _expect_shape(out, (M, k_in if bwd else n_out), "out")
+    return r
+
+
+def _workspace(ws: torch.Tensor | None, need: int, device) -> tuple[torch.Tensor, int]:
+    """A caller workspace (contiguous CUDA memory, any dtype) or a fresh one; its size in bytes."""
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    elif not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ws, ws.numel() * ws.element_size()
+
+
+def _same_device(w, *ts):
+    dev = w.codes.device
+    for t in ts:
+        if t is not None and t.device != dev:
+            raise ValueError(f"tensor on {t.device}, the weight is on {dev}")
+
+
 def sizes(n_out: int, k_in: int):
     """(codes, absmax_q, group_scale, absmax_mean) byte sizes of a quantised weight."""
     a, b, c, d = (ctypes.c_size_t() for _ in range(4))
@@ -149,13 +194,16 @@ def nf4_quantize(W: torch.Tensor, out: NF4Weight | None = None, workspace: torch
                  stream=None) -> NF4Weight:
     """Quantise a bf16 (n_out x k_in) CUDA tensor to NF4 with double quantisation."""
     _dev_bf16(W, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D (n_out x k_in)")
     n, k = W.shape
     out = out or NF4Weight.empty(n, k, W.device)
-    need = quantize_workspace_size(n, k)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    if (out.n_out, out.k_in) != (n, k):
+        raise ValueError(f"out holds a {out.n_out} x {out.k_in} weight, W is {n} x {k}")
+    _same_device(out, W)
+    workspace, ws_bytes = _workspace(workspace, quantize_workspace_size(n, k), W.device)
     cw = out.c_struct()
-    _check(load().nf4_quantize(_ptr(W), ctypes.byref(cw), _ptr(workspace), workspace.numel(), _stream(stream)),
+    _check(load().nf4_quantize(_ptr(W), ctypes.byref(cw), _ptr(workspace), ws_bytes, _stream(stream)),
            "nf4_quantize")
     return out
 
@@ -165,6 +213,9 @@ def nf4_quantize_static_ws(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4W
     library allocates nothing (the output buffers are the caller's). See the header for the
     size limit and the rule that overlapping calls race."""
     _dev_bf16(W, "W")
+    if W.dim() != 2 or (out.n_out, out.k_in) != tuple(W.shape):
+        raise ValueError(f"W of shape {tuple(W.shape)} does not match a {out.n_out} x {out.k_in} weight")
+    _same_device(out, W)
     cw = out.c_struct()
     _check(load().nf4_quantize_static_ws(_ptr(W), ctypes.byref(cw), _stream(stream)), "nf4_quantize_static_ws")
     return out
@@ -173,6 +224,8 @@ def nf4_quantize_static_ws(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4W
 def nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     out = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
     _dev_bf16(out, "out")
+    _expect_shape(out, (w.n_out, w.k_in), "out")
+    _same_device(w, out)
     cw = w.c_struct()
     _check(load().nf4_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "nf4_dequantize")
     return out
@@ -191,17 +244,16 @@ def qlora_linear_fwd(w: NF4Weight, x: torch.Tensor, A: torch.Tensor | None, B: t
                      stream=None) -> torch.Tensor:
     """h = dequant(W) x + (alpha/r) B (A x); x is M x k_in, h is M x n_out (bf16)."""
     _dev_bf16(x, "x")
+    r = check_linear_shapes(w.n_out, w.k_in, x, A, B, out, bwd=False)
     M = x.shape[0]
-    r = 0 if A is None else A.shape[0]
     A, B = _lora(A, B, r)
     out = out if out is not None else torch.empty(M, w.n_out, dtype=torch.bfloat16, device=x.device)
     _dev_bf16(out, "out")
-    need = linear_workspace_size(M, w.n_out, w.k_in, r)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    _same_device(w, x, A, B, out)
+    workspace, ws_bytes = _workspace(workspace, linear_workspace_size(M, w.n_out, w.k_in, r), x.device)
     cw = w.c_struct()
     _check(load().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
-                                   _ptr(workspace), workspace.numel(), _stream(stream)), "qlora_linear_fwd")
+                                   _ptr(workspace), ws_bytes, _stream(stream)), "qlora_linear_fwd")
     return out
 
 
@@ -210,16 +262,15 @@ def qlora_linear_bwd_x(w: NF4Weight, grad_h: torch.Tensor, A: torch.Tensor | Non
                        stream=None) -> torch.Tensor:
     """grad_x = dequant(W)^T grad_h + (alpha/r) A^T (B^T grad_h); grad_h is M x n_out."""
     _dev_bf16(grad_h, "grad_h")
+    r = check_linear_shapes(w.n_out, w.k_in, grad_h, A, B, out, bwd=True)
     M = grad_h.shape[0]
-    r = 0 if A is None else A.shape[0]
     A, B = _lora(A, B, r)
     out = out if out is not None else torch.empty(M, w.k_in, dtype=torch.bfloat16, device=grad_h.device)
     _dev_bf16(out, "out")
-    need = linear_workspace_size(M, w.n_out, w.k_in, r)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=grad_h.device)
+    _same_device(w, grad_h, A, B, out)
+    workspace, ws_bytes = _workspace(workspace, linear_workspace_size(M, w.n_out, w.k_in, r), grad_h.device)
     cw = w.c_struct()
     _check(load().qlora_linear_bwd_x(ctypes.byref(cw), _ptr(grad_h), M, _ptr(A), _ptr(B), r, float(alpha),
-                                     _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+                                     _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
            "qlora_linear_bwd_x")
     return out

@@ -132,3 +132,51 @@ def test_empty_problems_enqueue_nothing(lib):
 def test_status_strings(lib):
     for s in range(6):
         assert lib.qn_status_string(s)
+
+
+# ------------------------------------------------- binding: shapes refused before the call
+# The library receives pointers and M only, so the binding refuses any tensor whose shape does
+# not match the weight (it would be read or written out of bounds).
+
+def _t(*shape):
+    import torch
+    return torch.empty(*shape, dtype=torch.bfloat16)
+
+
+def test_binding_accepts_matching_linear_shapes():
+    from bit_nf4_quantized_25_b200 import binding as qb
+    n, k, M, r = 96, 128, 5, 16
+    assert qb.check_linear_shapes(n, k, _t(M, k), _t(r, k), _t(n, r), _t(M, n), bwd=False) == r
+    assert qb.check_linear_shapes(n, k, _t(M, n), _t(r, k), _t(n, r), _t(M, k), bwd=True) == r
+    assert qb.check_linear_shapes(n, k, _t(M, k), None, None, None, bwd=False) == 0
+    assert qb.check_linear_shapes(n, k, _t(0, k), _t(0, k), _t(n, 0), _t(0, n), bwd=False) == 0
+
+
+@pytest.mark.parametrize("what", ["x_k", "x_1d", "out_fwd", "a_only", "a_cols", "b_rank", "b_rows", "gh_n",
+                                  "out_bwd"])
+def test_binding_refuses_mismatched_linear_shapes(what):
+    from bit_nf4_quantized_25_b200 import binding as qb
+    n, k, M, r = 96, 128, 5, 16
+    x, A, B, h, gh, gx = _t(M, k), _t(r, k), _t(n, r), _t(M, n), _t(M, n), _t(M, k)
+    bwd = what in ("gh_n", "out_bwd")
+    act, out = (gh, gx) if bwd else (x, h)
+    if what == "x_k":
+        act = _t(M, k + 64)
+    elif what == "x_1d":
+        act = _t(M * k)
+    elif what == "out_fwd":
+        out = _t(M, n + 1)
+    elif what == "a_only":
+        B = None
+    elif what == "a_cols":
+        A = _t(r, k - 64)
+    elif what == "b_rank":
+        B = _t(n, r + 1)
+    elif what == "b_rows":
+        B = _t(n - 8, r)
+    elif what == "gh_n":
+        act = _t(M, k)
+    elif what == "out_bwd":
+        out = _t(M, n)
+    with pytest.raises(ValueError):
+        qb.check_linear_shapes(n, k, act, A, B, out, bwd=bwd)
