@@ -534,12 +534,17 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
     } else {
         tm_lora = tm_act;  // never read
     }
-    static bool configured = false;
-    if (!configured) {
+    // The shared-memory limit is a per-device attribute: set once per (host thread, device).
+    static thread_local uint64_t configured = 0;  // bit d: device d is configured
+    int dev = 0;
+    cudaError_t ge = cudaGetDevice(&dev);
+    if (ge != cudaSuccess) return ge;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+    if (bit == 0 || !(configured & bit)) {
         cudaError_t e = cudaFuncSetAttribute(k_gemm_nf4<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kGemmSmem));
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured |= bit;
     }
     GemmParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, M, lora_rows, r, out, err};
     const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileM - 1) / kTileM;
