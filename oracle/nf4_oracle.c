@@ -3,7 +3,7 @@
  *
  * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
  * this file: only the tests, the smoke check and the benchmark's cpu_baseline
- * leg use it. It shares no code, header, table or helper with the CUDA library.
+ * leg and reference arm use it. It shares no code, header, table or helper with the CUDA library.
  *
  * What it computes, step by step, with the passage each step follows:
  *

@@ -1,7 +1,7 @@
 """CPU oracle for the NF4 + double-quant + LoRA linear layer (test infrastructure).
 
-Only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
-``bench.py`` may import this module. The product path (the CUDA library and its
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s ``cpu_baseline``
+leg and reference arm (``--impl reference``) may import this module. The product path (the CUDA library and its
 Python binding) never imports, links or executes anything under ``oracle/``.
 
 The arithmetic lives in ``nf4_oracle.c`` (plain C, fp64 sums, OpenMP over
