@@ -51,6 +51,18 @@ def linear_flops(n, k, M, r):
     return 2 * M * n * k + 2 * M * r * (k + n)
 
 
+def decode_config(layers, world):
+    """The `config` of the decode-step workload; both arms report the same one."""
+    shapes = [(n, k) for _ in range(layers) for (_, n, k) in SHAPES_7B]
+    per_m_bytes = sum(fwd_bytes(n, k, M, RANK_7B) for M in DECODE_M for (n, k) in shapes) / len(DECODE_M)
+    return {"workload": f"llama7b-decode: {layers} layers x 7 linears (4096x4096 x4, 11008x4096 x2, "
+                        f"4096x11008), LoRA r=16 alpha=32, M in {{1,4,16}} per step, forward",
+            "global_batch": sum(DECODE_M), "layer_calls_per_step": len(shapes) * len(DECODE_M),
+            "l2": f"inputs larger than L2: {per_m_bytes / 1e9:.2f} GB of weights streamed per M",
+            "parallelism": f"replicas x{world}",
+            "quantised_weight_bytes": int(sum(weight_bytes(n, k) for (n, k) in shapes))}
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -376,7 +388,6 @@ def run_ours(args):
 
     per_step_bytes = sum(fwd_bytes(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)
     per_step_flops = sum(linear_flops(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)
-    per_step_calls = len(stack) * len(DECODE_M)
 
     # warm-up (eager), then capture one step into a CUDA graph
     for _ in range(max(args.warmup, 1)):
@@ -469,12 +480,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nf4/bf16 in, fp32 accumulate, bf16 out",
             "data": "synthetic (seeded random Llama-7B-shaped weights, no checkpoint)",
-            "config": {"workload": f"llama7b-decode: {args.layers} layers x 7 linears (4096x4096 x4, 11008x4096 x2, "
-                                   f"4096x11008), LoRA r=16 alpha=32, M in {{1,4,16}} per step, forward",
-                       "global_batch": sum(DECODE_M), "layer_calls_per_step": per_step_calls,
-                       "l2": f"inputs larger than L2: {per_step_bytes / len(DECODE_M) / 1e9:.2f} GB of weights "
-                             f"streamed per M", "parallelism": f"replicas x{world}",
-                       "quantised_weight_bytes": int(sum(weight_bytes(n, k) for (_, n, k, *_r) in stack))},
+            "config": decode_config(args.layers, world),
             "tflops": round(tflops, 3),
             "gpu_launches": int(launches_per_step * args.steps),
             "roofline": {"bound": "hbm", "kernel": "k_decode_fwd (few-token NF4+LoRA forward)",
@@ -514,8 +520,7 @@ def run_reference(args):
     line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": steps, "warmup": warm, "ms_per_step": round(dt / steps * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama7b-decode (bounded sample on the host CPU: oracle)",
-                       "parallelism": "host cores"},
+            "config": decode_config(args.layers, world),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
                              "sample": last["sample"]},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -112,3 +112,24 @@ def test_sampler_falls_back_to_200_ms_when_the_interval_is_refused(monkeypatch, 
     s = clk.summary()
     assert clk.period_ms == 200
     assert s["samples"] >= 1 and s["sm_mhz"] == 1965.0
+
+
+def test_reference_arm_reports_our_config(monkeypatch, capsys):
+    import json
+    import types
+
+    class QuickSample:  # stands in for the oracle run; only the line's shape is checked here
+        def run(self, budget):
+            return {"value": 1.0, "cores": 4, "sample": "stand-in"}
+
+    monkeypatch.setattr(bench, "CpuSample", QuickSample)
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.run_reference(types.SimpleNamespace(steps=2, warmup=3, layers=32))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s" and line["higher_is_better"] is True
+    assert line["config"] == bench.decode_config(32, 1)
+    assert line["config"]["layer_calls_per_step"] == 672
+    assert line["config"]["quantised_weight_bytes"] == 3340772224
+    assert line["e2e"] == {"value": 1.0, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
