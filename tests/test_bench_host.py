@@ -133,3 +133,15 @@ def test_reference_arm_reports_our_config(monkeypatch, capsys):
     assert line["config"]["layer_calls_per_step"] == 672
     assert line["config"]["quantised_weight_bytes"] == 3340772224
     assert line["e2e"] == {"value": 1.0, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_algorithmic_bytes_per_launch_of_the_decode_step():
+    # 0.5159 B per weight (codes 0.5, FP8 constant 1/64, fp32 group scale 4/(64*256), plus the mean),
+    # x, A, B and h in bf16; averaged over the 21 launches of one layer (7 linears x M = 1, 4, 16).
+    per_layer = [bench.fwd_bytes(n, k, M, bench.RANK_7B) for M in bench.DECODE_M for (_, n, k) in bench.SHAPES_7B]
+    assert len(per_layer) == 21
+    assert round(sum(per_layer) / 21) == 15_427_259
+    # the weight part alone: codes + constants + scales + mean of a 4096 x 4096 weight
+    n = k = 4096
+    assert bench.weight_bytes(n, k) == n * k // 2 + n * k // 64 + 4 * ((n * k // 64 + 255) // 256) + 4
+    assert bench.fwd_bytes(n, k, 1, 16) == bench.weight_bytes(n, k) + 2 * k + 2 * 16 * k + 2 * n * 16 + 2 * n
