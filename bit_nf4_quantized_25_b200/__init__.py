@@ -5,7 +5,9 @@ The computation lives in ``libqlora_nf4.so`` (C ABI: ``include/qlora_nf4.h``); t
 the library; the first call does, and fails loudly if it is missing.
 """
 from .binding import (NF4Weight, QNError, linear_workspace_size, launch_count, load, nf4_dequantize,
-                      nf4_quantize, qlora_linear_bwd_x, qlora_linear_fwd, quantize_workspace_size, sizes)
+                      nf4_quantize, nf4_quantize_static_ws, qlora_linear_bwd_x, qlora_linear_fwd,
+                      quantize_workspace_size, sizes)
 
 __all__ = ["NF4Weight", "QNError", "linear_workspace_size", "launch_count", "load", "nf4_dequantize",
-           "nf4_quantize", "qlora_linear_bwd_x", "qlora_linear_fwd", "quantize_workspace_size", "sizes"]
+           "nf4_quantize", "nf4_quantize_static_ws", "qlora_linear_bwd_x", "qlora_linear_fwd",
+           "quantize_workspace_size", "sizes"]
