@@ -31,6 +31,12 @@
  *  - Input gradient through the frozen, dequantised base: "How QLoRA works"
  *    section 7 (the 4-bit weights are dequantised on the fly to compute
  *    gradients and are not updated).
+ *  - Gradients of the adapter weights A and B, the only trained parameters:
+ *    "How QLoRA works" sections 2 (W frozen; B and A trained) and 7; they
+ *    are the derivatives of h = W'x + s B (A x) with respect to B and A.
+ *  - Merging the adapter into a 16-bit weight, W' + s B A (the weight cannot
+ *    stay NF4 once merged): "QLoRA & PEFT family" section 3.6
+ *    (merge_and_unload) and "QLoRA paper notes", Introduction.
  *
  * All sums of the linear layer are taken in fp64 in plain loop order.
  */
@@ -431,5 +437,105 @@ void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, 
     }
     free(u);
     free(gs);
+    free(cp);
+}
+
+/* ------------------------------------------------- adapter weight gradients */
+
+/* Gradients of the adapter for M token rows (all of them):
+ *   t[m, j]      = sum_k A[j,k] x[m,k]          (the unscaled down-projection)
+ *   grad_B[n, j] = s * sum_m grad_h[m,n] t[m,j]
+ *   u[m, j]      = sum_n grad_h[m,n] B[n,j]
+ *   grad_A[j, k] = s * sum_m u[m,j] x[m,k]
+ * with s = fl32(alpha / r). x is M x k, grad_h M x n, A r x k, B n x r (bf16
+ * bits); grad_A (r x k) and grad_B (n x r) are fp64, all sums in fp64 in plain
+ * loop order. */
+void or_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, int64_t k,
+                   const uint16_t *A, const uint16_t *B, int r, float alpha, double *grad_A,
+                   double *grad_B) {
+    double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    double *t = (double *)malloc(sizeof(double) * (size_t)(M * (r > 0 ? r : 1) + 1));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(M * (r > 0 ? r : 1) + 1));
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int j = 0; j < r; ++j) {
+            double ta = 0.0, ua = 0.0;
+            for (int64_t kk = 0; kk < k; ++kk)
+                ta += bf16_bits_to_float(A[j * k + kk]) * (double)bf16_bits_to_float(x[m * k + kk]);
+            for (int64_t nn = 0; nn < n; ++nn)
+                ua += bf16_bits_to_float(gh[m * n + nn]) * (double)bf16_bits_to_float(B[nn * r + j]);
+            t[m * r + j] = ta;
+            u[m * r + j] = ua;
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t nn = 0; nn < n; ++nn)
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += bf16_bits_to_float(gh[m * n + nn]) * t[m * r + j];
+            grad_B[nn * r + j] = s * acc;
+        }
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < r; ++j)
+        for (int64_t kk = 0; kk < k; ++kk) {
+            double acc = 0.0;
+            for (int64_t m = 0; m < M; ++m) acc += u[m * r + j] * bf16_bits_to_float(x[m * k + kk]);
+            grad_A[(int64_t)j * k + kk] = s * acc;
+        }
+    free(u);
+    free(t);
+}
+
+/* ------------------------------------------------------------------ merge */
+
+/* fp64 -> bf16, round to nearest, ties to even, in one step (no fp32 on the way);
+ * finite inputs, overflow to infinity, bf16 subnormals kept. */
+uint16_t or_f64_to_bf16(double v) {
+    uint16_t sign = (v < 0.0 || (v == 0.0 && signbit(v))) ? 0x8000 : 0x0000;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    /* a = f * 2^e with f in [1, 2) */
+    int e;
+    double f = frexp(a, &e) * 2.0;
+    e -= 1;
+    if (e < -126) { /* subnormal range of bf16: units of 2^-133 */
+        double units = ldexp(a, 133);
+        double fl = floor(units), rem = units - fl;
+        uint32_t m = (uint32_t)fl;
+        if (rem > 0.5 || (rem == 0.5 && (m & 1u))) m += 1;
+        return (uint16_t)(sign | m); /* m == 128 becomes the smallest normal */
+    }
+    double scaled = ldexp(f, 7); /* in [128, 256) */
+    double fl = floor(scaled), rem = scaled - fl;
+    uint32_t m = (uint32_t)fl;
+    if (rem > 0.5 || (rem == 0.5 && (m & 1u))) m += 1;
+    if (m == 256) {
+        m = 128;
+        e += 1;
+    }
+    if (e > 127) return (uint16_t)(sign | 0x7f80);
+    return (uint16_t)(sign | ((uint32_t)(e + 127) << 7) | (m - 128));
+}
+
+/* W_merged[n, k] = bf16_rn( W'32[n,k] + s * sum_j B[n,j] A[j,k] ):
+ * W'32 = fl32(T[code] * c'_b), the dequantised weight as or_nf4_dequant rounds it to
+ * fp32, the adapter sum exact in fp64 (r products of bf16 values), one rounding of
+ * the fp64 total to bf16. A (r x k), B (n x r) bf16 bits; r == 0 gives the plain
+ * dequantised weight. */
+void or_merge_bf16(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
+                   int64_t k, const uint16_t *A, const uint16_t *B, int r, float alpha, uint16_t *out) {
+    int64_t nb = or_num_blocks(n, k);
+    float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    block_constants(q, sigma, mu, nb, cp);
+    double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+#pragma omp parallel for schedule(static)
+    for (int64_t nn = 0; nn < n; ++nn)
+        for (int64_t kk = 0; kk < k; ++kk) {
+            int64_t e = nn * k + kk;
+            float w = (float)OR_NF4[code_at(codes, e)] * cp[e / OR_BLOCK];
+            double ad = 0.0;
+            for (int j = 0; j < r; ++j)
+                ad += (double)bf16_bits_to_float(B[nn * r + j]) * (double)bf16_bits_to_float(A[(int64_t)j * k + kk]);
+            out[e] = or_f64_to_bf16((double)w + s * ad);
+        }
     free(cp);
 }

@@ -70,6 +70,10 @@ def _load():
         lib.or_qlora_fwd.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, i64, P, P,
                                      ctypes.c_int, ctypes.c_float, P]
         lib.or_qlora_bwd_x.argtypes = lib.or_qlora_fwd.argtypes
+        lib.or_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P, P]
+        lib.or_f64_to_bf16.argtypes = [ctypes.c_double]
+        lib.or_f64_to_bf16.restype = ctypes.c_uint16
+        lib.or_merge_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P]
         _lib = lib
         return lib
 
@@ -196,3 +200,31 @@ def qlora_bwd_x(qw: dict, n: int, k: int, gh_bits: np.ndarray, m: int, A_bits, B
     _load().or_qlora_bwd_x(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
                            _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(gx))
     return gx.reshape(rows.size, k)
+
+
+def lora_grads(x_bits: np.ndarray, gh_bits: np.ndarray, m: int, n: int, k: int, A_bits, B_bits, r: int,
+               alpha: float):
+    """(grad_A (r x k), grad_B (n x r)) in fp64 for all m token rows of x (m x k) and grad_h (m x n)."""
+    x = _bits16(x_bits).reshape(-1)
+    g = _bits16(gh_bits).reshape(-1)
+    assert x.size == m * k and g.size == m * n
+    A = _bits16(A_bits).reshape(-1)
+    B = _bits16(B_bits).reshape(-1)
+    gA = np.zeros(r * k, dtype=np.float64)
+    gB = np.zeros(n * r, dtype=np.float64)
+    _load().or_lora_grads(_ptr(x), _ptr(g), m, n, k, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(gA), _ptr(gB))
+    return gA.reshape(r, k), gB.reshape(n, r)
+
+
+def f64_to_bf16(v: float) -> int:
+    return int(_load().or_f64_to_bf16(float(v)))
+
+
+def merge_bf16(qw: dict, n: int, k: int, A_bits, B_bits, r: int, alpha: float) -> np.ndarray:
+    """bf16 bits (n x k) of the merged weight W' + s B A."""
+    A = _bits16(A_bits).reshape(-1) if r > 0 else None
+    B = _bits16(B_bits).reshape(-1) if r > 0 else None
+    out = np.zeros(n * k, dtype=np.uint16)
+    _load().or_merge_bf16(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
+                          _ptr(A), _ptr(B), int(r), float(alpha), _ptr(out))
+    return out.reshape(n, k)

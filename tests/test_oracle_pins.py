@@ -500,3 +500,139 @@ def test_dequant_reconstructs_weights(oracle, n, k):
     d16 = oracle.nf4_dequant_bf16(qw, n, k).reshape(-1)
     f16 = (d16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.all(np.abs(f16 - wf) <= bound + np.abs(d64) * 2.0 ** -8)
+
+
+# ------------------------------------------------------ adapter weight gradients
+# [aivaro] 2 and 7: W is frozen, only B and A are trained; their gradients are the
+# derivatives of h = W'x + s B (A x). The pins below compare or_lora_grads with the
+# forward oracle (h is linear in B and in A), with numpy on tiny shapes, and with the
+# per-token decomposition.
+
+def _grads(oracle, n, k, m, r, alpha, seed):
+    qw, A, B, x, gh = _layer(oracle, n, k, m, r, seed)
+    gA, gB = oracle.lora_grads(_bits(x), _bits(gh), m, n, k, _bits(A), _bits(B), r, alpha)
+    return qw, A, B, x, gh, gA, gB
+
+
+@pytest.mark.parametrize("alpha,r", [(8.0, 4), (32.0, 16), (16.0, 64)])
+def test_grad_B_is_adjoint_of_forward_in_B(oracle, alpha, r):
+    n, k, m = 48, 192, 5
+    qw, A, B, x, gh, gA, gB = _grads(oracle, n, k, m, r, alpha, 70 + r)
+    B2 = (torch.randn(n, r, generator=torch.Generator().manual_seed(5 + r)) * 0.01).to(torch.bfloat16)
+    h1 = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    h2 = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B2), r, alpha)
+    lhs = np.sum(gh.double().numpy() * (h2 - h1))
+    rhs = np.sum(gB * (B2.double().numpy() - B.double().numpy()))
+    assert abs(lhs - rhs) <= 1e-10 * (abs(lhs) + 1e-300) + 1e-13
+
+
+@pytest.mark.parametrize("alpha,r", [(8.0, 4), (32.0, 16), (16.0, 64)])
+def test_grad_A_is_adjoint_of_forward_in_A(oracle, alpha, r):
+    n, k, m = 48, 192, 5
+    qw, A, B, x, gh, gA, gB = _grads(oracle, n, k, m, r, alpha, 80 + r)
+    A2 = (torch.randn(r, k, generator=torch.Generator().manual_seed(9 + r)) * 0.01).to(torch.bfloat16)
+    h1 = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    h2 = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A2), _bits(B), r, alpha)
+    lhs = np.sum(gh.double().numpy() * (h2 - h1))
+    rhs = np.sum(gA * (A2.double().numpy() - A.double().numpy()))
+    assert abs(lhs - rhs) <= 1e-10 * (abs(lhs) + 1e-300) + 1e-13
+
+
+def test_lora_grads_match_numpy_on_tiny_shapes(oracle):
+    n, k, m, r, alpha = 16, 64, 3, 4, 8.0
+    qw, A, B, x, gh, gA, gB = _grads(oracle, n, k, m, r, alpha, 91)
+    s = alpha / r
+    xd, gd, Ad, Bd = (t.double().numpy() for t in (x, gh, A, B))
+    np.testing.assert_allclose(gB, s * gd.T @ (xd @ Ad.T), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(gA, s * (gd @ Bd).T @ xd, rtol=1e-12, atol=1e-15)
+
+
+def test_lora_grads_sum_over_tokens(oracle):
+    # the gradients of a batch are the sums of the per-token gradients
+    n, k, m, r, alpha = 32, 128, 4, 8, 16.0
+    qw, A, B, x, gh, gA, gB = _grads(oracle, n, k, m, r, alpha, 92)
+    sA, sB = np.zeros_like(gA), np.zeros_like(gB)
+    for i in range(m):
+        a1, b1 = oracle.lora_grads(_bits(x[i:i + 1]), _bits(gh[i:i + 1]), 1, n, k, _bits(A), _bits(B), r, alpha)
+        sA += a1
+        sB += b1
+    np.testing.assert_allclose(gA, sA, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(gB, sB, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------------------------------- merge
+# [codex] 3.6 merge_and_unload: the adapter is folded into a 16-bit weight W' + s B A
+# ([tqpw] Introduction: it cannot stay NF4).
+
+def test_f64_to_bf16_is_nearest_even(oracle):
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([rng.standard_normal(3000) * 10.0 ** rng.integers(-40, 38, 3000),
+                           np.ldexp(1.0 + np.arange(1, 256) / 256.0 + 2.0 ** -9, 0),  # exact ties
+                           [2.0 ** -133, 2.0 ** -134, 3.0 * 2.0 ** -134, 1e-45, 3.39e38, -0.0, 0.0]])
+    for v in vals:
+        b = oracle.f64_to_bf16(float(v))
+        got = float(np.array([b << 16], dtype=np.uint32).view(np.float32)[0])
+        # brute force: the two bf16 neighbours of v (truncation and the next one up in magnitude)
+        t32 = np.array([v], dtype=np.float64)
+        lo_bits = int(np.float32(v).view(np.uint32)) >> 16 if np.isfinite(np.float32(v)) else None
+        if lo_bits is None:
+            continue
+        cands = set()
+        for d in (-1, 0, 1):
+            c = (lo_bits + d) & 0xffff
+            f = float(np.array([c << 16], dtype=np.uint32).view(np.float32)[0])
+            if np.isfinite(f) and (f == 0 or np.sign(f) == np.sign(v) or v == 0):
+                cands.add((abs(f - v), c & 1, c, f))
+        best = min(cands)
+        ties = [c for c in cands if c[0] == best[0]]
+        want = min(ties, key=lambda c: c[1])[3] if len(ties) > 1 else best[3]
+        assert got == want or (got == 0 and want == 0), (v, got, want)
+        del t32
+
+
+def test_f64_to_bf16_matches_torch_on_fp32_values(oracle):
+    # for values exact in fp32 the one-step rounding equals torch's fp32 -> bf16 rounding
+    x = torch.randn(4000, dtype=torch.float32) * 3.0
+    want = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.f64_to_bf16(float(v)) for v in x.numpy()], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_merge_without_adapter_is_the_dequantised_weight(oracle):
+    n, k, m, r = 24, 192, 1, 4
+    qw, A, B, x, _ = _layer(oracle, n, k, m, r, 93, zero_b=True)
+    merged = oracle.merge_bf16(qw, n, k, _bits(A), _bits(B), r, 8.0)
+    assert np.array_equal(merged, oracle.nf4_dequant_bf16(qw, n, k))
+    assert np.array_equal(oracle.merge_bf16(qw, n, k, None, None, 0, 0.0), oracle.nf4_dequant_bf16(qw, n, k))
+
+
+def test_merge_of_zero_base_is_rounded_scaled_product(oracle):
+    n, k, m, r, alpha = 20, 128, 1, 8, 16.0
+    qw, A, B, x, _ = _layer(oracle, n, k, m, r, 94, zero_w=True)
+    merged = oracle.merge_bf16(qw, n, k, _bits(A), _bits(B), r, alpha)
+    prod = (alpha / r) * (B.double().numpy() @ A.double().numpy())
+    # r products of bf16 values sum exactly in fp64 here, so numpy's order cannot change them
+    want = np.array([oracle.f64_to_bf16(float(v)) for v in prod.reshape(-1)], dtype=np.uint16).reshape(n, k)
+    assert np.array_equal(merged, want)
+
+
+def test_merged_weight_reproduces_the_forward_pass(oracle):
+    # x W_merged^T agrees with the oracle forward within the bf16 rounding of the merged weight
+    n, k, m, r, alpha = 40, 256, 3, 16, 32.0
+    qw, A, B, x, _ = _layer(oracle, n, k, m, r, 95)
+    merged = oracle.merge_bf16(qw, n, k, _bits(A), _bits(B), r, alpha)
+    Wm = (merged.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    h = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    hm = x.double().numpy() @ Wm.T
+    bound = 2.0 ** -8 * (np.abs(x.double().numpy()) @ np.abs(Wm).T) + 1e-12
+    assert np.all(np.abs(h - hm) <= bound)
+
+
+def test_f64_to_bf16_overflow_threshold(oracle):
+    # IEEE round to nearest: magnitudes from max_finite + half an ulp up overflow to infinity
+    mx = (2.0 - 2.0 ** -7) * 2.0 ** 127
+    half = 2.0 ** 119
+    assert oracle.f64_to_bf16(mx) == 0x7f7f
+    assert oracle.f64_to_bf16(mx + half * 0.999) == 0x7f7f
+    assert oracle.f64_to_bf16(mx + half) == 0x7f80  # tie: the even neighbour is 2^128 -> inf
+    assert oracle.f64_to_bf16(-(mx + 2 * half)) == 0xff80
