@@ -4,10 +4,10 @@ The computation lives in ``libqlora_nf4.so`` (C ABI: ``include/qlora_nf4.h``); t
 ``binding`` module marshals torch tensors into it. Importing the package does not load
 the library; the first call does, and fails loudly if it is missing.
 """
-from .binding import (NF4Weight, QNError, linear_workspace_size, launch_count, load, nf4_dequantize,
+from .binding import (NF4Weight, QNError, linear_workspace_size, launch_count, load, new_workspace, nf4_dequantize,
                       nf4_quantize, nf4_quantize_static_ws, qlora_linear_bwd_x, qlora_linear_fwd,
-                      quantize_workspace_size, sizes)
+                      qlora_lora_grads, qlora_merge_bf16, quantize_workspace_size, sizes, workspace_check)
 
-__all__ = ["NF4Weight", "QNError", "linear_workspace_size", "launch_count", "load", "nf4_dequantize",
+__all__ = ["NF4Weight", "QNError", "linear_workspace_size", "launch_count", "load", "new_workspace", "nf4_dequantize",
            "nf4_quantize", "nf4_quantize_static_ws", "qlora_linear_bwd_x", "qlora_linear_fwd",
-           "quantize_workspace_size", "sizes"]
+           "qlora_lora_grads", "qlora_merge_bf16", "quantize_workspace_size", "sizes", "workspace_check"]

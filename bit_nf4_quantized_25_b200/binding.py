@@ -16,11 +16,12 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 
-QN_OK, QN_EINVAL, QN_ESHAPE, QN_EALIGN, QN_ECUDA, QN_EWORKSPACE = range(6)
+QN_OK, QN_EINVAL, QN_ESHAPE, QN_EALIGN, QN_ECUDA, QN_EWORKSPACE, QN_ETIMEOUT = range(7)
 BLOCK, GROUP, MAX_RANK = 64, 256, 256
 
 EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
-            "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x", "qn_status_string",
+            "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x",
+            "qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qn_status_string",
             "qn_last_error", "qn_launch_count")
 
 
@@ -59,10 +60,15 @@ def load(path: str | None = None):
         lib.nf4_dequantize.argtypes = [W, P, P]
         lib.nf4_quantize_static_ws.argtypes = [P, W, P]
         lib.qlora_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, sz]
+        lib.qlora_workspace_check.argtypes = [P, P]
         lib.qlora_linear_fwd.argtypes = [W, P, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, ctypes.c_size_t, P]
         lib.qlora_linear_bwd_x.argtypes = lib.qlora_linear_fwd.argtypes
-        for f in ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
-                  "qlora_workspace_size", "qlora_linear_fwd", "qlora_linear_bwd_x"):
+        lib.qlora_merge_bf16.argtypes = [W, P, P, ctypes.c_int, ctypes.c_float, P, P]
+        lib.qlora_lora_grads_workspace_size.argtypes = [i64, ctypes.c_int, sz]
+        lib.qlora_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, P,
+                                         ctypes.c_size_t, P]
+        for f in ("qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
+                  "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x"):
             getattr(lib, f).restype = st
         lib.qn_status_string.argtypes = [st]
         lib.qn_status_string.restype = ctypes.c_char_p
@@ -123,10 +129,22 @@ def check_linear_shapes(n_out: int, k_in: int, act: torch.Tensor, A, B, out, bwd
     return r
 
 
+def new_workspace(need: int, device="cuda") -> torch.Tensor:
+    """A linear-layer workspace of `need` bytes with its error word zeroed (see
+    qlora_workspace_size in the header); reusable across calls in stream order."""
+    return torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
+
+
+def workspace_check(ws: torch.Tensor, stream=None):
+    """Raise QNError(QN_ETIMEOUT) if a kernel that used `ws` gave up a bounded wait since the last
+    check (the error word is then cleared); synchronises the stream."""
+    _check(load().qlora_workspace_check(_ptr(ws), _stream(stream)), "qlora_workspace_check")
+
+
 def _workspace(ws: torch.Tensor | None, need: int, device) -> tuple[torch.Tensor, int]:
     """A caller workspace (contiguous CUDA memory, any dtype) or a fresh one; its size in bytes."""
     if ws is None:
-        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+        ws = new_workspace(need, device)
     elif not ws.is_cuda or not ws.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     return ws, ws.numel() * ws.element_size()
@@ -274,3 +292,67 @@ def qlora_linear_bwd_x(w: NF4Weight, grad_h: torch.Tensor, A: torch.Tensor | Non
                                      _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
            "qlora_linear_bwd_x")
     return out
+
+
+def qlora_merge_bf16(w: NF4Weight, A: torch.Tensor | None, B: torch.Tensor | None, alpha: float,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W' + (alpha/r) B A as a bf16 n_out x k_in tensor (merge and unload)."""
+    if (A is None) != (B is None):
+        raise ValueError("A and B are given together or not at all")
+    r = 0
+    if A is not None:
+        _dev_bf16(A, "A")
+        _dev_bf16(B, "B")
+        if A.dim() != 2:
+            raise ValueError("A must be 2-D (r x k_in)")
+        r = A.shape[0]
+        _expect_shape(A, (r, w.k_in), "A")
+        _expect_shape(B, (w.n_out, r), "B")
+    out = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    _dev_bf16(out, "out")
+    _expect_shape(out, (w.n_out, w.k_in), "out")
+    _same_device(w, A, B, out)
+    cw = w.c_struct()
+    _check(load().qlora_merge_bf16(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(out), _stream(stream)),
+           "qlora_merge_bf16")
+    return out
+
+
+def lora_grads_workspace_size(M: int, r: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().qlora_lora_grads_workspace_size(M, r, ctypes.byref(v)), "qlora_lora_grads_workspace_size")
+    return v.value
+
+
+def qlora_lora_grads(x: torch.Tensor, grad_h: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     grad_A: torch.Tensor | None = None, grad_B: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """(grad_A (r x k_in), grad_B (n_out x r)) in fp32 for x (M x k_in) and grad_h (M x n_out)."""
+    for t, nm in ((x, "x"), (grad_h, "grad_h"), (A, "A"), (B, "B")):
+        _dev_bf16(t, nm)
+    if x.dim() != 2 or grad_h.dim() != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError("x, grad_h, A and B must be 2-D")
+    M, k = x.shape
+    n = grad_h.shape[1]
+    r = A.shape[0]
+    _expect_shape(grad_h, (M, n), "grad_h")
+    _expect_shape(A, (r, k), "A")
+    _expect_shape(B, (n, r), "B")
+    f32 = dict(dtype=torch.float32, device=x.device)
+    grad_A = grad_A if grad_A is not None else torch.empty(r, k, **f32)
+    grad_B = grad_B if grad_B is not None else torch.empty(n, r, **f32)
+    for t, shp, nm in ((grad_A, (r, k), "grad_A"), (grad_B, (n, r), "grad_B")):
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous fp32 CUDA tensor")
+        _expect_shape(t, shp, nm)
+    if workspace is None:
+        workspace = torch.empty(max(lora_grads_workspace_size(M, r), 256), dtype=torch.uint8, device=x.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    for t in (grad_h, A, B, grad_A, grad_B, workspace):
+        if t.device != x.device:
+            raise ValueError(f"tensor on {t.device}, x is on {x.device}")
+    _check(load().qlora_lora_grads(_ptr(x), _ptr(grad_h), M, n, k, _ptr(A), _ptr(B), r, float(alpha), _ptr(grad_A),
+                                   _ptr(grad_B), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream)), "qlora_lora_grads")
+    return grad_A, grad_B

@@ -90,6 +90,7 @@ const char *qn_status_string(qn_status s) {
         case QN_EALIGN: return "misaligned pointer";
         case QN_ECUDA: return "CUDA error";
         case QN_EWORKSPACE: return "workspace missing or too small";
+        case QN_ETIMEOUT: return "a kernel gave up a bounded wait";
     }
     return "unknown status";
 }
@@ -172,6 +173,55 @@ qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream) {
                        "nf4_dequantize");
 }
 
+qn_status qlora_merge_bf16(const qn_nf4_weight *w, const void *A, const void *B, int r, float alpha, void *W_out,
+                           void *stream) {
+    qn_status s = check_weight(w);
+    if (s != QN_OK) return s;
+    s = check_lora(A, B, r, alpha);
+    if (s != QN_OK) return s;
+    if (w->n_out == 0 || w->k_in == 0) return QN_OK;
+    if (!W_out) return fail(QN_EINVAL, "null W_out");
+    if (!aligned16(W_out)) return fail(QN_EALIGN, "W_out not 16-byte aligned");
+    if (W_out == A || W_out == B) return fail(QN_EINVAL, "W_out aliases an adapter factor");
+    const float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
+    return cuda_status(launch_merge(view(w), static_cast<const uint16_t *>(A), static_cast<const uint16_t *>(B), r, sc,
+                                    static_cast<uint16_t *>(W_out), static_cast<cudaStream_t>(stream)),
+                       "qlora_merge_bf16");
+}
+
+qn_status qlora_lora_grads_workspace_size(int64_t M, int r, size_t *ws_bytes) {
+    if (!ws_bytes) return fail(QN_EINVAL, "null output pointer");
+    if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
+    if (r < 1 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [1, %d]", r, QN_MAX_RANK);
+    *ws_bytes = lora_grads_workspace_bytes(M, r);
+    g_err.clear();
+    return QN_OK;
+}
+
+qn_status qlora_lora_grads(const void *x, const void *grad_h, int64_t M, int64_t n_out, int64_t k_in, const void *A,
+                           const void *B, int r, float alpha, float *grad_A, float *grad_B, void *ws, size_t ws_bytes,
+                           void *stream) {
+    qn_status s = check_shape(n_out, k_in);
+    if (s != QN_OK) return s;
+    if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
+    if (r < 1 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [1, %d]", r, QN_MAX_RANK);
+    s = check_lora(A, B, r, alpha);
+    if (s != QN_OK) return s;
+    if (!grad_A || !grad_B) return fail(QN_EINVAL, "null gradient output");
+    if (n_out == 0 || k_in == 0) return QN_OK;
+    if (M > 0 && (!x || !grad_h)) return fail(QN_EINVAL, "null activation pointer");
+    if (M > 0 && (!aligned16(x) || !aligned16(grad_h))) return fail(QN_EALIGN, "x or grad_h not 16-byte aligned");
+    const size_t need = lora_grads_workspace_bytes(M, r);
+    if (!ws || ws_bytes < need) return fail(QN_EWORKSPACE, "adapter-gradient workspace needs %zu bytes", need);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
+    const float sc = alpha / static_cast<float>(r);
+    return cuda_status(launch_lora_grads(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(grad_h), M,
+                                         n_out, k_in, static_cast<const uint16_t *>(A),
+                                         static_cast<const uint16_t *>(B), r, sc, grad_A, grad_B, ws,
+                                         static_cast<cudaStream_t>(stream)),
+                       "qlora_lora_grads");
+}
+
 qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, size_t *ws_bytes) {
     if (!ws_bytes) return fail(QN_EINVAL, "null output pointer");
     qn_status s = check_shape(n_out, k_in);
@@ -180,7 +230,7 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
     if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
     // The few-token kernels need no workspace (256 bytes keep the pointer non-null); the
     // tensor-core path stores its error word and the adapter operand there.
-    *ws_bytes = M > kDecodeMaxM ? gemm_workspace_bytes(M, r) : 256;
+    *ws_bytes = (M > kDecodeMaxM || r > kDecodeMaxRank) ? gemm_workspace_bytes(M, r) : 256;
     g_err.clear();
     return QN_OK;
 }
@@ -202,6 +252,22 @@ static qn_status check_linear(const qn_nf4_weight *w, const void *in, int64_t M,
     return QN_OK;
 }
 
+qn_status qlora_workspace_check(void *ws, void *stream) {
+    if (!ws) return fail(QN_EINVAL, "null workspace");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_status(e, "qlora_workspace_check");
+    if (word == 0) return cuda_status(cudaSuccess, "");
+    e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_status(e, "qlora_workspace_check");
+    return fail(QN_ETIMEOUT,
+                "a kernel that used this workspace gave up a bounded wait (error word %d); its output is incomplete",
+                word);
+}
+
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B, int r,
                            float alpha, void *h, void *ws, size_t ws_bytes, void *stream) {
     qn_status s = check_linear(w, x, M, A, B, r, alpha, h, ws, ws_bytes);
@@ -213,16 +279,19 @@ qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, con
     const uint16_t *xp = static_cast<const uint16_t *>(x);
     uint16_t *hp = static_cast<uint16_t *>(h);
     const uint16_t *Ap = static_cast<const uint16_t *>(A), *Bp = static_cast<const uint16_t *>(B);
-    if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, false)) {
-        if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
-        return cuda_status(launch_gemm_fwd(wv, xp, M, Ap, Bp, r, sc, hp, ws, st), "qlora_linear_fwd");
+    // few tokens and adapters of rank <= 64: the streamed kernel, 16 tokens per launch;
+    // otherwise the tensor-core GEMM (any token count; the forward operand always suits TMA)
+    if (M <= kDecodeMaxM && r <= kDecodeMaxRank) {
+        int *err = static_cast<int *>(ws);
+        for (int64_t m0 = 0; m0 < M; m0 += kDecodeTokens) {
+            const int mc = static_cast<int>(M - m0 < kDecodeTokens ? M - m0 : kDecodeTokens);
+            cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, Ap, Bp, r, sc, hp + m0 * w->n_out, err, st);
+            if (e != cudaSuccess) return cuda_status(e, "qlora_linear_fwd");
+        }
+        return cuda_status(cudaSuccess, "");
     }
-    for (int64_t m0 = 0; m0 < M; m0 += kDecodeMaxM) {
-        const int mc = static_cast<int>(M - m0 < kDecodeMaxM ? M - m0 : kDecodeMaxM);
-        cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, Ap, Bp, r, sc, hp + m0 * w->n_out, st);
-        if (e != cudaSuccess) return cuda_status(e, "qlora_linear_fwd");
-    }
-    return cuda_status(cudaSuccess, "");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
+    return cuda_status(launch_gemm_fwd(wv, xp, M, Ap, Bp, r, sc, hp, ws, st), "qlora_linear_fwd");
 }
 
 qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A, const void *B,
@@ -236,10 +305,23 @@ qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t
     const uint16_t *gp = static_cast<const uint16_t *>(grad_h);
     uint16_t *xp = static_cast<uint16_t *>(grad_x);
     const uint16_t *Ap = static_cast<const uint16_t *>(A), *Bp = static_cast<const uint16_t *>(B);
-    if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, true)) {
+    // few tokens and adapters of rank <= 64: the streamed kernel, 16 tokens per launch
+    if (M <= kDecodeMaxM && r <= kDecodeMaxRank) {
+        int *err = static_cast<int *>(ws);
+        for (int64_t m0 = 0; m0 < M; m0 += kDecodeTokens) {
+            const int mc = static_cast<int>(M - m0 < kDecodeTokens ? M - m0 : kDecodeTokens);
+            cudaError_t e =
+                launch_decode_bwd_stream(wv, gp + m0 * w->n_out, mc, Ap, Bp, r, sc, xp + m0 * w->k_in, err, st);
+            if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
+        }
+        return cuda_status(cudaSuccess, "");
+    }
+    if (gemm_supported(w->n_out, w->k_in, M, true)) {
         if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
         return cuda_status(launch_gemm_bwd(wv, gp, M, Ap, Bp, r, sc, xp, ws, st), "qlora_linear_bwd_x");
     }
+    // many tokens with n_out % 8 != 0 (the GEMM's TMA row-stride rule), or few tokens with a rank
+    // above 64: the earlier few-token kernel in chunks of 32 tokens
     constexpr int kChunk = 32;
     for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
         const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);

@@ -9,6 +9,7 @@
 // lanes of a block load the same constant inputs), looks the values up in a 16-entry shared
 // table and writes 16 bytes of bf16, so every warp load and store is fully contiguous.
 #include "common.cuh"
+#include "host_cache.h"
 #include "kernels.h"
 
 namespace qn {
@@ -53,15 +54,11 @@ k_dequant(const uint32_t *__restrict__ codes, const uint8_t *__restrict__ q, con
 cudaError_t launch_dequant(const WeightView &w, uint16_t *out, cudaStream_t s) {
     const int64_t n_words = w.n * w.k / 8;  // 4 bytes of codes each
     if (n_words == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    static int occ = 0;  // resident CTAs per SM
-    if (occ == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_dequant, kDeqThreads, 0) != cudaSuccess ||
-                     occ <= 0)) {
-        (void)cudaGetLastError();
-        occ = 4;
-    }
+    int sms = 148, occ = 4;
+    cudaError_t e = device_sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    e = resident_ctas(reinterpret_cast<const void *>(k_dequant), kDeqThreads, 0, &occ);
+    if (e != cudaSuccess) return e;
     int64_t grid = (n_words + 2 * kDeqThreads - 1) / (2 * kDeqThreads);
     const int64_t cap = static_cast<int64_t>(sms) * occ;  // one wave
     if (grid > cap) grid = cap;

@@ -582,13 +582,11 @@ cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, c
     int *err = static_cast<int *>(ws);
     uint16_t *t = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
     const int RT = (r + 63) / 64 * 64;
-    cudaError_t e;
+    // the error word is sticky: kernels only ever set it (qlora_workspace_check reads and clears it)
     if (r > 0) {
-        e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, err, st);
-    } else {
-        e = cudaMemsetAsync(err, 0, sizeof(int), st);
+        cudaError_t e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, st);
+        if (e != cudaSuccess) return e;
     }
-    if (e != cudaSuccess) return e;
     return launch_gemm_impl<false>(w, x, M, B, r, t, RT, h, err, st);
 }
 
@@ -597,13 +595,10 @@ cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, 
     int *err = static_cast<int *>(ws);
     uint16_t *u = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
     const int RT = (r + 63) / 64 * 64;
-    cudaError_t e;
     if (r > 0) {
-        e = launch_lora_down(gh, M, w.n, B, 1, r, r, s, u, RT, err, st);
-    } else {
-        e = cudaMemsetAsync(err, 0, sizeof(int), st);
+        cudaError_t e = launch_lora_down(gh, M, w.n, B, 1, r, r, s, u, RT, st);
+        if (e != cudaSuccess) return e;
     }
-    if (e != cudaSuccess) return e;
     return launch_gemm_impl<true>(w, gh, M, A, r, u, RT, gx, err, st);
 }
 

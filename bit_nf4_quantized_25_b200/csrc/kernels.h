@@ -38,20 +38,39 @@ cudaError_t static_scratch_address(void **out);
 // nf4_dequantize.
 cudaError_t launch_dequant(const WeightView &w, uint16_t *out, cudaStream_t s);
 
-// Token-count bound of the decode kernels (M <= kDecodeMaxM).
-constexpr int kDecodeMaxM = 64;
+// qlora_merge_bf16: out = bf16(fl32(NF4[code] c'_b) + s B A), A r x k, B n x r (r may be 0).
+cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *out,
+                         cudaStream_t st);
 
-// h = dequant(W) x + s B (A x) for M <= kDecodeMaxM tokens, one launch.
+// Token-count bound of the few-token path (M <= kDecodeMaxM tokens go there; the forward
+// kernel takes kDecodeTokens tokens per launch and adapters of rank <= kDecodeMaxRank).
+constexpr int kDecodeMaxM = 64;
+constexpr int kDecodeTokens = 16;
+constexpr int kDecodeMaxRank = 64;
+
+// h = dequant(W) x + s B (A x) for M <= kDecodeTokens tokens and r <= kDecodeMaxRank, one
+// launch; a timeout of a bounded wait is recorded in *err.
 cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A,
-                              const uint16_t *B, int r, float s, uint16_t *h, cudaStream_t st);
+                              const uint16_t *B, int r, float s, uint16_t *h, int *err, cudaStream_t st);
+// grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h), streamed kernel: M <= kDecodeTokens tokens,
+// r <= kDecodeMaxRank, one launch; a timeout of a bounded wait is recorded in *err.
+cudaError_t launch_decode_bwd_stream(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
+                                     const uint16_t *B, int r, float s, uint16_t *gx, int *err, cudaStream_t st);
 // grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h) for M <= kDecodeMaxM tokens.
 cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
                               const uint16_t *B, int r, float s, uint16_t *gx, cudaStream_t st);
 
 // Adapter down-projection for many tokens: out[m, j] = bf16(s * sum_i act[m,i] S(j,i)),
-// S(j,i) = small[j*ldj + i*ldk]; out is M x RT with zeros for j >= r. Clears *err.
+// S(j,i) = small[j*ldj + i*ldk]; out is M x RT with zeros for j >= r.
 cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
-                             int64_t ldk, int r, float s, uint16_t *out, int RT, int *err, cudaStream_t st);
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st);
+
+// Gradients of the adapter weights (fp32): grad_A (r x k), grad_B (n x r); workspace of
+// lora_grads_workspace_bytes(M, r) bytes holds t = x A^T and u = grad_h B (bf16).
+size_t lora_grads_workspace_bytes(int64_t M, int r);
+cudaError_t launch_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, int64_t k,
+                              const uint16_t *A, const uint16_t *B, int r, float s, float *grad_A, float *grad_B,
+                              void *ws, cudaStream_t st);
 
 // tcgen05 fused dequant-GEMM for many tokens (the LoRA down-projection runs first, into
 // the workspace). Workspace: a 256-byte header (error word) then the M x RT adapter operand.

@@ -7,7 +7,7 @@
 //
 // HBM-bound on the activations (read once). One CTA = 16 tokens; its 4 warps split the
 // reduction, each running mma.sync m16n8k16 (tokens x adapter rank), and reduce through
-// shared memory. Thread 0 of CTA 0 also clears the GEMM's error word.
+// shared memory in a fixed order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,13 +26,20 @@ struct LoraDownParams {
     float s;
     uint16_t *out;  // M x RT
     int RT;
-    int *err;
 };
 
-template <int NT>  // 8*NT adapter columns per pass
+// bf16 pair (v[i], v[i + 1]); kEven: i is even and v 4-byte aligned, so one 4-byte load.
+template <bool kEven>
+__device__ __forceinline__ uint32_t load_pair(const uint16_t *v) {
+    if (kEven) return ld_ro_u32(v);
+    return static_cast<uint32_t>(ld_ro_u16(v)) | (static_cast<uint32_t>(ld_ro_u16(v + 1)) << 16);
+}
+
+// kEven: the reduction length (the activation row stride) is even, so every activation pair
+// and every pair of a row-major small operand is 4-byte aligned.
+template <int NT, bool kEven>  // 8*NT adapter columns per pass
 __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParams p) {
     __shared__ float red[kLdWarps][16][8 * NT];
-    if (blockIdx.x == 0 && threadIdx.x == 0 && p.err) *p.err = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 16;
@@ -40,7 +47,7 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
     const bool vA = rowA < p.M, vB = rowB < p.M;
     const uint16_t *aA = p.act + (vA ? rowA : 0) * p.red;
     const uint16_t *aB = p.act + (vB ? rowB : 0) * p.red;
-    const int64_t steps = (p.red + 15) / 16;  // red is even; a partial last step reads zeros
+    const int64_t steps = (p.red + 15) / 16;  // a partial last step reads zeros
     const int64_t s_lo = steps * warp / kLdWarps, s_hi = steps * (warp + 1) / kLdWarps;
 
     for (int j0 = 0; j0 < p.RT; j0 += 8 * NT) {
@@ -51,10 +58,16 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
             for (int64_t st = s_lo; st < s_hi; ++st) {
                 const int64_t k0 = st * 16;
                 const bool lo_ok = k0 + 2 * t < p.red, hi_ok = k0 + 2 * t + 8 < p.red;
-                const uint32_t a0 = (vA && lo_ok) ? ld_ro_u32(aA + k0 + 2 * t) : 0u;
-                const uint32_t a1 = (vB && lo_ok) ? ld_ro_u32(aB + k0 + 2 * t) : 0u;
-                const uint32_t a2 = (vA && hi_ok) ? ld_ro_u32(aA + k0 + 2 * t + 8) : 0u;
-                const uint32_t a3 = (vB && hi_ok) ? ld_ro_u32(aB + k0 + 2 * t + 8) : 0u;
+                // a pair never straddles the row end: red is even, or (odd red) the last pair is
+                // read element-wise below
+                auto pair = [&](const uint16_t *row, int64_t kk) -> uint32_t {
+                    if (kk + 1 < p.red) return load_pair<kEven>(row + kk);
+                    return kk < p.red ? static_cast<uint32_t>(ld_ro_u16(row + kk)) : 0u;
+                };
+                const uint32_t a0 = (vA && lo_ok) ? pair(aA, k0 + 2 * t) : 0u;
+                const uint32_t a1 = (vB && lo_ok) ? pair(aB, k0 + 2 * t) : 0u;
+                const uint32_t a2 = (vA && hi_ok) ? pair(aA, k0 + 2 * t + 8) : 0u;
+                const uint32_t a3 = (vB && hi_ok) ? pair(aB, k0 + 2 * t + 8) : 0u;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int j = j0 + nt * 8 + g;
@@ -62,16 +75,20 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
                     if (j < p.r) {
                         const uint16_t *sp = p.small + static_cast<int64_t>(j) * p.ldj;
                         if (p.ldk == 1) {
-                            if (lo_ok) b0 = ld_ro_u32(sp + k0 + 2 * t);
-                            if (hi_ok) b1 = ld_ro_u32(sp + k0 + 2 * t + 8);
+                            if (lo_ok) b0 = pair(sp, k0 + 2 * t);
+                            if (hi_ok) b1 = pair(sp, k0 + 2 * t + 8);
                         } else {
                             const int64_t L = p.ldk;
                             if (lo_ok)
                                 b0 = ld_ro_u16(sp + (k0 + 2 * t) * L) |
-                                     (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 1) * L)) << 16);
+                                     (k0 + 2 * t + 1 < p.red
+                                          ? static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 1) * L)) << 16
+                                          : 0u);
                             if (hi_ok)
                                 b1 = ld_ro_u16(sp + (k0 + 2 * t + 8) * L) |
-                                     (static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 9) * L)) << 16);
+                                     (k0 + 2 * t + 9 < p.red
+                                          ? static_cast<uint32_t>(ld_ro_u16(sp + (k0 + 2 * t + 9) * L)) << 16
+                                          : 0u);
                         }
                     }
                     mma_16816(d[nt], a0, a1, a2, a3, b0, b1);
@@ -107,17 +124,19 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
 }  // namespace
 
 cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
-                             int64_t ldk, int r, float s, uint16_t *out, int RT, int *err, cudaStream_t st) {
-    LoraDownParams p{act, M, red, small, ldj, ldk, r, s, out, RT, err};
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st) {
+    LoraDownParams p{act, M, red, small, ldj, ldk, r, s, out, RT};
     const unsigned grid = static_cast<unsigned>((M + 15) / 16);
+    const bool even = (red & 1) == 0;
+    auto go = [&](auto kern) { kern<<<grid, kLdWarps * 32, 0, st>>>(p); };
     if (r <= 8)
-        k_lora_down<1><<<grid, kLdWarps * 32, 0, st>>>(p);
+        even ? go(k_lora_down<1, true>) : go(k_lora_down<1, false>);
     else if (r <= 16)
-        k_lora_down<2><<<grid, kLdWarps * 32, 0, st>>>(p);
+        even ? go(k_lora_down<2, true>) : go(k_lora_down<2, false>);
     else if (r <= 32)
-        k_lora_down<4><<<grid, kLdWarps * 32, 0, st>>>(p);
+        even ? go(k_lora_down<4, true>) : go(k_lora_down<4, false>);
     else
-        k_lora_down<8><<<grid, kLdWarps * 32, 0, st>>>(p);
+        even ? go(k_lora_down<8, true>) : go(k_lora_down<8, false>);
     count_launch();
     return cudaGetLastError();
 }

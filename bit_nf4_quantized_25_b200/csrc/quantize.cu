@@ -20,8 +20,10 @@
 // The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
+#include "host_cache.h"
 #include "kernels.h"
 
 namespace qn {
@@ -299,24 +301,35 @@ __device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
 
 size_t static_scratch_bytes() { return kStaticScratchBytes; }
 
-// Device address of g_quant_scratch on the current device. The symbol's host-side name is not
-// a device address, so it is resolved with cudaGetSymbolAddress, once per device (with that
-// device current), and cached.
+// Device address of g_quant_scratch in the current context. The symbol's host-side name is not
+// a device address, so it is resolved with cudaGetSymbolAddress (with the device current) and
+// cached per context: a device reset creates a new context, where the module and its array are
+// loaded again, so the address is looked up again there.
 cudaError_t static_scratch_address(void **out) {
+    struct Entry {
+        uint64_t ctx;
+        int dev;
+        void *addr;
+    };
     static std::mutex lock;
-    static void *addr[64] = {};
+    static std::vector<Entry> cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    uint64_t ctx = current_context_id();
     std::lock_guard<std::mutex> guard(lock);
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_quant_scratch);
-        if (e != cudaSuccess) return e;
-        addr[dev] = p;
-    }
-    *out = addr[dev];
+    if (ctx != 0)
+        for (const Entry &c : cache)
+            if (c.ctx == ctx && c.dev == dev) {
+                *out = c.addr;
+                return cudaSuccess;
+            }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_quant_scratch);
+    if (e != cudaSuccess) return e;
+    ctx = current_context_id();  // the lookup makes the device's primary context current
+    if (ctx != 0) cache.push_back(Entry{ctx, dev, p});
+    *out = p;
     return cudaSuccess;
 }
 
@@ -336,15 +349,11 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     auto *cblk = reinterpret_cast<float *>(static_cast<char *>(ws) + kHeaderBytes);
     cudaError_t e = cudaMemsetAsync(bins, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    static int occ = 0;  // resident CTAs per SM
-    if (occ == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_blocks, kQuantThreads, 0) != cudaSuccess ||
-                     occ <= 0)) {
-        (void)cudaGetLastError();
-        occ = 4;
-    }
+    int sms = 148, occ = 4;
+    e = device_sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    e = resident_ctas(reinterpret_cast<const void *>(k_quant_blocks), kQuantThreads, 0, &occ);
+    if (e != cudaSuccess) return e;
     // 32 blocks per CTA per pass; exactly one wave of resident CTAs, never more than needed,
     // and few enough passes per thread that the 32-bit smem bins cannot overflow.
     int64_t grid = (nb + 31) / 32;

@@ -56,7 +56,8 @@ typedef enum {
     QN_ESHAPE = 2,     /* k_in not a multiple of 64, or a size above the limits */
     QN_EALIGN = 3,     /* a tensor pointer is not 16-byte aligned               */
     QN_ECUDA = 4,      /* a CUDA launch or attribute call failed                */
-    QN_EWORKSPACE = 5  /* workspace pointer null or smaller than required       */
+    QN_EWORKSPACE = 5, /* workspace pointer null or smaller than required       */
+    QN_ETIMEOUT = 6    /* a kernel gave up a bounded wait (qlora_workspace_check) */
 } qn_status;
 
 /* Blocking of the format: one absmax per QN_BLOCK consecutive weights of the
@@ -124,7 +125,8 @@ qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t
  * every GPU that loads the library holds until the process exits; it fits weights of at most
  * 4,193,728 blocks of 64 (268,398,592 weights; 28672 x 8192 fits). Larger weights are
  * rejected with QN_EWORKSPACE before anything is enqueued.
- * Results are bit-identical to nf4_quantize. The first call on each device looks up the
+ * Results are bit-identical to nf4_quantize. The first call in each CUDA context (on each
+ * device, and again after a device reset, which loads the library's module anew) looks up the
  * scratch address (cudaGetSymbolAddress) with that device current, so make it before any
  * stream capture. Every call shares the one scratch array (the part that must start at zero is
  * cleared by each call): calls whose work overlaps on the GPU -- on different streams, or from
@@ -141,9 +143,42 @@ qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *
  * aligned), QN_ECUDA. */
 qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream);
 
+/* qlora_merge_bf16 -- fold the adapter into a 16-bit weight (merge and unload):
+ *   W_out[n, k] = bf16_rn( fl32(NF4[code] * c'_b) + s * sum_j B[n,j] A[j,k] ),  s = alpha / r.
+ * A : r x k_in bf16, B : n_out x r bf16 (r == 0: A = B = NULL, W_out is the
+ * dequantised weight); W_out : n_out x k_in bf16 (written; must not alias A or B).
+ * The adapter product is accumulated in fp32 on the tensor cores and added to
+ * the fp32 dequantised weight with one fp32 rounding before the bf16 rounding,
+ * so a result may differ from the exactly rounded sum by one bf16 unit.
+ * Source: "QLoRA & PEFT family" (ai-reference-codex) 3.6 (merge_and_unload);
+ * "QLoRA paper notes" (tqpw.cn), Introduction (the merged weight is 16-bit:
+ * it cannot be folded back into NF4).
+ * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (codes, A, B or W_out not 16-byte
+ * aligned), QN_ECUDA. */
+qn_status qlora_merge_bf16(const qn_nf4_weight *w, const void *A, const void *B, int r, float alpha, void *W_out,
+                           void *stream);
+
 /* Workspace bytes qlora_linear_fwd / qlora_linear_bwd_x need for M tokens,
- * an n_out x k_in weight and rank r (0 <= r <= 256). Host-only. */
+ * an n_out x k_in weight and rank r (0 <= r <= 256). Host-only.
+ *
+ * The linear-layer workspace: device memory of at least this many bytes,
+ * 256-byte aligned. Its first 4 bytes are an error word. Zero them when the
+ * workspace is allocated (or call qlora_workspace_check once); the kernels
+ * never clear the word, they only set it (to 1) when a bounded wait inside
+ * them runs out, in which case that call's output is incomplete. The rest of
+ * the workspace is scratch whose contents on entry do not matter. One
+ * workspace may serve any number of calls in stream order, of any shapes,
+ * as long as it is large enough for each; calls that run concurrently on the
+ * GPU need separate workspaces. */
 qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, size_t *ws_bytes);
+
+/* qlora_workspace_check -- read back and clear the workspace error word.
+ * Synchronises `stream` (the stream the calls that used `ws` ran on).
+ * Returns QN_OK when no kernel that used `ws` since the last check gave up a
+ * bounded wait, QN_ETIMEOUT (and clears the word) otherwise.
+ * No counterpart in the pages: this is the library's failure report.
+ * Errors: QN_EINVAL (null ws), QN_ECUDA, QN_ETIMEOUT. */
+qn_status qlora_workspace_check(void *ws, void *stream);
 
 /* qlora_linear_fwd -- h = dequant(W) x + (alpha/r) B (A x), per token row:
  *   h[m, n] = sum_k W'[n,k] x[m,k] + s * sum_j B[n,j] sum_k A[j,k] x[m,k].
@@ -156,8 +191,9 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
  * r == 0 means no adapter (A and B must then be NULL; alpha is ignored).
  * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), forward
  * equations; "How does QLoRA work for training?" (aivaro.ru) 2.
- * ws: device workspace of at least qlora_workspace_size() bytes, 256-byte
- * aligned, contents on entry irrelevant. M may be 0 (nothing is enqueued).
+ * ws: the linear-layer workspace (see qlora_workspace_size: at least that many
+ * bytes, 256-byte aligned, error word zeroed once). M may be 0 (nothing is
+ * enqueued).
  * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (x, h, codes, A or B not 16-byte
  * aligned), QN_EWORKSPACE, QN_ECUDA. */
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
@@ -175,6 +211,28 @@ qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, con
 qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A,
                              const void *B, int r, float alpha, void *grad_x, void *ws, size_t ws_bytes,
                              void *stream);
+
+/* Workspace bytes qlora_lora_grads needs for M tokens and rank r (1..256).
+ * Host-only. The workspace's contents on entry do not matter. */
+qn_status qlora_lora_grads_workspace_size(int64_t M, int r, size_t *ws_bytes);
+
+/* qlora_lora_grads -- gradients of the adapter weights, the only trained
+ * parameters of the layer (W is frozen):
+ *   grad_B[n, j] = s * sum_m grad_h[m,n] t[m,j],  t = x A^T        (n_out x r)
+ *   grad_A[j, k] = s * sum_m u[m,j] x[m,k],       u = grad_h B     (r x k_in)
+ * with s = alpha / r. x : M x k_in bf16, grad_h : M x n_out bf16, A : r x k_in
+ * bf16, B : n_out x r bf16; grad_A, grad_B : fp32 device buffers (written).
+ * t and u are rounded to bf16 (the tensor-core operands); all sums are fp32.
+ * Source: "How does QLoRA work for training?" (aivaro.ru) 2 (only B and A are
+ * trained) and 7 (gradients through the frozen base; only the adapters are
+ * updated); the derivatives of the forward equation of "Quantized LoRA (QLoRA)
+ * and 4-bit training" (apxml.com).
+ * ws: at least qlora_lora_grads_workspace_size() bytes, 256-byte aligned.
+ * Errors: QN_EINVAL (null pointer, r outside 1..256, alpha not finite),
+ * QN_ESHAPE, QN_EALIGN, QN_EWORKSPACE, QN_ECUDA. */
+qn_status qlora_lora_grads(const void *x, const void *grad_h, int64_t M, int64_t n_out, int64_t k_in,
+                           const void *A, const void *B, int r, float alpha, float *grad_A, float *grad_B,
+                           void *ws, size_t ws_bytes, void *stream);
 
 /* Static description of a status code. */
 const char *qn_status_string(qn_status s);

@@ -180,3 +180,13 @@ def test_binding_refuses_mismatched_linear_shapes(what):
         out = _t(M, n)
     with pytest.raises(ValueError):
         qb.check_linear_shapes(n, k, act, A, B, out, bwd=bwd)
+
+
+def test_workspace_check_rejects_null(lib):
+    # argument errors are returned before any GPU work
+    assert lib.qlora_workspace_check(None, None) == 1  # QN_EINVAL
+    assert "null workspace" in lib.qn_last_error().decode()
+
+
+def test_timeout_status_has_a_description(lib):
+    assert lib.qn_status_string(6).decode() == "a kernel gave up a bounded wait"

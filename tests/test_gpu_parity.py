@@ -192,17 +192,31 @@ def test_gemm_small(oracle, n, k, M, r):
     run_case(oracle, synth.LayerCase(f"gemm{n}x{k}M{M}r{r}", n, k, M, r, 2.0 * max(r, 1), 0.02, n * 3 + k + M))
 
 
-def test_gemm_error_word_stays_clear(oracle):
-    case = synth.LayerCase("gemm_err", 256, 512, 300, 16, 32.0, 0.02, 99)
+@pytest.mark.parametrize("M", [300, 5])
+def test_error_word_stays_clear(oracle, M):
+    # tensor-core path (M > 64) and few-token path: a run without a timeout leaves the
+    # workspace error word at zero, and qlora_workspace_check reports success
+    case = synth.LayerCase("err_word", 256, 512, M, 16, 32.0, 0.02, 99)
     W, A, B, x, gh = synth.layer_inputs(case, DEV)
     w = qb.nf4_quantize(W)
-    ws = torch.full((qb.linear_workspace_size(300, 256, 512, 16),), 0xAB, dtype=torch.uint8, device=DEV)
+    ws = qb.new_workspace(qb.linear_workspace_size(M, 256, 512, 16))
     qb.qlora_linear_fwd(w, x, A, B, 32.0, workspace=ws)
-    torch.cuda.synchronize()
-    assert int(ws[:4].view(torch.int32).item()) == 0
     qb.qlora_linear_bwd_x(w, gh, A, B, 32.0, workspace=ws)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+    qb.workspace_check(ws)
+
+
+def test_error_word_is_reported_and_cleared():
+    # a set error word (what a kernel writes when a bounded wait runs out) is reported as
+    # QN_ETIMEOUT by the check, which clears it
+    ws = qb.new_workspace(256)
+    ws[:4].view(torch.int32).fill_(1)
+    with pytest.raises(qb.QNError) as e:
+        qb.workspace_check(ws)
+    assert e.value.status == qb.QN_ETIMEOUT
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    qb.workspace_check(ws)
 
 
 def test_tiny_fwd_bwd(oracle):
@@ -306,3 +320,86 @@ def test_repeat_runs_bit_identical(n, k, M, bwd):
         else:
             assert torch.equal(got, first), f"run-to-run difference in {int((got != first).sum())} elements"
     assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+# ------------------------------------------------------------------------- merge
+
+def _ulp_diff_bf16(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in bf16 units between two arrays of bf16 bit patterns (finite values)."""
+    def key(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, -(u & 0x7fff), u & 0x7fff)
+    return np.abs(key(a) - key(b))
+
+
+@pytest.mark.parametrize("n,k,r,alpha", [(256, 256, 4, 8.0), (200, 448, 5, 10.0), (4096, 4096, 16, 32.0),
+                                         (1000, 64 * 19, 64, 16.0), (130, 256, 256, 16.0), (64, 128, 0, 0.0)])
+def test_merge_matches_oracle(oracle, n, k, r, alpha):
+    # "QLoRA & PEFT family" 3.6 (merge_and_unload): W' + s B A as bf16. The GPU adds the fp32
+    # tensor-core product to the fp32 dequantised weight (one fp32 rounding) before rounding to
+    # bf16, so it may differ from the exactly rounded oracle by one bf16 unit.
+    case = synth.LayerCase(f"merge{n}x{k}r{r}", n, k, 1, max(r, 1), alpha, 0.02, 7 * n + k + r)
+    W, A, B, _, _ = synth.layer_inputs(case, DEV, need_grad=False)
+    w = qb.nf4_quantize(W)
+    Ad, Bd = (A, B) if r > 0 else (None, None)
+    got = bits(qb.qlora_merge_bf16(w, Ad, Bd, alpha)).reshape(n, k)
+    torch.cuda.synchronize()
+    hw = to_host_weight(w)
+    ref = oracle.merge_bf16(hw, n, k, bits(A) if r > 0 else None, bits(B) if r > 0 else None, r, alpha)
+    # within the stated tolerance everywhere; off by more than one bf16 unit only where the sum
+    # cancels (the fp32 rounding of the product then spans several units of the small result)
+    assert_close(torch.from_numpy(got.view(np.int16)).view(torch.bfloat16), bf16_to_f64(ref), "merge")
+    d = _ulp_diff_bf16(got, ref)
+    assert float(np.mean(d <= 1)) > 0.999, f"{int((d > 1).sum())} merged weights more than one bf16 unit off"
+    assert float(np.mean(d == 0)) > 0.98
+    if r == 0:
+        assert np.array_equal(got, oracle.nf4_dequant_bf16(hw, n, k))
+
+
+# --------------------------------------------------------- adapter weight gradients
+
+def _assert_close_f32(got: torch.Tensor, ref: np.ndarray, what: str):
+    g = got.detach().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    err = np.abs(g - ref)
+    bound = RTOL * np.abs(ref) + STOL * rms
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} elements outside tolerance; "
+                           f"worst err/bound = {np.max(err / np.maximum(bound, 1e-300)):.3g}")
+
+
+@pytest.mark.parametrize("n,k,M,r,alpha", [(256, 256, 8, 4, 8.0), (200, 448, 129, 5, 10.0), (17, 64, 33, 16, 32.0),
+                                           (4096, 4096, 4096, 16, 32.0), (11008, 4096, 512, 16, 32.0),
+                                           (8192, 28672, 256, 64, 16.0), (320, 192, 70, 200, 400.0)])
+def test_lora_grads_match_oracle(oracle, n, k, M, r, alpha):
+    # "How does QLoRA work for training?" 2 and 7: only B and A are trained; grad_B = s grad_h^T (x A^T),
+    # grad_A = s (grad_h B)^T x, fp32 outputs within the stated tolerance of the fp64 oracle.
+    case = synth.LayerCase(f"grads{n}x{k}M{M}r{r}", n, k, M, r, alpha, 0.02, 3 * n + k + M + r)
+    _, A, B, x, gh = synth.layer_inputs(case, DEV)
+    gA, gB = qb.qlora_lora_grads(x, gh, A, B, alpha)
+    torch.cuda.synchronize()
+    rA, rB = oracle.lora_grads(bits(x), bits(gh), M, n, k, bits(A), bits(B), r, alpha)
+    _assert_close_f32(gA, rA, "grad_A")
+    _assert_close_f32(gB, rB, "grad_B")
+
+
+def test_lora_grads_repeat_bit_identical():
+    case = synth.LayerCase("grads_repeat", 1024, 2048, 777, 16, 32.0, 0.02, 5)
+    _, A, B, x, gh = synth.layer_inputs(case, DEV)
+    ws = torch.empty(qb.lora_grads_workspace_size(777, 16), dtype=torch.uint8, device=DEV)
+    first = None
+    for _ in range(4):
+        gA, gB = qb.qlora_lora_grads(x, gh, A, B, 32.0, workspace=ws)
+        torch.cuda.synchronize()
+        cur = (gA.clone(), gB.clone())
+        if first is None:
+            first = cur
+        else:
+            assert torch.equal(cur[0], first[0]) and torch.equal(cur[1], first[1])
+
+
+@pytest.mark.parametrize("n,M,r", [(204, 129, 16), (200 + 4, 65, 4), (100, 70, 100)])
+def test_bwd_many_tokens_with_unaligned_rows(oracle, n, M, r):
+    # more than 64 tokens with n_out % 8 != 0 (the tensor-core path's TMA row-stride rule fails),
+    # and few-token input gradients with a rank above 64: the fallback few-token kernel in chunks
+    run_case(oracle, synth.LayerCase(f"bwd_unaligned{n}M{M}r{r}", n, 256, M, r, 2.0 * r, 0.02, 11 * n + M + r))
