@@ -64,3 +64,33 @@ def test_static_scratch_rejects_weights_above_the_limit():
     st = lib.nf4_quantize_static_ws(ctypes.c_void_p(base + 0x4000000), ctypes.byref(cw), None)
     assert st == qb.QN_EWORKSPACE
     assert "static scratch" in lib.qn_last_error().decode()
+
+
+def test_static_scratch_inside_a_stream_capture_allocates_nothing():
+    # The case the entry point exists for: after one warm-up call (which resolves the scratch
+    # address), a call captured into a CUDA graph and replayed gives the same bits as the
+    # workspace entry point, and neither the capture nor the replays allocate device memory.
+    n, k = 2048, 4096
+    W = synth.student_t_bf16((n, k), 0.02, 41, device="cuda")
+    ref = qb.nf4_quantize(W)
+    out = qb.NF4Weight.empty(n, k)
+    qb.nf4_quantize_static_ws(W, out)  # warm-up outside the capture
+    torch.cuda.synchronize()
+    out.codes.fill_(0)
+    out.absmax_q.fill_(0)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    free_before, _ = torch.cuda.mem_get_info()
+    with torch.cuda.graph(graph, stream=stream):
+        qb.nf4_quantize_static_ws(W, out, stream=stream)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+        torch.cuda.synchronize()
+        _same(out, ref)
+    free_after, _ = torch.cuda.mem_get_info()
+    # the graph's own bookkeeping may take a little device memory; the quantiser's scratch
+    # (up to 16 MiB) must not appear as an allocation
+    assert free_before - free_after < (8 << 20)
+    del graph
