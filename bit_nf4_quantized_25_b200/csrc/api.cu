@@ -55,7 +55,8 @@ qn_status check_weight(const qn_nf4_weight *w) {
     if (w->n_out == 0 || w->k_in == 0) return QN_OK;
     if (!w->codes || !w->absmax_q || !w->group_scale || !w->absmax_mean)
         return fail(QN_EINVAL, "null pointer in the quantised weight");
-    if (!aligned16(w->codes)) return fail(QN_EALIGN, "codes not 16-byte aligned");
+    if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale))
+        return fail(QN_EALIGN, "codes, absmax_q or group_scale not 16-byte aligned");
     return QN_OK;
 }
 
@@ -228,9 +229,10 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
     if (s != QN_OK) return s;
     if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
     if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
-    // The few-token kernels need no workspace (256 bytes keep the pointer non-null); the
-    // tensor-core path stores its error word and the adapter operand there.
-    *ws_bytes = (M > kDecodeMaxM || r > kDecodeMaxRank) ? gemm_workspace_bytes(M, r) : 256;
+    // The few-token kernels keep the error word, the adapter product and its ready flag there
+    // (4 KB); the tensor-core path the error word and the adapter operand.
+    const size_t few = decode_fwd_workspace_bytes() > 4096 ? decode_fwd_workspace_bytes() : 4096;
+    *ws_bytes = (M > kDecodeMaxM || r > kDecodeMaxRank) ? gemm_workspace_bytes(M, r) : few;
     g_err.clear();
     return QN_OK;
 }
@@ -264,8 +266,8 @@ qn_status qlora_workspace_check(void *ws, void *stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_status(e, "qlora_workspace_check");
     return fail(QN_ETIMEOUT,
-                "a kernel that used this workspace gave up a bounded wait (error word %d); its output is incomplete",
-                word);
+                "a kernel that used this workspace stopped early (error word %d: %s); its output is incomplete", word,
+                word == 2 ? "dynamic shared memory not 1024-byte aligned" : "a bounded wait ran out");
 }
 
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B, int r,
@@ -305,8 +307,9 @@ qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t
     const uint16_t *gp = static_cast<const uint16_t *>(grad_h);
     uint16_t *xp = static_cast<uint16_t *>(grad_x);
     const uint16_t *Ap = static_cast<const uint16_t *>(A), *Bp = static_cast<const uint16_t *>(B);
-    // few tokens and adapters of rank <= 64: the streamed kernel, 16 tokens per launch
-    if (M <= kDecodeMaxM && r <= kDecodeMaxRank) {
+    // few tokens, adapters of rank <= 64 and TMA-friendly rows: the streamed kernel, 16 tokens per
+    // launch
+    if (M <= kDecodeMaxM && r <= kDecodeMaxRank && decode_bwd_stream_supported(w->n_out, w->k_in, r)) {
         int *err = static_cast<int *>(ws);
         for (int64_t m0 = 0; m0 < M; m0 += kDecodeTokens) {
             const int mc = static_cast<int>(M - m0 < kDecodeTokens ? M - m0 : kDecodeTokens);
@@ -316,12 +319,13 @@ qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t
         }
         return cuda_status(cudaSuccess, "");
     }
-    if (gemm_supported(w->n_out, w->k_in, M, true)) {
+    if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, true)) {
         if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
         return cuda_status(launch_gemm_bwd(wv, gp, M, Ap, Bp, r, sc, xp, ws, st), "qlora_linear_bwd_x");
     }
     // many tokens with n_out % 8 != 0 (the GEMM's TMA row-stride rule), or few tokens with a rank
-    // above 64: the earlier few-token kernel in chunks of 32 tokens
+    // above 64 or rows the streamed kernel's boxes cannot read: the register-streaming few-token
+    // kernel in chunks of 32 tokens
     constexpr int kChunk = 32;
     for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
         const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);

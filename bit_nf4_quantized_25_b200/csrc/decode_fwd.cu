@@ -1,6 +1,6 @@
 // decode_fwd.cu -- QLoRA linear forward for few tokens (M <= 16 per launch) on sm_100a.
 //
-//   h[m,n] = sum_k W'[n,k] x[m,k] + sum_j B[n,j] t[m,j],  t = s A x,  W'[n,k] = NF4[code] * c'_b
+//   h[m,n] = sum_k W'[n,k] x[m,k] + sum_j B[n,j] t[m,j],  t = bf16(s A x),  W'[n,k] = NF4[code] * c'_b
 // ("Quantized LoRA (QLoRA) and 4-bit training", apxml.com, forward equations; "How does QLoRA
 // work for training?", aivaro.ru, section 2).
 //
@@ -13,29 +13,37 @@
 //
 // Work split. One CTA per SM. A CTA owns R = 16 m weight rows over one K-slice; the C K-slices
 // of a row chunk form a thread-block cluster (R and C are chosen on the host so that the grid
-// fills the SMs evenly). The CTA streams its (R rows x K-slice) tile through a ring of stages;
-// a stage is R rows x 4 blocks of codes (one TMA box: one large box per stage keeps the copy
-// engine near the HBM rate, several small boxes do not), the matching 4 x 64 columns of x and
-// of the adapter A, and the inputs of the R x 4 block constants.
-//   warp 0      : producer. Lane 0 issues the codes box; the 32 lanes copy x, A (16-byte
-//                 cp.async into the 128-byte swizzled layout) and the constant inputs (the
-//                 FP8 codes and group scales) with cp.async; every copy completes on the
-//                 stage's full barrier.
+// fills the SMs and each CTA moves the fewest bytes). The CTA streams its (R rows x K-slice)
+// tile through a ring of stages. A stage holds R rows x 4 blocks of codes (one TMA box, 128-byte
+// swizzled so that the 8-byte reads of eight rows hit eight different bank groups) and the
+// matching 4 x 64 columns of the M token rows of x (one 3-D TMA box, [block][token][64 values],
+// same swizzle). The FP8 block codes and group scales of the CTA's whole slice are staged once.
+//   warp 0      : producer (one lane issues the TMA boxes; all lanes stage the constants and
+//                 the rows of B the CTA's up-projection needs).
 //   warps 1..16 : consumers. Warp (kg, rg) takes block kg of every stage and the m-tiles
 //                 rg, rg + 4, ... of the chunk: codes -> pair table -> mma.sync with x, one fp32
-//                 fragment per block scaled by c'_b into the accumulators. The four lanes of a
-//                 quad compute the block constants c'_b = fma(e4m3(q_b), sigma_g, mu) the quad
-//                 needs and share them by shuffles. Each warp also runs a share of the adapter
-//                 down-projection t_c = A x over the stage (mma.sync).
-// After the loop the four block-warps of each m-tile are summed in a fixed order, the slice's
-// adapter term B (s t_c) is added on the tensor cores, and the partial sums are pushed with DSMEM
-// stores into the CTA of the cluster that finalises those rows; one cluster barrier later that
-// CTA sums the slices in rank order and stores h. Results are bit-reproducible.
+//                 fragment per block scaled by c'_b = fma(e4m3(q_b), sigma_g, mu) into the
+//                 accumulators (the four lanes of a quad compute the constants the quad needs and
+//                 share them by shuffles).
+// The adapter down-projection t = bf16(s A x) is computed once per call by one more cluster (the
+// first row of the grid, so that it is dispatched first): its CTAs stream x and A over the same K-slices, reduce their partial
+// sums into rank 0 (DSMEM), and rank 0 publishes t in the workspace and raises a flag. The other
+// CTAs' producers wait for the flag after their last stage and copy t to shared memory; the last
+// of them to do so lowers the flag again for the next call.
+// After the loop the four block-warps of each m-tile are summed in a fixed order; one CTA per
+// m-tile adds B t on the tensor cores; the partial sums go by asynchronous DSMEM stores to the
+// CTA of the cluster that finalises those rows, which waits on its own mbarrier for the bytes,
+// sums the slices in rank order and stores h. Results are bit-reproducible.
 //
-// Nothing is read from global memory before the programmatic-launch wait. Every mbarrier wait
-// is bounded; a timeout records an error code in the workspace error word, stops the CTA's
-// work (cluster and named barriers are still passed, so no CTA waits forever) and drains the
-// loads already issued.
+// Programmatic launch: the packed weight (codes, FP8 codes, group scales) is requested BEFORE the
+// dependency wait, so the first stages of the ring fill while the preceding kernel finishes; x,
+// A and B are read, and h written, only after it. The caller guarantees that the preceding
+// kernel on the stream, if it signals its dependents early, does not write the packed weight
+// (no kernel of this library that signals early writes one). The codes are read with an L2
+// evict-first policy: they are used once, and the activations and adapters should stay cached.
+//
+// Every wait is bounded; a timeout records an error code in the workspace error word, stops the
+// CTA's work and drains the loads already issued.
 #include <cudaTypedefs.h>
 
 #include "host_cache.h"
@@ -45,17 +53,20 @@ namespace qn {
 
 #ifdef QN_TIMELINE
 // Per-CTA timestamps (globaltimer, ns) of the forward kernel's phases, for profiling builds only.
-__device__ unsigned long long g_fwd_timeline[1024][8];
-__device__ __forceinline__ void tl_mark(int slot) {
+// Two buffers, used by alternate launches, so that a chain's last two launches can be compared.
+__device__ unsigned long long g_fwd_timeline[2][1024][16];
+__device__ __forceinline__ void tl_mark(int buf, int slot) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
-    if (cta < 1024) g_fwd_timeline[cta][slot] = t;
+    if (cta < 1024) g_fwd_timeline[buf & 1][cta][slot] = t;
 }
 #define QN_TL(slot, cond) \
     do {                  \
-        if (cond) tl_mark(slot); \
+        if (cond) tl_mark(p.tl_buf, slot); \
     } while (0)
+static int g_last_plan[6];  // R, C, stages, chunks, shared bytes, bytes of the busiest CTA (KB)
+static int g_launches_tl = 0;
 #else
 #define QN_TL(slot, cond) \
     do {                  \
@@ -75,88 +86,327 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxCluster = 8;
 constexpr size_t kSmemLimit = 227 * 1024;
 
+// Workspace of the few-token path: error word, t-ready flag, reader count, t.
+constexpr size_t kWsFlag = 64, kWsReaders = 128, kWsT = 256;
+
 struct FwdArgs {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
     const uint16_t *B;  // n x r
-    const uint16_t *x;  // M x k
-    const uint16_t *A;  // r x k
     uint16_t *h;        // M x n
     int *err;
+    uint16_t *t_ws;     // [MP][rk16] bf16: bf16(s A x), published by the adapter cluster
+    unsigned *flag;     // 1 while t_ws holds this call's t
+    unsigned *readers;  // CTAs that have copied t_ws
     int64_t n, k;
+    int64_t row_lo, row_hi;  // rows of W this launch covers (chunk c: row_lo + c R ..)
     int nbr;     // blocks per row (k / 64)
     int ncol;    // stage columns (ceil(nbr / 4))
-    int M, r, rpad;  // rpad: r rounded up to 8, 16, 32 or 64 (0 without adapter)
+    int M, r, rpad, rk16;  // rpad: r rounded up to 8, 16, 32 or 64; rk16: to 16 (0 without adapter)
     float s;
     int R, m;    // rows and m-tiles per chunk
     int C;       // K-slices (cluster size)
+    int chunks;  // row chunks: grid rows 1 .. chunks when r > 0 (row 0 is the adapter cluster), else 0 .. chunks - 1
     int stages;
+    int evict_first;  // the codes are read with an L2 evict-first policy
     // shared-memory layout (byte offsets from the start of dynamic shared memory)
-    uint32_t slot_bytes, x_off, a_off, q_off, s_off;  // inside a slot
-    uint32_t ring_off, recv_off, bar_off, post_off;
-    uint32_t tx_bytes;
+    uint32_t slot_bytes, x_off;  // chunk CTAs: codes [R][128 B], x [4][M][128 B] at x_off
+    uint32_t a_off;              // adapter CTAs: x [4][MP][128 B] at 0, A [4][rpad][128 B] at a_off
+    uint32_t ring_off, qs_off, ss_off, tb_off, bs_off, recv_off, bar_off, post_off;
+    uint32_t qs_stride;  // bytes per chunk row of the staged FP8 codes
+    uint32_t bs_stride;  // bytes per staged row of B
+    uint32_t codes_bytes, x_bytes, xa_bytes;  // transaction bytes: codes box; x box; adapter x + A boxes
+#ifdef QN_TIMELINE
+    int tl_buf;
+#endif
 };
 
+// Barrier block: full[kMaxStages], empty[kMaxStages], consts, recv, abort flag.
+struct Bars {
+    uint64_t *full, *empty, *consts, *recv;
+    volatile uint32_t *abort_flag;
+};
+
+__device__ __forceinline__ Bars bars_of(uint8_t *smem, const FwdArgs &p) {
+    Bars b;
+    b.full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
+    b.empty = b.full + kMaxStages;
+    b.consts = b.empty + kMaxStages;
+    b.recv = b.consts + 1;
+    b.abort_flag = reinterpret_cast<volatile uint32_t *>(b.recv + 1);
+    return b;
+}
+
+// ------------------------------------------------------------------------------ adapter cluster
+// t_c = A x over this CTA's K-slice (mma.sync, the 16 consumer warps split the stage's (rank
+// tile, k16 step) jobs), summed into rank 0, which publishes bf16(s t).
+template <int NG>
+__device__ __forceinline__ void adapter_body(const CUtensorMap *tm_xp, const CUtensorMap *tm_a, const FwdArgs &p,
+                                             uint8_t *smem) {
+    constexpr int MP = 8 * NG;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int C = p.C;
+    const int crank = C > 1 ? static_cast<int>(cg::this_cluster().block_rank()) : 0;
+    const int col_lo = p.ncol * crank / C, col_hi = p.ncol * (crank + 1) / C;
+    const int ns = col_hi - col_lo;
+    const int S = p.stages;
+    const uint32_t s_base = saddr(smem);
+    const uint32_t s_ring = s_base + p.ring_off;
+    const Bars bb = bars_of(smem, p);
+    const uint32_t recv_bytes = static_cast<uint32_t>(C * MP * p.rpad * 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bb.full[s], 1);
+            mbar_init(&bb.empty[s], kConsumers);
+        }
+        mbar_init(bb.recv, 1);
+        if (C > 1 && crank == 0) mbar_arrive_expect_tx(bb.recv, recv_bytes);
+        *bb.abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch_desc(tm_xp);
+        tma_prefetch_desc(tm_a);
+    }
+    __syncthreads();
+    if (C > 1) cluster_arrive_relaxed();  // phase 1: this CTA runs (its shared memory may be written)
+    grid_dependents_launch();
+    grid_dependency_wait();  // x and A may come from the preceding kernel
+
+    auto fail = [&]() {
+        if (atomicExch(const_cast<uint32_t *>(bb.abort_flag), 1u) == 0u) record_error(p.err, kErrTimeout);
+    };
+    const int cw = warp - 1;
+    float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int NT = p.rpad / 8;  // rank tiles of 8 (1, 2, 4 or 8); 16 NT jobs per stage
+    if (warp == 0) {
+        int ni = 0;
+        if (lane == 0) {
+            for (int s = 0; s < ns; ++s) {
+                const int slot = s % S;
+                if (*bb.abort_flag) break;
+                if (s >= S && !mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_expect_tx(&bb.full[slot], p.xa_bytes);
+                const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+                tma_load_3d_saddr(sl, tm_xp, &bb.full[slot], 0, 0, 4 * (col_lo + s));
+                tma_load_3d_saddr(sl + p.a_off, tm_a, &bb.full[slot], 0, 0, 4 * (col_lo + s));
+                ni = s + 1;
+            }
+            for (int s = (ni > S ? ni - S : 0); s < ni; ++s) mbar_wait(&bb.full[s % S], (s / S) & 1);
+        }
+        __syncwarp();
+    } else {
+        const int nt_job = cw % NT;
+        const int kq_step = 16 / NT;
+        const int kq0 = cw / NT;
+        const int jrow = nt_job * 8 + g;  // rank row of this lane's B fragment
+        for (int s = 0; s < ns; ++s) {
+            const int slot = s % S;
+            if (*bb.abort_flag) break;
+            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
+                fail();
+                break;
+            }
+            const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+            for (int j = 0; j < NT; ++j) {
+                const int kq = kq0 + kq_step * j;
+                const int blk = kq >> 2, q4 = kq & 3;
+                const uint32_t xa = sl + blk * MP * 128;
+                const uint32_t aa = sl + p.a_off + blk * p.rpad * 128;
+                const uint32_t c0 = static_cast<uint32_t>(((2 * q4) ^ g) << 4) + 4 * t;
+                const uint32_t c1 = static_cast<uint32_t>(((2 * q4 + 1) ^ g) << 4) + 4 * t;
+                const uint32_t a0 = lds32(xa + g * 128 + c0), a2 = lds32(xa + g * 128 + c1);
+                uint32_t a1 = 0u, a3 = 0u;
+                if (NG > 1) {
+                    a1 = lds32(xa + (g + 8) * 128 + c0);
+                    a3 = lds32(xa + (g + 8) * 128 + c1);
+                }
+                const uint32_t jc0 = static_cast<uint32_t>(((2 * q4) ^ (jrow & 7)) << 4) + 4 * t;
+                const uint32_t jc1 = static_cast<uint32_t>(((2 * q4 + 1) ^ (jrow & 7)) << 4) + 4 * t;
+                const uint32_t b0 = lds32(aa + jrow * 128 + jc0), b1 = lds32(aa + jrow * 128 + jc1);
+                mma_16816(tacc, a0, a1, a2, a3, b0, b1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bb.empty[slot]);
+        }
+    }
+    __syncthreads();
+    // Per-CTA sum of the rank tiles (warps cw, cw + NT, ... in that order) into rank 0's
+    // receive buffer [src][MP tokens][rpad] fp32.
+    const uint32_t tbuf = s_base + p.post_off;  // [16 warps][32 lanes][4] f32, in the idle ring
+    if (warp > 0)
+        asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(tbuf + static_cast<uint32_t>(cw * 32 + lane) * 16),
+                     "f"(tacc[0]), "f"(tacc[1]), "f"(tacc[2]), "f"(tacc[3])
+                     : "memory");
+    __syncthreads();
+    const uint32_t recv = s_base + p.recv_off;
+    if (C > 1) cluster_wait();  // phase 1: every CTA of the cluster runs
+    if (warp > 0 && cw < NT) {
+        float tt[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int w = cw; w < kConsumers; w += NT) {
+            const uint4 v = lds128(tbuf + static_cast<uint32_t>(w * 32 + lane) * 16);
+            tt[0] += __uint_as_float(v.x);
+            tt[1] += __uint_as_float(v.y);
+            tt[2] += __uint_as_float(v.z);
+            tt[3] += __uint_as_float(v.w);
+        }
+        // fragment: tokens g / g + 8, ranks 8 cw + 2 t (+1)
+        const int j = 8 * cw + 2 * t;
+        const uint32_t o0 = recv + static_cast<uint32_t>(((crank * MP + g) * p.rpad + j) * 4);
+        const uint32_t o1 = recv + static_cast<uint32_t>(((crank * MP + g + 8) * p.rpad + j) * 4);
+        if (C > 1) {
+            const uint32_t bar = mapa(saddr(bb.recv), 0);
+            st_async_v2(mapa(o0, 0), tt[0], tt[1], bar);
+            if (NG > 1) st_async_v2(mapa(o1, 0), tt[2], tt[3], bar);
+        } else {
+            asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(o0), "f"(tt[0]), "f"(tt[1]) : "memory");
+            if (NG > 1) asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(o1), "f"(tt[2]), "f"(tt[3]) : "memory");
+        }
+    }
+    if (crank != 0) return;
+    bool ok = true;
+    if (C > 1) {
+        ok = mbar_wait(bb.recv, 0);
+        if (!ok && threadIdx.x == 0) record_error(p.err, kErrTimeout);
+    } else {
+        __syncthreads();
+    }
+    // t = bf16(s t) in rank order, [MP tokens][rk16] with zeros past rpad
+    const int half = p.rk16 / 2;
+    const float *rv = reinterpret_cast<const float *>(smem + p.recv_off);
+    for (int i = threadIdx.x; i < MP * half; i += kThreads) {
+        const int tok = i / half, j = 2 * (i - tok * half);
+        float v0 = 0.0f, v1 = 0.0f;
+        if (j < p.rpad)
+            for (int src = 0; src < C; ++src) {
+                v0 += rv[(src * MP + tok) * p.rpad + j];
+                v1 += rv[(src * MP + tok) * p.rpad + j + 1];
+            }
+        reinterpret_cast<uint32_t *>(p.t_ws)[i] = pack_bf16x2(p.s * v0, p.s * v1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && ok && !*bb.abort_flag) {
+        __threadfence();
+        st_release_u32(p.flag, 1u);
+    }
+}
+
+// ------------------------------------------------------------------------------ chunk clusters
 template <int NG, bool kFixedBase>
-__device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdArgs &p, uint8_t *smem) {
+__device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CUtensorMap *tm_x, const FwdArgs &p,
+                                           uint8_t *smem) {
     constexpr int MP = 8 * NG;  // padded tokens
     constexpr int MW = 4 / NG;  // m-tiles per warp at most (m <= 4 MW)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int C = p.C;
     const int crank = C > 1 ? static_cast<int>(cg::this_cluster().block_rank()) : 0;
-    const int chunk = blockIdx.y;
-    const int64_t row0 = static_cast<int64_t>(chunk) * p.R;
+    const int chunk = static_cast<int>(blockIdx.y) - (p.r > 0 ? 1 : 0);
+    const int64_t row0 = p.row_lo + static_cast<int64_t>(chunk) * p.R;
+    const int64_t nrow = p.row_hi;  // rows at or past nrow are not this launch's
     const int col_lo = p.ncol * crank / C, col_hi = p.ncol * (crank + 1) / C;
     const int ns = col_hi - col_lo;
     const int S = p.stages;
+    const int npre = ns < S ? ns : S;  // stages whose codes are requested before the dependency wait
+    // rows [r_lo, r_hi) of the chunk are finalised by this CTA (C > 1)
+    const int r_lo = p.R * crank / C, r_hi = p.R * (crank + 1) / C, nr = r_hi - r_lo;
+    const int nrmax = (p.R + C - 1) / C;
 
     uint8_t *lut = smem;
     const uint32_t s_base = saddr(smem);
     const uint32_t s_ring = s_base + p.ring_off;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-    uint64_t *empty = full + kMaxStages;
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(empty + kMaxStages);
+    const uint32_t s_qs = s_base + p.qs_off;
+    const uint32_t s_ss = s_base + p.ss_off;
+    const uint32_t tb = s_base + p.tb_off;  // [MP tokens][rk16] bf16 t
+    const uint32_t bs = s_base + p.bs_off;  // [assigned m-tiles x 16 rows][bs_stride] B rows
+    const Bars bb = bars_of(smem, p);
+    // the staged group scales start at index s_lo (that of the chunk's first block of the slice)
+    const int64_t s_lo = (row0 * p.nbr + 4 * col_lo) >> 8;
+
+    auto load_codes = [&](int s, uint64_t pol) {
+        const int slot = s % S;
+        const uint32_t dst = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+        const int32_t c0 = (col_lo + s) * 128, c1 = static_cast<int32_t>(row0);
+        if (p.evict_first)
+            tma_load_2d_saddr_hint(dst, tm_codes, &bb.full[slot], c0, c1, pol);
+        else
+            tma_load_2d_saddr(dst, tm_codes, &bb.full[slot], c0, c1);
+    };
 
     QN_TL(0, threadIdx.x == 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 32);  // the producer's 32 lanes (cp.async arrivals) + TMA bytes
-            mbar_init(&empty[s], kConsumers);
+            mbar_init(&bb.full[s], 1);  // lane 0's arrive.expect_tx (x) + the boxes' bytes
+            mbar_init(&bb.empty[s], kConsumers);
         }
-        *abort_flag = 0u;
+        mbar_init(bb.consts, kConsumers * 32);  // one cp.async arrival per consumer thread
+        mbar_init(bb.recv, 1);
+        if (C > 1) mbar_arrive_expect_tx(bb.recv, static_cast<uint32_t>(C * nr * MP * 4));
+        *bb.abort_flag = 0u;
         fence_barrier_init();
-        tma_prefetch_desc(tm_codes);
     }
-    build_pair_lut(lut, threadIdx.x, kThreads);
-    // rows M .. MP-1 of x and r .. rpad-1 of A are read by the fragments but never copied: zero
-    // them once in every slot
-    for (int sidx = 0; sidx < S; ++sidx) {
-        const uint32_t sl = s_ring + sidx * p.slot_bytes;
-        const int xw = kStageBlocks * (MP - p.M) * 32, aw = kStageBlocks * (p.rpad - p.r) * 32;
-        for (int i = threadIdx.x; i < xw; i += kThreads) {
-            const int b = i / ((MP - p.M) * 32), rem = i % ((MP - p.M) * 32);
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sl + p.x_off + b * MP * 128 + (p.M + rem / 32) * 128 + (rem % 32) * 4),
-                         "r"(0u)
-                         : "memory");
+    __syncthreads();  // barriers initialised
+    if (warp == 0) {
+        // ------------------------------------------ producer, before the dependency wait: weights
+        if (lane == 0) {
+            tma_prefetch_desc(tm_codes);
+            tma_prefetch_desc(tm_x);
+            const uint64_t pol = l2_policy_evict_first();
+            for (int s = 0; s < npre; ++s) {
+                mbar_expect_tx(&bb.full[s], p.codes_bytes);
+                load_codes(s, pol);
+            }
         }
-        for (int i = threadIdx.x; i < aw; i += kThreads) {
-            const int b = i / ((p.rpad - p.r) * 32), rem = i % ((p.rpad - p.r) * 32);
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(sl + p.a_off + b * p.rpad * 128 + (p.r + rem / 32) * 128 +
-                                                      (rem % 32) * 4),
-                         "r"(0u)
-                         : "memory");
+        __syncwarp();
+        QN_TL(14, lane == 0);
+    } else {
+        // ------------------------------------------ consumers, before the wait: constants, table
+        // FP8 codes of the slice: chunk row i holds the 16-byte aligned chunks from the one that
+        // contains block 4 col_lo of that row on; the group scales of every block of the chunk
+        // rows from the slice's first to its last, in whole 16-byte chunks. Bytes past the arrays
+        // read as zero.
+        const int ct = threadIdx.x - 32;
+        {
+            const int64_t nbq = p.n * p.nbr;
+            const int nch = static_cast<int>(p.qs_stride >> 4);
+            const int items = p.R * nch;
+            for (int it = ct; it < items; it += kConsumers * 32) {
+                const int i = it / nch, c = it - (it / nch) * nch;
+                const int64_t row = row0 + i;
+                const int64_t cb = (((row < nrow ? row : row0) * p.nbr + 4 * col_lo) >> 4) + c;  // 16-byte chunk
+                const int64_t avail = row < nrow ? nbq - 16 * cb : 0;
+                const uint32_t bytes = avail >= 16 ? 16u : (avail > 0 ? static_cast<uint32_t>(avail) : 0u);
+                cp_async16_zfill(s_qs + static_cast<uint32_t>(i) * p.qs_stride + 16u * c, p.q + (bytes ? 16 * cb : 0),
+                                 bytes);
+            }
+            const int64_t ngs = (nbq + kGroup - 1) / kGroup;
+            const int64_t rend = row0 + p.R < nrow ? row0 + p.R : nrow;
+            const int64_t bend = 4 * col_hi < p.nbr ? 4 * col_hi : p.nbr;
+            const int64_t s_hi = ((rend - 1) * p.nbr + bend - 1) >> 8;
+            const int scnt = static_cast<int>((s_hi >> 2) - (s_lo >> 2) + 1);  // 16-byte chunks
+            for (int c = ct; c < scnt; c += kConsumers * 32) {
+                const int64_t f = ((s_lo >> 2) + c) * 4;  // first float of the chunk
+                const int64_t avail = 4 * (ngs - f);
+                const uint32_t bytes = avail >= 16 ? 16u : (avail > 0 ? static_cast<uint32_t>(avail) : 0u);
+                cp_async16_zfill(s_ss + 16u * c, p.sigma + (bytes ? f : 0), bytes);
+            }
         }
+        cp_async_arrive_noinc(bb.consts);
+        QN_TL(8, ct == 0);
+        build_pair_lut(lut, ct, kConsumers * 32);
+        named_sync(1, kConsumers * 32);  // the table is complete
     }
-    __syncthreads();
     if (C > 1) cluster_arrive_relaxed();  // phase 1: this CTA runs (its shared memory may be written)
     grid_dependents_launch();
-    grid_dependency_wait();  // x, A and B may come from the preceding kernel
+    grid_dependency_wait();  // x, A and B may come from the preceding kernel; h may be read by it
     QN_TL(1, threadIdx.x == 0);
 
     auto fail = [&]() {
-        if (atomicExch(const_cast<uint32_t *>(abort_flag), 1u) == 0u) record_error(p.err, kErrTimeout);
+        if (atomicExch(const_cast<uint32_t *>(bb.abort_flag), 1u) == 0u) record_error(p.err, kErrTimeout);
     };
 
     const int cw = warp - 1;  // consumer index
@@ -166,151 +416,175 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
     for (int i = 0; i < MW; ++i)
 #pragma unroll
         for (int tg = 0; tg < NG; ++tg) acc[i][tg][0] = acc[i][tg][1] = acc[i][tg][2] = acc[i][tg][3] = 0.0f;
-    float tacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const int NT = p.rpad / 8;  // adapter n-tiles of 8 ranks (1, 2, 4 or 8)
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        // Stage s: wait for its slot; lane 0 issues the TMA loads (codes, x, A); every lane copies
-        // the constant inputs of its chunk rows (the aligned 8-byte window of q that holds the
-        // stage's four FP8 codes, and the group scales of the first and last of the four blocks)
-        // with cp.async, whose completion arrives on the same full barrier.
-        const int RJ = (p.R + 31) >> 5;  // chunk rows per lane: lane + 32 j
-        const int64_t nb = p.n * p.nbr;
-        const int64_t ng = (nb + kGroup - 1) / kGroup;
-        // the chunk's rows of B, read after the loop by the up-projection: into L2 now
-        if (p.r > 0) {
-            const int64_t nrows = (row0 + p.R <= p.n ? p.R : p.n - row0);
-            const char *b0 = reinterpret_cast<const char *>(p.B + row0 * p.r);
-            const int64_t bytes = nrows * p.r * 2;
-            for (int64_t off = static_cast<int64_t>(lane) * 128; off < bytes; off += 32 * 128)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(b0 + off) : "memory");
-        }
-        __syncwarp();
-        int ni = 0;  // stages issued
+        // Stage s: wait for its slot (from the second round on, then request its codes); arm the
+        // full barrier with the x bytes and request the x box. After the first round is armed,
+        // stage the B rows of this CTA's up-projection (m-tiles mt = crank mod C).
+        int ni = 0;  // stages armed
+        const int nassign = p.r > 0 ? (p.m - crank + C - 1) / C : 0;
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*abort_flag) break;
-            if (s >= S && !mbar_wait(&empty[slot], ((s / S) & 1) ^ 1)) {
-                fail();
-                break;
-            }
-            const int col = col_lo + s;
-            const uint32_t sl = s_ring + slot * p.slot_bytes;
+            if (*bb.abort_flag) break;
             if (lane == 0) {
-                mbar_expect_tx(&full[slot], p.tx_bytes);
-                tma_load_2d_saddr(sl, tm_codes, &full[slot], col * 128, static_cast<int32_t>(row0));
-            }
-            // x and A columns [256 col, 256 col + 256): row by row, lane j copies 16-byte chunk j & 7
-            // of block j >> 3 into the 128-byte swizzled layout (chunk c of row rr at c ^ (rr & 7))
-            {
-                const int b = lane >> 3, c = lane & 7;
-                const bool bvalid = 4 * col + b < p.nbr;
-                const int64_t kcol = static_cast<int64_t>(4 * col + b) * 64 + 8 * c;
-                for (int rr = 0; rr < p.M; ++rr) {
-                    const uint32_t dst = sl + p.x_off + static_cast<uint32_t>(b * MP * 128 + rr * 128 + ((c ^ (rr & 7)) << 4));
-                    cp_async16_zfill(dst, bvalid ? p.x + rr * p.k + kcol : p.x, bvalid ? 16u : 0u);
+                bool ok = true;
+                if (s >= S) {
+                    ok = mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1);
+                    if (ok) {
+                        mbar_expect_tx(&bb.full[slot], p.codes_bytes);
+                        load_codes(s, l2_policy_evict_first());
+                    } else {
+                        fail();
+                    }
                 }
-                for (int rr = 0; rr < p.r; ++rr) {
-                    const uint32_t dst =
-                        sl + p.a_off + static_cast<uint32_t>(b * p.rpad * 128 + rr * 128 + ((c ^ (rr & 7)) << 4));
-                    cp_async16_zfill(dst, bvalid ? p.A + rr * p.k + kcol : p.A, bvalid ? 16u : 0u);
+                if (ok) {
+                    mbar_arrive_expect_tx(&bb.full[slot], p.x_bytes);
+                    const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+                    tma_load_3d_saddr(sl + p.x_off, tm_x, &bb.full[slot], 0, 0, 4 * (col_lo + s));
                 }
             }
-            for (int j = 0; j < RJ; ++j) {
-                const int i = lane + 32 * j;
-                const int64_t row = row0 + i;
-                if (i < p.R && row < p.n) {
-                    const int64_t e0 = row * p.nbr + 4 * col;
-                    const int64_t e3 = e0 + 3 < nb ? e0 + 3 : nb - 1;
-                    const int64_t w0 = e0 & ~int64_t(3), w1 = w0 + 4;
-                    const uint32_t qd = sl + p.q_off + static_cast<uint32_t>(i) * 8u;
-                    const uint32_t sd = sl + p.s_off + static_cast<uint32_t>(i) * 8u;
-                    cp_async4_zfill(qd, p.q + w0, 4);
-                    const int64_t rest = nb - w1;
-                    cp_async4_zfill(qd + 4, p.q + (rest > 0 ? w1 : w0), rest >= 4 ? 4u : (rest > 0 ? static_cast<uint32_t>(rest) : 0u));
-                    cp_async4_zfill(sd, p.sigma + (e0 >> 8), 4);
-                    cp_async4_zfill(sd + 4, p.sigma + ((e3 >> 8) < ng ? (e3 >> 8) : ng - 1), 4);
-                }
-            }
-            cp_async_arrive_noinc(&full[slot]);  // one arrival per lane when its copies have landed
+            __syncwarp();
+            if (*bb.abort_flag) break;
             ni = s + 1;
             QN_TL(2, lane == 0 && s == S - 1);
+            if (s == npre - 1 && nassign > 0) {
+                // B rows 16 mt .. 16 mt + 16 of the assigned m-tiles, ranks 0 .. rk16 (zeros past
+                // r and past the last row)
+                const int cpr = p.rk16 / 8;  // 16-byte chunks per row
+                const bool r8 = (p.r & 7) == 0;
+                for (int i = lane; i < nassign * 16 * cpr; i += 32) {
+                    const int rr = i / cpr, c = i - (i / cpr) * cpr;
+                    const int mt = (rr >> 4) * C + crank;
+                    const int64_t row = row0 + 16 * mt + (rr & 15);
+                    const uint32_t dst = bs + static_cast<uint32_t>(rr) * p.bs_stride + 16u * c;
+                    if (r8) {
+                        const bool v = row < nrow && 8 * c < p.r;
+                        cp_async16_zfill(dst, v ? p.B + row * p.r + 8 * c : p.B, v ? 16u : 0u);
+                    } else {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 8 * c + 2 * e;
+                            const uint32_t lo = (row < nrow && j < p.r) ? ld_ro_u16(p.B + row * p.r + j) : 0u;
+                            const uint32_t hi = (row < nrow && j + 1 < p.r) ? ld_ro_u16(p.B + row * p.r + j + 1) : 0u;
+                            w[e] = lo | (hi << 16);
+                        }
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]),
+                                     "r"(w[2]), "r"(w[3])
+                                     : "memory");
+                    }
+                }
+            }
         }
-        // drain: every copy this warp issued has landed before the CTA can exit
+        // drain: the stages whose codes were requested before the wait but that were never
+        // armed get their arrival now; then every requested stage lands before the CTA exits
+        if (lane == 0) {
+            for (int s = ni; s < npre; ++s) mbar_arrive(&bb.full[s]);
+            const int hi = ni > npre ? ni : npre;
+            for (int s = (hi > S ? hi - S : 0); s < hi; ++s) mbar_wait(&bb.full[s % S], (s / S) & 1);
+        }
+        // t from the adapter cluster
+        if (p.r > 0) {
+            bool ok = true;
+            if (lane == 0) ok = wait_flag(p.flag);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) fail();
+            } else {
+                for (int i = lane; i < MP * p.rk16 / 2; i += 32)
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(tb + 4u * i), "r"(ld_cg_u32(p.t_ws + 2 * i))
+                                 : "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    const unsigned old = atomicAdd(p.readers, 1u);
+                    if (old == static_cast<unsigned>(p.chunks * C) - 1u) {
+                        // every CTA has its copy: lower the flag for the next call
+                        atomicExch(p.readers, 0u);
+                        atomicExch(p.flag, 0u);
+                    }
+                }
+            }
+            QN_TL(15, lane == 0);
+        }
         cp_async_wait_all();
-        if (lane == 0)
-            for (int s = (ni > S ? ni - S : 0); s < ni; ++s) mbar_wait(&full[s % S], (s / S) & 1);
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ consumers
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
         const float mu = __ldg(p.mu);
-        // x rows of this lane's tokens (tokens beyond M read a valid token; their columns of
-        // the result are never stored), swizzle chunk offsets of x[tok][16 t .. 16 t + 16)
+        // x rows of this lane's tokens (tokens beyond M read token tok % M; their columns of the
+        // result are never stored): row kg M + tok of the x box, 16-byte chunks 2 t and 2 t + 1
+        // of it, stored at chunk ^ (row & 7)
         uint32_t xr[NG], xc0[NG], xc1[NG];
 #pragma unroll
         for (int tg = 0; tg < NG; ++tg) {
-            int tok = tg * 8 + g;
-            if (tok >= p.M) tok = tok % p.M;
-            xr[tg] = static_cast<uint32_t>(tok) * 128u;
-            xc0[tg] = static_cast<uint32_t>(((2 * t) ^ (tok & 7)) << 4);
-            xc1[tg] = static_cast<uint32_t>(((2 * t + 1) ^ (tok & 7)) << 4);
+            const int tok = (tg * 8 + g) % p.M;
+            const int row = kg * p.M + tok;
+            xr[tg] = static_cast<uint32_t>(row) * 128u;
+            xc0[tg] = static_cast<uint32_t>(((2 * t) ^ (row & 7)) << 4);
+            xc1[tg] = static_cast<uint32_t>(((2 * t + 1) ^ (row & 7)) << 4);
         }
-        const int nt_job = NT > 0 ? cw % NT : 0;
-        const int kq_step = NT > 0 ? 16 / NT : 0;
-        const int kq0 = NT > 0 ? cw / NT : 0;
-        const int jrow = nt_job * 8 + g;  // adapter rank row of this lane's B fragment
-        // The block constant this lane computes each stage: m-tile rg + 4 (t >> 1), row g + 8 (t & 1)
-        // of it, block kg. The quad's four lanes cover the (up to) two m-tiles x two rows the quad
-        // needs and share them with shuffles (MW = 4: a second pass for m-tiles rg + 8, rg + 12).
-        int c_row[MW / 2 > 0 ? MW / 2 : 1];
-        int64_t c_rowbase[MW / 2 > 0 ? MW / 2 : 1];
-        uint32_t c_qoff[MW / 2 > 0 ? MW / 2 : 1];
+        // The block constant this lane computes each stage: m-tile rg + 4 (2 pass + (t >> 1)), row
+        // g + 8 (t & 1) of it, block kg. The quad's four lanes cover the (up to) two m-tiles x two
+        // rows the quad needs and share them with shuffles (MW = 4: a second pass for m-tiles
+        // rg + 8, rg + 12). c_q: staged FP8 code of block kg of the first stage; c_e: its block
+        // index relative to the first staged group scale (its scale is staged at c_e >> 8).
+        constexpr int NP = (MW + 1) / 2;
+        bool c_ok[NP];
+        uint32_t c_q[NP];
+        int64_t c_e[NP];
 #pragma unroll
-        for (int pass = 0; pass < (MW + 1) / 2; ++pass) {
+        for (int pass = 0; pass < NP; ++pass) {
             const int mt = rg + 4 * (2 * pass + (t >> 1));
             const int i = 16 * mt + g + 8 * (t & 1);
-            c_row[pass] = (mt < p.m && row0 + i < p.n) ? i : -1;
-            c_rowbase[pass] = (row0 + i) * p.nbr;
-            c_qoff[pass] = static_cast<uint32_t>(c_rowbase[pass] & 3);
+            const int64_t e0 = (row0 + i) * p.nbr + 4 * col_lo;
+            c_ok[pass] = mt < p.m && row0 + i < nrow;
+            c_q[pass] = s_qs + static_cast<uint32_t>(i) * p.qs_stride + static_cast<uint32_t>(e0 & 15) + kg;
+            c_e[pass] = e0 + kg - ((s_lo & ~int64_t(3)) << 8);  // staged scales start at s_lo & ~3
+        }
+        int nsc = ns;
+        if (!mbar_wait(bb.consts, 0)) {
+            fail();
+            nsc = 0;
         }
 
-        for (int s = 0; s < ns; ++s) {
+        for (int s = 0; s < nsc; ++s) {
             const int slot = s % S;
-            if (*abort_flag) break;
-            if (!mbar_wait(&full[slot], (s / S) & 1)) {
+            if (*bb.abort_flag) break;
+            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
                 fail();
                 break;
             }
             QN_TL(3, threadIdx.x == 32 && s == 0);
             QN_TL(4, threadIdx.x == 32 && s == ns - 1);
             const int col = col_lo + s;
-            const uint32_t sl = s_ring + slot * p.slot_bytes;
+            const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+            const bool blk_ok = 4 * col + kg < p.nbr;
             // block constants c'_b = fma(e4m3(q_b), sigma_g, mu) of this lane's rows, block kg
-            float cmine[(MW + 1) / 2];
+            float cmine[NP];
 #pragma unroll
-            for (int pass = 0; pass < (MW + 1) / 2; ++pass) {
+            for (int pass = 0; pass < NP; ++pass) {
                 float c = 0.0f;
-                const int i = c_row[pass];
-                if (i >= 0 && 4 * col + kg < p.nbr) {
-                    const uint32_t qw = lds32(sl + p.q_off + i * 8 + (((c_qoff[pass] + kg) >> 2) << 2));
-                    const uint32_t qb = (qw >> (8 * ((c_qoff[pass] + kg) & 3))) & 0xffu;
-                    const int64_t e = c_rowbase[pass] + 4 * col;
-                    const bool same = ((e + kg) >> 8) == (e >> 8);
-                    const float sg = __uint_as_float(lds32(sl + p.s_off + i * 8 + (same ? 0 : 4)));
+                if (c_ok[pass] && blk_ok) {
+                    const uint32_t qb = lds8(c_q[pass] + 4u * s);
+                    const int64_t si = (c_e[pass] + 4 * s) >> 8;
+                    const float sg = __uint_as_float(lds32(s_ss + 4u * static_cast<uint32_t>(si)));
                     c = block_constant(static_cast<uint8_t>(qb), sg, mu);
                 }
                 cmine[pass] = c;
             }
-            const uint32_t xb = sl + p.x_off + kg * MP * 128;
+            const uint32_t xb = sl + p.x_off;
             uint4 x0[NG], x1[NG];
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) {
                 x0[tg] = lds128(xb + xr[tg] + xc0[tg]);
                 x1[tg] = lds128(xb + xr[tg] + xc1[tg]);
             }
+            // codes of row (16 mt + g), bytes 32 kg + 8 t .. + 8: 16-byte chunk 2 kg + (t >> 1) of
+            // the 128-byte row, stored at chunk index ^ (row & 7) = ^ g
+            const uint32_t cchunk = static_cast<uint32_t>(((2 * kg + (t >> 1)) ^ g) << 4) + 8u * (t & 1);
 #pragma unroll
             for (int i = 0; i < MW; ++i) {
                 const int mt = rg + 4 * i;
@@ -318,7 +592,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
                 const float cA = __shfl_sync(0xffffffffu, cmine[i >> 1], (lane & ~3) | (2 * (i & 1)));
                 const float cB = __shfl_sync(0xffffffffu, cmine[i >> 1], (lane & ~3) | (2 * (i & 1) + 1));
                 if (mt < p.m) {
-                    const uint32_t cr = sl + static_cast<uint32_t>(16 * mt + g) * 128u + kg * 32 + 8 * t;
+                    const uint32_t cr = sl + static_cast<uint32_t>(16 * mt + g) * 128u + cchunk;
                     const uint2 ca = lds64(cr), cb = lds64(cr + 8 * 128);
                     uint32_t af[4][4];
 #pragma unroll
@@ -344,47 +618,19 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
                     }
                 }
             }
-            // adapter down-projection jobs: n-tile nt_job, k16 steps kq0 + kq_step * j of the stage
-            for (int j = 0; j < NT; ++j) {
-                const int kq = kq0 + kq_step * j;
-                const int blk = kq >> 2, q4 = kq & 3;
-                const uint32_t xa = sl + p.x_off + blk * MP * 128;
-                const uint32_t aa = sl + p.a_off + blk * p.rpad * 128;
-                const uint32_t c0 = static_cast<uint32_t>(((2 * q4) ^ g) << 4) + 4 * t;
-                const uint32_t c1 = static_cast<uint32_t>(((2 * q4 + 1) ^ g) << 4) + 4 * t;
-                const uint32_t a0 = lds32(xa + g * 128 + c0), a2 = lds32(xa + g * 128 + c1);
-                uint32_t a1 = 0u, a3 = 0u;
-                if (NG > 1) {
-                    a1 = lds32(xa + (g + 8) * 128 + c0);
-                    a3 = lds32(xa + (g + 8) * 128 + c1);
-                }
-                const uint32_t jc0 = static_cast<uint32_t>(((2 * q4) ^ (jrow & 7)) << 4) + 4 * t;
-                const uint32_t jc1 = static_cast<uint32_t>(((2 * q4 + 1) ^ (jrow & 7)) << 4) + 4 * t;
-                const uint32_t b0 = lds32(aa + jrow * 128 + jc0), b1 = lds32(aa + jrow * 128 + jc1);
-                mma_16816(tacc, a0, a1, a2, a3, b0, b1);
-            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (lane == 0) mbar_arrive(&bb.empty[slot]);
         }
+        cp_async_wait_all();  // the constants' copies (complete already unless a wait ran out)
     }
 
     // ---------------------------------------------------------------------- reduction
     // The ring is idle from here on (every stage was consumed, the producer drained its loads):
-    // its space holds the exchange buffers.
+    // its space holds the exchange buffer of the four block-warps.
     QN_TL(5, threadIdx.x == 32);
     __syncthreads();
     QN_TL(6, threadIdx.x == 0);
-    const uint32_t post = s_base + p.post_off;
-    const uint32_t tbuf = post;                                  // [16 warps][32 lanes][4] f32
-    const uint32_t tb = post + kConsumers * 32 * 16;             // [MP tokens][rk16] bf16 (s t_c)
-    const int rk16 = (p.rpad + 15) & ~15;
-    const uint32_t red = tb + ((MP * rk16 * 2 + 255) & ~255);    // [3][16 m-tiles][32 lanes][NG*4] f32
-    if (warp > 0 && p.r > 0) {
-        const uint32_t o = tbuf + static_cast<uint32_t>(cw * 32 + lane) * 16;
-        asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(o), "f"(tacc[0]), "f"(tacc[1]), "f"(tacc[2]),
-                     "f"(tacc[3])
-                     : "memory");
-    }
+    const uint32_t red = s_base + p.post_off;  // [3][16 m-tiles][32 lanes][NG*4] f32
     if (warp > 0 && kg > 0) {
 #pragma unroll
         for (int i = 0; i < MW; ++i) {
@@ -401,39 +647,11 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
         }
     }
     __syncthreads();
-    // t_c of n-tile cw (cw < NT): the warps cw, cw + NT, ... in that order; s t_c to bf16
-    if (warp > 0 && cw < NT) {
-        float tt[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int w = cw; w < kConsumers; w += NT) {
-            const uint4 v = lds128(tbuf + static_cast<uint32_t>(w * 32 + lane) * 16);
-            tt[0] += __uint_as_float(v.x);
-            tt[1] += __uint_as_float(v.y);
-            tt[2] += __uint_as_float(v.z);
-            tt[3] += __uint_as_float(v.w);
-        }
-        // fragment: tokens g / g + 8, ranks 8 cw + 2 t (+1)
-        const int j = 8 * cw + 2 * t;
-        const uint32_t v0 = pack_bf16x2(p.s * tt[0], p.s * tt[1]);
-        const uint32_t v1 = pack_bf16x2(p.s * tt[2], p.s * tt[3]);
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(tb + static_cast<uint32_t>(g * rk16 + j) * 2), "r"(v0) : "memory");
-        if (NG > 1)
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tb + static_cast<uint32_t>((g + 8) * rk16 + j) * 2), "r"(v1)
-                         : "memory");
-    }
-    // ranks beyond rpad (up to the k16 boundary) read as zero
-    if (p.r > 0 && rk16 > p.rpad) {
-        for (int i = threadIdx.x; i < MP * (rk16 - p.rpad) / 2; i += kThreads) {
-            const int tok = i / ((rk16 - p.rpad) / 2), jj = p.rpad + 2 * (i % ((rk16 - p.rpad) / 2));
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tb + static_cast<uint32_t>(tok * rk16 + jj) * 2), "r"(0u)
-                         : "memory");
-        }
-    }
-    __syncthreads();
-
-    const int nrmax = (p.R + C - 1) / C;
-    float *recv = reinterpret_cast<float *>(smem + p.recv_off);
+    QN_TL(9, threadIdx.x == 0);
+    const bool run_ok = !*bb.abort_flag;
     if (warp > 0 && kg == 0) {
-        // sum the four block-warps of each m-tile (kg = 0, 1, 2, 3 in order), add B (s t_c)
+        // sum the four block-warps of each m-tile (kg = 0, 1, 2, 3 in order); the CTA that owns
+        // the m-tile's adapter term (mt = crank mod C) adds B t
 #pragma unroll
         for (int i = 0; i < MW; ++i) {
             const int mt = rg + 4 * i;
@@ -449,42 +667,43 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
                     acc[i][tg][3] += __uint_as_float(v.w);
                 }
             }
-            const int64_t rA = row0 + 16 * mt + g, rB = rA + 8;
-            const bool vA = rA < p.n, vB = rB < p.n;
-            for (int kc = 0; kc < rk16 / 16 && p.r > 0; ++kc) {
-                const int j = 16 * kc + 2 * t;
-                const uint32_t a0 = load_pair_rowmajor(p.B, rA, vA, j, p.r);
-                const uint32_t a1 = load_pair_rowmajor(p.B, rB, vB, j, p.r);
-                const uint32_t a2 = load_pair_rowmajor(p.B, rA, vA, j + 8, p.r);
-                const uint32_t a3 = load_pair_rowmajor(p.B, rB, vB, j + 8, p.r);
-#pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    const uint32_t tr = tb + static_cast<uint32_t>((tg * 8 + g) * rk16 + j) * 2;
-                    mma_16816(acc[i][tg], a0, a1, a2, a3, lds32(tr), lds32(tr + 16));
-                }
-            }
-            if (C == 1) {
-                if (!*abort_flag) {
+            if (p.r > 0 && mt % C == crank) {
+                const uint32_t brow = bs + static_cast<uint32_t>(((mt / C) * 16 + g) * p.bs_stride);
+                for (int kc = 0; kc < p.rk16 / 16; ++kc) {
+                    const uint32_t j2 = static_cast<uint32_t>(16 * kc + 2 * t) * 2u;
+                    const uint32_t a0 = lds32(brow + j2), a2 = lds32(brow + j2 + 16);
+                    const uint32_t a1 = lds32(brow + 8 * p.bs_stride + j2), a3 = lds32(brow + 8 * p.bs_stride + j2 + 16);
 #pragma unroll
                     for (int tg = 0; tg < NG; ++tg) {
-                        const int tok = tg * 8 + 2 * t;
+                        const uint32_t tr = tb + static_cast<uint32_t>((tg * 8 + g) * p.rk16) * 2u + j2;
+                        mma_16816(acc[i][tg], a0, a1, a2, a3, lds32(tr), lds32(tr + 16));
+                    }
+                }
+            }
+            if (C == 1 && run_ok) {
+                const int64_t rA = row0 + 16 * mt + g, rB = rA + 8;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int64_t row = (e < 2) ? rA : rB;
-                            const int tk = tok + (e & 1);
-                            if (row < p.n && tk < p.M)
-                                p.h[static_cast<int64_t>(tk) * p.n + row] =
-                                    __bfloat16_as_ushort(__float2bfloat16_rn(acc[i][tg][e]));
-                        }
+                for (int tg = 0; tg < NG; ++tg) {
+                    const int tok = tg * 8 + 2 * t;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int64_t row = (e < 2) ? rA : rB;
+                        const int tk = tok + (e & 1);
+                        if (row < nrow && tk < p.M)
+                            p.h[static_cast<int64_t>(tk) * p.n + row] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(acc[i][tg][e]));
                     }
                 }
             }
         }
     }
+    QN_TL(10, threadIdx.x == 32);
     if (C > 1) {
-        cluster_wait();  // phase 1: every CTA of the cluster runs
+        // partial sums of every row, all MP token columns, to the row's owner [src][row][MP] f32
+        cluster_wait();  // phase 1: every CTA of the cluster runs (its barriers are initialised)
+        QN_TL(11, threadIdx.x == 32);
         if (warp > 0 && kg == 0) {
-            cg::cluster_group cluster = cg::this_cluster();
+            const uint32_t recv = s_base + p.recv_off;
 #pragma unroll
             for (int i = 0; i < MW; ++i) {
                 const int mt = rg + 4 * i;
@@ -494,24 +713,28 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
                     const int rl = 16 * mt + g + 8 * hh;
                     const int owner = (rl * C + C - 1) / p.R;
                     const int rr = rl - p.R * owner / C;
-                    float *dst = cluster.map_shared_rank(recv, owner) + (crank * nrmax + rr) * MP + 2 * t;
+                    const uint32_t dst = mapa(recv + static_cast<uint32_t>(((crank * nrmax + rr) * MP + 2 * t) * 4),
+                                              static_cast<uint32_t>(owner));
+                    const uint32_t bar = mapa(saddr(bb.recv), static_cast<uint32_t>(owner));
 #pragma unroll
                     for (int tg = 0; tg < NG; ++tg)
-                        *reinterpret_cast<float2 *>(dst + tg * 8) = make_float2(acc[i][tg][2 * hh], acc[i][tg][2 * hh + 1]);
+                        st_async_v2(dst + 32u * tg, acc[i][tg][2 * hh], acc[i][tg][2 * hh + 1], bar);
                 }
             }
         }
-        cluster_arrive_release();
-        cluster_wait_acquire();  // phase 2: every partial has landed
-        // rows [R crank / C, R (crank + 1) / C) of the chunk
-        const int r_lo = p.R * crank / C, r_hi = p.R * (crank + 1) / C, nr = r_hi - r_lo;
-        if (!*abort_flag) {
+        QN_TL(12, threadIdx.x == 32);
+        // rows [r_lo, r_hi): wait for the C partials, sum them in rank order
+        const bool ok = mbar_wait(bb.recv, 0);
+        if (!ok && threadIdx.x == 0) record_error(p.err, kErrTimeout);
+        QN_TL(13, threadIdx.x == 0);
+        if (ok && run_ok) {
+            const float *recvf = reinterpret_cast<const float *>(smem + p.recv_off);
             for (int it = threadIdx.x; it < nr * p.M; it += kThreads) {
                 const int rr = it % nr, tok = it / nr;
                 const int64_t row = row0 + r_lo + rr;
-                if (row >= p.n) continue;
+                if (row >= nrow) continue;
                 float sum = 0.0f;
-                for (int src = 0; src < C; ++src) sum += recv[(src * nrmax + rr) * MP + tok];
+                for (int src = 0; src < C; ++src) sum += recvf[(src * nrmax + rr) * MP + tok];
                 p.h[static_cast<int64_t>(tok) * p.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
             }
         }
@@ -521,12 +744,22 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap *tm_codes, const FwdA
 
 template <int NG>
 __global__ void __launch_bounds__(kThreads, 1)
-k_decode_fwd(const __grid_constant__ CUtensorMap tm_codes, const FwdArgs p) {
+k_decode_fwd(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+             const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_a, const FwdArgs p) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    if ((saddr(smem) & 0x00ffffffu) == kDynSmemBase)
-        fwd_body<NG, true>(&tm_codes, p, smem);
-    else
-        fwd_body<NG, false>(&tm_codes, p, smem);
+    // the 128-byte-swizzled boxes need 1024-byte aligned slots (uniform over the grid: every CTA
+    // leaves here together, before any barrier)
+    if (saddr(smem) & 1023u) {
+        if (threadIdx.x == 0) record_error(p.err, kErrLayout);
+        return;
+    }
+    if (p.r > 0 && blockIdx.y == 0) {
+        adapter_body<NG>(&tm_xp, &tm_a, p, smem);
+    } else if ((saddr(smem) & 0x00ffffffu) == kDynSmemBase) {
+        chunk_body<NG, true>(&tm_codes, &tm_x, p, smem);
+    } else {
+        chunk_body<NG, false>(&tm_codes, &tm_x, p, smem);
+    }
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -545,60 +778,162 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t cols, uint64_t rows,
-               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+// Tiled tensor map of `rank` dimensions: dims[0] is contiguous; strides[i] is the byte stride of
+// dimension i + 1.
+bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+            const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    cuuint64_t d[3], st[2];
+    cuuint32_t b[3], es[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    return fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, st, b, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// x (M x k) or A (r x k), bf16, as the stage boxes read it: 3-D {64 values, rows, blocks}, box
+// {64, box_rows, 4} (rows past `rows` read as zero), 128-byte swizzle.
+bool encode_operand(CUtensorMap *m, const uint16_t *base, int64_t rows, int64_t k, int box_rows) {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(k / 64)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(k) * 2, 128};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(box_rows), kStageBlocks};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int round_rank(int r) { return r <= 0 ? 0 : r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : 64; }
 
-// Shared-memory layout of one launch shape; false if it does not fit with at least two stages.
+uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory layout of one launch shape; false if it does not fit.
 bool layout(FwdArgs &a, int MP) {
-    const uint32_t codes = static_cast<uint32_t>(a.R) * 128u;
-    const uint32_t xb = kStageBlocks * MP * 128u;
-    const uint32_t ab = kStageBlocks * a.rpad * 128u;
-    const uint32_t qb = static_cast<uint32_t>(a.R) * 8u;  // q windows of the chunk rows
-    const uint32_t sb = static_cast<uint32_t>(a.R) * 8u;  // group scales of the chunk rows
+    const uint32_t codes = static_cast<uint32_t>(a.R) * 128u;  // multiple of 2048 (R = 16 m)
+    const uint32_t xb = kStageBlocks * static_cast<uint32_t>(a.M) * 128u;
+    const uint32_t xpb = kStageBlocks * MP * 128u;
+    const uint32_t ab = a.r > 0 ? kStageBlocks * a.rpad * 128u : 0u;
     a.x_off = codes;
-    a.a_off = codes + xb;
-    a.q_off = codes + xb + ab;
-    a.s_off = a.q_off + qb;
-    a.slot_bytes = (a.s_off + sb + 1023u) & ~1023u;
-    a.tx_bytes = codes;
-    const int rk16 = (a.rpad + 15) & ~15;
-    const uint32_t post = kConsumers * 32 * 16 + ((MP * rk16 * 2 + 255) & ~255) + 3 * kMaxM * 32 * 16 * (MP / 8);
-    const uint32_t recv = a.C > 1 ? (static_cast<uint32_t>(a.C * ((a.R + a.C - 1) / a.C) * MP * 4) + 1023u) & ~1023u : 0u;
-    a.ring_off = kLutBytes;
-    const uint32_t fixed = kLutBytes + recv + 1024;  // + barriers and flag
-    if (fixed >= kSmemLimit) return false;
+    a.a_off = xpb;
+    a.slot_bytes = align_up(codes + xb > xpb + ab ? codes + xb : xpb + ab, 1024);
+    a.codes_bytes = codes;
+    a.x_bytes = xb;
+    a.xa_bytes = xpb + ab;
+    const int nsmax = (a.ncol + a.C - 1) / a.C;
+    // staged FP8 codes: 16-byte chunks per chunk row, an odd count so that rows fall on
+    // distinct bank groups
+    const int nch = (15 + 4 * nsmax + 15) / 16;
+    a.qs_stride = 16u * static_cast<uint32_t>(nch | 1);
+    // staged group scales: at most R nbr / 256 + 2 of them, in whole 16-byte chunks
+    const int64_t s_max = static_cast<int64_t>(a.R) * a.nbr / 256 + 8;
+    if (s_max > (int64_t(1) << 20)) return false;
+    const uint32_t qs = align_up(static_cast<uint32_t>(a.R) * a.qs_stride, 128);
+    const uint32_t ss = align_up(static_cast<uint32_t>(s_max) * 4u, 128);
+    const uint32_t tbb = a.r > 0 ? align_up(static_cast<uint32_t>(MP * a.rk16 * 2), 128) : 0u;
+    // staged B rows: the CTA's m-tiles (mt = crank mod C), 16 rows each, padded so that the eight
+    // fragment rows fall on distinct bank groups
+    a.bs_stride = static_cast<uint32_t>(2 * a.rk16 + 16);
+    const uint32_t bsb = a.r > 0 ? align_up(static_cast<uint32_t>((a.m + a.C - 1) / a.C * 16) * a.bs_stride, 128) : 0u;
+    const uint32_t post_chunk = 3 * kMaxM * 32 * 16 * (MP / 8);
+    const uint32_t post_adapter = kConsumers * 32 * 16;
+    const uint32_t post = post_chunk > post_adapter ? post_chunk : post_adapter;
+    const uint32_t recv_chunk = a.C > 1 ? static_cast<uint32_t>(a.C * ((a.R + a.C - 1) / a.C) * MP * 4) : 0u;
+    const uint32_t recv_adapter = a.r > 0 ? static_cast<uint32_t>(a.C * MP * a.rpad * 4) : 0u;
+    const uint32_t recv = align_up(recv_chunk > recv_adapter ? recv_chunk : recv_adapter, 128);
+    const uint32_t bars = 256;
+    const uint64_t fixed = static_cast<uint64_t>(kLutBytes) + qs + ss + tbb + bsb + recv + bars;
+    if (fixed + a.slot_bytes > kSmemLimit) return false;
     int stages = static_cast<int>((kSmemLimit - fixed) / a.slot_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
-    if (stages < 2) return false;
-    const uint32_t ring = static_cast<uint32_t>(stages) * a.slot_bytes;
-    if (ring < post) {
-        // the exchange buffers outgrow the ring: give them room of their own
-        if (fixed + ring + post > kSmemLimit) {
-            stages = static_cast<int>((kSmemLimit - fixed - post) / a.slot_bytes);
-            if (stages < 2) return false;
-        }
+    if (stages > nsmax) stages = nsmax;
+    const int need = nsmax < 2 ? nsmax : 2;
+    if (stages < need) return false;
+    uint32_t ring = static_cast<uint32_t>(stages) * a.slot_bytes;
+    bool post_in_ring = ring >= post;
+    if (!post_in_ring && fixed + ring + post > kSmemLimit) {
+        // the exchange buffer outgrows the ring: give it room of its own
+        stages = static_cast<int>((kSmemLimit - fixed - post) / a.slot_bytes);
+        if (stages < need) return false;
+        ring = static_cast<uint32_t>(stages) * a.slot_bytes;
+        post_in_ring = ring >= post;
     }
     a.stages = stages;
-    const uint32_t ring_bytes = static_cast<uint32_t>(a.stages) * a.slot_bytes;
-    a.post_off = a.ring_off + (ring_bytes >= post ? 0u : ring_bytes);
-    const uint32_t after = a.ring_off + (ring_bytes >= post ? ring_bytes : ring_bytes + post);
-    a.recv_off = after;
-    a.bar_off = after + recv;
-    return true;
+    a.ring_off = kLutBytes;
+    uint32_t off = a.ring_off + ring;
+    if (post_in_ring) {
+        a.post_off = a.ring_off;
+    } else {
+        a.post_off = off;
+        off += align_up(post, 128);
+    }
+    a.qs_off = off;
+    off += qs;
+    a.ss_off = off;
+    off += ss;
+    a.tb_off = off;
+    off += tbb;
+    a.bs_off = off;
+    off += bsb;
+    a.recv_off = off;
+    off += recv;
+    a.bar_off = off;
+    return static_cast<uint64_t>(off) + bars <= kSmemLimit;
 }
 
-size_t smem_bytes(const FwdArgs &a) { return static_cast<size_t>(a.bar_off) + 2 * kMaxStages * 8 + 16; }
+size_t smem_bytes(const FwdArgs &a) { return static_cast<size_t>(a.bar_off) + 256; }
+
+// Bytes the busiest CTA moves: chunk CTAs codes + x per stage, adapter CTAs x + A per stage.
+double cta_bytes(const FwdArgs &a) {
+    const int nsmax = (a.ncol + a.C - 1) / a.C;
+    const double chunk = static_cast<double>(a.codes_bytes + a.x_bytes) * nsmax;
+    const double adapter = a.r > 0 ? static_cast<double>(a.xa_bytes) * nsmax : 0.0;
+    return chunk > adapter ? chunk : adapter;
+}
+
+// Launch shape for `rows` weight rows: R = 16 m rows per chunk and C K-slices per cluster with
+// (chunks + 1) x C <= SMs and every cluster resident at once; the shape whose busiest CTA moves
+// the fewest bytes (ties: the first found, i.e. smaller clusters, then shorter chunks).
+template <int NG>
+cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
+    constexpr int MP = 8 * NG;
+    const void *kern = reinterpret_cast<const void *>(k_decode_fwd<NG>);
+    const int extra = a.r > 0 ? 1 : 0;  // the adapter cluster
+    double best_cost = 0.0;
+    FwdArgs best = a;
+    found = false;
+    // m is a multiple of 4 (every consumer warp holds the same number of m-tiles) unless the
+    // weight has fewer than 64 rows
+    const int m_max = 16 / NG;  // four m-tile rows of warps, 4 / NG m-tiles each
+    const int m_min = rows < 64 ? static_cast<int>((rows + 15) / 16) : 4;
+    const int m_step = rows < 64 ? 1 : 4;
+    for (int C = 1; C <= kMaxCluster && C <= a.ncol; ++C) {
+        for (int m = m_min; m <= m_max; m += m_step) {
+            FwdArgs c = a;
+            c.m = m;
+            c.R = 16 * m;
+            c.C = C;
+            const int64_t chunks = (rows + c.R - 1) / c.R;
+            if ((chunks + extra) * C > sms) continue;
+            c.chunks = static_cast<int>(chunks);
+            if (!layout(c, MP)) continue;
+            const double cost = cta_bytes(c);
+            if (found && cost >= best_cost * (1.0 - 1e-9)) continue;
+            if (C > 1) {
+                int nc = 0;
+                const cudaError_t e = resident_clusters(kern, kThreads, C, smem_bytes(c), &nc);
+                if (e != cudaSuccess) return e;
+                if (nc < c.chunks + extra) continue;
+            }
+            best = c;
+            best_cost = cost;
+            found = true;
+        }
+    }
+    if (found) a = best;
+    return cudaSuccess;
+}
 
 template <int NG>
 cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint16_t *A, const uint16_t *B, int r,
@@ -614,10 +949,12 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
     a.sigma = w.sigma;
     a.mu = w.mu;
     a.B = B;
-    a.x = x;
-    a.A = A;
     a.h = h;
     a.err = err;
+    char *wsb = reinterpret_cast<char *>(err);
+    a.flag = reinterpret_cast<unsigned *>(wsb + kWsFlag);
+    a.readers = reinterpret_cast<unsigned *>(wsb + kWsReaders);
+    a.t_ws = reinterpret_cast<uint16_t *>(wsb + kWsT);
     a.n = w.n;
     a.k = w.k;
     a.nbr = static_cast<int>(w.k / kBlock);
@@ -625,83 +962,89 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
     a.M = M;
     a.r = r;
     a.rpad = round_rank(r);
+    a.rk16 = (a.rpad + 15) & ~15;
     a.s = s;
+#ifdef QN_FWD_NO_EVICT_HINT
+    a.evict_first = 0;
+#else
+    a.evict_first = 1;
+#endif
+    const int extra = r > 0 ? 1 : 0;  // the adapter cluster
 
-    // Launch shape: R = 16 m rows per chunk and C K-slices per cluster with chunks x C <= SMs
-    // and every cluster resident at once; per-CTA work is R x ceil(ncol / C) stage columns: take
-    // the shape with the least of it (ties: smaller clusters, then shorter chunks).
-    double best_work = 0.0;
-    FwdArgs best = a;
+    // Every CTA of a launch must be resident at once (the chunk CTAs wait for the adapter
+    // cluster): a weight taller than one wave runs as several launches over row ranges of equal
+    // size (multiples of 256 rows), each with its own adapter cluster.
+    int64_t part = w.n;
     bool found = false;
-    // m is a multiple of 4 (every consumer warp holds the same number of m-tiles) unless the
-    // weight has fewer than 64 rows
-    const int m_max = 16 / NG;  // four m-tile rows of warps, 4 / NG m-tiles each
-    const int m_min = w.n < 64 ? static_cast<int>((w.n + 15) / 16) : 4;
-    const int m_step = w.n < 64 ? 1 : 4;
-    for (int C = 1; C <= kMaxCluster && C <= a.ncol; ++C) {
-        for (int m = m_min; m <= m_max; m += m_step) {
-            FwdArgs c = a;
-            c.m = m;
-            c.R = 16 * m;
-            c.C = C;
-            const int64_t chunks = (w.n + c.R - 1) / c.R;
-            if (chunks * C > sms || chunks > 65535) continue;
-            const double work = static_cast<double>(c.R) * ((a.ncol + C - 1) / C);
-            if (found && work >= best_work * (1.0 - 1e-9)) continue;
-            if (!layout(c, MP)) continue;
-            if (C > 1) {
-                int nc = 0;
-                e = resident_clusters(kern, kThreads, C, smem_bytes(c), &nc);
-                if (e != cudaSuccess) return e;
-                if (nc < chunks) continue;
-            }
-            best = c;
-            best_work = work;
-            found = true;
-        }
+    for (;;) {
+        e = plan<NG>(a, part, sms, found);
+        if (e != cudaSuccess) return e;
+        if (found) break;
+        if (part <= 256) return cudaErrorInvalidConfiguration;
+        part = ((part + 1) / 2 + 255) / 256 * 256;
     }
-    if (!found) {
-        // more rows than one wave of the tallest chunks holds: several waves, no split
-        best.m = m_max;
-        best.R = 16 * m_max;
-        best.C = 1;
-        while (!layout(best, MP)) {
-            if (best.m == 1) return cudaErrorInvalidConfiguration;
-            best.m -= 1;
-            best.R = 16 * best.m;
-        }
-    }
-    a = best;
     const size_t smem = smem_bytes(a);
 
-    CUtensorMap tm_codes;
-    if (!encode_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, static_cast<uint64_t>(w.k / 2),
-                   static_cast<uint64_t>(w.n), 128, static_cast<uint32_t>(a.R), CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    CUtensorMap tm_codes, tm_x, tm_xp, tm_a;
+    {
+        const uint64_t dims[2] = {static_cast<uint64_t>(w.k / 2), static_cast<uint64_t>(w.n)};
+        const uint64_t strides[1] = {static_cast<uint64_t>(w.k / 2)};
+        const uint32_t box[2] = {128, static_cast<uint32_t>(a.R)};
+        if (!encode(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.codes, dims, strides, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    if (!encode_operand(&tm_x, x, M, w.k, M)) return cudaErrorInvalidValue;
+    if (r > 0) {
+        if (!encode_operand(&tm_xp, x, M, w.k, MP) || !encode_operand(&tm_a, A, r, w.k, a.rpad))
+            return cudaErrorInvalidValue;
+    } else {
+        tm_xp = tm_x;  // never read
+        tm_a = tm_x;
+    }
     e = ensure_smem_limit(kern, smem);
     if (e != cudaSuccess) return e;
 
-    const int64_t chunks = (w.n + a.R - 1) / a.R;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(a.C), static_cast<unsigned>(chunks), 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = a.C;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = a.C > 1 ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, k_decode_fwd<NG>, tm_codes, a);
-    count_launch();
+    for (int64_t lo = 0; lo < w.n; lo += part) {
+        FwdArgs b = a;
+#ifdef QN_TIMELINE
+        b.tl_buf = g_launches_tl++ & 1;
+#endif
+        b.row_lo = lo;
+        b.row_hi = lo + part < w.n ? lo + part : w.n;
+        b.chunks = static_cast<int>((b.row_hi - lo + b.R - 1) / b.R);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(b.C), static_cast<unsigned>(b.chunks + extra), 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = b.C;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = b.C > 1 ? 2 : 1;
+        e = cudaLaunchKernelEx(&cfg, k_decode_fwd<NG>, tm_codes, tm_x, tm_xp, tm_a, b);
+        count_launch();
+        if (e != cudaSuccess) return e;
+    }
+#ifdef QN_TIMELINE
+    g_last_plan[0] = a.R;
+    g_last_plan[1] = a.C;
+    g_last_plan[2] = a.stages;
+    g_last_plan[3] = a.chunks;
+    g_last_plan[4] = static_cast<int>(smem);
+    g_last_plan[5] = static_cast<int>(cta_bytes(a) / 1024);
+#endif
     return e;
 }
 
 }  // namespace
+
+size_t decode_fwd_workspace_bytes() { return kWsT + 16 * 64 * 2; }
 
 cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A, const uint16_t *B,
                               int r, float s, uint16_t *h, int *err, cudaStream_t st) {
@@ -712,9 +1055,14 @@ cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, con
 }
 
 #ifdef QN_TIMELINE
-extern "C" int qn_debug_fwd_timeline(unsigned long long *out, int n) {
-    return cudaMemcpyFromSymbol(out, g_fwd_timeline, sizeof(unsigned long long) * 8 * (n < 1024 ? n : 1024)) ==
-                   cudaSuccess
+extern "C" void qn_debug_fwd_plan(int *out) {
+    for (int i = 0; i < 6; ++i) out[i] = g_last_plan[i];
+}
+// buf 0: the last launch's timeline, 1: the one before it
+extern "C" int qn_debug_fwd_timeline(unsigned long long *out, int n, int buf) {
+    const int which = (g_launches_tl - 1 - buf) & 1;
+    return cudaMemcpyFromSymbol(out, g_fwd_timeline, sizeof(unsigned long long) * 16 * (n < 1024 ? n : 1024),
+                                sizeof(unsigned long long) * 16 * 1024 * which) == cudaSuccess
                ? 0
                : 1;
 }

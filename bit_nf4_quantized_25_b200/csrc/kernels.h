@@ -48,14 +48,21 @@ constexpr int kDecodeMaxM = 64;
 constexpr int kDecodeTokens = 16;
 constexpr int kDecodeMaxRank = 64;
 
-// h = dequant(W) x + s B (A x) for M <= kDecodeTokens tokens and r <= kDecodeMaxRank, one
-// launch; a timeout of a bounded wait is recorded in *err.
+// h = dequant(W) x + s B (A x) for M <= kDecodeTokens tokens and r <= kDecodeMaxRank (one
+// launch, several for weights taller than one wave). err is the workspace (its first word the
+// error word; it also holds the adapter product t and its ready flag, see
+// decode_fwd_workspace_bytes); a timeout of a bounded wait is recorded in the error word.
 cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A,
                               const uint16_t *B, int r, float s, uint16_t *h, int *err, cudaStream_t st);
+// Workspace bytes launch_decode_fwd uses (zeroed once before the first call).
+size_t decode_fwd_workspace_bytes();
 // grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h), streamed kernel: M <= kDecodeTokens tokens,
-// r <= kDecodeMaxRank, one launch; a timeout of a bounded wait is recorded in *err.
+// r <= kDecodeMaxRank, shapes with decode_bwd_stream_supported(), one launch; err is the
+// workspace (as for launch_decode_fwd).
 cudaError_t launch_decode_bwd_stream(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
                                      const uint16_t *B, int r, float s, uint16_t *gx, int *err, cudaStream_t st);
+// n_out % 8 == 0, r % 8 == 0 (or r == 0) and few enough 256-feature chunks for one wave.
+bool decode_bwd_stream_supported(int64_t n, int64_t k, int r);
 // grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h) for M <= kDecodeMaxM tokens.
 cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
                               const uint16_t *B, int r, float s, uint16_t *gx, cudaStream_t st);

@@ -75,6 +75,34 @@ __device__ __forceinline__ void tma_load_2d_saddr(uint32_t dst, const CUtensorMa
         : "memory");
 }
 
+// Same with an L2 cache policy (createpolicy) attached to the global reads.
+__device__ __forceinline__ void tma_load_2d_saddr_hint(uint32_t dst, const CUtensorMap *m, uint64_t *bar, int32_t c0,
+                                                       int32_t c1, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+// 3-D tiled bulk tensor load into this CTA's shared memory (destination as a shared-window address).
+__device__ __forceinline__ void tma_load_3d_saddr(uint32_t dst, const CUtensorMap *m, uint64_t *bar, int32_t c0,
+                                                  int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// L2 policy for data read once (streamed weights): evict first, so that the small operands
+// read by every CTA stay cached.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // Add `bytes` to the transaction count the current phase of `bar` expects (no arrival).
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)

@@ -26,6 +26,7 @@ constexpr int kLutBytes = 256 * 256;
 // sits above them. Kernels check it at run time and otherwise take the generic table path.
 constexpr uint32_t kDynSmemBase = 1024;
 constexpr int kErrTimeout = 1;  // error word value: a bounded wait ran out
+constexpr int kErrLayout = 2;   // error word value: dynamic shared memory not 1024-byte aligned
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -40,6 +41,11 @@ __device__ __forceinline__ uint32_t saddr(const void *p) { return static_cast<ui
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
@@ -141,6 +147,43 @@ __device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier
 __device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// Shared-window address `a` of this CTA mapped into the window of cluster rank `rank`.
+__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// Asynchronous 8-byte store into a cluster CTA's shared memory; completes `bytes` on that
+// CTA's mbarrier (both addresses from mapa).
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "f"(a), "f"(b), "r"(mbar)
+                 : "memory");
+}
+// 4-byte global load that bypasses L1 (data another CTA published).
+__device__ __forceinline__ uint32_t ld_cg_u32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait (nanosleep between polls, about a second in all) for a flag another CTA of the
+// grid sets with release semantics; false when it runs out.
+__device__ __forceinline__ bool wait_flag(const unsigned *flag) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        if (ld_acquire_u32(flag) != 0u) return true;
+        __nanosleep(128);
+    }
+    return false;
+}
 
 // Named barrier over `nthreads` threads (id 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(int id, int nthreads) {

@@ -57,7 +57,7 @@ typedef enum {
     QN_EALIGN = 3,     /* a tensor pointer is not 16-byte aligned               */
     QN_ECUDA = 4,      /* a CUDA launch or attribute call failed                */
     QN_EWORKSPACE = 5, /* workspace pointer null or smaller than required       */
-    QN_ETIMEOUT = 6    /* a kernel gave up a bounded wait (qlora_workspace_check) */
+    QN_ETIMEOUT = 6    /* a kernel stopped early: a bounded wait ran out (qlora_workspace_check) */
 } qn_status;
 
 /* Blocking of the format: one absmax per QN_BLOCK consecutive weights of the
@@ -68,7 +68,8 @@ typedef enum {
 #define QN_MAX_RANK 256
 
 /* A quantised weight. The struct is host memory; the four buffers are device
- * memory owned by the caller, with the sizes qn_nf4_sizes() returns.
+ * memory owned by the caller, with the sizes qn_nf4_sizes() returns; codes,
+ * absmax_q and group_scale start on 16-byte boundaries (QN_EALIGN otherwise).
  *   codes        : n_out*k_in/2 bytes. Weight e = n*k_in + k (row-major) is the
  *                  low nibble of byte e/2 when e is even, the high nibble when e
  *                  is odd. A nibble is an index 0..15 into the NF4 table
@@ -112,8 +113,8 @@ qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_byt
  * W must not contain NaN or Inf (the result is then unspecified).
  * ws: device workspace of at least qn_quantize_workspace_size() bytes, 256-byte
  * aligned; its contents on entry do not matter.
- * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (W or codes not 16-byte aligned),
- * QN_EWORKSPACE, QN_ECUDA. */
+ * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (W, codes, absmax_q or group_scale not
+ * 16-byte aligned), QN_EWORKSPACE, QN_ECUDA. */
 qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t ws_bytes, void *stream);
 
 /* nf4_quantize_static_ws -- nf4_quantize without a caller workspace and without allocating.
@@ -162,14 +163,17 @@ qn_status qlora_merge_bf16(const qn_nf4_weight *w, const void *A, const void *B,
  * an n_out x k_in weight and rank r (0 <= r <= 256). Host-only.
  *
  * The linear-layer workspace: device memory of at least this many bytes,
- * 256-byte aligned. Its first 4 bytes are an error word. Zero them when the
- * workspace is allocated (or call qlora_workspace_check once); the kernels
- * never clear the word, they only set it (to 1) when a bounded wait inside
- * them runs out, in which case that call's output is incomplete. The rest of
- * the workspace is scratch whose contents on entry do not matter. One
- * workspace may serve any number of calls in stream order, of any shapes,
- * as long as it is large enough for each; calls that run concurrently on the
- * GPU need separate workspaces. */
+ * 256-byte aligned. Zero all of it once when it is allocated. Its first 4
+ * bytes are an error word: the kernels never clear it, they only set it when
+ * a bounded wait inside them runs out (1) or the launch could not run (2), in
+ * which case that call's output is incomplete; qlora_workspace_check reads and
+ * clears it. The next bytes hold state the few-token kernels hand from one CTA
+ * to another within a call (the adapter product and its ready flag); every
+ * call leaves that state as it found it, so the workspace needs no clearing
+ * between calls, but after an error (QN_ETIMEOUT) zero it all again before
+ * reusing it. One workspace may serve any number of calls in stream order, of
+ * any shapes, as long as it is large enough for each; calls that run
+ * concurrently on the GPU need separate workspaces. */
 qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, size_t *ws_bytes);
 
 /* qlora_workspace_check -- read back and clear the workspace error word.
@@ -194,6 +198,11 @@ qn_status qlora_workspace_check(void *ws, void *stream);
  * ws: the linear-layer workspace (see qlora_workspace_size: at least that many
  * bytes, 256-byte aligned, error word zeroed once). M may be 0 (nothing is
  * enqueued).
+ * Ordering: the call may start reading the quantised weight (not x, A, B or h)
+ * before the preceding kernel on the stream has finished when that kernel
+ * signals its dependents early (griddepcontrol.launch_dependents); such a
+ * kernel must not write the quantised weight. No kernel of this library that
+ * signals early writes one.
  * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (x, h, codes, A or B not 16-byte
  * aligned), QN_EWORKSPACE, QN_ECUDA. */
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
