@@ -308,7 +308,7 @@ def detail_measurements(hbm_peak, tc_peak):
         g = synth.normal_bf16((M, n), 1.0, 15, dev)
         h = torch.empty(M, n, dtype=torch.bfloat16, device=dev)
         gx = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(qb.linear_workspace_size(M, n, k, r), 256), dtype=torch.uint8, device=dev)
+        ws = qb.new_workspace(qb.linear_workspace_size(M, n, k, r))  # zeroed once, as the header asks
         tf = time_fn(lambda: qb.qlora_linear_fwd(w, x, A, B, alpha, out=h, workspace=ws), reps=5, flush=flush)
         tb = time_fn(lambda: qb.qlora_linear_bwd_x(w, g, A, B, alpha, out=gx, workspace=ws), reps=5, flush=flush)
         fl = linear_flops(n, k, M, r)
@@ -383,7 +383,9 @@ def run_ours(args):
     stack = build_stack(args.layers, dev)
     xs = {(M, k): synth.normal_bf16((M, k), 1.0, 7000 + M + k, dev) for M in DECODE_M for k in (4096, 11008)}
     outs = {(M, n): torch.empty(M, n, dtype=torch.bfloat16, device=dev) for M in DECODE_M for n in (4096, 11008)}
-    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    # one workspace for every call of the step (stream order), zeroed once, as the header asks
+    ws = qb.new_workspace(max(qb.linear_workspace_size(M, n, k, RANK_7B) for M in DECODE_M
+                              for (_, n, k) in SHAPES_7B))
     step = decode_step_fn(stack, xs, outs, ws)
 
     per_step_bytes = sum(fwd_bytes(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)

@@ -130,8 +130,8 @@ def check_linear_shapes(n_out: int, k_in: int, act: torch.Tensor, A, B, out, bwd
 
 
 def new_workspace(need: int, device="cuda") -> torch.Tensor:
-    """A linear-layer workspace of `need` bytes with its error word zeroed (see
-    qlora_workspace_size in the header); reusable across calls in stream order."""
+    """A linear-layer workspace of `need` bytes, all zero as the header asks of a new workspace (see
+    qlora_workspace_size there); reusable across calls in stream order."""
     return torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
 
 

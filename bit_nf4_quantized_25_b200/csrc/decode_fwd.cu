@@ -54,19 +54,27 @@ namespace qn {
 #ifdef QN_TIMELINE
 // Per-CTA timestamps (globaltimer, ns) of the forward kernel's phases, for profiling builds only.
 // Two buffers, used by alternate launches, so that a chain's last two launches can be compared.
+// Slots 0 and 1 (start, past the wait): globaltimer (ns); the other slots: SM cycles since the
+// marking thread entered the kernel (clock64: one counter per SM, exact within a CTA).
 __device__ unsigned long long g_fwd_timeline[2][1024][16];
-__device__ __forceinline__ void tl_mark(int buf, int slot) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+__device__ __forceinline__ void tl_mark(int buf, int slot, long long c0) {
     const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
-    if (cta < 1024) g_fwd_timeline[buf & 1][cta][slot] = t;
+    if (cta >= 1024) return;
+    unsigned long long t;
+    if (slot <= 1) {
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    } else {
+        t = static_cast<unsigned long long>(clock64() - c0);
+    }
+    g_fwd_timeline[buf & 1][cta][slot] = t;
 }
 #define QN_TL(slot, cond) \
     do {                  \
-        if (cond) tl_mark(p.tl_buf, slot); \
+        if (cond) tl_mark(p.tl_buf, slot, tl_c0); \
     } while (0)
 static int g_last_plan[6];  // R, C, stages, chunks, shared bytes, bytes of the busiest CTA (KB)
 static int g_launches_tl = 0;
+__device__ int g_fwd_smid[2][1024];
 #else
 #define QN_TL(slot, cond) \
     do {                  \
@@ -301,6 +309,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                                            uint8_t *smem) {
     constexpr int MP = 8 * NG;  // padded tokens
     constexpr int MW = 4 / NG;  // m-tiles per warp at most (m <= 4 MW)
+#ifdef QN_TIMELINE
+    const long long tl_c0 = clock64();
+#endif
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int C = p.C;
@@ -338,6 +349,14 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     };
 
     QN_TL(0, threadIdx.x == 0);
+#ifdef QN_TIMELINE
+    if (threadIdx.x == 0) {
+        unsigned sm;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+        const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
+        if (cta < 1024) g_fwd_smid[p.tl_buf & 1][cta] = static_cast<int>(sm);
+    }
+#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&bb.full[s], 1);  // lane 0's arrive.expect_tx (x) + the boxes' bytes
@@ -505,7 +524,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                     }
                 }
             }
-            QN_TL(15, lane == 0);
+            QN_TL(12, lane == 0);
         }
         cp_async_wait_all();
         __syncwarp();
@@ -701,7 +720,6 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     if (C > 1) {
         // partial sums of every row, all MP token columns, to the row's owner [src][row][MP] f32
         cluster_wait();  // phase 1: every CTA of the cluster runs (its barriers are initialised)
-        QN_TL(11, threadIdx.x == 32);
         if (warp > 0 && kg == 0) {
             const uint32_t recv = s_base + p.recv_off;
 #pragma unroll
@@ -722,7 +740,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 }
             }
         }
-        QN_TL(12, threadIdx.x == 32);
+        QN_TL(11, threadIdx.x == 32);
         // rows [r_lo, r_hi): wait for the C partials, sum them in rank order
         const bool ok = mbar_wait(bb.recv, 0);
         if (!ok && threadIdx.x == 0) record_error(p.err, kErrTimeout);
@@ -1057,6 +1075,13 @@ cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, con
 #ifdef QN_TIMELINE
 extern "C" void qn_debug_fwd_plan(int *out) {
     for (int i = 0; i < 6; ++i) out[i] = g_last_plan[i];
+}
+extern "C" int qn_debug_fwd_smid(int *out, int n, int buf) {
+    const int which = (g_launches_tl - 1 - buf) & 1;
+    return cudaMemcpyFromSymbol(out, g_fwd_smid, sizeof(int) * (n < 1024 ? n : 1024), sizeof(int) * 1024 * which) ==
+                   cudaSuccess
+               ? 0
+               : 1;
 }
 // buf 0: the last launch's timeline, 1: the one before it
 extern "C" int qn_debug_fwd_timeline(unsigned long long *out, int n, int buf) {

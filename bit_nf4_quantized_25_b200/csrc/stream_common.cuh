@@ -5,8 +5,9 @@
 // The pair table: a code byte (two nibbles) maps to a bf16 pair of NF4 values,
 // bf16x2(NF4[byte & 15], NF4[byte >> 4]). It is stored once per lane in 256-byte rows, so the
 // byte permute that extracts a byte also forms the conflict-free address (byte << 8 | lane << 2);
-// 64 KB per CTA, of which the second half of every row is unused. NF4 values: "QLoRA paper
-// notes" (tqpw.cn), "NormalFloat Quantization (NF4)".
+// 64 KB per CTA, of which the second half of every row is unused (a packed 32 KB table needs one
+// more shift per lookup and measured slower). NF4 values: "QLoRA paper notes" (tqpw.cn),
+// "NormalFloat Quantization (NF4)".
 #pragma once
 
 #include <cooperative_groups.h>
