@@ -37,6 +37,15 @@
  *  - Merging the adapter into a 16-bit weight, W' + s B A (the weight cannot
  *    stay NF4 once merged): "QLoRA & PEFT family" section 3.6
  *    (merge_and_unload) and "QLoRA paper notes", Introduction.
+ *  - LoRA dropout on the adapter's input (training): "QLoRA & PEFT family"
+ *    section 3.4 (dropout 0.05-0.1) and the lora_dropout setting of the
+ *    configuration in "How does QLoRA work for training?". The pages give the
+ *    rate only; the reading taken: inverted dropout of x on the adapter branch
+ *    only (the base path sees x), element (m, k) of x kept when the 32-bit
+ *    output of a counter-based generator is >= floor(p 2^32), kept elements
+ *    scaled by 1 / (1 - p); the generator is Philox4x32-10 (Salmon, Moraes,
+ *    Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
+ *    written here from that definition.
  *
  * All sums of the linear layer are taken in fp64 in plain loop order.
  */
@@ -336,29 +345,90 @@ void or_nf4_dequant_f64(const uint8_t *codes, const uint8_t *q, const float *sig
     free(cp);
 }
 
+/* ---------------------------------------------------------------- dropout */
+
+/* Philox4x32 with 10 rounds: each round multiplies words 0 and 2 of the counter
+ * by the two round multipliers, mixes the high and low halves of the products
+ * with words 1 and 3 and the key, and the key is bumped by the two Weyl
+ * constants between rounds. */
+void or_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+    const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u, W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t p0 = (uint64_t)M0 * c0, p1 = (uint64_t)M1 * c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/* Keep threshold of rate p (0 <= p < 1): floor(p * 2^32), computed in fp64. */
+uint32_t or_dropout_threshold(double p) {
+    if (!(p > 0.0)) return 0u;
+    return (uint32_t)floor(p * 4294967296.0);
+}
+
+/* 32-bit generator output for element index e (already offset): word e % 4 of
+ * Philox4x32-10 at counter (e / 4 low word, e / 4 high word, 0, 0), key (seed
+ * low word, seed high word). */
+uint32_t or_dropout_bits(uint64_t seed, uint64_t e) {
+    const uint64_t blk = e >> 2;
+    const uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    or_philox4x32_10(ctr, key, out);
+    return out[e & 3];
+}
+
+/* 1 when element (m, kk) of the M x k activation survives dropout. */
+static int keep_at(uint64_t seed, uint64_t offset, uint32_t thr, int64_t m, int64_t k, int64_t kk) {
+    if (thr == 0u) return 1;
+    return or_dropout_bits(seed, offset + (uint64_t)(m * k + kk)) >= thr;
+}
+
 /* ------------------------------------------------------ linear layer */
 
 /* h[i, j] for the selected token rows rows[i] (i < nsel) of x (m x k):
  *   h = sum_k W'[j,k] x[row,k] + s * sum_r B[j,r] * (sum_k A[r,k] x[row,k])
  * with W' = T[code] * c' in fp64, s = fl32(alpha / r). A (r x k) and B (n x r)
- * may be NULL when r == 0. Output h is nsel x n, fp64. */
+ * may be NULL when r == 0. With dropout (p_drop > 0) the adapter's x[row,k] is
+ * kept or zeroed by keep_at(seed, offset, row, k) and s becomes s / (1 - p).
+ * Output h is nsel x n, fp64. */
 void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
                   int64_t k, const uint16_t *x, const int64_t *rows, int64_t nsel, const uint16_t *A,
-                  const uint16_t *B, int r, float alpha, double *h) {
+                  const uint16_t *B, int r, float alpha, double p_drop, uint64_t seed, uint64_t offset,
+                  double *h) {
     int64_t nb = or_num_blocks(n, k);
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
     block_constants(q, sigma, mu, nb, cp);
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    const uint32_t thr = or_dropout_threshold(p_drop);
+    if (thr != 0u) s = s / (1.0 - p_drop);
     double *xs = (double *)malloc(sizeof(double) * (size_t)(nsel * k + 1));
     double *t = (double *)malloc(sizeof(double) * (size_t)(nsel * (r > 0 ? r : 1) + 1));
     for (int64_t i = 0; i < nsel; ++i)
         for (int64_t kk = 0; kk < k; ++kk) xs[i * k + kk] = bf16_bits_to_float(x[rows[i] * k + kk]);
-    /* t[i, rr] = sum_k A[rr, k] x[row_i, k] */
+    /* t[i, rr] = sum_k A[rr, k] x[row_i, k] keep(row_i, k) (the dropout scale is in s) */
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < nsel; ++i)
         for (int rr = 0; rr < r; ++rr) {
             double acc = 0.0;
-            for (int64_t kk = 0; kk < k; ++kk) acc += bf16_bits_to_float(A[rr * k + kk]) * xs[i * k + kk];
+            for (int64_t kk = 0; kk < k; ++kk)
+                if (keep_at(seed, offset, thr, rows[i], k, kk))
+                    acc += bf16_bits_to_float(A[rr * k + kk]) * xs[i * k + kk];
             t[i * r + rr] = acc;
         }
 #pragma omp parallel
@@ -385,14 +455,18 @@ void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, fl
 
 /* grad_x[i, kk] for the selected rows of grad_h (m x n):
  *   grad_x = sum_j grad_h[row,j] W'[j,kk] + s * sum_r A[r,kk] * (sum_j grad_h[row,j] B[j,r])
- * Output nsel x k, fp64. */
+ * With dropout the adapter term of (row, kk) is zeroed where the forward's mask
+ * zeroed x[row, kk], and s becomes s / (1 - p). Output nsel x k, fp64. */
 void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
                     int64_t k, const uint16_t *gh, const int64_t *rows, int64_t nsel,
-                    const uint16_t *A, const uint16_t *B, int r, float alpha, double *gx) {
+                    const uint16_t *A, const uint16_t *B, int r, float alpha, double p_drop,
+                    uint64_t seed, uint64_t offset, double *gx) {
     int64_t nb = or_num_blocks(n, k);
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
     block_constants(q, sigma, mu, nb, cp);
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    const uint32_t thr = or_dropout_threshold(p_drop);
+    if (thr != 0u) s = s / (1.0 - p_drop);
     double *gs = (double *)malloc(sizeof(double) * (size_t)(nsel * n + 1));
     double *u = (double *)malloc(sizeof(double) * (size_t)(nsel * (r > 0 ? r : 1) + 1));
     for (int64_t i = 0; i < nsel; ++i)
@@ -429,6 +503,7 @@ void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, 
                 for (int64_t kk = k0; kk < k1; ++kk) {
                     double lora = 0.0;
                     for (int rr = 0; rr < r; ++rr) lora += bf16_bits_to_float(A[rr * k + kk]) * u[i * r + rr];
+                    if (!keep_at(seed, offset, thr, rows[i], k, kk)) lora = 0.0;
                     gx[i * k + kk] = acc[i * CH + (kk - k0)] + s * lora;
                 }
         }
@@ -447,13 +522,16 @@ void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, 
  *   grad_B[n, j] = s * sum_m grad_h[m,n] t[m,j]
  *   u[m, j]      = sum_n grad_h[m,n] B[n,j]
  *   grad_A[j, k] = s * sum_m u[m,j] x[m,k]
- * with s = fl32(alpha / r). x is M x k, grad_h M x n, A r x k, B n x r (bf16
+ * with s = fl32(alpha / r); with dropout x is the forward's masked x and s
+ * becomes s / (1 - p). x is M x k, grad_h M x n, A r x k, B n x r (bf16
  * bits); grad_A (r x k) and grad_B (n x r) are fp64, all sums in fp64 in plain
  * loop order. */
 void or_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, int64_t k,
-                   const uint16_t *A, const uint16_t *B, int r, float alpha, double *grad_A,
-                   double *grad_B) {
+                   const uint16_t *A, const uint16_t *B, int r, float alpha, double p_drop, uint64_t seed,
+                   uint64_t offset, double *grad_A, double *grad_B) {
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
+    const uint32_t thr = or_dropout_threshold(p_drop);
+    if (thr != 0u) s = s / (1.0 - p_drop);
     double *t = (double *)malloc(sizeof(double) * (size_t)(M * (r > 0 ? r : 1) + 1));
     double *u = (double *)malloc(sizeof(double) * (size_t)(M * (r > 0 ? r : 1) + 1));
 #pragma omp parallel for schedule(static)
@@ -461,7 +539,8 @@ void or_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, 
         for (int j = 0; j < r; ++j) {
             double ta = 0.0, ua = 0.0;
             for (int64_t kk = 0; kk < k; ++kk)
-                ta += bf16_bits_to_float(A[j * k + kk]) * (double)bf16_bits_to_float(x[m * k + kk]);
+                if (keep_at(seed, offset, thr, m, k, kk))
+                    ta += bf16_bits_to_float(A[j * k + kk]) * (double)bf16_bits_to_float(x[m * k + kk]);
             for (int64_t nn = 0; nn < n; ++nn)
                 ua += bf16_bits_to_float(gh[m * n + nn]) * (double)bf16_bits_to_float(B[nn * r + j]);
             t[m * r + j] = ta;
@@ -478,7 +557,8 @@ void or_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, 
     for (int j = 0; j < r; ++j)
         for (int64_t kk = 0; kk < k; ++kk) {
             double acc = 0.0;
-            for (int64_t m = 0; m < M; ++m) acc += u[m * r + j] * bf16_bits_to_float(x[m * k + kk]);
+            for (int64_t m = 0; m < M; ++m)
+                if (keep_at(seed, offset, thr, m, k, kk)) acc += u[m * r + j] * bf16_bits_to_float(x[m * k + kk]);
             grad_A[(int64_t)j * k + kk] = s * acc;
         }
     free(u);

@@ -67,10 +67,17 @@ def _load():
         lib.or_block_constant.restype = ctypes.c_float
         lib.or_nf4_dequant_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
         lib.or_nf4_dequant_f64.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
+        u64, f64 = ctypes.c_uint64, ctypes.c_double
         lib.or_qlora_fwd.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, i64, P, P,
-                                     ctypes.c_int, ctypes.c_float, P]
+                                     ctypes.c_int, ctypes.c_float, f64, u64, u64, P]
         lib.or_qlora_bwd_x.argtypes = lib.or_qlora_fwd.argtypes
-        lib.or_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P, P]
+        lib.or_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, f64, u64, u64,
+                                      P, P]
+        lib.or_philox4x32_10.argtypes = [P, P, P]
+        lib.or_dropout_threshold.argtypes = [f64]
+        lib.or_dropout_threshold.restype = ctypes.c_uint32
+        lib.or_dropout_bits.argtypes = [u64, u64]
+        lib.or_dropout_bits.restype = ctypes.c_uint32
         lib.or_f64_to_bf16.argtypes = [ctypes.c_double]
         lib.or_f64_to_bf16.restype = ctypes.c_uint16
         lib.or_merge_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P]
@@ -174,9 +181,35 @@ def _rows(m: int, rows) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
 
 
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """The four 32-bit words of Philox4x32-10 at counter `ctr` (4 words) and key `key` (2 words)."""
+    c = np.ascontiguousarray(np.asarray(ctr, dtype=np.uint32))
+    kk = np.ascontiguousarray(np.asarray(key, dtype=np.uint32))
+    out = np.zeros(4, dtype=np.uint32)
+    _load().or_philox4x32_10(_ptr(c), _ptr(kk), _ptr(out))
+    return out
+
+
+def dropout_threshold(p: float) -> int:
+    return int(_load().or_dropout_threshold(float(p)))
+
+
+def dropout_bits(seed: int, e: int) -> int:
+    """The generator's 32-bit output for (offset) element index e."""
+    return int(_load().or_dropout_bits(int(seed), int(e)))
+
+
+def dropout_keep(seed: int, offset: int, p: float, m: int, k: int) -> np.ndarray:
+    """m x k boolean mask of the adapter input's surviving elements (slow; small shapes)."""
+    thr = dropout_threshold(p)
+    return np.array([[thr == 0 or dropout_bits(seed, offset + i * k + j) >= thr for j in range(k)]
+                     for i in range(m)], dtype=bool)
+
+
 def qlora_fwd(qw: dict, n: int, k: int, x_bits: np.ndarray, m: int, A_bits, B_bits, r: int,
-              alpha: float, rows=None) -> np.ndarray:
-    """h (fp64) for the selected token rows of x (m x k bf16 bits); shape len(rows) x n."""
+              alpha: float, rows=None, p_drop: float = 0.0, seed: int = 0, offset: int = 0) -> np.ndarray:
+    """h (fp64) for the selected token rows of x (m x k bf16 bits); shape len(rows) x n.
+    p_drop > 0: LoRA dropout of the adapter's input with generator (seed, offset)."""
     rows = _rows(m, rows)
     x = _bits16(x_bits).reshape(-1)
     assert x.size == m * k
@@ -184,12 +217,13 @@ def qlora_fwd(qw: dict, n: int, k: int, x_bits: np.ndarray, m: int, A_bits, B_bi
     B = _bits16(B_bits).reshape(-1) if r > 0 else None
     h = np.zeros(rows.size * n, dtype=np.float64)
     _load().or_qlora_fwd(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
-                         _ptr(x), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(h))
+                         _ptr(x), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), float(p_drop),
+                         int(seed), int(offset), _ptr(h))
     return h.reshape(rows.size, n)
 
 
 def qlora_bwd_x(qw: dict, n: int, k: int, gh_bits: np.ndarray, m: int, A_bits, B_bits, r: int,
-                alpha: float, rows=None) -> np.ndarray:
+                alpha: float, rows=None, p_drop: float = 0.0, seed: int = 0, offset: int = 0) -> np.ndarray:
     """grad_x (fp64) for the selected token rows of grad_h (m x n bf16 bits); shape len(rows) x k."""
     rows = _rows(m, rows)
     g = _bits16(gh_bits).reshape(-1)
@@ -198,12 +232,13 @@ def qlora_bwd_x(qw: dict, n: int, k: int, gh_bits: np.ndarray, m: int, A_bits, B
     B = _bits16(B_bits).reshape(-1) if r > 0 else None
     gx = np.zeros(rows.size * k, dtype=np.float64)
     _load().or_qlora_bwd_x(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
-                           _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(gx))
+                           _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), float(p_drop),
+                           int(seed), int(offset), _ptr(gx))
     return gx.reshape(rows.size, k)
 
 
 def lora_grads(x_bits: np.ndarray, gh_bits: np.ndarray, m: int, n: int, k: int, A_bits, B_bits, r: int,
-               alpha: float):
+               alpha: float, p_drop: float = 0.0, seed: int = 0, offset: int = 0):
     """(grad_A (r x k), grad_B (n x r)) in fp64 for all m token rows of x (m x k) and grad_h (m x n)."""
     x = _bits16(x_bits).reshape(-1)
     g = _bits16(gh_bits).reshape(-1)
@@ -212,7 +247,8 @@ def lora_grads(x_bits: np.ndarray, gh_bits: np.ndarray, m: int, n: int, k: int, 
     B = _bits16(B_bits).reshape(-1)
     gA = np.zeros(r * k, dtype=np.float64)
     gB = np.zeros(n * r, dtype=np.float64)
-    _load().or_lora_grads(_ptr(x), _ptr(g), m, n, k, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(gA), _ptr(gB))
+    _load().or_lora_grads(_ptr(x), _ptr(g), m, n, k, _ptr(A), _ptr(B), int(r), float(alpha), float(p_drop),
+                          int(seed), int(offset), _ptr(gA), _ptr(gB))
     return gA.reshape(r, k), gB.reshape(n, r)
 
 

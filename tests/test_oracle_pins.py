@@ -636,3 +636,127 @@ def test_f64_to_bf16_overflow_threshold(oracle):
     assert oracle.f64_to_bf16(mx + half * 0.999) == 0x7f7f
     assert oracle.f64_to_bf16(mx + half) == 0x7f80  # tie: the even neighbour is 2^128 -> inf
     assert oracle.f64_to_bf16(-(mx + 2 * half)) == 0xff80
+
+
+# ---------------------------------------------------------------- LoRA dropout
+# [codex] 3.4 and the lora_dropout setting in [aivaro]'s configuration: dropout on the adapter's
+# input. Reading (the pages give only the rate): inverted dropout of x on the adapter branch only,
+# element kept when the Philox4x32-10 output is >= floor(p 2^32), kept elements scaled 1 / (1 - p).
+# Pins: the generator's published known-answer vectors; the threshold's closed form; the keep rate
+# within a binomial bound; the counter/offset layout; p = 0 reducing to the plain layer exactly;
+# the masked input gradient being the adjoint of the masked forward; the mean over seeds of the
+# masked adapter term converging to the unmasked one; the gradients' adjointness with dropout.
+
+def _kat():
+    rows = []
+    with open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                w = [int(v, 16) for v in line.split()]
+                rows.append((w[0:4], w[4:6], w[6:10]))
+    return rows
+
+
+def test_philox_known_answers(oracle):
+    for ctr, key, want in _kat():
+        assert [int(v) for v in oracle.philox4x32_10(ctr, key)] == want
+
+
+def test_dropout_threshold_closed_form(oracle):
+    assert oracle.dropout_threshold(0.0) == 0
+    assert oracle.dropout_threshold(0.5) == 2 ** 31
+    assert oracle.dropout_threshold(0.25) == 2 ** 30
+    assert oracle.dropout_threshold(0.05) == math.floor(0.05 * 2 ** 32)
+    assert oracle.dropout_threshold(0.1) == math.floor(0.1 * 2 ** 32)
+
+
+def test_dropout_bits_counter_layout(oracle):
+    # element e draws word e % 4 of the block e // 4; the seed is the key (low, high word)
+    seed = 0x0123456789ABCDEF
+    for e in (0, 1, 2, 3, 4, 7, 1 << 33, (1 << 34) + 3):
+        blk = e >> 2
+        words = oracle.philox4x32_10([blk & 0xFFFFFFFF, blk >> 32, 0, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        assert oracle.dropout_bits(seed, e) == int(words[e & 3])
+
+
+def test_dropout_keep_rate_and_offset(oracle):
+    p, m, k = 0.1, 40, 1024
+    keep = oracle.dropout_keep(1234, 0, p, m, k)
+    n = keep.size
+    rate = keep.mean()
+    sd = math.sqrt(p * (1 - p) / n)
+    assert abs(rate - (1 - p)) < 5 * sd
+    # the offset shifts the element index: element (0, j) at offset d is element (0, j + d) at 0
+    k2 = oracle.dropout_keep(1234, 5, p, 1, k - 5)
+    assert np.array_equal(k2[0], keep[0, 5:])
+    # another seed gives another mask
+    assert not np.array_equal(oracle.dropout_keep(1235, 0, p, m, k), keep)
+
+
+def test_dropout_zero_rate_is_the_plain_layer(oracle):
+    n, k, m, r, alpha = 48, 192, 5, 8, 16.0
+    qw, A, B, x, gh = _layer(oracle, n, k, m, r, 123)
+    for fn, inp in ((oracle.qlora_fwd, x), (oracle.qlora_bwd_x, gh)):
+        a = fn(qw, n, k, _bits(inp), m, _bits(A), _bits(B), r, alpha)
+        b = fn(qw, n, k, _bits(inp), m, _bits(A), _bits(B), r, alpha, p_drop=0.0, seed=77, offset=9)
+        assert np.array_equal(a, b)
+    ga = oracle.lora_grads(_bits(x), _bits(gh), m, n, k, _bits(A), _bits(B), r, alpha)
+    gb = oracle.lora_grads(_bits(x), _bits(gh), m, n, k, _bits(A), _bits(B), r, alpha, 0.0, 77, 9)
+    assert np.array_equal(ga[0], gb[0]) and np.array_equal(ga[1], gb[1])
+
+
+@pytest.mark.parametrize("p", [0.05, 0.3])
+def test_dropout_adjoint_identity(oracle, p):
+    # with one mask, the layer is linear in x and the input gradient is its adjoint
+    n, k, m, r, alpha = 64, 256, 4, 16, 32.0
+    qw, A, B, x, gh = _layer(oracle, n, k, m, r, 140)
+    h = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha, p_drop=p, seed=9, offset=100)
+    gx = oracle.qlora_bwd_x(qw, n, k, _bits(gh), m, _bits(A), _bits(B), r, alpha, p_drop=p, seed=9, offset=100)
+    lhs = np.sum(gh.double().numpy() * h)
+    rhs = np.sum(gx * x.double().numpy())
+    assert abs(lhs - rhs) <= 1e-11 * (abs(lhs) + np.sqrt(np.sum(h * h)))
+    # and the mask matters: without it the adapter part differs
+    h0 = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    assert not np.allclose(h, h0)
+
+
+def test_dropout_adapter_term_is_the_masked_product(oracle):
+    # zero base: h = s / (1 - p) B A (keep * x), keep from the generator (brute force, tiny shape)
+    n, k, m, r, alpha, p = 16, 64, 3, 4, 8.0, 0.25
+    zero, A, B, x, gh = _layer(oracle, n, k, m, r, 150, zero_w=True)
+    keep = oracle.dropout_keep(31, 7, p, m, k)
+    h = oracle.qlora_fwd(zero, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha, p_drop=p, seed=31, offset=7)
+    xd = x.double().numpy() * keep
+    ref = (alpha / r) / (1 - p) * (xd @ A.double().numpy().T) @ B.double().numpy().T
+    np.testing.assert_allclose(h, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_dropout_mean_over_seeds_is_the_plain_adapter(oracle):
+    # inverted dropout is unbiased: the mean of the masked adapter term over independent masks
+    # tends to the unmasked term (zero base isolates the adapter)
+    n, k, m, r, alpha, p = 8, 64, 2, 4, 8.0, 0.3
+    zero, A, B, x, gh = _layer(oracle, n, k, m, r, 160, zero_w=True)
+    plain = oracle.qlora_fwd(zero, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    runs = np.stack([oracle.qlora_fwd(zero, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha, p_drop=p, seed=s)
+                     for s in range(400)])
+    mean, sem = runs.mean(axis=0), runs.std(axis=0) / math.sqrt(runs.shape[0])
+    assert np.all(np.abs(mean - plain) <= 5 * sem + 1e-12)
+
+
+def test_dropout_grads_are_adjoint_of_forward(oracle):
+    n, k, m, r, alpha, p = 48, 192, 5, 16, 32.0, 0.1
+    qw, A, B, x, gh = _layer(oracle, n, k, m, r, 170)
+    gA, gB = oracle.lora_grads(_bits(x), _bits(gh), m, n, k, _bits(A), _bits(B), r, alpha, p, 5, 11)
+    B2 = (torch.randn(n, r, generator=torch.Generator().manual_seed(171)) * 0.01).to(torch.bfloat16)
+    A2 = (torch.randn(r, k, generator=torch.Generator().manual_seed(172)) * 0.01).to(torch.bfloat16)
+    fwd = lambda AA, BB: oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(AA), _bits(BB), r, alpha, p_drop=p, seed=5,
+                                          offset=11)
+    h1 = fwd(A, B)
+    g = gh.double().numpy()
+    lhs = np.sum(g * (fwd(A, B2) - h1))
+    rhs = np.sum(gB * (B2.double().numpy() - B.double().numpy()))
+    assert abs(lhs - rhs) <= 1e-10 * (abs(lhs) + 1e-300) + 1e-13
+    lhs = np.sum(g * (fwd(A2, B) - h1))
+    rhs = np.sum(gA * (A2.double().numpy() - A.double().numpy()))
+    assert abs(lhs - rhs) <= 1e-10 * (abs(lhs) + 1e-300) + 1e-13
