@@ -21,7 +21,8 @@ BLOCK, GROUP, MAX_RANK = 64, 256, 256
 
 EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
             "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x",
-            "qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qn_status_string",
+            "qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qlora_linear_fwd_dropout",
+            "qlora_linear_bwd_x_dropout", "qlora_lora_grads_dropout", "qn_status_string",
             "qn_last_error", "qn_launch_count")
 
 
@@ -35,6 +36,16 @@ class CWeight(ctypes.Structure):
     _fields_ = [("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64), ("codes", ctypes.c_void_p),
                 ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
                 ("absmax_mean", ctypes.c_void_p)]
+
+
+class CDropout(ctypes.Structure):
+    """qn_lora_dropout (see the header): rate p, generator key and element-index offset."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+
+
+def _dropout_struct(dropout) -> CDropout:
+    p, seed, offset = dropout
+    return CDropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFFFFFFFFFF)
 
 
 _lock = threading.Lock()
@@ -67,8 +78,15 @@ def load(path: str | None = None):
         lib.qlora_lora_grads_workspace_size.argtypes = [i64, ctypes.c_int, sz]
         lib.qlora_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, P,
                                          ctypes.c_size_t, P]
+        D = ctypes.POINTER(CDropout)
+        lib.qlora_linear_fwd_dropout.argtypes = [W, P, i64, P, P, ctypes.c_int, ctypes.c_float, D, P, P,
+                                                 ctypes.c_size_t, P]
+        lib.qlora_linear_bwd_x_dropout.argtypes = lib.qlora_linear_fwd_dropout.argtypes
+        lib.qlora_lora_grads_dropout.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, D, P, P,
+                                                 P, ctypes.c_size_t, P]
         for f in ("qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
-                  "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x"):
+                  "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x",
+                  "qlora_linear_fwd_dropout", "qlora_linear_bwd_x_dropout", "qlora_lora_grads_dropout"):
             getattr(lib, f).restype = st
         lib.qn_status_string.argtypes = [st]
         lib.qn_status_string.restype = ctypes.c_char_p
@@ -259,8 +277,9 @@ def _lora(A, B, r):
 
 def qlora_linear_fwd(w: NF4Weight, x: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
                      alpha: float, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                     stream=None) -> torch.Tensor:
-    """h = dequant(W) x + (alpha/r) B (A x); x is M x k_in, h is M x n_out (bf16)."""
+                     stream=None, dropout=None) -> torch.Tensor:
+    """h = dequant(W) x + (alpha/r) B (A x); x is M x k_in, h is M x n_out (bf16).
+    dropout = (p, seed, offset): LoRA dropout of the adapter's input (qlora_linear_fwd_dropout)."""
     _dev_bf16(x, "x")
     r = check_linear_shapes(w.n_out, w.k_in, x, A, B, out, bwd=False)
     M = x.shape[0]
@@ -270,15 +289,22 @@ def qlora_linear_fwd(w: NF4Weight, x: torch.Tensor, A: torch.Tensor | None, B: t
     _same_device(w, x, A, B, out)
     workspace, ws_bytes = _workspace(workspace, linear_workspace_size(M, w.n_out, w.k_in, r), x.device)
     cw = w.c_struct()
-    _check(load().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
-                                   _ptr(workspace), ws_bytes, _stream(stream)), "qlora_linear_fwd")
+    if dropout is None:
+        _check(load().qlora_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                                       _ptr(workspace), ws_bytes, _stream(stream)), "qlora_linear_fwd")
+    else:
+        d = _dropout_struct(dropout)
+        _check(load().qlora_linear_fwd_dropout(ctypes.byref(cw), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                               ctypes.byref(d), _ptr(out), _ptr(workspace), ws_bytes,
+                                               _stream(stream)), "qlora_linear_fwd_dropout")
     return out
 
 
 def qlora_linear_bwd_x(w: NF4Weight, grad_h: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
                        alpha: float, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                       stream=None) -> torch.Tensor:
-    """grad_x = dequant(W)^T grad_h + (alpha/r) A^T (B^T grad_h); grad_h is M x n_out."""
+                       stream=None, dropout=None) -> torch.Tensor:
+    """grad_x = dequant(W)^T grad_h + (alpha/r) A^T (B^T grad_h); grad_h is M x n_out.
+    dropout = (p, seed, offset): the forward's LoRA-dropout mask (qlora_linear_bwd_x_dropout)."""
     _dev_bf16(grad_h, "grad_h")
     r = check_linear_shapes(w.n_out, w.k_in, grad_h, A, B, out, bwd=True)
     M = grad_h.shape[0]
@@ -288,9 +314,15 @@ def qlora_linear_bwd_x(w: NF4Weight, grad_h: torch.Tensor, A: torch.Tensor | Non
     _same_device(w, grad_h, A, B, out)
     workspace, ws_bytes = _workspace(workspace, linear_workspace_size(M, w.n_out, w.k_in, r), grad_h.device)
     cw = w.c_struct()
-    _check(load().qlora_linear_bwd_x(ctypes.byref(cw), _ptr(grad_h), M, _ptr(A), _ptr(B), r, float(alpha),
-                                     _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
-           "qlora_linear_bwd_x")
+    if dropout is None:
+        _check(load().qlora_linear_bwd_x(ctypes.byref(cw), _ptr(grad_h), M, _ptr(A), _ptr(B), r, float(alpha),
+                                         _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)),
+               "qlora_linear_bwd_x")
+    else:
+        d = _dropout_struct(dropout)
+        _check(load().qlora_linear_bwd_x_dropout(ctypes.byref(cw), _ptr(grad_h), M, _ptr(A), _ptr(B), r,
+                                                 float(alpha), ctypes.byref(d), _ptr(out), _ptr(workspace),
+                                                 ws_bytes, _stream(stream)), "qlora_linear_bwd_x_dropout")
     return out
 
 
@@ -326,8 +358,9 @@ def lora_grads_workspace_size(M: int, r: int) -> int:
 
 def qlora_lora_grads(x: torch.Tensor, grad_h: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      grad_A: torch.Tensor | None = None, grad_B: torch.Tensor | None = None,
-                     workspace: torch.Tensor | None = None, stream=None):
-    """(grad_A (r x k_in), grad_B (n_out x r)) in fp32 for x (M x k_in) and grad_h (M x n_out)."""
+                     workspace: torch.Tensor | None = None, stream=None, dropout=None):
+    """(grad_A (r x k_in), grad_B (n_out x r)) in fp32 for x (M x k_in) and grad_h (M x n_out).
+    dropout = (p, seed, offset): the forward's LoRA-dropout mask (qlora_lora_grads_dropout)."""
     for t, nm in ((x, "x"), (grad_h, "grad_h"), (A, "A"), (B, "B")):
         _dev_bf16(t, nm)
     if x.dim() != 2 or grad_h.dim() != 2 or A.dim() != 2 or B.dim() != 2:
@@ -352,7 +385,14 @@ def qlora_lora_grads(x: torch.Tensor, grad_h: torch.Tensor, A: torch.Tensor, B: 
     for t in (grad_h, A, B, grad_A, grad_B, workspace):
         if t.device != x.device:
             raise ValueError(f"tensor on {t.device}, x is on {x.device}")
-    _check(load().qlora_lora_grads(_ptr(x), _ptr(grad_h), M, n, k, _ptr(A), _ptr(B), r, float(alpha), _ptr(grad_A),
-                                   _ptr(grad_B), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                   _stream(stream)), "qlora_lora_grads")
+    wsb = workspace.numel() * workspace.element_size()
+    if dropout is None:
+        _check(load().qlora_lora_grads(_ptr(x), _ptr(grad_h), M, n, k, _ptr(A), _ptr(B), r, float(alpha),
+                                       _ptr(grad_A), _ptr(grad_B), _ptr(workspace), wsb, _stream(stream)),
+               "qlora_lora_grads")
+    else:
+        d = _dropout_struct(dropout)
+        _check(load().qlora_lora_grads_dropout(_ptr(x), _ptr(grad_h), M, n, k, _ptr(A), _ptr(B), r, float(alpha),
+                                               ctypes.byref(d), _ptr(grad_A), _ptr(grad_B), _ptr(workspace), wsb,
+                                               _stream(stream)), "qlora_lora_grads_dropout")
     return grad_A, grad_B

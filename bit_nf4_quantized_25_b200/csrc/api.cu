@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" boundary declared in include/qlora_nf4.h: argument checks,
 // size queries, path selection (few-token decode kernels or the tcgen05 GEMM) and launches.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -73,6 +74,19 @@ qn_status check_lora(const void *A, const void *B, int r, float alpha) {
     if (!A || !B) return fail(QN_EINVAL, "null adapter pointer with r=%d", r);
     if (!aligned16(A) || !aligned16(B)) return fail(QN_EALIGN, "A or B not 16-byte aligned");
     if (!(alpha == alpha) || alpha - alpha != 0.0f) return fail(QN_EINVAL, "alpha is not finite");
+    return QN_OK;
+}
+
+// The kernels' mask parameters and the adapter scale under dropout (s / (1 - p)); off when d is
+// null, p == 0 or there is no adapter.
+qn_status resolve_dropout(const qn_lora_dropout *d, int r, float sc, DropoutArgs *drop, float *sc_eff) {
+    *drop = DropoutArgs{0, 0, 0};
+    *sc_eff = sc;
+    if (!d || d->p == 0.0f || r == 0) return QN_OK;
+    if (!(d->p > 0.0f && d->p < 1.0f)) return fail(QN_EINVAL, "dropout rate p=%g outside [0, 1)", (double)d->p);
+    const double thr = floor(static_cast<double>(d->p) * 4294967296.0);
+    *drop = DropoutArgs{d->seed, d->offset, static_cast<uint32_t>(thr)};
+    *sc_eff = static_cast<float>(static_cast<double>(sc) / (1.0 - static_cast<double>(d->p)));
     return QN_OK;
 }
 
@@ -202,6 +216,13 @@ qn_status qlora_lora_grads_workspace_size(int64_t M, int r, size_t *ws_bytes) {
 qn_status qlora_lora_grads(const void *x, const void *grad_h, int64_t M, int64_t n_out, int64_t k_in, const void *A,
                            const void *B, int r, float alpha, float *grad_A, float *grad_B, void *ws, size_t ws_bytes,
                            void *stream) {
+    return qlora_lora_grads_dropout(x, grad_h, M, n_out, k_in, A, B, r, alpha, nullptr, grad_A, grad_B, ws, ws_bytes,
+                                    stream);
+}
+
+qn_status qlora_lora_grads_dropout(const void *x, const void *grad_h, int64_t M, int64_t n_out, int64_t k_in,
+                                   const void *A, const void *B, int r, float alpha, const qn_lora_dropout *dropout,
+                                   float *grad_A, float *grad_B, void *ws, size_t ws_bytes, void *stream) {
     qn_status s = check_shape(n_out, k_in);
     if (s != QN_OK) return s;
     if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
@@ -215,10 +236,13 @@ qn_status qlora_lora_grads(const void *x, const void *grad_h, int64_t M, int64_t
     const size_t need = lora_grads_workspace_bytes(M, r);
     if (!ws || ws_bytes < need) return fail(QN_EWORKSPACE, "adapter-gradient workspace needs %zu bytes", need);
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
-    const float sc = alpha / static_cast<float>(r);
+    DropoutArgs drop;
+    float sc = alpha / static_cast<float>(r);
+    s = resolve_dropout(dropout, r, sc, &drop, &sc);
+    if (s != QN_OK) return s;
     return cuda_status(launch_lora_grads(static_cast<const uint16_t *>(x), static_cast<const uint16_t *>(grad_h), M,
                                          n_out, k_in, static_cast<const uint16_t *>(A),
-                                         static_cast<const uint16_t *>(B), r, sc, grad_A, grad_B, ws,
+                                         static_cast<const uint16_t *>(B), r, sc, drop, grad_A, grad_B, ws,
                                          static_cast<cudaStream_t>(stream)),
                        "qlora_lora_grads");
 }
@@ -230,9 +254,11 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
     if (M < 0 || M > kMaxDim) return fail(QN_EINVAL, "M=%lld out of range", (long long)M);
     if (r < 0 || r > QN_MAX_RANK) return fail(QN_EINVAL, "rank r=%d outside [0, %d]", r, QN_MAX_RANK);
     // The few-token kernels keep the error word, the adapter product and its ready flag there
-    // (4 KB); the tensor-core path the error word and the adapter operand.
+    // (4 KB); the tensor-core path and the paths that add a dropout-masked adapter term after a
+    // base-only pass the error word and the M x roundup(r, 64) adapter operand.
     const size_t few = decode_fwd_workspace_bytes() > 4096 ? decode_fwd_workspace_bytes() : 4096;
-    *ws_bytes = (M > kDecodeMaxM || r > kDecodeMaxRank) ? gemm_workspace_bytes(M, r) : few;
+    const size_t op = gemm_workspace_bytes(M, r);
+    *ws_bytes = op > few ? op : few;
     g_err.clear();
     return QN_OK;
 }
@@ -272,10 +298,19 @@ qn_status qlora_workspace_check(void *ws, void *stream) {
 
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B, int r,
                            float alpha, void *h, void *ws, size_t ws_bytes, void *stream) {
+    return qlora_linear_fwd_dropout(w, x, M, A, B, r, alpha, nullptr, h, ws, ws_bytes, stream);
+}
+
+qn_status qlora_linear_fwd_dropout(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
+                                   int r, float alpha, const qn_lora_dropout *dropout, void *h, void *ws,
+                                   size_t ws_bytes, void *stream) {
     qn_status s = check_linear(w, x, M, A, B, r, alpha, h, ws, ws_bytes);
     if (s != QN_OK) return s;
+    DropoutArgs drop;
+    float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
+    s = resolve_dropout(dropout, r, sc, &drop, &sc);
+    if (s != QN_OK) return s;
     if (M == 0 || w->n_out == 0) return QN_OK;
-    const float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
     const WeightView wv = view(w);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *xp = static_cast<const uint16_t *>(x);
@@ -287,21 +322,33 @@ qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, con
         int *err = static_cast<int *>(ws);
         for (int64_t m0 = 0; m0 < M; m0 += kDecodeTokens) {
             const int mc = static_cast<int>(M - m0 < kDecodeTokens ? M - m0 : kDecodeTokens);
-            cudaError_t e = launch_decode_fwd(wv, xp + m0 * w->k_in, mc, Ap, Bp, r, sc, hp + m0 * w->n_out, err, st);
+            DropoutArgs dc = drop;
+            dc.offset += static_cast<uint64_t>(m0 * w->k_in);  // element index of token m0
+            cudaError_t e =
+                launch_decode_fwd(wv, xp + m0 * w->k_in, mc, Ap, Bp, r, sc, dc, hp + m0 * w->n_out, err, st);
             if (e != cudaSuccess) return cuda_status(e, "qlora_linear_fwd");
         }
         return cuda_status(cudaSuccess, "");
     }
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
-    return cuda_status(launch_gemm_fwd(wv, xp, M, Ap, Bp, r, sc, hp, ws, st), "qlora_linear_fwd");
+    return cuda_status(launch_gemm_fwd(wv, xp, M, Ap, Bp, r, sc, hp, ws, st, &drop), "qlora_linear_fwd");
 }
 
 qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A, const void *B,
                              int r, float alpha, void *grad_x, void *ws, size_t ws_bytes, void *stream) {
+    return qlora_linear_bwd_x_dropout(w, grad_h, M, A, B, r, alpha, nullptr, grad_x, ws, ws_bytes, stream);
+}
+
+qn_status qlora_linear_bwd_x_dropout(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A,
+                                     const void *B, int r, float alpha, const qn_lora_dropout *dropout, void *grad_x,
+                                     void *ws, size_t ws_bytes, void *stream) {
     qn_status s = check_linear(w, grad_h, M, A, B, r, alpha, grad_x, ws, ws_bytes);
     if (s != QN_OK) return s;
+    DropoutArgs drop;
+    float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
+    s = resolve_dropout(dropout, r, sc, &drop, &sc);
+    if (s != QN_OK) return s;
     if (M == 0 || w->k_in == 0) return QN_OK;
-    const float sc = r > 0 ? alpha / static_cast<float>(r) : 0.0f;
     const WeightView wv = view(w);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *gp = static_cast<const uint16_t *>(grad_h);
@@ -313,23 +360,38 @@ qn_status qlora_linear_bwd_x(const qn_nf4_weight *w, const void *grad_h, int64_t
         int *err = static_cast<int *>(ws);
         for (int64_t m0 = 0; m0 < M; m0 += kDecodeTokens) {
             const int mc = static_cast<int>(M - m0 < kDecodeTokens ? M - m0 : kDecodeTokens);
+            DropoutArgs dc = drop;
+            dc.offset += static_cast<uint64_t>(m0 * w->k_in);  // element index of token m0
             cudaError_t e =
-                launch_decode_bwd_stream(wv, gp + m0 * w->n_out, mc, Ap, Bp, r, sc, xp + m0 * w->k_in, err, st);
+                launch_decode_bwd_stream(wv, gp + m0 * w->n_out, mc, Ap, Bp, r, sc, dc, xp + m0 * w->k_in, err, st);
             if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
         }
         return cuda_status(cudaSuccess, "");
     }
+    // Under dropout the other paths run base-only and the masked adapter term is added after them
+    // (u = s B^T grad_h into the workspace, then grad_x += mask * u A).
+    const bool masked = drop.thr != 0u;
+    const int ra = masked ? 0 : r;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
     if (M > kDecodeMaxM && gemm_supported(w->n_out, w->k_in, M, true)) {
-        if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
-        return cuda_status(launch_gemm_bwd(wv, gp, M, Ap, Bp, r, sc, xp, ws, st), "qlora_linear_bwd_x");
+        cudaError_t e = launch_gemm_bwd(wv, gp, M, Ap, Bp, ra, sc, xp, ws, st);
+        if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
+    } else {
+        // many tokens with n_out % 8 != 0 (the GEMM's TMA row-stride rule), or few tokens with a
+        // rank above 64 or rows the streamed kernel's boxes cannot read: the register-streaming
+        // few-token kernel in chunks of 32 tokens
+        constexpr int kChunk = 32;
+        for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
+            const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);
+            cudaError_t e = launch_decode_bwd(wv, gp + m0 * w->n_out, mc, Ap, Bp, ra, sc, xp + m0 * w->k_in, st);
+            if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
+        }
     }
-    // many tokens with n_out % 8 != 0 (the GEMM's TMA row-stride rule), or few tokens with a rank
-    // above 64 or rows the streamed kernel's boxes cannot read: the register-streaming few-token
-    // kernel in chunks of 32 tokens
-    constexpr int kChunk = 32;
-    for (int64_t m0 = 0; m0 < M; m0 += kChunk) {
-        const int mc = static_cast<int>(M - m0 < kChunk ? M - m0 : kChunk);
-        cudaError_t e = launch_decode_bwd(wv, gp + m0 * w->n_out, mc, Ap, Bp, r, sc, xp + m0 * w->k_in, st);
+    if (masked) {
+        const int RT = (r + 63) / 64 * 64;
+        uint16_t *u = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
+        cudaError_t e = launch_lora_down(gp, M, w->n_out, Bp, 1, r, r, sc, u, RT, st);
+        if (e == cudaSuccess) e = launch_adapter_up_masked(u, M, RT, Ap, r, w->k_in, drop, xp, st);
         if (e != cudaSuccess) return cuda_status(e, "qlora_linear_bwd_x");
     }
     return cuda_status(cudaSuccess, "");

@@ -37,6 +37,7 @@
 // other shapes to the register-streaming kernel of decode_bwd.cu.
 #include <cudaTypedefs.h>
 
+#include "dropout.cuh"
 #include "host_cache.h"
 #include "stream_common.cuh"
 
@@ -70,7 +71,8 @@ struct BwdArgs {
     int nrs;     // row stages (ceil(n / kSR))
     int chunks;  // feature chunks (ceil(k / 256)): grid rows 1 .. chunks when r > 0, else 0 ..
     int M, r, rpad, rk16;
-    float s;
+    float s;           // adapter scale (divided by 1 - p under dropout)
+    DropoutArgs drop;  // mask of the forward's adapter input (thr == 0: none); offset of token 0
     int C, stages;
     int q_tma;  // FP8 codes by a TMA box (rows of FP8 codes 16-byte aligned), else per-row copies
     uint32_t slot_bytes, g_off, q_off, s_off;  // chunk slot: codes, grad_h, FP8 codes, group scales
@@ -180,9 +182,10 @@ __device__ __forceinline__ void adapter_body(const CUtensorMap *tm_g, const CUte
     } else {
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
-            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
-                fail();
+            // every lane waits for the stage; the warp leaves together (mma.sync and shuffles below)
+            const bool ok = !*bb.abort_flag && mbar_wait(&bb.full[slot], (s / S) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (!ok) fail();
                 break;
             }
             const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
@@ -397,12 +400,15 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
-            bool ok = true;
-            if (lane == 0 && s >= S) ok = mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) {
-                if (lane == 0) fail();
+            // lane 0 decides (abort flag, slot wait) and the warp follows it as one
+            int st = 0;  // 0 go on, 1 aborted elsewhere, 2 this wait ran out
+            if (lane == 0) {
+                if (*bb.abort_flag) st = 1;
+                else if (s >= S && !mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1)) st = 2;
+            }
+            st = __shfl_sync(0xffffffffu, st, 0);
+            if (st != 0) {
+                if (lane == 0 && st == 2) fail();
                 break;
             }
             if (s >= S) stage_weights(s, l2_policy_evict_first());
@@ -458,9 +464,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         const bool blk_ok = 4 * col + kg < p.nbr;
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
-            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
-                fail();
+            // every lane waits for the stage; the warp leaves together (mma.sync and shuffles below)
+            const bool ok = !*bb.abort_flag && mbar_wait(&bb.full[slot], (s / S) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (!ok) fail();
                 break;
             }
             const int64_t n0 = static_cast<int64_t>(rs_lo + s) * kSR;
@@ -555,7 +562,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                     acc[f][tg][3] += __uint_as_float(v.w);
                 }
         // adapter term of block kg (this CTA's when kg = crank mod C): A^T u from the staged tile
-        // [rpad ranks][64 features] (128-byte swizzle: chunk c of rank row j at c ^ (j & 7))
+        // [rpad ranks][64 features] (128-byte swizzle: chunk c of rank row j at c ^ (j & 7)); under
+        // dropout only the elements whose input survived the forward's mask receive it
         if (p.r > 0 && kg % C == crank) {
             const uint32_t ab = at + static_cast<uint32_t>((kg / C) * p.rpad * 128);
             auto a_el = [&](int j, int feat) -> uint32_t {  // A[j][64 kg + feat] (bf16 bits)
@@ -564,21 +572,42 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
                 return v;
             };
-            for (int kc = 0; kc < p.rk16 / 16; ++kc) {
-                const int j = 16 * kc + 2 * t;
+            auto pair = [&](int jj, int feat) -> uint32_t {
+                if (jj >= p.rpad) return 0u;
+                return a_el(jj, feat) | (a_el(jj + 1, feat) << 16);
+            };
 #pragma unroll
-                for (int f = 0; f < 4; ++f) {
-                    const int fa = 8 * g + 2 * f, fb = fa + 1;
-                    auto pair = [&](int jj, int feat) -> uint32_t {
-                        if (jj >= p.rpad) return 0u;
-                        return a_el(jj, feat) | (a_el(jj + 1, feat) << 16);
-                    };
+            for (int f = 0; f < 4; ++f) {
+                const int fa = 8 * g + 2 * f, fb = fa + 1;
+                float ad[NG][4];
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) ad[tg][0] = ad[tg][1] = ad[tg][2] = ad[tg][3] = 0.0f;
+                for (int kc = 0; kc < p.rk16 / 16; ++kc) {
+                    const int j = 16 * kc + 2 * t;
                     const uint32_t a0 = pair(j, fa), a1 = pair(j, fb), a2 = pair(j + 8, fa), a3 = pair(j + 8, fb);
 #pragma unroll
                     for (int tg = 0; tg < NG; ++tg) {
                         const uint32_t ur = ut + static_cast<uint32_t>((tg * 8 + g) * p.rk16 + j) * 2u;
-                        mma_16816(acc[f][tg], a0, a1, a2, a3, lds32(ur), lds32(ur + 16));
+                        mma_16816(ad[tg], a0, a1, a2, a3, lds32(ur), lds32(ur + 16));
                     }
+                }
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) {
+                    // fragment element e: feature 64 kg + fa + (e >> 1), token tg 8 + 2 t + (e & 1)
+                    uint32_t keep = 0xfu;
+                    if (p.drop.thr != 0u) {
+                        const int64_t feat = f0 + 64 * kg + fa;
+                        const int tok = tg * 8 + 2 * t;
+                        const uint32_t k0 =
+                            dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(tok * p.k + feat), 2);
+                        const uint32_t k1 = dropout_keep_bits(
+                            p.drop, p.drop.offset + static_cast<uint64_t>((tok + 1) * p.k + feat), 2);
+                        // e = 0: (fa, tok), 1: (fa, tok + 1), 2: (fb, tok), 3: (fb, tok + 1)
+                        keep = (k0 & 1u) | ((k1 & 1u) << 1) | ((k0 & 2u) << 1) | ((k1 & 2u) << 2);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (keep & (1u << e)) acc[f][tg][e] += ad[tg][e];
                 }
             }
         }
@@ -755,7 +784,7 @@ size_t smem_bytes(const BwdArgs &a) { return static_cast<size_t>(a.bar_off) + 25
 
 template <int NG>
 cudaError_t launch_ng(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A, const uint16_t *B, int r,
-                      float s, uint16_t *gx, int *err, cudaStream_t st) {
+                      float s, const DropoutArgs &drop, uint16_t *gx, int *err, cudaStream_t st) {
     constexpr int MP = 8 * NG;
     const void *kern = reinterpret_cast<const void *>(k_decode_bwd<NG>);
     int sms = 148;
@@ -781,6 +810,7 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *gh, int M, const uint
     a.rpad = round_rank(r);
     a.rk16 = (a.rpad + 15) & ~15;
     a.s = s;
+    a.drop = drop;
     a.q_tma = (a.nbr % 16) == 0 ? 1 : 0;
     const int extra = r > 0 ? 1 : 0;
     // cluster size: the largest C <= 8 with (chunks + 1) x C <= SMs, every cluster resident and
@@ -874,12 +904,13 @@ bool decode_bwd_stream_supported(int64_t n, int64_t k, int r) {
 }
 
 cudaError_t launch_decode_bwd_stream(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
-                                     const uint16_t *B, int r, float s, uint16_t *gx, int *err, cudaStream_t st) {
+                                     const uint16_t *B, int r, float s, const DropoutArgs &drop, uint16_t *gx,
+                                     int *err, cudaStream_t st) {
     if (M <= 0 || w.k == 0) return cudaSuccess;
     if (M > kDecodeTokens || r > kDecodeMaxRank || !decode_bwd_stream_supported(w.n, w.k, r))
         return cudaErrorInvalidValue;
-    if (M <= 8) return launch_ng<1>(w, gh, M, A, B, r, s, gx, err, st);
-    return launch_ng<2>(w, gh, M, A, B, r, s, gx, err, st);
+    if (M <= 8) return launch_ng<1>(w, gh, M, A, B, r, s, drop, gx, err, st);
+    return launch_ng<2>(w, gh, M, A, B, r, s, drop, gx, err, st);
 }
 
 }  // namespace qn

@@ -46,6 +46,7 @@
 // CTA's work and drains the loads already issued.
 #include <cudaTypedefs.h>
 
+#include "dropout.cuh"
 #include "host_cache.h"
 #include "stream_common.cuh"
 
@@ -56,7 +57,7 @@ namespace qn {
 // Two buffers, used by alternate launches, so that a chain's last two launches can be compared.
 // Slots 0 and 1 (start, past the wait): globaltimer (ns); the other slots: SM cycles since the
 // marking thread entered the kernel (clock64: one counter per SM, exact within a CTA).
-__device__ unsigned long long g_fwd_timeline[2][1024][16];
+__device__ unsigned long long g_fwd_timeline[2][1024][24];
 __device__ __forceinline__ void tl_mark(int buf, int slot, long long c0) {
     const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
     if (cta >= 1024) return;
@@ -102,6 +103,7 @@ struct FwdArgs {
     const float *sigma;
     const float *mu;
     const uint16_t *B;  // n x r
+    const uint16_t *x;  // M x k (the chunk CTAs' stage copies)
     uint16_t *h;        // M x n
     int *err;
     uint16_t *t_ws;     // [MP][rk16] bf16: bf16(s A x), published by the adapter cluster
@@ -112,7 +114,8 @@ struct FwdArgs {
     int nbr;     // blocks per row (k / 64)
     int ncol;    // stage columns (ceil(nbr / 4))
     int M, r, rpad, rk16;  // rpad: r rounded up to 8, 16, 32 or 64; rk16: to 16 (0 without adapter)
-    float s;
+    float s;     // adapter scale (divided by 1 - p under dropout)
+    DropoutArgs drop;  // mask of the adapter's input x (thr == 0: none); offset of this launch's token 0
     int R, m;    // rows and m-tiles per chunk
     int C;       // K-slices (cluster size)
     int chunks;  // row chunks: grid rows 1 .. chunks when r > 0 (row 0 is the adapter cluster), else 0 .. chunks - 1
@@ -130,9 +133,9 @@ struct FwdArgs {
 #endif
 };
 
-// Barrier block: full[kMaxStages], empty[kMaxStages], consts, recv, abort flag.
+// Barrier block: full[kMaxStages], empty[kMaxStages], consts, recv, tready, abort flag.
 struct Bars {
-    uint64_t *full, *empty, *consts, *recv;
+    uint64_t *full, *empty, *consts, *recv, *tready;
     volatile uint32_t *abort_flag;
 };
 
@@ -142,7 +145,8 @@ __device__ __forceinline__ Bars bars_of(uint8_t *smem, const FwdArgs &p) {
     b.empty = b.full + kMaxStages;
     b.consts = b.empty + kMaxStages;
     b.recv = b.consts + 1;
-    b.abort_flag = reinterpret_cast<volatile uint32_t *>(b.recv + 1);
+    b.tready = b.recv + 1;
+    b.abort_flag = reinterpret_cast<volatile uint32_t *>(b.tready + 1);
     return b;
 }
 
@@ -214,12 +218,37 @@ __device__ __forceinline__ void adapter_body(const CUtensorMap *tm_xp, const CUt
         const int jrow = nt_job * 8 + g;  // rank row of this lane's B fragment
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
-            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
-                fail();
+            // every lane waits for the stage; the warp leaves together (mma.sync and shuffles below)
+            const bool ok = !*bb.abort_flag && mbar_wait(&bb.full[slot], (s / S) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (!ok) fail();
                 break;
             }
             const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
+            if (p.drop.thr != 0u) {
+                // LoRA dropout: zero the dropped elements of the stage's x box in place, one
+                // 16-byte chunk (8 elements of one token row) per consumer thread
+                const int items = kStageBlocks * p.M * 8;
+                for (int i = threadIdx.x - 32; i < items; i += kConsumers * 32) {
+                    const int blk = i / (p.M * 8), rem = i - blk * (p.M * 8), tok = rem >> 3, c = rem & 7;
+                    const int64_t kk0 = static_cast<int64_t>(4 * (col_lo + s) + blk) * 64 + 8 * c;
+                    if (kk0 >= p.k) continue;
+                    const uint32_t a = sl + static_cast<uint32_t>(blk * MP * 128 + tok * 128 + ((c ^ (tok & 7)) << 4));
+                    const uint32_t keep =
+                        dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(tok * p.k + kk0), 8);
+                    uint4 v = lds128(a);
+                    v.x = mask_pair(v.x, keep);
+                    v.y = mask_pair(v.y, keep >> 2);
+                    v.z = mask_pair(v.z, keep >> 4);
+                    v.w = mask_pair(v.w, keep >> 6);
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+                                 "r"(v.w)
+                                 : "memory");
+                }
+                // these writes precede the TMA that refills the slot (async proxy)
+                fence_proxy_async_smem();
+                named_sync(4, kConsumers * 32);
+            }
             for (int j = 0; j < NT; ++j) {
                 const int kq = kq0 + kq_step * j;
                 const int blk = kq >> 2, q4 = kq & 3;
@@ -322,7 +351,11 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     const int col_lo = p.ncol * crank / C, col_hi = p.ncol * (crank + 1) / C;
     const int ns = col_hi - col_lo;
     const int S = p.stages;
+#ifdef QN_NPRE_MAX
+    const int npre = ns < S ? (ns < QN_NPRE_MAX ? ns : QN_NPRE_MAX) : (S < QN_NPRE_MAX ? S : QN_NPRE_MAX);
+#else
     const int npre = ns < S ? ns : S;  // stages whose codes are requested before the dependency wait
+#endif
     // rows [r_lo, r_hi) of the chunk are finalised by this CTA (C > 1)
     const int r_lo = p.R * crank / C, r_hi = p.R * (crank + 1) / C, nr = r_hi - r_lo;
     const int nrmax = (p.R + C - 1) / C;
@@ -333,7 +366,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     const uint32_t s_qs = s_base + p.qs_off;
     const uint32_t s_ss = s_base + p.ss_off;
     const uint32_t tb = s_base + p.tb_off;  // [MP tokens][rk16] bf16 t
-    const uint32_t bs = s_base + p.bs_off;  // [assigned m-tiles x 16 rows][bs_stride] B rows
+    const uint32_t bs = s_base + p.bs_off;  // [rows r_lo .. r_hi of the chunk][bs_stride] B rows
     const Bars bb = bars_of(smem, p);
     // the staged group scales start at index s_lo (that of the chunk's first block of the slice)
     const int64_t s_lo = (row0 * p.nbr + 4 * col_lo) >> 8;
@@ -359,12 +392,13 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 #endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&bb.full[s], 1);  // lane 0's arrive.expect_tx (x) + the boxes' bytes
+            mbar_init(&bb.full[s], 33);  // lane 0 + the producer lanes' x copies; codes by bytes
             mbar_init(&bb.empty[s], kConsumers);
         }
         mbar_init(bb.consts, kConsumers * 32);  // one cp.async arrival per consumer thread
         mbar_init(bb.recv, 1);
         if (C > 1) mbar_arrive_expect_tx(bb.recv, static_cast<uint32_t>(C * nr * MP * 4));
+        mbar_init(bb.tready, 1);  // the producer: t and the B rows are in shared memory
         *bb.abort_flag = 0u;
         fence_barrier_init();
     }
@@ -373,7 +407,6 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // ------------------------------------------ producer, before the dependency wait: weights
         if (lane == 0) {
             tma_prefetch_desc(tm_codes);
-            tma_prefetch_desc(tm_x);
             const uint64_t pol = l2_policy_evict_first();
             for (int s = 0; s < npre; ++s) {
                 mbar_expect_tx(&bb.full[s], p.codes_bytes);
@@ -439,43 +472,54 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
         // Stage s: wait for its slot (from the second round on, then request its codes); arm the
-        // full barrier with the x bytes and request the x box. After the first round is armed,
-        // stage the B rows of this CTA's up-projection (m-tiles mt = crank mod C).
+        // full barrier (lane 0's arrival) and copy the stage's x. After the first round is armed,
+        // stage the B rows of the rows this CTA finalises (r_lo .. r_hi; all rows when C == 1).
         int ni = 0;  // stages armed
-        const int nassign = p.r > 0 ? (p.m - crank + C - 1) / C : 0;
         for (int s = 0; s < ns; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
+            // lane 0 decides (abort flag, slot wait) and the warp follows it as one
+            bool ok = true;
             if (lane == 0) {
-                bool ok = true;
-                if (s >= S) {
+                if (*bb.abort_flag) ok = false;
+                if (ok && s >= S) {
                     ok = mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1);
-                    if (ok) {
-                        mbar_expect_tx(&bb.full[slot], p.codes_bytes);
-                        load_codes(s, l2_policy_evict_first());
-                    } else {
-                        fail();
-                    }
+                    if (!ok) fail();
                 }
-                if (ok) {
-                    mbar_arrive_expect_tx(&bb.full[slot], p.x_bytes);
-                    const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes;
-                    tma_load_3d_saddr(sl + p.x_off, tm_x, &bb.full[slot], 0, 0, 4 * (col_lo + s));
+                if (ok && s >= npre) {
+                    mbar_expect_tx(&bb.full[slot], p.codes_bytes);
+                    load_codes(s, l2_policy_evict_first());
                 }
+                if (ok) mbar_arrive(&bb.full[slot]);
             }
-            __syncwarp();
-            if (*bb.abort_flag) break;
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            // x of the stage by the lanes' 16-byte copies (not TMA: these small loads must not
+            // queue behind the code boxes): [block][token][64 values], 16-byte chunk c of row
+            // b M + tok at c ^ (row & 7); blocks past the row read as zero
+            {
+                const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes + p.x_off;
+                const int items = kStageBlocks * p.M * 8;
+                for (int i = lane; i < items; i += 32) {
+                    const int b = i / (p.M * 8), rem = i - b * (p.M * 8), tok = rem >> 3, c = rem & 7;
+                    const int row = b * p.M + tok;
+                    const int64_t kk = static_cast<int64_t>(4 * (col_lo + s) + b) * 64 + 8 * c;
+                    const bool v = kk < p.k;
+                    cp_async16_zfill(sl + static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
+                                     v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
+                }
+                cp_async_arrive_noinc(&bb.full[slot]);
+            }
+            QN_TL(16 + (s < 4 ? s : 3), lane == 0 && s < 4);
             ni = s + 1;
             QN_TL(2, lane == 0 && s == S - 1);
-            if (s == npre - 1 && nassign > 0) {
-                // B rows 16 mt .. 16 mt + 16 of the assigned m-tiles, ranks 0 .. rk16 (zeros past
-                // r and past the last row)
+            if (s == npre - 1 && p.r > 0) {
+                // B rows r_lo .. r_hi of the chunk, ranks 0 .. rk16 (zeros past r and past the
+                // last row)
                 const int cpr = p.rk16 / 8;  // 16-byte chunks per row
                 const bool r8 = (p.r & 7) == 0;
-                for (int i = lane; i < nassign * 16 * cpr; i += 32) {
+                for (int i = lane; i < nr * cpr; i += 32) {
                     const int rr = i / cpr, c = i - (i / cpr) * cpr;
-                    const int mt = (rr >> 4) * C + crank;
-                    const int64_t row = row0 + 16 * mt + (rr & 15);
+                    const int64_t row = row0 + r_lo + rr;
                     const uint32_t dst = bs + static_cast<uint32_t>(rr) * p.bs_stride + 16u * c;
                     if (r8) {
                         const bool v = row < nrow && 8 * c < p.r;
@@ -497,9 +541,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             }
         }
         // drain: the stages whose codes were requested before the wait but that were never
-        // armed get their arrival now; then every requested stage lands before the CTA exits
+        // armed get their 33 arrivals now; then every requested stage lands before the CTA exits
         if (lane == 0) {
-            for (int s = ni; s < npre; ++s) mbar_arrive(&bb.full[s]);
+            for (int s = ni; s < npre; ++s) mbar_arrive_cnt(&bb.full[s], 33);
             const int hi = ni > npre ? ni : npre;
             for (int s = (hi > S ? hi - S : 0); s < hi; ++s) mbar_wait(&bb.full[s % S], (s / S) & 1);
         }
@@ -526,8 +570,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             }
             QN_TL(12, lane == 0);
         }
-        cp_async_wait_all();
+        cp_async_wait_all();  // the B rows
         __syncwarp();
+        if (lane == 0) mbar_arrive(bb.tready);
+        if (C > 1) cluster_wait();  // phase 1 (every thread waits once)
     } else {
         // ------------------------------------------------------------------ consumers
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
@@ -571,9 +617,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 
         for (int s = 0; s < nsc; ++s) {
             const int slot = s % S;
-            if (*bb.abort_flag) break;
-            if (!mbar_wait(&bb.full[slot], (s / S) & 1)) {
-                fail();
+            // every lane waits for the stage; the warp leaves together (mma.sync and shuffles below)
+            const bool ok = !*bb.abort_flag && mbar_wait(&bb.full[slot], (s / S) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (!ok) fail();
                 break;
             }
             QN_TL(3, threadIdx.x == 32 && s == 0);
@@ -644,13 +691,12 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     }
 
     // ---------------------------------------------------------------------- reduction
-    // The ring is idle from here on (every stage was consumed, the producer drained its loads):
-    // its space holds the exchange buffer of the four block-warps.
+    // The ring is idle once every consumer has left its loop (they waited for every stage, so
+    // every box has landed): its space holds the exchange buffer of the four block-warps. The
+    // consumers sum the block-warps of each m-tile in a fixed order (kg = 0, 1, 2, 3).
     QN_TL(5, threadIdx.x == 32);
-    __syncthreads();
-    QN_TL(6, threadIdx.x == 0);
     const uint32_t red = s_base + p.post_off;  // [3][16 m-tiles][32 lanes][NG*4] f32
-    if (warp > 0 && kg > 0) {
+    auto store_partials = [&]() {
 #pragma unroll
         for (int i = 0; i < MW; ++i) {
             const int mt = rg + 4 * i;
@@ -664,63 +710,85 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 }
             }
         }
-    }
-    __syncthreads();
-    QN_TL(9, threadIdx.x == 0);
-    const bool run_ok = !*bb.abort_flag;
-    if (warp > 0 && kg == 0) {
-        // sum the four block-warps of each m-tile (kg = 0, 1, 2, 3 in order); the CTA that owns
-        // the m-tile's adapter term (mt = crank mod C) adds B t
+    };
+    auto sum_partials = [&](int i) {
+        const int mt = rg + 4 * i;
 #pragma unroll
-        for (int i = 0; i < MW; ++i) {
-            const int mt = rg + 4 * i;
-            if (mt >= p.m) continue;
+        for (int q = 0; q < 3; ++q) {
 #pragma unroll
-            for (int q = 0; q < 3; ++q) {
-#pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    const uint4 v = lds128(red + static_cast<uint32_t>(((q * kMaxM + mt) * 32 + lane) * NG + tg) * 16);
-                    acc[i][tg][0] += __uint_as_float(v.x);
-                    acc[i][tg][1] += __uint_as_float(v.y);
-                    acc[i][tg][2] += __uint_as_float(v.z);
-                    acc[i][tg][3] += __uint_as_float(v.w);
-                }
+            for (int tg = 0; tg < NG; ++tg) {
+                const uint4 v = lds128(red + static_cast<uint32_t>(((q * kMaxM + mt) * 32 + lane) * NG + tg) * 16);
+                acc[i][tg][0] += __uint_as_float(v.x);
+                acc[i][tg][1] += __uint_as_float(v.y);
+                acc[i][tg][2] += __uint_as_float(v.z);
+                acc[i][tg][3] += __uint_as_float(v.w);
             }
-            if (p.r > 0 && mt % C == crank) {
-                const uint32_t brow = bs + static_cast<uint32_t>(((mt / C) * 16 + g) * p.bs_stride);
-                for (int kc = 0; kc < p.rk16 / 16; ++kc) {
-                    const uint32_t j2 = static_cast<uint32_t>(16 * kc + 2 * t) * 2u;
-                    const uint32_t a0 = lds32(brow + j2), a2 = lds32(brow + j2 + 16);
-                    const uint32_t a1 = lds32(brow + 8 * p.bs_stride + j2), a3 = lds32(brow + 8 * p.bs_stride + j2 + 16);
+        }
+    };
+
+    if (C == 1) {
+        // one CTA holds whole rows: add B t to the summed fragments on the tensor cores and store
+        __syncthreads();  // every consumer has left its loop; the producer has t and the B rows
+        QN_TL(6, threadIdx.x == 0);
+        if (warp > 0 && kg > 0) store_partials();
+        __syncthreads();
+        QN_TL(9, threadIdx.x == 0);
+        const bool run_ok = !*bb.abort_flag;
+        if (warp > 0 && kg == 0) {
 #pragma unroll
-                    for (int tg = 0; tg < NG; ++tg) {
-                        const uint32_t tr = tb + static_cast<uint32_t>((tg * 8 + g) * p.rk16) * 2u + j2;
-                        mma_16816(acc[i][tg], a0, a1, a2, a3, lds32(tr), lds32(tr + 16));
+            for (int i = 0; i < MW; ++i) {
+                const int mt = rg + 4 * i;
+                if (mt >= p.m) continue;
+                sum_partials(i);
+                if (p.r > 0) {
+                    const uint32_t brow = bs + static_cast<uint32_t>((16 * mt + g) * p.bs_stride);
+                    for (int kc = 0; kc < p.rk16 / 16; ++kc) {
+                        const uint32_t j2 = static_cast<uint32_t>(16 * kc + 2 * t) * 2u;
+                        const uint32_t a0 = lds32(brow + j2), a2 = lds32(brow + j2 + 16);
+                        const uint32_t a1 = lds32(brow + 8 * p.bs_stride + j2),
+                                       a3 = lds32(brow + 8 * p.bs_stride + j2 + 16);
+#pragma unroll
+                        for (int tg = 0; tg < NG; ++tg) {
+                            const uint32_t tr = tb + static_cast<uint32_t>((tg * 8 + g) * p.rk16) * 2u + j2;
+                            mma_16816(acc[i][tg], a0, a1, a2, a3, lds32(tr), lds32(tr + 16));
+                        }
                     }
                 }
-            }
-            if (C == 1 && run_ok) {
-                const int64_t rA = row0 + 16 * mt + g, rB = rA + 8;
+                if (run_ok) {
+                    const int64_t rA = row0 + 16 * mt + g, rB = rA + 8;
 #pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    const int tok = tg * 8 + 2 * t;
+                    for (int tg = 0; tg < NG; ++tg) {
+                        const int tok = tg * 8 + 2 * t;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int64_t row = (e < 2) ? rA : rB;
-                        const int tk = tok + (e & 1);
-                        if (row < nrow && tk < p.M)
-                            p.h[static_cast<int64_t>(tk) * p.n + row] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(acc[i][tg][e]));
+                        for (int e = 0; e < 4; ++e) {
+                            const int64_t row = (e < 2) ? rA : rB;
+                            const int tk = tok + (e & 1);
+                            if (row < nrow && tk < p.M)
+                                p.h[static_cast<int64_t>(tk) * p.n + row] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(acc[i][tg][e]));
+                        }
                     }
                 }
             }
         }
-    }
-    QN_TL(10, threadIdx.x == 32);
-    if (C > 1) {
-        // partial sums of every row, all MP token columns, to the row's owner [src][row][MP] f32
+        QN_TL(10, threadIdx.x == 32);
+    } else if (warp > 0) {
+        // Cluster: the consumers reduce among themselves and push each row's partial sums (all MP
+        // token columns) to the row's owner [src][row][MP] f32 right away; the owner adds B t while
+        // it sums the C partials, so t from the adapter cluster is needed only there.
+        named_sync(2, kConsumers * 32);  // every consumer has left its loop: the ring is idle
+        QN_TL(6, threadIdx.x == 32);
+        if (kg > 0) store_partials();
+        named_sync(3, kConsumers * 32);
+        QN_TL(9, threadIdx.x == 32);
+        if (kg == 0) {
+#pragma unroll
+            for (int i = 0; i < MW; ++i)
+                if (rg + 4 * i < p.m) sum_partials(i);
+            QN_TL(10, threadIdx.x == 32);
+        }
         cluster_wait();  // phase 1: every CTA of the cluster runs (its barriers are initialised)
-        if (warp > 0 && kg == 0) {
+        if (kg == 0) {
             const uint32_t recv = s_base + p.recv_off;
 #pragma unroll
             for (int i = 0; i < MW; ++i) {
@@ -739,25 +807,46 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                         st_async_v2(dst + 32u * tg, acc[i][tg][2 * hh], acc[i][tg][2 * hh + 1], bar);
                 }
             }
+            QN_TL(11, threadIdx.x == 32);
         }
-        QN_TL(11, threadIdx.x == 32);
-        // rows [r_lo, r_hi): wait for the C partials, sum them in rank order
-        const bool ok = mbar_wait(bb.recv, 0);
-        if (!ok && threadIdx.x == 0) record_error(p.err, kErrTimeout);
-        QN_TL(13, threadIdx.x == 0);
-        if (ok && run_ok) {
+        // rows [r_lo, r_hi): the C partials in rank order, plus B t
+        bool ok = mbar_wait(bb.recv, 0);
+        if (ok && !mbar_wait(bb.tready, 0)) ok = false;
+        if (!ok && threadIdx.x == 32) record_error(p.err, kErrTimeout);
+        QN_TL(13, threadIdx.x == 32);
+        if (ok && !*bb.abort_flag) {
             const float *recvf = reinterpret_cast<const float *>(smem + p.recv_off);
-            for (int it = threadIdx.x; it < nr * p.M; it += kThreads) {
+            for (int it = threadIdx.x - 32; it < nr * p.M; it += kConsumers * 32) {
                 const int rr = it % nr, tok = it / nr;
                 const int64_t row = row0 + r_lo + rr;
                 if (row >= nrow) continue;
                 float sum = 0.0f;
                 for (int src = 0; src < C; ++src) sum += recvf[(src * nrmax + rr) * MP + tok];
+                if (p.r > 0) {
+                    const uint32_t brow = bs + static_cast<uint32_t>(rr) * p.bs_stride;
+                    const uint32_t trow = tb + static_cast<uint32_t>(tok * p.rk16) * 2u;
+                    float bt = 0.0f;
+                    for (int j = 0; j < p.rpad; j += 2) {
+                        const uint32_t bv = lds32(brow + 2u * j), tv = lds32(trow + 2u * j);
+                        bt = __fmaf_rn(bf16_lo(bv), bf16_lo(tv), bt);
+                        bt = __fmaf_rn(bf16_hi(bv), bf16_hi(tv), bt);
+                    }
+                    sum += bt;
+                }
                 p.h[static_cast<int64_t>(tok) * p.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
             }
         }
+        QN_TL(20, threadIdx.x == 32);
     }
     QN_TL(7, threadIdx.x == 0);
+#ifdef QN_TIMELINE
+    if (threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
+        if (cta < 1024) g_fwd_timeline[p.tl_buf & 1][cta][15] = t;  // end in ns: with slot 7 gives the clock
+    }
+#endif
 }
 
 template <int NG>
@@ -850,10 +939,10 @@ bool layout(FwdArgs &a, int MP) {
     const uint32_t qs = align_up(static_cast<uint32_t>(a.R) * a.qs_stride, 128);
     const uint32_t ss = align_up(static_cast<uint32_t>(s_max) * 4u, 128);
     const uint32_t tbb = a.r > 0 ? align_up(static_cast<uint32_t>(MP * a.rk16 * 2), 128) : 0u;
-    // staged B rows: the CTA's m-tiles (mt = crank mod C), 16 rows each, padded so that the eight
+    // staged B rows: the rows the CTA finalises (all R when C == 1), padded so that the eight
     // fragment rows fall on distinct bank groups
     a.bs_stride = static_cast<uint32_t>(2 * a.rk16 + 16);
-    const uint32_t bsb = a.r > 0 ? align_up(static_cast<uint32_t>((a.m + a.C - 1) / a.C * 16) * a.bs_stride, 128) : 0u;
+    const uint32_t bsb = a.r > 0 ? align_up(static_cast<uint32_t>((a.R + a.C - 1) / a.C) * a.bs_stride, 128) : 0u;
     const uint32_t post_chunk = 3 * kMaxM * 32 * 16 * (MP / 8);
     const uint32_t post_adapter = kConsumers * 32 * 16;
     const uint32_t post = post_chunk > post_adapter ? post_chunk : post_adapter;
@@ -955,7 +1044,7 @@ cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
 
 template <int NG>
 cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint16_t *A, const uint16_t *B, int r,
-                      float s, uint16_t *h, int *err, cudaStream_t st) {
+                      float s, const DropoutArgs &drop, uint16_t *h, int *err, cudaStream_t st) {
     constexpr int MP = 8 * NG;
     const void *kern = reinterpret_cast<const void *>(k_decode_fwd<NG>);
     int sms = 148;
@@ -967,6 +1056,7 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
     a.sigma = w.sigma;
     a.mu = w.mu;
     a.B = B;
+    a.x = x;
     a.h = h;
     a.err = err;
     char *wsb = reinterpret_cast<char *>(err);
@@ -982,6 +1072,7 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
     a.rpad = round_rank(r);
     a.rk16 = (a.rpad + 15) & ~15;
     a.s = s;
+    a.drop = drop;
 #ifdef QN_FWD_NO_EVICT_HINT
     a.evict_first = 0;
 #else
@@ -1065,11 +1156,11 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
 size_t decode_fwd_workspace_bytes() { return kWsT + 16 * 64 * 2; }
 
 cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A, const uint16_t *B,
-                              int r, float s, uint16_t *h, int *err, cudaStream_t st) {
+                              int r, float s, const DropoutArgs &drop, uint16_t *h, int *err, cudaStream_t st) {
     if (M <= 0 || w.n == 0) return cudaSuccess;
     if (M > kDecodeTokens || r > kDecodeMaxRank) return cudaErrorInvalidValue;
-    if (M <= 8) return launch_ng<1>(w, x, M, A, B, r, s, h, err, st);
-    return launch_ng<2>(w, x, M, A, B, r, s, h, err, st);
+    if (M <= 8) return launch_ng<1>(w, x, M, A, B, r, s, drop, h, err, st);
+    return launch_ng<2>(w, x, M, A, B, r, s, drop, h, err, st);
 }
 
 #ifdef QN_TIMELINE
@@ -1086,8 +1177,8 @@ extern "C" int qn_debug_fwd_smid(int *out, int n, int buf) {
 // buf 0: the last launch's timeline, 1: the one before it
 extern "C" int qn_debug_fwd_timeline(unsigned long long *out, int n, int buf) {
     const int which = (g_launches_tl - 1 - buf) & 1;
-    return cudaMemcpyFromSymbol(out, g_fwd_timeline, sizeof(unsigned long long) * 16 * (n < 1024 ? n : 1024),
-                                sizeof(unsigned long long) * 16 * 1024 * which) == cudaSuccess
+    return cudaMemcpyFromSymbol(out, g_fwd_timeline, sizeof(unsigned long long) * 24 * (n < 1024 ? n : 1024),
+                                sizeof(unsigned long long) * 24 * 1024 * which) == cudaSuccess
                ? 0
                : 1;
 }

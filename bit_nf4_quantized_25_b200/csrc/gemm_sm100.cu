@@ -578,13 +578,13 @@ bool gemm_supported(int64_t n, int64_t k, int64_t M, bool bwd) {
 }
 
 cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, const uint16_t *A, const uint16_t *B,
-                            int r, float s, uint16_t *h, void *ws, cudaStream_t st) {
+                            int r, float s, uint16_t *h, void *ws, cudaStream_t st, const DropoutArgs *drop) {
     int *err = static_cast<int *>(ws);
     uint16_t *t = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + 256);
     const int RT = (r + 63) / 64 * 64;
     // the error word is sticky: kernels only ever set it (qlora_workspace_check reads and clears it)
     if (r > 0) {
-        cudaError_t e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, st);
+        cudaError_t e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, st, drop);
         if (e != cudaSuccess) return e;
     }
     return launch_gemm_impl<false>(w, x, M, B, r, t, RT, h, err, st);

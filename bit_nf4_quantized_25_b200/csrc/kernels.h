@@ -14,6 +14,15 @@ struct WeightView {
     const float *mu;
 };
 
+// LoRA dropout of the adapter's input (dropout.cuh): element e = offset + m k_in + k of the
+// activation is kept when its Philox draw is >= thr; thr == 0 turns it off. The kernels take the
+// adapter scale already divided by 1 - p.
+struct DropoutArgs {
+    uint64_t seed;
+    uint64_t offset;
+    uint32_t thr;
+};
+
 // Lookup used by the quantiser: the interval [-1, 1] split into 64 cells of
 // width 1/32 plus the point 1.0; for cell j, `base[j]` is the number of code
 // thresholds below the cell and `thr[j]` the single threshold inside the cell
@@ -53,14 +62,16 @@ constexpr int kDecodeMaxRank = 64;
 // error word; it also holds the adapter product t and its ready flag, see
 // decode_fwd_workspace_bytes); a timeout of a bounded wait is recorded in the error word.
 cudaError_t launch_decode_fwd(const WeightView &w, const uint16_t *x, int M, const uint16_t *A,
-                              const uint16_t *B, int r, float s, uint16_t *h, int *err, cudaStream_t st);
+                              const uint16_t *B, int r, float s, const DropoutArgs &drop, uint16_t *h, int *err,
+                              cudaStream_t st);
 // Workspace bytes launch_decode_fwd uses (zeroed once before the first call).
 size_t decode_fwd_workspace_bytes();
 // grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h), streamed kernel: M <= kDecodeTokens tokens,
 // r <= kDecodeMaxRank, shapes with decode_bwd_stream_supported(), one launch; err is the
 // workspace (as for launch_decode_fwd).
 cudaError_t launch_decode_bwd_stream(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A,
-                                     const uint16_t *B, int r, float s, uint16_t *gx, int *err, cudaStream_t st);
+                                     const uint16_t *B, int r, float s, const DropoutArgs &drop, uint16_t *gx,
+                                     int *err, cudaStream_t st);
 // n_out % 8 == 0, r % 8 == 0 (or r == 0) and few enough 256-feature chunks for one wave.
 bool decode_bwd_stream_supported(int64_t n, int64_t k, int r);
 // grad_x = dequant(W)^T grad_h + s A^T (B^T grad_h) for M <= kDecodeMaxM tokens.
@@ -68,23 +79,30 @@ cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, co
                               const uint16_t *B, int r, float s, uint16_t *gx, cudaStream_t st);
 
 // Adapter down-projection for many tokens: out[m, j] = bf16(s * sum_i act[m,i] S(j,i)),
-// S(j,i) = small[j*ldj + i*ldk]; out is M x RT with zeros for j >= r.
+// S(j,i) = small[j*ldj + i*ldk]; out is M x RT with zeros for j >= r. With a dropout mask the
+// activation element (m, i) enters only when it survives (element index offset + m red + i).
 cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
-                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st);
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st,
+                             const DropoutArgs *drop = nullptr);
+// gx[m, k] = bf16(gx[m, k] + keep(m, k) sum_j u[m, j] A[j, k]): the adapter term of the input
+// gradient under dropout, added to a base-only gradient (u: M x RT bf16, already scaled).
+cudaError_t launch_adapter_up_masked(const uint16_t *u, int64_t M, int RT, const uint16_t *A, int r, int64_t k,
+                                     const DropoutArgs &drop, uint16_t *gx, cudaStream_t st);
 
 // Gradients of the adapter weights (fp32): grad_A (r x k), grad_B (n x r); workspace of
 // lora_grads_workspace_bytes(M, r) bytes holds t = x A^T and u = grad_h B (bf16).
 size_t lora_grads_workspace_bytes(int64_t M, int r);
 cudaError_t launch_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, int64_t k,
-                              const uint16_t *A, const uint16_t *B, int r, float s, float *grad_A, float *grad_B,
-                              void *ws, cudaStream_t st);
+                              const uint16_t *A, const uint16_t *B, int r, float s, const DropoutArgs &drop,
+                              float *grad_A, float *grad_B, void *ws, cudaStream_t st);
 
 // tcgen05 fused dequant-GEMM for many tokens (the LoRA down-projection runs first, into
 // the workspace). Workspace: a 256-byte header (error word) then the M x RT adapter operand.
 size_t gemm_workspace_bytes(int64_t M, int r);
 bool gemm_supported(int64_t n, int64_t k, int64_t M, bool bwd);
 cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, const uint16_t *A, const uint16_t *B,
-                            int r, float s, uint16_t *h, void *ws, cudaStream_t st);
+                            int r, float s, uint16_t *h, void *ws, cudaStream_t st,
+                            const DropoutArgs *drop = nullptr);
 cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, const uint16_t *A, const uint16_t *B,
                             int r, float s, uint16_t *gx, void *ws, cudaStream_t st);
 

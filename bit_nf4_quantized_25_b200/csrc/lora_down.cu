@@ -9,6 +9,7 @@
 // reduction, each running mma.sync m16n8k16 (tokens x adapter rank), and reduce through
 // shared memory in a fixed order.
 #include "common.cuh"
+#include "dropout.cuh"
 #include "kernels.h"
 
 namespace qn {
@@ -26,6 +27,7 @@ struct LoraDownParams {
     float s;
     uint16_t *out;  // M x RT
     int RT;
+    DropoutArgs drop;  // mask of act's elements (thr == 0: none)
 };
 
 // bf16 pair (v[i], v[i + 1]); kEven: i is even and v 4-byte aligned, so one 4-byte load.
@@ -64,10 +66,19 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
                     if (kk + 1 < p.red) return load_pair<kEven>(row + kk);
                     return kk < p.red ? static_cast<uint32_t>(ld_ro_u16(row + kk)) : 0u;
                 };
-                const uint32_t a0 = (vA && lo_ok) ? pair(aA, k0 + 2 * t) : 0u;
-                const uint32_t a1 = (vB && lo_ok) ? pair(aB, k0 + 2 * t) : 0u;
-                const uint32_t a2 = (vA && hi_ok) ? pair(aA, k0 + 2 * t + 8) : 0u;
-                const uint32_t a3 = (vB && hi_ok) ? pair(aB, k0 + 2 * t + 8) : 0u;
+                uint32_t a0 = (vA && lo_ok) ? pair(aA, k0 + 2 * t) : 0u;
+                uint32_t a1 = (vB && lo_ok) ? pair(aB, k0 + 2 * t) : 0u;
+                uint32_t a2 = (vA && hi_ok) ? pair(aA, k0 + 2 * t + 8) : 0u;
+                uint32_t a3 = (vB && hi_ok) ? pair(aB, k0 + 2 * t + 8) : 0u;
+                if (p.drop.thr != 0u) {
+                    // LoRA dropout of the activation: element (m, i) at index offset + m red + i
+                    const uint64_t eA = p.drop.offset + static_cast<uint64_t>(rowA * p.red + k0 + 2 * t);
+                    const uint64_t eB = p.drop.offset + static_cast<uint64_t>(rowB * p.red + k0 + 2 * t);
+                    a0 = mask_pair(a0, dropout_keep_bits(p.drop, eA, 2));
+                    a1 = mask_pair(a1, dropout_keep_bits(p.drop, eB, 2));
+                    a2 = mask_pair(a2, dropout_keep_bits(p.drop, eA + 8, 2));
+                    a3 = mask_pair(a3, dropout_keep_bits(p.drop, eB + 8, 2));
+                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int j = j0 + nt * 8 + g;
@@ -121,11 +132,84 @@ __global__ void __launch_bounds__(kLdWarps * 32) k_lora_down(const LoraDownParam
     }
 }
 
+// Adapter term of the input gradient under dropout: gx[m, k] += keep(m, k) sum_j u[m, j] A[j, k].
+// A CTA owns 32 tokens x 128 features; thread (ty, tx) accumulates tokens 4 ty .. + 4 and features
+// 4 tx .. + 4 in fp32 over rank chunks of 64 staged in shared memory (u transposed, A row-major).
+constexpr int kUpTok = 32, kUpFeat = 128, kUpRank = 64;
+
+struct UpParams {
+    const uint16_t *u;  // M x RT
+    int64_t M;
+    int RT;
+    const uint16_t *A;  // r x k
+    int r;
+    int64_t k;
+    DropoutArgs drop;
+    uint16_t *gx;  // M x k
+};
+
+__global__ void __launch_bounds__(256) k_adapter_up_masked(const UpParams p) {
+    __shared__ __align__(16) uint16_t uT[kUpRank][kUpTok];
+    __shared__ __align__(16) uint16_t As[kUpRank][kUpFeat];
+    const int ty = threadIdx.x >> 5, tx = threadIdx.x & 31;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kUpTok, f0 = static_cast<int64_t>(blockIdx.x) * kUpFeat;
+    float acc[4][4] = {};
+    for (int j0 = 0; j0 < p.RT && j0 < p.r; j0 += kUpRank) {
+        for (int i = threadIdx.x; i < kUpRank * kUpTok; i += 256) {
+            const int j = i / kUpTok, tk = i % kUpTok;
+            const int64_t m = m0 + tk;
+            uT[j][tk] = (m < p.M && j0 + j < p.RT) ? ld_ro_u16(p.u + m * p.RT + j0 + j) : static_cast<uint16_t>(0);
+        }
+        for (int i = threadIdx.x; i < kUpRank * kUpFeat; i += 256) {
+            const int j = i / kUpFeat, f = i % kUpFeat;
+            As[j][f] = (j0 + j < p.r && f0 + f < p.k) ? ld_ro_u16(p.A + static_cast<int64_t>(j0 + j) * p.k + f0 + f)
+                                                      : static_cast<uint16_t>(0);
+        }
+        __syncthreads();
+        for (int j = 0; j < kUpRank; ++j) {
+            const uint2 uv = *reinterpret_cast<const uint2 *>(&uT[j][4 * ty]);
+            const uint2 av = *reinterpret_cast<const uint2 *>(&As[j][4 * tx]);
+            const float uu[4] = {bf16_lo(uv.x), bf16_hi(uv.x), bf16_lo(uv.y), bf16_hi(uv.y)};
+            const float aa[4] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y)};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(uu[a], aa[b], acc[a][b]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int64_t m = m0 + 4 * ty + a;
+        const int64_t f = f0 + 4 * tx;
+        if (m >= p.M) continue;
+        const uint32_t keep = dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(m * p.k + f), 4);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (f + b >= p.k || !(keep & (1u << b))) continue;
+            uint16_t *dst = p.gx + m * p.k + f + b;
+            const float v = __uint_as_float(static_cast<uint32_t>(*dst) << 16) + acc[a][b];
+            *dst = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+    }
+}
+
 }  // namespace
 
+cudaError_t launch_adapter_up_masked(const uint16_t *u, int64_t M, int RT, const uint16_t *A, int r, int64_t k,
+                                     const DropoutArgs &drop, uint16_t *gx, cudaStream_t st) {
+    if (M <= 0 || k <= 0 || r <= 0) return cudaSuccess;
+    UpParams p{u, M, RT, A, r, k, drop, gx};
+    const dim3 grid(static_cast<unsigned>((k + kUpFeat - 1) / kUpFeat), static_cast<unsigned>((M + kUpTok - 1) / kUpTok));
+    k_adapter_up_masked<<<grid, 256, 0, st>>>(p);
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_lora_down(const uint16_t *act, int64_t M, int64_t red, const uint16_t *small, int64_t ldj,
-                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st) {
-    LoraDownParams p{act, M, red, small, ldj, ldk, r, s, out, RT};
+                             int64_t ldk, int r, float s, uint16_t *out, int RT, cudaStream_t st,
+                             const DropoutArgs *drop) {
+    LoraDownParams p{act, M, red, small, ldj, ldk, r, s, out, RT, drop ? *drop : DropoutArgs{0, 0, 0}};
     const unsigned grid = static_cast<unsigned>((M + 15) / 16);
     const bool even = (red & 1) == 0;
     auto go = [&](auto kern) { kern<<<grid, kLdWarps * 32, 0, st>>>(p); };

@@ -14,6 +14,7 @@
 // fp32 accumulation over all M tokens in a fixed order (bit-reproducible); results are fp32,
 // grad_A written transposed from its C = grad_A^T.
 #include "common.cuh"
+#include "dropout.cuh"
 #include "host_cache.h"
 #include "kernels.h"
 
@@ -37,6 +38,7 @@ struct TnArgs {
     float *C;        // output
     int64_t ldC;     // C[p * ldC + q] (transpose = false) or C[q * ldC + p] (transpose = true)
     bool transpose;
+    DropoutArgs drop;  // mask of L's elements (m, p) at index offset + m P + p (thr == 0: none)
 };
 
 __device__ __forceinline__ uint32_t saddr32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -104,6 +106,23 @@ __global__ void __launch_bounds__(kGThreads) k_tn(const TnArgs p) {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
+        if (p.drop.thr != 0u) {
+            // LoRA dropout: L is the forward's adapter input; zero its dropped elements in place
+            for (int i = threadIdx.x; i < kGM * (kGP / 8); i += kGThreads) {
+                const int row = i / (kGP / 8), seg = i % (kGP / 8);
+                const int64_t m = c * kGM + row, col = p0 + 8 * seg;
+                if (m >= p.M || col >= p.P) continue;
+                const uint32_t keep = dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(m * p.P + col), 8);
+                uint4 *v = reinterpret_cast<uint4 *>(&Ls[buf][row][8 * seg]);
+                uint4 w = *v;
+                w.x = mask_pair(w.x, keep);
+                w.y = mask_pair(w.y, keep >> 2);
+                w.z = mask_pair(w.z, keep >> 4);
+                w.w = mask_pair(w.w, keep >> 6);
+                *v = w;
+            }
+            __syncthreads();
+        }
 #pragma unroll
         for (int ks = 0; ks < kGM / 16; ++ks) {
             // A operand: L^T[p][m] for p = 16 warp .. + 16, m = 16 ks .. + 16 (matrix i: p half i & 1,
@@ -186,26 +205,26 @@ size_t lora_grads_workspace_bytes(int64_t M, int r) {
 }
 
 cudaError_t launch_lora_grads(const uint16_t *x, const uint16_t *gh, int64_t M, int64_t n, int64_t k,
-                              const uint16_t *A, const uint16_t *B, int r, float s, float *grad_A, float *grad_B,
-                              void *ws, cudaStream_t st) {
+                              const uint16_t *A, const uint16_t *B, int r, float s, const DropoutArgs &drop,
+                              float *grad_A, float *grad_B, void *ws, cudaStream_t st) {
     if (r <= 0) return cudaSuccess;
     const int RT = (r + 63) / 64 * 64;
     const size_t half = (static_cast<size_t>(M * RT) * 2 + 255) & ~size_t(255);
     uint16_t *t = static_cast<uint16_t *>(ws);
     uint16_t *u = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + half);
     if (M > 0) {
-        // t = x A^T and u = grad_h B (unscaled), bf16, M x RT
-        cudaError_t e = launch_lora_down(x, M, k, A, k, 1, r, 1.0f, t, RT, st);
+        // t = (mask x) A^T and u = grad_h B (unscaled), bf16, M x RT
+        cudaError_t e = launch_lora_down(x, M, k, A, k, 1, r, 1.0f, t, RT, st, &drop);
         if (e != cudaSuccess) return e;
         e = launch_lora_down(gh, M, n, B, 1, r, r, 1.0f, u, RT, st);
         if (e != cudaSuccess) return e;
     }
     // grad_B = s grad_h^T t   (n x r)
-    TnArgs gb{gh, n, t, RT, M, n, r, s, grad_B, r, false};
+    TnArgs gb{gh, n, t, RT, M, n, r, s, grad_B, r, false, DropoutArgs{0, 0, 0}};
     cudaError_t e = launch_tn(gb, st);
     if (e != cudaSuccess) return e;
-    // grad_A^T = s x^T u     (k x r), stored as grad_A (r x k)
-    TnArgs ga{x, k, u, RT, M, k, r, s, grad_A, k, true};
+    // grad_A^T = s (mask x)^T u     (k x r), stored as grad_A (r x k)
+    TnArgs ga{x, k, u, RT, M, k, r, s, grad_A, k, true, drop};
     return launch_tn(ga, st);
 }
 

@@ -243,6 +243,45 @@ qn_status qlora_lora_grads(const void *x, const void *grad_h, int64_t M, int64_t
                            const void *A, const void *B, int r, float alpha, float *grad_A, float *grad_B,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* LoRA dropout of the adapter's input (training). "QLoRA & PEFT family"
+ * (ai-reference-codex) 3.4 gives the rate (0.05-0.1) and the configuration in
+ * "How does QLoRA work for training?" (aivaro.ru) sets lora_dropout; the pages
+ * say no more. This library's reading: inverted dropout of x on the adapter
+ * branch only (the frozen base sees x unchanged). Element (m, k) of the M x
+ * k_in activation has index e = offset + m * k_in + k; it survives when word
+ * (e mod 4) of Philox4x32-10 (Salmon, Moraes, Dror and Shaw, SC 2011) at
+ * counter (e / 4 low 32 bits, e / 4 high 32 bits, 0, 0) with key (seed low 32
+ * bits, seed high 32 bits) is >= floor(p * 2^32); survivors are scaled by
+ * 1 / (1 - p) (folded into the adapter scale: alpha / r / (1 - p)). The same
+ * (seed, offset) in the forward, the input gradient and the adapter gradients
+ * gives the same mask. A null pointer or p == 0 turns it off. */
+typedef struct {
+    float p;          /* drop rate, 0 <= p < 1 */
+    uint64_t seed;    /* the generator's key */
+    uint64_t offset;  /* added to every element index */
+} qn_lora_dropout;
+
+/* qlora_linear_fwd with LoRA dropout of the adapter's input:
+ *   h = dequant(W) x + s / (1 - p) B (A (mask * x)).
+ * Arguments, workspace and errors as qlora_linear_fwd; QN_EINVAL also for p
+ * outside [0, 1). */
+qn_status qlora_linear_fwd_dropout(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
+                                   int r, float alpha, const qn_lora_dropout *dropout, void *h, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* qlora_linear_bwd_x under the forward's dropout mask:
+ *   grad_x = dequant(W)^T grad_h + mask * (s / (1 - p) A^T (B^T grad_h)).
+ * Arguments, workspace and errors as qlora_linear_bwd_x. */
+qn_status qlora_linear_bwd_x_dropout(const qn_nf4_weight *w, const void *grad_h, int64_t M, const void *A,
+                                     const void *B, int r, float alpha, const qn_lora_dropout *dropout, void *grad_x,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* qlora_lora_grads under the forward's dropout mask (x replaced by mask * x,
+ * s by s / (1 - p)). Arguments, workspace and errors as qlora_lora_grads. */
+qn_status qlora_lora_grads_dropout(const void *x, const void *grad_h, int64_t M, int64_t n_out, int64_t k_in,
+                                   const void *A, const void *B, int r, float alpha, const qn_lora_dropout *dropout,
+                                   float *grad_A, float *grad_B, void *ws, size_t ws_bytes, void *stream);
+
 /* Static description of a status code. */
 const char *qn_status_string(qn_status s);
 

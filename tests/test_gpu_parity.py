@@ -403,3 +403,87 @@ def test_bwd_many_tokens_with_unaligned_rows(oracle, n, M, r):
     # more than 64 tokens with n_out % 8 != 0 (the tensor-core path's TMA row-stride rule fails),
     # and few-token input gradients with a rank above 64: the fallback few-token kernel in chunks
     run_case(oracle, synth.LayerCase(f"bwd_unaligned{n}M{M}r{r}", n, 256, M, r, 2.0 * r, 0.02, 11 * n + M + r))
+
+
+# ---------------------------------------------------------------- LoRA dropout
+# "QLoRA & PEFT family" 3.4 and the lora_dropout setting of "How does QLoRA work for training?":
+# dropout of the adapter's input. With a zero base and identity adapters the layer returns the
+# masked, scaled input itself, so the mask is compared bit for bit with the oracle's generator;
+# the other tests compare whole layers (adapter-dominated, so that a wrong mask shows).
+
+def _zero_weight(n, k):
+    return qb.nf4_quantize(torch.zeros(n, k, dtype=torch.bfloat16, device=DEV))
+
+
+def _identity_adapters(r):
+    eye = torch.eye(r, dtype=torch.bfloat16, device=DEV)
+    return eye.contiguous(), eye.clone()
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 40, 100])
+def test_dropout_mask_is_the_generators(oracle, M):
+    n = k = r = 64
+    p, seed, offset = 0.25, 0x1234_5678_9ABC_DEF0, 12345
+    w = _zero_weight(n, k)
+    A, B = _identity_adapters(r)
+    x = (torch.rand(M, k, generator=torch.Generator().manual_seed(M)) + 0.5).to(torch.bfloat16).to(DEV)
+    # h = s / (1 - p) B (A (mask x)) = s / (1 - p) (mask x), s = alpha / r = 1
+    h = qb.qlora_linear_fwd(w, x, A, B, float(r) * (1 - p), dropout=(p, seed, offset))
+    gh = x.clone()
+    gx = qb.qlora_linear_bwd_x(w, gh, A, B, float(r) * (1 - p), dropout=(p, seed, offset))
+    torch.cuda.synchronize()
+    keep = oracle.dropout_keep(seed, offset, p, M, k)
+    for got, what in ((h, "fwd"), (gx, "bwd_x")):
+        g = got.float().cpu().numpy()
+        assert np.array_equal(g != 0, keep), f"{what}: {int(np.sum((g != 0) != keep))} mask bits differ"
+        np.testing.assert_allclose(g[keep], x.float().cpu().numpy()[keep], rtol=1e-2)
+
+
+@pytest.mark.parametrize("n,k,M,r,zero_base", [(4096, 4096, 1, 16, True), (4096, 4096, 5, 16, False),
+                                               (11008, 4096, 16, 16, True), (4096, 11008, 3, 64, True),
+                                               (256, 512, 300, 16, True), (204, 256, 40, 16, True),
+                                               (200, 448, 129, 8, True)])
+def test_dropout_layer_matches_oracle(oracle, n, k, M, r, zero_base):
+    # few-token kernels (M <= 16 per launch), the tensor-core path (M > 64) and the fallback
+    # paths (n_out % 8 != 0; M > 64 with n_out % 8 != 0): forward and input gradient vs the oracle
+    p, seed, offset = 0.1, 987654321, 3 * n + k
+    case = synth.LayerCase(f"drop{n}x{k}M{M}", n, k, M, r, 2.0 * r, 0.02, n + k + M)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV)
+    if zero_base:
+        W = torch.zeros_like(W)
+    A, B = A * 30, B * 30  # an adapter term comparable to the base
+    w = qb.nf4_quantize(W)
+    h = qb.qlora_linear_fwd(w, x, A, B, case.alpha, dropout=(p, seed, offset))
+    gx = qb.qlora_linear_bwd_x(w, gh, A, B, case.alpha, dropout=(p, seed, offset))
+    torch.cuda.synchronize()
+    hw = to_host_weight(w)
+    ref_h = oracle.qlora_fwd(hw, n, k, bits(x), M, bits(A), bits(B), r, case.alpha, p_drop=p, seed=seed,
+                             offset=offset)
+    ref_g = oracle.qlora_bwd_x(hw, n, k, bits(gh), M, bits(A), bits(B), r, case.alpha, p_drop=p, seed=seed,
+                               offset=offset)
+    assert_close(h, ref_h, f"{case.name} fwd")
+    assert_close(gx, ref_g, f"{case.name} bwd_x")
+
+
+@pytest.mark.parametrize("n,k,M,r", [(256, 256, 8, 4), (1024, 2048, 300, 16), (512, 4096, 33, 64)])
+def test_dropout_lora_grads_match_oracle(oracle, n, k, M, r):
+    p, seed, offset = 0.2, 42, 7
+    case = synth.LayerCase(f"dropgrads{n}x{k}M{M}", n, k, M, r, 2.0 * r, 0.02, 2 * n + k + M)
+    _, A, B, x, gh = synth.layer_inputs(case, DEV)
+    gA, gB = qb.qlora_lora_grads(x, gh, A, B, case.alpha, dropout=(p, seed, offset))
+    torch.cuda.synchronize()
+    rA, rB = oracle.lora_grads(bits(x), bits(gh), M, n, k, bits(A), bits(B), r, case.alpha, p, seed, offset)
+    _assert_close_f32(gA, rA, "grad_A")
+    _assert_close_f32(gB, rB, "grad_B")
+
+
+def test_dropout_rate_zero_is_the_plain_call():
+    case = synth.LayerCase("drop0", 1024, 2048, 9, 16, 32.0, 0.02, 5)
+    W, A, B, x, gh = synth.layer_inputs(case, DEV)
+    w = qb.nf4_quantize(W)
+    a = qb.qlora_linear_fwd(w, x, A, B, 32.0)
+    b = qb.qlora_linear_fwd(w, x, A, B, 32.0, dropout=(0.0, 11, 13))
+    c = qb.qlora_linear_bwd_x(w, gh, A, B, 32.0)
+    d = qb.qlora_linear_bwd_x(w, gh, A, B, 32.0, dropout=(0.0, 11, 13))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(c, d)
