@@ -122,7 +122,9 @@ struct FwdArgs {
     int stages;
     int evict_first;  // the codes are read with an L2 evict-first policy
     // shared-memory layout (byte offsets from the start of dynamic shared memory)
-    uint32_t slot_bytes, x_off;  // chunk CTAs: codes [R][128 B], x [4][M][128 B] at x_off
+    uint32_t slot_bytes, x_off;  // chunk CTAs: codes [R][128 B], x [4][M][128 B] at x_off (x_once == 0)
+    int x_once;                  // chunk CTAs stage the x of every stage once, after the dependency wait
+    uint32_t xs_off, xs_stage;   // ... at xs_off, xs_stage bytes per stage ([4][M][128 B])
     uint32_t a_off;              // adapter CTAs: x [4][MP][128 B] at 0, A [4][rpad][128 B] at a_off
     uint32_t ring_off, qs_off, ss_off, tb_off, bs_off, recv_off, bar_off, post_off;
     uint32_t qs_stride;  // bytes per chunk row of the staged FP8 codes
@@ -365,6 +367,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     const uint32_t s_ring = s_base + p.ring_off;
     const uint32_t s_qs = s_base + p.qs_off;
     const uint32_t s_ss = s_base + p.ss_off;
+    const uint32_t s_xs = s_base + p.xs_off;  // x of every stage (x_once)
     const uint32_t tb = s_base + p.tb_off;  // [MP tokens][rk16] bf16 t
     const uint32_t bs = s_base + p.bs_off;  // [rows r_lo .. r_hi of the chunk][bs_stride] B rows
     const Bars bb = bars_of(smem, p);
@@ -392,7 +395,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 #endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&bb.full[s], 33);  // lane 0 + the producer lanes' x copies; codes by bytes
+            // codes by bytes; one arrival, plus the producer lanes' x copies when x comes per stage
+            mbar_init(&bb.full[s], p.x_once ? 1 : 33);
             mbar_init(&bb.empty[s], kConsumers);
         }
         mbar_init(bb.consts, kConsumers * 32);  // one cp.async arrival per consumer thread
@@ -409,7 +413,11 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             tma_prefetch_desc(tm_codes);
             const uint64_t pol = l2_policy_evict_first();
             for (int s = 0; s < npre; ++s) {
-                mbar_expect_tx(&bb.full[s], p.codes_bytes);
+                // with x staged once, the stage is complete when its codes land: arm it now
+                if (p.x_once)
+                    mbar_arrive_expect_tx(&bb.full[s], p.codes_bytes);
+                else
+                    mbar_expect_tx(&bb.full[s], p.codes_bytes);
                 load_codes(s, pol);
             }
         }
@@ -451,6 +459,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         QN_TL(8, ct == 0);
         build_pair_lut(lut, ct, kConsumers * 32);
         named_sync(1, kConsumers * 32);  // the table is complete
+        QN_TL(23, ct == 0);
     }
     if (C > 1) cluster_arrive_relaxed();  // phase 1: this CTA runs (its shared memory may be written)
     grid_dependents_launch();
@@ -471,79 +480,106 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        // Stage s: wait for its slot (from the second round on, then request its codes); arm the
-        // full barrier (lane 0's arrival) and copy the stage's x. After the first round is armed,
-        // stage the B rows of the rows this CTA finalises (r_lo .. r_hi; all rows when C == 1).
-        int ni = 0;  // stages armed
-        for (int s = 0; s < ns; ++s) {
-            const int slot = s % S;
-            // lane 0 decides (abort flag, slot wait) and the warp follows it as one
-            bool ok = true;
-            if (lane == 0) {
-                if (*bb.abort_flag) ok = false;
-                if (ok && s >= S) {
-                    ok = mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1);
-                    if (!ok) fail();
-                }
-                if (ok && s >= npre) {
-                    mbar_expect_tx(&bb.full[slot], p.codes_bytes);
-                    load_codes(s, l2_policy_evict_first());
-                }
-                if (ok) mbar_arrive(&bb.full[slot]);
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            // x of the stage by the lanes' 16-byte copies (not TMA: these small loads must not
-            // queue behind the code boxes): [block][token][64 values], 16-byte chunk c of row
-            // b M + tok at c ^ (row & 7); blocks past the row read as zero
-            {
-                const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes + p.x_off;
-                const int items = kStageBlocks * p.M * 8;
-                for (int i = lane; i < items; i += 32) {
-                    const int b = i / (p.M * 8), rem = i - b * (p.M * 8), tok = rem >> 3, c = rem & 7;
-                    const int row = b * p.M + tok;
-                    const int64_t kk = static_cast<int64_t>(4 * (col_lo + s) + b) * 64 + 8 * c;
-                    const bool v = kk < p.k;
-                    cp_async16_zfill(sl + static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
-                                     v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
-                }
-                cp_async_arrive_noinc(&bb.full[slot]);
-            }
-            QN_TL(16 + (s < 4 ? s : 3), lane == 0 && s < 4);
-            ni = s + 1;
-            QN_TL(2, lane == 0 && s == S - 1);
-            if (s == npre - 1 && p.r > 0) {
-                // B rows r_lo .. r_hi of the chunk, ranks 0 .. rk16 (zeros past r and past the
-                // last row)
-                const int cpr = p.rk16 / 8;  // 16-byte chunks per row
-                const bool r8 = (p.r & 7) == 0;
-                for (int i = lane; i < nr * cpr; i += 32) {
-                    const int rr = i / cpr, c = i - (i / cpr) * cpr;
-                    const int64_t row = row0 + r_lo + rr;
-                    const uint32_t dst = bs + static_cast<uint32_t>(rr) * p.bs_stride + 16u * c;
-                    if (r8) {
-                        const bool v = row < nrow && 8 * c < p.r;
-                        cp_async16_zfill(dst, v ? p.B + row * p.r + 8 * c : p.B, v ? 16u : 0u);
-                    } else {
-                        uint32_t w[4];
+        // B rows r_lo .. r_hi of the chunk (all rows when C == 1), ranks 0 .. rk16 (zeros past r
+        // and past the last row)
+        auto stage_brows = [&]() {
+            if (p.r == 0) return;
+            const int cpr = p.rk16 / 8;  // 16-byte chunks per row
+            const bool r8 = (p.r & 7) == 0;
+            for (int i = lane; i < nr * cpr; i += 32) {
+                const int rr = i / cpr, c = i - (i / cpr) * cpr;
+                const int64_t row = row0 + r_lo + rr;
+                const uint32_t dst = bs + static_cast<uint32_t>(rr) * p.bs_stride + 16u * c;
+                if (r8) {
+                    const bool v = row < nrow && 8 * c < p.r;
+                    cp_async16_zfill(dst, v ? p.B + row * p.r + 8 * c : p.B, v ? 16u : 0u);
+                } else {
+                    uint32_t w[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 8 * c + 2 * e;
-                            const uint32_t lo = (row < nrow && j < p.r) ? ld_ro_u16(p.B + row * p.r + j) : 0u;
-                            const uint32_t hi = (row < nrow && j + 1 < p.r) ? ld_ro_u16(p.B + row * p.r + j + 1) : 0u;
-                            w[e] = lo | (hi << 16);
-                        }
-                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]),
-                                     "r"(w[2]), "r"(w[3])
-                                     : "memory");
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 8 * c + 2 * e;
+                        const uint32_t lo = (row < nrow && j < p.r) ? ld_ro_u16(p.B + row * p.r + j) : 0u;
+                        const uint32_t hi = (row < nrow && j + 1 < p.r) ? ld_ro_u16(p.B + row * p.r + j + 1) : 0u;
+                        w[e] = lo | (hi << 16);
                     }
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                                 "r"(w[3])
+                                 : "memory");
                 }
+            }
+        };
+        int ni = 0;  // stages armed
+        if (p.x_once) {
+            // The first round was armed with its code requests; from then on lane 0 waits for a
+            // free slot and requests the next stage's codes.
+            stage_brows();
+            ni = npre;
+            if (lane == 0) {
+                for (int s = npre; s < ns; ++s) {
+                    const int slot = s % S;
+                    if (*bb.abort_flag) break;
+                    if (!mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1)) {
+                        fail();
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bb.full[slot], p.codes_bytes);
+                    load_codes(s, l2_policy_evict_first());
+                    ni = s + 1;
+                }
+            }
+            ni = __shfl_sync(0xffffffffu, ni, 0);
+        } else {
+            // Stage s: wait for its slot (from the second round on, then request its codes); arm
+            // the full barrier (lane 0's arrival) and copy the stage's x. After the first round
+            // is armed, stage the B rows.
+            for (int s = 0; s < ns; ++s) {
+                const int slot = s % S;
+                // lane 0 decides (abort flag, slot wait) and the warp follows it as one
+                bool ok = true;
+                if (lane == 0) {
+                    if (*bb.abort_flag) ok = false;
+                    if (ok && s >= S) {
+                        ok = mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1);
+                        if (!ok) fail();
+                    }
+                    if (ok && s >= npre) {
+                        mbar_expect_tx(&bb.full[slot], p.codes_bytes);
+                        load_codes(s, l2_policy_evict_first());
+                    }
+                    if (ok) mbar_arrive(&bb.full[slot]);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                QN_TL(21, lane == 0 && s == 0);
+                // x of the stage by the lanes' 16-byte copies (not TMA: these small loads must
+                // not queue behind the code boxes): [block][token][64 values], 16-byte chunk c of
+                // row b M + tok at c ^ (row & 7); blocks past the row read as zero
+                {
+                    const uint32_t sl = s_ring + static_cast<uint32_t>(slot) * p.slot_bytes + p.x_off;
+                    const int items = kStageBlocks * p.M * 8;
+                    for (int i = lane; i < items; i += 32) {
+                        const int b = i / (p.M * 8), rem = i - b * (p.M * 8), tok = rem >> 3, c = rem & 7;
+                        const int row = b * p.M + tok;
+                        const int64_t kk = static_cast<int64_t>(4 * (col_lo + s) + b) * 64 + 8 * c;
+                        const bool v = kk < p.k;
+                        cp_async16_zfill(sl + static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
+                                         v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
+                    }
+                    QN_TL(22, lane == 0 && s == 0);
+                    cp_async_arrive_noinc(&bb.full[slot]);
+                }
+                QN_TL(16 + (s < 4 ? s : 3), lane == 0 && s < 4);
+                ni = s + 1;
+                QN_TL(2, lane == 0 && s == S - 1);
+                if (s == npre - 1) stage_brows();
             }
         }
-        // drain: the stages whose codes were requested before the wait but that were never
-        // armed get their 33 arrivals now; then every requested stage lands before the CTA exits
+        // drain: in the per-stage mode, the stages whose codes were requested before the wait but
+        // that were never armed get their 33 arrivals now; then every requested stage lands
+        // before the CTA exits
         if (lane == 0) {
-            for (int s = ni; s < npre; ++s) mbar_arrive_cnt(&bb.full[s], 33);
+            if (!p.x_once)
+                for (int s = ni; s < npre; ++s) mbar_arrive_cnt(&bb.full[s], 33);
             const int hi = ni > npre ? ni : npre;
             for (int s = (hi > S ? hi - S : 0); s < hi; ++s) mbar_wait(&bb.full[s % S], (s / S) & 1);
         }
@@ -576,6 +612,25 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         if (C > 1) cluster_wait();  // phase 1 (every thread waits once)
     } else {
         // ------------------------------------------------------------------ consumers
+        if (p.x_once) {
+            // x of every stage of the slice, [stage][block][token][64 values] with 16-byte chunk c
+            // of row b M + tok at c ^ (row & 7); blocks past the row read as zero
+            const int ct = threadIdx.x - 32;
+            const int per = kStageBlocks * p.M * 8;  // 16-byte chunks per stage
+            for (int i = ct; i < ns * per; i += kConsumers * 32) {
+                const int sx = i / per, j = i - sx * per;
+                const int b = j / (p.M * 8), rem = j - b * (p.M * 8), tok = rem >> 3, c = rem & 7;
+                const int row = b * p.M + tok;
+                const int64_t kk = static_cast<int64_t>(4 * (col_lo + sx) + b) * 64 + 8 * c;
+                const bool v = kk < p.k;
+                cp_async16_zfill(s_xs + static_cast<uint32_t>(sx) * p.xs_stage +
+                                     static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
+                                 v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
+            }
+            cp_async_wait_all();
+            named_sync(5, kConsumers * 32);  // every consumer's copies have landed
+            QN_TL(22, ct == 0);
+        }
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
         const float mu = __ldg(p.mu);
@@ -641,7 +696,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 }
                 cmine[pass] = c;
             }
-            const uint32_t xb = sl + p.x_off;
+            const uint32_t xb = p.x_once ? s_xs + static_cast<uint32_t>(s) * p.xs_stage : sl + p.x_off;
             uint4 x0[NG], x1[NG];
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) {
@@ -916,19 +971,24 @@ int round_rank(int r) { return r <= 0 ? 0 : r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 
 
 uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Shared-memory layout of one launch shape; false if it does not fit.
-bool layout(FwdArgs &a, int MP) {
+// Shared-memory layout of one launch shape, x staged once (x_once) or per stage in the ring
+// slots; false if it does not fit.
+bool layout_mode(FwdArgs &a, int MP, bool x_once) {
     const uint32_t codes = static_cast<uint32_t>(a.R) * 128u;  // multiple of 2048 (R = 16 m)
     const uint32_t xb = kStageBlocks * static_cast<uint32_t>(a.M) * 128u;
     const uint32_t xpb = kStageBlocks * MP * 128u;
     const uint32_t ab = a.r > 0 ? kStageBlocks * a.rpad * 128u : 0u;
-    a.x_off = codes;
+    const int nsmax = (a.ncol + a.C - 1) / a.C;
+    a.x_once = x_once ? 1 : 0;
+    a.x_off = x_once ? 0u : codes;
+    a.xs_stage = xb;
+    const uint32_t chunk_slot = x_once ? codes : codes + xb;
     a.a_off = xpb;
-    a.slot_bytes = align_up(codes + xb > xpb + ab ? codes + xb : xpb + ab, 1024);
+    a.slot_bytes = align_up(chunk_slot > xpb + ab ? chunk_slot : xpb + ab, 1024);
     a.codes_bytes = codes;
     a.x_bytes = xb;
     a.xa_bytes = xpb + ab;
-    const int nsmax = (a.ncol + a.C - 1) / a.C;
+    const uint32_t xs = x_once ? align_up(static_cast<uint32_t>(nsmax) * xb, 128) : 0u;
     // staged FP8 codes: 16-byte chunks per chunk row, an odd count so that rows fall on
     // distinct bank groups
     const int nch = (15 + 4 * nsmax + 15) / 16;
@@ -950,7 +1010,7 @@ bool layout(FwdArgs &a, int MP) {
     const uint32_t recv_adapter = a.r > 0 ? static_cast<uint32_t>(a.C * MP * a.rpad * 4) : 0u;
     const uint32_t recv = align_up(recv_chunk > recv_adapter ? recv_chunk : recv_adapter, 128);
     const uint32_t bars = 256;
-    const uint64_t fixed = static_cast<uint64_t>(kLutBytes) + qs + ss + tbb + bsb + recv + bars;
+    const uint64_t fixed = static_cast<uint64_t>(kLutBytes) + qs + ss + tbb + bsb + xs + recv + bars;
     if (fixed + a.slot_bytes > kSmemLimit) return false;
     int stages = static_cast<int>((kSmemLimit - fixed) / a.slot_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -983,10 +1043,19 @@ bool layout(FwdArgs &a, int MP) {
     off += tbb;
     a.bs_off = off;
     off += bsb;
+    a.xs_off = off;
+    off += xs;
     a.recv_off = off;
     off += recv;
     a.bar_off = off;
     return static_cast<uint64_t>(off) + bars <= kSmemLimit;
+}
+
+bool layout(FwdArgs &a, int MP) {
+#ifndef QN_FWD_NO_X_ONCE
+    if (layout_mode(a, MP, true)) return true;
+#endif
+    return layout_mode(a, MP, false);
 }
 
 size_t smem_bytes(const FwdArgs &a) { return static_cast<size_t>(a.bar_off) + 256; }

@@ -50,11 +50,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+#ifdef QN_WAIT_HINT
+// try_wait with a suspend-time hint (ns): the thread may sleep until the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(QN_WAIT_HINT))
+        : "memory");
+    return ok != 0;
+}
+#endif
+
 // Bounded wait: returns false (and never spins forever) when the phase does not
 // complete within `limit` polls. Each try_wait already blocks for a while in hardware.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = (1u << 24)) {
     for (uint32_t i = 0; i < limit; ++i)
+#ifdef QN_WAIT_HINT
+        if (mbar_try_wait_hint(bar, parity)) return true;
+#else
         if (mbar_try_wait(bar, parity)) return true;
+#endif
     return false;
 }
 
