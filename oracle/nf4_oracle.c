@@ -46,6 +46,21 @@
  *    scaled by 1 / (1 - p); the generator is Philox4x32-10 (Salmon, Moraes,
  *    Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
  *    written here from that definition.
+ *  - The two other settings of the 4-bit load: the quant type (NF4 or the
+ *    standard 4-bit float; "Quantized LoRA (QLoRA) and 4-bit training", the
+ *    four configuration knobs, and the bnb_4bit_quant_type setting of "How
+ *    does QLoRA work for training?" section 6; NF4 measured better than FP4 in
+ *    "QLoRA paper notes", Experiments) and double quantisation on or off (the
+ *    same knobs; without it the block constants stay fp32, 0.5 bit per
+ *    parameter in "QLoRA & PEFT family" section 3.3). The pages do not define
+ *    the 4-bit float; the reading taken: E2M1 (sign, two exponent bits with
+ *    bias 1, one mantissa bit, no infinities or NaN), magnitudes 0, 0.5, 1,
+ *    1.5, 2, 3, 4, 6, normalised onto [-1, 1] like NF4 by the largest, 6, and
+ *    rounded to fp32; code = sign bit (bit 3) and magnitude index (bits 0-2),
+ *    so code 8 is -0. Codes are chosen, as for NF4, as the nearest table
+ *    value to w / c with ties to the lower code index (so -0 never occurs and
+ *    ties go toward zero); an all-zero block gets the lowest code of value 0.
+ *    Without double quantisation the block constant is the exact absmax c_b.
  *
  * All sums of the linear layer are taken in fp64 in plain loop order.
  */
@@ -81,10 +96,42 @@ static const double OR_NF4[16] = {
     1.0,
 };
 
+/* The 4-bit float (E2M1) values in code order: codes 0-7 are +m/6 for the
+ * magnitudes m = 0, 0.5, 1, 1.5, 2, 3, 4, 6; codes 8-15 are their negatives
+ * (code 8 is -0). Each is the fp32 value nearest to m/6. */
+#define OR_E2M1(m) ((double)(float)((m) / 6.0))
+static const double OR_FP4[16] = {
+    OR_E2M1(0.0),  OR_E2M1(0.5),  OR_E2M1(1.0),  OR_E2M1(1.5),  OR_E2M1(2.0),  OR_E2M1(3.0),
+    OR_E2M1(4.0),  OR_E2M1(6.0),  -OR_E2M1(0.0), -OR_E2M1(0.5), -OR_E2M1(1.0), -OR_E2M1(1.5),
+    -OR_E2M1(2.0), -OR_E2M1(3.0), -OR_E2M1(4.0), -OR_E2M1(6.0),
+};
+
+#define OR_QT_NF4 0
+#define OR_QT_FP4 1
+
+static const double *table_of(int qtype) { return qtype == OR_QT_FP4 ? OR_FP4 : OR_NF4; }
+
+/* A quantised weight: codes, the quant type's table, and its block constants,
+ * either double quantised (q, sigma, mu) or fp32 (absmax). */
+typedef struct {
+    int qtype; /* OR_QT_NF4 or OR_QT_FP4 */
+    int dq;    /* 1: q, sigma, mu; 0: absmax */
+    const uint8_t *codes;
+    const uint8_t *q;
+    const float *sigma;
+    float mu;
+    const float *absmax;
+} or_weight;
+
 /* ------------------------------------------------------------------ scalars */
 
 void or_nf4_table(double *out16) {
     for (int i = 0; i < 16; ++i) out16[i] = OR_NF4[i];
+}
+
+void or_4bit_table(int qtype, double *out16) {
+    const double *T = table_of(qtype);
+    for (int i = 0; i < 16; ++i) out16[i] = T[i];
 }
 
 int or_threads(void) {
@@ -228,11 +275,11 @@ float or_exact_mean_f32(const float *c, int64_t nb) {
 
 /* ------------------------------------------------------------- quantiser */
 
-static int nearest_code(float x) {
+static int nearest_code(const double *T, float x) {
     int best = 0;
-    double best_err = fabs((double)x - OR_NF4[0]);
+    double best_err = fabs((double)x - T[0]);
     for (int i = 1; i < 16; ++i) {
-        double err = fabs((double)x - OR_NF4[i]);
+        double err = fabs((double)x - T[i]);
         if (err < best_err) { /* strict: ties keep the lower index */
             best = i;
             best_err = err;
@@ -241,22 +288,28 @@ static int nearest_code(float x) {
     return best;
 }
 
-/* Code of one bf16 weight w in a block with absmax c (exposed for tests). */
-int or_nf4_code(float w, float c) {
-    if (c == 0.0f) return 7;
+/* Code of one bf16 weight w in a block with absmax c under quant type qtype:
+ * the nearest value to fl32(w / c); an all-zero block takes the lowest code of
+ * the value 0 (7 for NF4, 0 for the 4-bit float). Exposed for tests. */
+int or_4bit_code(int qtype, float w, float c) {
+    const double *T = table_of(qtype);
+    if (c == 0.0f) return nearest_code(T, 0.0f);
     float x = w / c;
-    return nearest_code(x);
+    return nearest_code(T, x);
 }
+
+int or_nf4_code(float w, float c) { return or_4bit_code(OR_QT_NF4, w, c); }
 
 int64_t or_num_blocks(int64_t n, int64_t k) { return n * k / OR_BLOCK; }
 int64_t or_num_groups(int64_t n, int64_t k) { return (or_num_blocks(n, k) + OR_GROUP - 1) / OR_GROUP; }
 
-/* W: n x k bf16 bits, row-major. Outputs: codes (n*k/2 bytes, element e in the
- * low nibble of byte e/2 when e is even, high nibble when odd), q (nb bytes
- * E4M3), sigma (ng floats), mu (1 float), absmax (nb floats, may be NULL).
- * Returns 0, or -1 when k is not a multiple of 64. */
-int or_nf4_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q,
-                    float *sigma, float *mu, float *absmax) {
+/* W: n x k bf16 bits, row-major; qtype OR_QT_NF4 or OR_QT_FP4. Outputs: codes
+ * (n*k/2 bytes, element e in the low nibble of byte e/2 when e is even, high
+ * nibble when odd); with dq: q (nb bytes E4M3), sigma (ng floats), mu (1 float);
+ * absmax (nb floats): required without dq, may be NULL with it. Returns 0, or
+ * -1 when k is not a multiple of 64. */
+int or_quantize4(int qtype, int dq, const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q,
+                 float *sigma, float *mu, float *absmax) {
     if (k % OR_BLOCK != 0 || n < 0 || k < 0) return -1;
     int64_t nb = or_num_blocks(n, k), ng = or_num_groups(n, k);
     float *c = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
@@ -272,10 +325,15 @@ int or_nf4_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uin
         }
         c[b] = m;
         for (int i = 0; i < OR_BLOCK; i += 2) {
-            int lo = or_nf4_code(bf16_bits_to_float(w[i]), m);
-            int hi = or_nf4_code(bf16_bits_to_float(w[i + 1]), m);
+            int lo = or_4bit_code(qtype, bf16_bits_to_float(w[i]), m);
+            int hi = or_4bit_code(qtype, bf16_bits_to_float(w[i + 1]), m);
             codes[(b * OR_BLOCK + i) / 2] = (uint8_t)(lo | (hi << 4));
         }
+    }
+    if (!dq) {
+        memcpy(absmax, c, sizeof(float) * (size_t)nb);
+        free(c);
+        return 0;
     }
 
     float m_all = or_exact_mean_f32(c, nb);
@@ -302,6 +360,11 @@ int or_nf4_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uin
     return 0;
 }
 
+int or_nf4_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q,
+                    float *sigma, float *mu, float *absmax) {
+    return or_quantize4(OR_QT_NF4, 1, W, n, k, codes, q, sigma, mu, absmax);
+}
+
 /* ---------------------------------------------------------- dequantiser */
 
 /* c'_b = fma(decode(q_b), sigma_g, mu), one rounding, fp32. */
@@ -309,9 +372,15 @@ float or_block_constant(uint8_t qb, float sg, float mu) {
     return fmaf((float)or_e4m3_decode(qb), sg, mu);
 }
 
-static void block_constants(const uint8_t *q, const float *sigma, float mu, int64_t nb, float *cp) {
+/* The block constants the dequantiser multiplies by: c'_b with double
+ * quantisation, else the stored fp32 absmax c_b itself. */
+static void block_constants(const or_weight *w, int64_t nb, float *cp) {
+    if (!w->dq) {
+        memcpy(cp, w->absmax, sizeof(float) * (size_t)nb);
+        return;
+    }
 #pragma omp parallel for schedule(static)
-    for (int64_t b = 0; b < nb; ++b) cp[b] = or_block_constant(q[b], sigma[b / OR_GROUP], mu);
+    for (int64_t b = 0; b < nb; ++b) cp[b] = or_block_constant(w->q[b], w->sigma[b / OR_GROUP], w->mu);
 }
 
 static int code_at(const uint8_t *codes, int64_t e) {
@@ -320,14 +389,14 @@ static int code_at(const uint8_t *codes, int64_t e) {
 }
 
 /* Dequantise into bf16: bf16_rn( fl32( T32[code] * c'_b ) ). */
-void or_nf4_dequant_bf16(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu,
-                         int64_t n, int64_t k, uint16_t *out) {
+void or_dequant_bf16(const or_weight *w, int64_t n, int64_t k, uint16_t *out) {
     int64_t nb = or_num_blocks(n, k);
+    const double *T = table_of(w->qtype);
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    block_constants(q, sigma, mu, nb, cp);
+    block_constants(w, nb, cp);
 #pragma omp parallel for schedule(static)
     for (int64_t e = 0; e < n * k; ++e) {
-        float t = (float)OR_NF4[code_at(codes, e)];
+        float t = (float)T[code_at(w->codes, e)];
         float v = t * cp[e / OR_BLOCK];
         out[e] = or_f32_to_bf16(v);
     }
@@ -335,13 +404,13 @@ void or_nf4_dequant_bf16(const uint8_t *codes, const uint8_t *q, const float *si
 }
 
 /* Dequantise into fp64 without rounding: T[code] * c'_b. */
-void or_nf4_dequant_f64(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu,
-                        int64_t n, int64_t k, double *out) {
+void or_dequant_f64(const or_weight *w, int64_t n, int64_t k, double *out) {
     int64_t nb = or_num_blocks(n, k);
+    const double *T = table_of(w->qtype);
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    block_constants(q, sigma, mu, nb, cp);
+    block_constants(w, nb, cp);
 #pragma omp parallel for schedule(static)
-    for (int64_t e = 0; e < n * k; ++e) out[e] = OR_NF4[code_at(codes, e)] * (double)cp[e / OR_BLOCK];
+    for (int64_t e = 0; e < n * k; ++e) out[e] = T[code_at(w->codes, e)] * (double)cp[e / OR_BLOCK];
     free(cp);
 }
 
@@ -407,13 +476,14 @@ static int keep_at(uint64_t seed, uint64_t offset, uint32_t thr, int64_t m, int6
  * may be NULL when r == 0. With dropout (p_drop > 0) the adapter's x[row,k] is
  * kept or zeroed by keep_at(seed, offset, row, k) and s becomes s / (1 - p).
  * Output h is nsel x n, fp64. */
-void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
-                  int64_t k, const uint16_t *x, const int64_t *rows, int64_t nsel, const uint16_t *A,
-                  const uint16_t *B, int r, float alpha, double p_drop, uint64_t seed, uint64_t offset,
-                  double *h) {
+void or_qlora_fwd(const or_weight *w, int64_t n, int64_t k, const uint16_t *x, const int64_t *rows,
+                  int64_t nsel, const uint16_t *A, const uint16_t *B, int r, float alpha, double p_drop,
+                  uint64_t seed, uint64_t offset, double *h) {
     int64_t nb = or_num_blocks(n, k);
+    const double *T = table_of(w->qtype);
+    const uint8_t *codes = w->codes;
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    block_constants(q, sigma, mu, nb, cp);
+    block_constants(w, nb, cp);
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
     const uint32_t thr = or_dropout_threshold(p_drop);
     if (thr != 0u) s = s / (1.0 - p_drop);
@@ -437,7 +507,7 @@ void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, fl
 #pragma omp for schedule(static)
         for (int64_t j = 0; j < n; ++j) {
             for (int64_t kk = 0; kk < k; ++kk)
-                wrow[kk] = OR_NF4[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
+                wrow[kk] = T[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
             for (int64_t i = 0; i < nsel; ++i) {
                 double acc = 0.0;
                 for (int64_t kk = 0; kk < k; ++kk) acc += wrow[kk] * xs[i * k + kk];
@@ -457,13 +527,14 @@ void or_qlora_fwd(const uint8_t *codes, const uint8_t *q, const float *sigma, fl
  *   grad_x = sum_j grad_h[row,j] W'[j,kk] + s * sum_r A[r,kk] * (sum_j grad_h[row,j] B[j,r])
  * With dropout the adapter term of (row, kk) is zeroed where the forward's mask
  * zeroed x[row, kk], and s becomes s / (1 - p). Output nsel x k, fp64. */
-void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
-                    int64_t k, const uint16_t *gh, const int64_t *rows, int64_t nsel,
-                    const uint16_t *A, const uint16_t *B, int r, float alpha, double p_drop,
+void or_qlora_bwd_x(const or_weight *w, int64_t n, int64_t k, const uint16_t *gh, const int64_t *rows,
+                    int64_t nsel, const uint16_t *A, const uint16_t *B, int r, float alpha, double p_drop,
                     uint64_t seed, uint64_t offset, double *gx) {
     int64_t nb = or_num_blocks(n, k);
+    const double *T = table_of(w->qtype);
+    const uint8_t *codes = w->codes;
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    block_constants(q, sigma, mu, nb, cp);
+    block_constants(w, nb, cp);
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
     const uint32_t thr = or_dropout_threshold(p_drop);
     if (thr != 0u) s = s / (1.0 - p_drop);
@@ -493,7 +564,7 @@ void or_qlora_bwd_x(const uint8_t *codes, const uint8_t *q, const float *sigma, 
             memset(acc, 0, sizeof(double) * (size_t)(nsel * CH));
             for (int64_t j = 0; j < n; ++j) {
                 for (int64_t kk = k0; kk < k1; ++kk)
-                    wseg[kk - k0] = OR_NF4[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
+                    wseg[kk - k0] = T[code_at(codes, j * k + kk)] * (double)cp[(j * k + kk) / OR_BLOCK];
                 for (int64_t i = 0; i < nsel; ++i) {
                     double g = gs[i * n + j];
                     for (int64_t kk = 0; kk < w; ++kk) acc[i * CH + kk] += g * wseg[kk];
@@ -601,17 +672,19 @@ uint16_t or_f64_to_bf16(double v) {
  * fp32, the adapter sum exact in fp64 (r products of bf16 values), one rounding of
  * the fp64 total to bf16. A (r x k), B (n x r) bf16 bits; r == 0 gives the plain
  * dequantised weight. */
-void or_merge_bf16(const uint8_t *codes, const uint8_t *q, const float *sigma, float mu, int64_t n,
-                   int64_t k, const uint16_t *A, const uint16_t *B, int r, float alpha, uint16_t *out) {
+void or_merge_bf16(const or_weight *wq, int64_t n, int64_t k, const uint16_t *A, const uint16_t *B, int r,
+                   float alpha, uint16_t *out) {
     int64_t nb = or_num_blocks(n, k);
+    const double *T = table_of(wq->qtype);
+    const uint8_t *codes = wq->codes;
     float *cp = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    block_constants(q, sigma, mu, nb, cp);
+    block_constants(wq, nb, cp);
     double s = (r > 0) ? (double)(alpha / (float)r) : 0.0;
 #pragma omp parallel for schedule(static)
     for (int64_t nn = 0; nn < n; ++nn)
         for (int64_t kk = 0; kk < k; ++kk) {
             int64_t e = nn * k + kk;
-            float w = (float)OR_NF4[code_at(codes, e)] * cp[e / OR_BLOCK];
+            float w = (float)T[code_at(codes, e)] * cp[e / OR_BLOCK];
             double ad = 0.0;
             for (int j = 0; j < r; ++j)
                 ad += (double)bf16_bits_to_float(B[nn * r + j]) * (double)bf16_bits_to_float(A[(int64_t)j * k + kk]);

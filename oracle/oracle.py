@@ -1,5 +1,9 @@
 """CPU oracle for the NF4 + double-quant + LoRA linear layer (test infrastructure).
 
+Quantised weights are dicts: ``codes`` and either ``q``, ``sigma``, ``mu`` (double
+quantisation, ``dq`` True, the default) or ``absmax`` (fp32 block constants, ``dq``
+False); ``qtype`` is "nf4" (default) or "fp4" (the 4-bit float, E2M1).
+
 Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s ``cpu_baseline``
 leg and reference arm (``--impl reference``) may import this module. The product path (the CUDA library and its
 Python binding) never imports, links or executes anything under ``oracle/``.
@@ -37,6 +41,23 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+QTYPES = {"nf4": 0, "fp4": 1}
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("qtype", ctypes.c_int), ("dq", ctypes.c_int), ("codes", ctypes.c_void_p),
+                ("q", ctypes.c_void_p), ("sigma", ctypes.c_void_p), ("mu", ctypes.c_float),
+                ("absmax", ctypes.c_void_p)]
+
+
+def _weight(qw: dict) -> _Weight:
+    """The C view of a quantised-weight dict (its arrays stay owned by the dict)."""
+    dq = bool(qw.get("dq", True))
+    return _Weight(QTYPES[qw.get("qtype", "nf4")], int(dq), _ptr(qw["codes"]),
+                   _ptr(qw["q"]) if dq else None, _ptr(qw["sigma"]) if dq else None,
+                   float(qw["mu"]) if dq else 0.0, None if dq else _ptr(qw["absmax"]))
+
+
 def _load():
     global _lib
     with _lock:
@@ -46,6 +67,12 @@ def _load():
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
         lib.or_nf4_table.argtypes = [P]
+        lib.or_4bit_table.argtypes = [ctypes.c_int, P]
+        lib.or_4bit_code.argtypes = [ctypes.c_int, ctypes.c_float, ctypes.c_float]
+        lib.or_4bit_code.restype = ctypes.c_int
+        lib.or_quantize4.argtypes = [ctypes.c_int, ctypes.c_int, P, i64, i64, P, P, P, P, P]
+        lib.or_quantize4.restype = ctypes.c_int
+        WP = ctypes.POINTER(_Weight)
         lib.or_threads.restype = ctypes.c_int
         lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.or_f32_to_bf16.restype = ctypes.c_uint16
@@ -65,11 +92,11 @@ def _load():
         lib.or_nf4_quantize.restype = ctypes.c_int
         lib.or_block_constant.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
         lib.or_block_constant.restype = ctypes.c_float
-        lib.or_nf4_dequant_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
-        lib.or_nf4_dequant_f64.argtypes = [P, P, P, ctypes.c_float, i64, i64, P]
+        lib.or_dequant_bf16.argtypes = [WP, i64, i64, P]
+        lib.or_dequant_f64.argtypes = [WP, i64, i64, P]
         u64, f64 = ctypes.c_uint64, ctypes.c_double
-        lib.or_qlora_fwd.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, i64, P, P,
-                                     ctypes.c_int, ctypes.c_float, f64, u64, u64, P]
+        lib.or_qlora_fwd.argtypes = [WP, i64, i64, P, P, i64, P, P, ctypes.c_int, ctypes.c_float, f64, u64, u64,
+                                     P]
         lib.or_qlora_bwd_x.argtypes = lib.or_qlora_fwd.argtypes
         lib.or_lora_grads.argtypes = [P, P, i64, i64, i64, P, P, ctypes.c_int, ctypes.c_float, f64, u64, u64,
                                       P, P]
@@ -80,7 +107,7 @@ def _load():
         lib.or_dropout_bits.restype = ctypes.c_uint32
         lib.or_f64_to_bf16.argtypes = [ctypes.c_double]
         lib.or_f64_to_bf16.restype = ctypes.c_uint16
-        lib.or_merge_bf16.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P]
+        lib.or_merge_bf16.argtypes = [WP, i64, i64, P, P, ctypes.c_int, ctypes.c_float, P]
         _lib = lib
         return lib
 
@@ -107,6 +134,18 @@ def nf4_table() -> np.ndarray:
     out = np.zeros(16, dtype=np.float64)
     _load().or_nf4_table(_ptr(out))
     return out
+
+
+def table(qtype: str = "nf4") -> np.ndarray:
+    """The 16 code values of a quant type, in code order (fp32 values as fp64)."""
+    out = np.zeros(16, dtype=np.float64)
+    _load().or_4bit_table(QTYPES[qtype], _ptr(out))
+    return out
+
+
+def code4(qtype: str, w: float, c: float) -> int:
+    """Code of weight w in a block of absmax c under quant type qtype."""
+    return int(_load().or_4bit_code(QTYPES[qtype], float(w), float(c)))
 
 
 def f32_to_bf16(v: float) -> int:
@@ -142,10 +181,11 @@ def block_constant(qb: int, sigma: float, mu: float) -> np.float32:
     return np.float32(_load().or_block_constant(int(qb), float(sigma), float(mu)))
 
 
-def nf4_quantize(W_bits: np.ndarray, n: int, k: int):
-    """Quantise a row-major n x k bf16 matrix (given as uint16 bits).
+def quantize4(W_bits: np.ndarray, n: int, k: int, qtype: str = "nf4", double_quant: bool = True):
+    """Quantise a row-major n x k bf16 matrix (given as uint16 bits) with quant type qtype.
 
-    Returns dict(codes=u8[n*k/2], q=u8[nb], sigma=f32[ng], mu=f32, absmax=f32[nb]).
+    Returns dict(codes=u8[n*k/2], absmax=f32[nb], qtype, dq) plus, with double quantisation,
+    q=u8[nb], sigma=f32[ng], mu=f32.
     """
     W = _bits16(W_bits).reshape(-1)
     assert W.size == n * k
@@ -155,23 +195,34 @@ def nf4_quantize(W_bits: np.ndarray, n: int, k: int):
     sigma = np.zeros(ng, dtype=np.float32)
     mu = np.zeros(1, dtype=np.float32)
     absmax = np.zeros(nb, dtype=np.float32)
-    rc = _load().or_nf4_quantize(_ptr(W), n, k, _ptr(codes), _ptr(q), _ptr(sigma), _ptr(mu), _ptr(absmax))
+    rc = _load().or_quantize4(QTYPES[qtype], int(bool(double_quant)), _ptr(W), n, k, _ptr(codes), _ptr(q),
+                              _ptr(sigma), _ptr(mu), _ptr(absmax))
     if rc != 0:
-        raise ValueError(f"or_nf4_quantize failed: {rc} (k must be a multiple of 64)")
-    return dict(codes=codes, q=q, sigma=sigma, mu=np.float32(mu[0]), absmax=absmax)
+        raise ValueError(f"or_quantize4 failed: {rc} (k must be a multiple of 64)")
+    out = dict(codes=codes, absmax=absmax, qtype=qtype, dq=bool(double_quant))
+    if double_quant:
+        out.update(q=q, sigma=sigma, mu=np.float32(mu[0]))
+    return out
+
+
+def nf4_quantize(W_bits: np.ndarray, n: int, k: int):
+    """NF4 with double quantisation: dict(codes, q, sigma, mu, absmax)."""
+    return quantize4(W_bits, n, k, "nf4", True)
 
 
 def nf4_dequant_bf16(qw: dict, n: int, k: int) -> np.ndarray:
+    """bf16 bits of the dequantised weight (any quant type and constant format)."""
     out = np.zeros(n * k, dtype=np.uint16)
-    _load().or_nf4_dequant_bf16(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]),
-                                n, k, _ptr(out))
+    w = _weight(qw)
+    _load().or_dequant_bf16(ctypes.byref(w), n, k, _ptr(out))
     return out.reshape(n, k)
 
 
 def nf4_dequant_f64(qw: dict, n: int, k: int) -> np.ndarray:
+    """The dequantised weight in fp64, unrounded (any quant type and constant format)."""
     out = np.zeros(n * k, dtype=np.float64)
-    _load().or_nf4_dequant_f64(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]),
-                               n, k, _ptr(out))
+    w = _weight(qw)
+    _load().or_dequant_f64(ctypes.byref(w), n, k, _ptr(out))
     return out.reshape(n, k)
 
 
@@ -216,9 +267,9 @@ def qlora_fwd(qw: dict, n: int, k: int, x_bits: np.ndarray, m: int, A_bits, B_bi
     A = _bits16(A_bits).reshape(-1) if r > 0 else None
     B = _bits16(B_bits).reshape(-1) if r > 0 else None
     h = np.zeros(rows.size * n, dtype=np.float64)
-    _load().or_qlora_fwd(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
-                         _ptr(x), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), float(p_drop),
-                         int(seed), int(offset), _ptr(h))
+    w = _weight(qw)
+    _load().or_qlora_fwd(ctypes.byref(w), n, k, _ptr(x), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r),
+                         float(alpha), float(p_drop), int(seed), int(offset), _ptr(h))
     return h.reshape(rows.size, n)
 
 
@@ -231,9 +282,9 @@ def qlora_bwd_x(qw: dict, n: int, k: int, gh_bits: np.ndarray, m: int, A_bits, B
     A = _bits16(A_bits).reshape(-1) if r > 0 else None
     B = _bits16(B_bits).reshape(-1) if r > 0 else None
     gx = np.zeros(rows.size * k, dtype=np.float64)
-    _load().or_qlora_bwd_x(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
-                           _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r), float(alpha), float(p_drop),
-                           int(seed), int(offset), _ptr(gx))
+    w = _weight(qw)
+    _load().or_qlora_bwd_x(ctypes.byref(w), n, k, _ptr(g), _ptr(rows), rows.size, _ptr(A), _ptr(B), int(r),
+                           float(alpha), float(p_drop), int(seed), int(offset), _ptr(gx))
     return gx.reshape(rows.size, k)
 
 
@@ -261,6 +312,6 @@ def merge_bf16(qw: dict, n: int, k: int, A_bits, B_bits, r: int, alpha: float) -
     A = _bits16(A_bits).reshape(-1) if r > 0 else None
     B = _bits16(B_bits).reshape(-1) if r > 0 else None
     out = np.zeros(n * k, dtype=np.uint16)
-    _load().or_merge_bf16(_ptr(qw["codes"]), _ptr(qw["q"]), _ptr(qw["sigma"]), float(qw["mu"]), n, k,
-                          _ptr(A), _ptr(B), int(r), float(alpha), _ptr(out))
+    w = _weight(qw)
+    _load().or_merge_bf16(ctypes.byref(w), n, k, _ptr(A), _ptr(B), int(r), float(alpha), _ptr(out))
     return out.reshape(n, k)

@@ -760,3 +760,157 @@ def test_dropout_grads_are_adjoint_of_forward(oracle):
     lhs = np.sum(g * (fwd(A2, B) - h1))
     rhs = np.sum(gA * (A2.double().numpy() - A.double().numpy()))
     assert abs(lhs - rhs) <= 1e-10 * (abs(lhs) + 1e-300) + 1e-13
+
+
+# ------------------------------------------- the 4-bit float and fp32 constants
+# [apxml] (the four configuration knobs) and [aivaro] 6 (bnb_4bit_quant_type,
+# bnb_4bit_use_double_quant): the quant type is NF4 or the standard 4-bit float, and
+# double quantisation can be off; [tqpw] Experiments compares NF4 with FP4; [codex] 3.3
+# gives the 0.5 bit per parameter of fp32 constants. The reading of "4-bit float": E2M1
+# (sign, two exponent bits with bias 1, one mantissa bit), normalised by its largest
+# magnitude 6 onto [-1, 1]. The pins derive the values from the bit fields here.
+
+def _e2m1(code):
+    s, e, m = code >> 3, (code >> 1) & 3, code & 1
+    mag = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0)
+    return -mag if s else mag
+
+
+def test_fp4_table_from_e2m1_bit_fields(oracle):
+    T = oracle.table("fp4")
+    want = np.array([np.float32(_e2m1(c) / 6.0) for c in range(16)], dtype=np.float64)
+    np.testing.assert_array_equal(T, want)
+    assert sorted({abs(_e2m1(c)) for c in range(16)}) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_fp4_table_invariants(oracle):
+    T = oracle.table("fp4")
+    assert T[7] == 1.0 and T[15] == -1.0 and T[0] == 0.0 and T[8] == 0.0
+    np.testing.assert_array_equal(T[8:], -T[:8])
+    assert len(set(T.tolist())) == 15  # +0 and -0 are one value
+    assert np.all(np.diff(T[:8]) > 0)
+    np.testing.assert_array_equal(oracle.table("nf4"), oracle.nf4_table())
+
+
+def test_fp4_code_special_cases(oracle):
+    for c in (1.0, 0.02, 3.0e-5, 1.5e38):
+        c = float(np.float32(torch.tensor(c).to(torch.bfloat16).float()))
+        assert oracle.code4("fp4", c, c) == 7
+        assert oracle.code4("fp4", -c, c) == 15
+        assert oracle.code4("fp4", 0.0, c) == 0
+        assert oracle.code4("fp4", -c * 2.0 ** -10, c) == 0  # rounds to zero: +0, never -0
+    assert oracle.code4("fp4", 0.0, 0.0) == 0
+    assert oracle.code4("nf4", 0.0, 0.0) == 7
+
+
+@pytest.mark.parametrize("c", [1.0, 0.0234375, 3.0])
+def test_fp4_code_is_nearest_table_value_all_bf16(oracle, c):
+    # Brute force over every finite bf16 weight with |w| <= c against the values derived
+    # from the bit fields: a nearest value, the lowest such code on a tie, never -0.
+    c = np.float32(torch.tensor(c).to(torch.bfloat16).float().item())
+    _, f = _bf16_all_finite()
+    f = f[np.abs(f) <= c]
+    T = np.array([np.float32(_e2m1(k) / 6.0) for k in range(16)], dtype=np.float64)
+    x = (f / c).astype(np.float32).astype(np.float64)
+    codes = np.array([oracle.code4("fp4", float(w), float(c)) for w in f])
+    err = np.abs(x[:, None] - T[None, :])
+    best = err.min(axis=1)
+    assert np.all(err[np.arange(len(x)), codes] == best)
+    assert np.array_equal(codes, np.argmax(err == best[:, None], axis=1))
+    assert not np.any(codes == 8)
+
+
+def test_fp4_ties_go_toward_zero(oracle):
+    # Every midpoint of neighbouring values that an fp32 x can equal exactly: the code
+    # of the smaller magnitude (the lower code index on both sides of zero).
+    T = oracle.table("fp4")
+    mags = T[:8]
+    hits = 0
+    for i in range(7):
+        m = (mags[i] + mags[i + 1]) / 2.0
+        if float(np.float32(m)) != m:
+            continue
+        hits += 1
+        assert oracle.code4("fp4", float(m), 1.0) == i
+        assert oracle.code4("fp4", -float(m), 1.0) == (i + 8 if i > 0 else 0)
+    assert hits >= 1
+
+
+def test_fp4_roundtrip_bound(oracle):
+    # Every weight decodes (exact absmax) within half the widest gap, (1 - 2/3) / 2.
+    rng = np.random.default_rng(11)
+    n, k = 4, 256
+    w = torch.from_numpy(rng.standard_t(4, (n, k)).astype(np.float32) * 0.02).to(torch.bfloat16)
+    qw = oracle.quantize4(_bits(w), n, k, "fp4", False)
+    wf = w.float().numpy().astype(np.float64).reshape(-1)
+    c = np.abs(wf).reshape(-1, 64).max(axis=1)
+    np.testing.assert_array_equal(qw["absmax"].astype(np.float64), c)
+    codes = np.empty(n * k, dtype=np.int64)
+    codes[0::2] = qw["codes"] & 15
+    codes[1::2] = qw["codes"] >> 4
+    T = np.array([np.float32(_e2m1(j) / 6.0) for j in range(16)], dtype=np.float64)
+    recon = T[codes] * np.repeat(c, 64)
+    assert np.all(np.abs(recon - wf) <= (1.0 / 6.0) * np.repeat(c, 64) * (1 + 1e-6))
+
+
+@pytest.mark.parametrize("qtype", ["nf4", "fp4"])
+def test_codes_do_not_depend_on_double_quant(oracle, qtype):
+    # Codes are chosen against the exact block absmax; double quantisation only changes
+    # how the constants are stored.
+    rng = np.random.default_rng(3)
+    n, k = 5, 64 * 9
+    w = torch.from_numpy(rng.normal(0, 0.02, (n, k)).astype(np.float32)).to(torch.bfloat16)
+    a = oracle.quantize4(_bits(w), n, k, qtype, True)
+    b = oracle.quantize4(_bits(w), n, k, qtype, False)
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    np.testing.assert_array_equal(a["absmax"], b["absmax"])
+    assert "q" not in b and "sigma" not in b
+
+
+@pytest.mark.parametrize("qtype", ["nf4", "fp4"])
+def test_fp32_constants_dequant_is_table_times_absmax(oracle, qtype):
+    # Without double quantisation the dequantised weight is T[code] * c_b with c_b the
+    # numpy block absmax; the bf16 form is its round-to-nearest-even (torch).
+    rng = np.random.default_rng(8)
+    n, k = 3, 64 * 5
+    w = torch.from_numpy(rng.normal(0, 0.02, (n, k)).astype(np.float32)).to(torch.bfloat16)
+    qw = oracle.quantize4(_bits(w), n, k, qtype, False)
+    c = np.abs(w.float().numpy()).reshape(-1, 64).max(axis=1).astype(np.float64)
+    codes = np.empty(n * k, dtype=np.int64)
+    codes[0::2] = qw["codes"] & 15
+    codes[1::2] = qw["codes"] >> 4
+    T = oracle.table(qtype)
+    want = T[codes] * np.repeat(c, 64)
+    np.testing.assert_array_equal(oracle.nf4_dequant_f64(qw, n, k).reshape(-1), want)
+    want16 = torch.from_numpy((T[codes].astype(np.float32) * np.repeat(c.astype(np.float32), 64))).to(torch.bfloat16)
+    np.testing.assert_array_equal(oracle.nf4_dequant_bf16(qw, n, k).reshape(-1), _bits(want16))
+
+
+@pytest.mark.parametrize("qtype,dq", [("fp4", True), ("fp4", False), ("nf4", False)])
+def test_formats_layer_is_dequant_matmul_plus_adapter(oracle, qtype, dq):
+    # The layer with another format is the same contraction: numpy over the independently
+    # dequantised weight (fp32 constants) or the oracle's dequantisation (double quant),
+    # plus s B (A x); and the adjoint identity between forward and input gradient.
+    n, k, m, r, alpha = 24, 64 * 3, 3, 4, 8.0
+    g = torch.Generator().manual_seed(21)
+    W = (torch.randn(n, k, generator=g) * 0.02).to(torch.bfloat16)
+    A = (torch.randn(r, k, generator=g) * 0.01).to(torch.bfloat16)
+    B = (torch.randn(n, r, generator=g) * 0.01).to(torch.bfloat16)
+    x = torch.randn(m, k, generator=g).to(torch.bfloat16)
+    gh = torch.randn(m, n, generator=g).to(torch.bfloat16)
+    qw = oracle.quantize4(_bits(W), n, k, qtype, dq)
+    if dq:
+        Wd = oracle.nf4_dequant_f64(qw, n, k)
+    else:
+        codes = np.empty(n * k, dtype=np.int64)
+        codes[0::2] = qw["codes"] & 15
+        codes[1::2] = qw["codes"] >> 4
+        c = np.abs(W.float().numpy()).reshape(-1, 64).max(axis=1).astype(np.float64)
+        Wd = (oracle.table(qtype)[codes] * np.repeat(c, 64)).reshape(n, k)
+    xf, Af, Bf, gf = (t.double().numpy() for t in (x, A, B, gh))
+    s = float(np.float32(alpha / r))
+    h = oracle.qlora_fwd(qw, n, k, _bits(x), m, _bits(A), _bits(B), r, alpha)
+    np.testing.assert_allclose(h, xf @ Wd.T + s * (xf @ Af.T) @ Bf.T, rtol=1e-12, atol=1e-12)
+    gx = oracle.qlora_bwd_x(qw, n, k, _bits(gh), m, _bits(A), _bits(B), r, alpha)
+    np.testing.assert_allclose(gx, gf @ Wd + s * (gf @ Bf) @ Af, rtol=1e-12, atol=1e-12)
+    assert abs(np.sum(gf * h) - np.sum(gx * xf)) <= 1e-10 * (np.abs(gf * h).sum() + 1.0)
