@@ -18,8 +18,10 @@ LIB_PATH = os.path.join(_PKG, "libqlora_nf4.so")
 
 QN_OK, QN_EINVAL, QN_ESHAPE, QN_EALIGN, QN_ECUDA, QN_EWORKSPACE, QN_ETIMEOUT = range(7)
 BLOCK, GROUP, MAX_RANK = 64, 256, 256
+QUANT_TYPES = {"nf4": 0, "fp4": 1}  # QN_QUANT_NF4, QN_QUANT_FP4
+CONST_DQ, CONST_F32 = 0, 1           # QN_CONST_DQ, QN_CONST_F32
 
-EXPORTED = ("qn_nf4_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
+EXPORTED = ("qn_nf4_sizes", "qn_weight_sizes", "qn_quantize_workspace_size", "nf4_quantize", "nf4_quantize_static_ws", "nf4_dequantize",
             "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x",
             "qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qlora_linear_fwd_dropout",
             "qlora_linear_bwd_x_dropout", "qlora_lora_grads_dropout", "qn_status_string",
@@ -33,9 +35,11 @@ class QNError(RuntimeError):
 
 
 class CWeight(ctypes.Structure):
+    """qn_nf4_weight (see the header); fields left at zero mean NF4 with double quantisation."""
     _fields_ = [("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64), ("codes", ctypes.c_void_p),
                 ("absmax_q", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
-                ("absmax_mean", ctypes.c_void_p)]
+                ("absmax_mean", ctypes.c_void_p), ("quant_type", ctypes.c_int32), ("const_format", ctypes.c_int32),
+                ("absmax", ctypes.c_void_p)]
 
 
 class CDropout(ctypes.Structure):
@@ -66,6 +70,7 @@ def load(path: str | None = None):
         W = ctypes.POINTER(CWeight)
         st = ctypes.c_int
         lib.qn_nf4_sizes.argtypes = [i64, i64, sz, sz, sz, sz]
+        lib.qn_weight_sizes.argtypes = [i64, i64, ctypes.c_int, sz, sz, sz, sz, sz]
         lib.qn_quantize_workspace_size.argtypes = [i64, i64, sz]
         lib.nf4_quantize.argtypes = [P, W, P, ctypes.c_size_t, P]
         lib.nf4_dequantize.argtypes = [W, P, P]
@@ -183,6 +188,14 @@ def sizes(n_out: int, k_in: int):
     return a.value, b.value, c.value, d.value
 
 
+def weight_sizes(n_out: int, k_in: int, double_quant: bool = True):
+    """(codes, absmax_q, group_scale, absmax_mean, absmax fp32) byte sizes for a constant format."""
+    v = [ctypes.c_size_t() for _ in range(5)]
+    _check(load().qn_weight_sizes(n_out, k_in, CONST_DQ if double_quant else CONST_F32, *(ctypes.byref(x) for x in v)),
+           "qn_weight_sizes")
+    return tuple(x.value for x in v)
+
+
 def quantize_workspace_size(n_out: int, k_in: int) -> int:
     v = ctypes.c_size_t()
     _check(load().qn_quantize_workspace_size(n_out, k_in, ctypes.byref(v)), "qn_quantize_workspace_size")
@@ -201,39 +214,53 @@ def launch_count(reset: bool = False) -> int:
 
 @dataclasses.dataclass
 class NF4Weight:
-    """A quantised weight: four device buffers plus the shape (see include/qlora_nf4.h)."""
+    """A quantised weight: its device buffers plus the shape and format (see include/qlora_nf4.h).
+    quant_type "nf4" or "fp4"; double_quant True: absmax_q, group_scale, absmax_mean hold the
+    constants; False: absmax (fp32 per block) does, and the other three are empty."""
     n_out: int
     k_in: int
     codes: torch.Tensor        # uint8 [n_out*k_in/2]
     absmax_q: torch.Tensor     # uint8 [nb], E4M3 bits
     group_scale: torch.Tensor  # float32 [ng]
     absmax_mean: torch.Tensor  # float32 [1]
+    quant_type: str = "nf4"
+    double_quant: bool = True
+    absmax: torch.Tensor | None = None  # float32 [nb] (double_quant False)
 
     @staticmethod
-    def empty(n_out: int, k_in: int, device="cuda") -> "NF4Weight":
-        cb, ab, sb, _ = sizes(n_out, k_in)
+    def empty(n_out: int, k_in: int, device="cuda", quant_type: str = "nf4", double_quant: bool = True) -> "NF4Weight":
+        if quant_type not in QUANT_TYPES:
+            raise ValueError(f"quant_type {quant_type!r} is not one of {sorted(QUANT_TYPES)}")
+        cb, ab, sb, mb, fb = weight_sizes(n_out, k_in, double_quant)
         u8 = dict(dtype=torch.uint8, device=device)
         f32 = dict(dtype=torch.float32, device=device)
-        return NF4Weight(n_out, k_in, torch.empty(cb, **u8), torch.empty(ab, **u8),
-                         torch.empty(sb // 4, **f32), torch.empty(1, **f32))
+        return NF4Weight(n_out, k_in, torch.empty(cb, **u8), torch.empty(ab, **u8), torch.empty(sb // 4, **f32),
+                         torch.empty(mb // 4, **f32), quant_type, bool(double_quant),
+                         None if double_quant else torch.empty(fb // 4, **f32))
 
     def c_struct(self) -> CWeight:
-        return CWeight(self.n_out, self.k_in, self.codes.data_ptr(), self.absmax_q.data_ptr(),
-                       self.group_scale.data_ptr(), self.absmax_mean.data_ptr())
+        if self.double_quant:
+            return CWeight(self.n_out, self.k_in, self.codes.data_ptr(), self.absmax_q.data_ptr(),
+                           self.group_scale.data_ptr(), self.absmax_mean.data_ptr(), QUANT_TYPES[self.quant_type],
+                           CONST_DQ, None)
+        return CWeight(self.n_out, self.k_in, self.codes.data_ptr(), None, None, None, QUANT_TYPES[self.quant_type],
+                       CONST_F32, self.absmax.data_ptr())
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.codes, self.absmax_q, self.group_scale,
-                                                          self.absmax_mean))
+        ts = (self.codes, self.absmax_q, self.group_scale, self.absmax_mean) + (
+            () if self.absmax is None else (self.absmax,))
+        return sum(t.numel() * t.element_size() for t in ts)
 
 
 def nf4_quantize(W: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
-                 stream=None) -> NF4Weight:
-    """Quantise a bf16 (n_out x k_in) CUDA tensor to NF4 with double quantisation."""
+                 stream=None, quant_type: str = "nf4", double_quant: bool = True) -> NF4Weight:
+    """Quantise a bf16 (n_out x k_in) CUDA tensor: NF4 (or "fp4") codes with double-quantised (or
+    fp32) block constants; an `out` given keeps its own format."""
     _dev_bf16(W, "W")
     if W.dim() != 2:
         raise ValueError("W must be 2-D (n_out x k_in)")
     n, k = W.shape
-    out = out or NF4Weight.empty(n, k, W.device)
+    out = out or NF4Weight.empty(n, k, W.device, quant_type, double_quant)
     if (out.n_out, out.k_in) != (n, k):
         raise ValueError(f"out holds a {out.n_out} x {out.k_in} weight, W is {n} x {k}")
     _same_device(out, W)

@@ -53,7 +53,16 @@ qn_status check_weight(const qn_nf4_weight *w) {
     if (!w) return fail(QN_EINVAL, "null weight struct");
     qn_status s = check_shape(w->n_out, w->k_in);
     if (s != QN_OK) return s;
+    if (w->quant_type != QN_QUANT_NF4 && w->quant_type != QN_QUANT_FP4)
+        return fail(QN_EINVAL, "unknown quant_type %d", w->quant_type);
+    if (w->const_format != QN_CONST_DQ && w->const_format != QN_CONST_F32)
+        return fail(QN_EINVAL, "unknown const_format %d", w->const_format);
     if (w->n_out == 0 || w->k_in == 0) return QN_OK;
+    if (w->const_format == QN_CONST_F32) {
+        if (!w->codes || !w->absmax) return fail(QN_EINVAL, "null pointer in the quantised weight");
+        if (!aligned16(w->codes) || !aligned16(w->absmax)) return fail(QN_EALIGN, "codes or absmax not 16-byte aligned");
+        return QN_OK;
+    }
     if (!w->codes || !w->absmax_q || !w->group_scale || !w->absmax_mean)
         return fail(QN_EINVAL, "null pointer in the quantised weight");
     if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale))
@@ -62,7 +71,24 @@ qn_status check_weight(const qn_nf4_weight *w) {
 }
 
 WeightView view(const qn_nf4_weight *w) {
-    return WeightView{w->n_out, w->k_in, w->codes, w->absmax_q, w->group_scale, w->absmax_mean};
+    const bool f32 = w->const_format == QN_CONST_F32;
+    return WeightView{w->n_out,
+                      w->k_in,
+                      w->codes,
+                      f32 ? nullptr : w->absmax_q,
+                      f32 ? nullptr : w->group_scale,
+                      f32 ? nullptr : w->absmax_mean,
+                      w->quant_type == QN_QUANT_FP4 ? 1 : 0,
+                      f32 ? w->absmax : nullptr};
+}
+
+qn_status launch_quantize_into(const void *W, const qn_nf4_weight *out, void *ws, cudaStream_t st) {
+    const bool f32 = out->const_format == QN_CONST_F32;
+    return cuda_status(launch_quantize(static_cast<const uint16_t *>(W), out->n_out, out->k_in,
+                                       out->quant_type == QN_QUANT_FP4 ? 1 : 0, out->codes,
+                                       f32 ? nullptr : out->absmax_q, f32 ? nullptr : out->group_scale,
+                                       f32 ? nullptr : out->absmax_mean, f32 ? out->absmax : nullptr, ws, st),
+                       "nf4_quantize");
 }
 
 qn_status check_lora(const void *A, const void *B, int r, float alpha) {
@@ -132,6 +158,21 @@ qn_status qn_nf4_sizes(int64_t n_out, int64_t k_in, size_t *codes_bytes, size_t 
     return QN_OK;
 }
 
+qn_status qn_weight_sizes(int64_t n_out, int64_t k_in, int const_format, size_t *codes_bytes, size_t *absmax_bytes,
+                          size_t *scale_bytes, size_t *mean_bytes, size_t *absmax_f32_bytes) {
+    if (!absmax_f32_bytes) return fail(QN_EINVAL, "null output pointer");
+    if (const_format != QN_CONST_DQ && const_format != QN_CONST_F32)
+        return fail(QN_EINVAL, "unknown const_format %d", const_format);
+    qn_status s = qn_nf4_sizes(n_out, k_in, codes_bytes, absmax_bytes, scale_bytes, mean_bytes);
+    if (s != QN_OK) return s;
+    *absmax_f32_bytes = 0;
+    if (const_format == QN_CONST_F32) {
+        *absmax_f32_bytes = sizeof(float) * *absmax_bytes;
+        *absmax_bytes = *scale_bytes = *mean_bytes = 0;
+    }
+    return QN_OK;
+}
+
 qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_bytes) {
     if (!ws_bytes) return fail(QN_EINVAL, "null output pointer");
     qn_status s = check_shape(n_out, k_in);
@@ -150,10 +191,7 @@ qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t
     const size_t need = quantize_workspace_bytes(out->n_out, out->k_in);
     if (!ws || ws_bytes < need) return fail(QN_EWORKSPACE, "quantize workspace needs %zu bytes", need);
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(QN_EALIGN, "workspace not 256-byte aligned");
-    return cuda_status(launch_quantize(static_cast<const uint16_t *>(W), out->n_out, out->k_in, out->codes,
-                                       out->absmax_q, out->group_scale, out->absmax_mean, ws,
-                                       static_cast<cudaStream_t>(stream)),
-                       "nf4_quantize");
+    return launch_quantize_into(W, out, ws, static_cast<cudaStream_t>(stream));
 }
 
 qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *stream) {
@@ -172,10 +210,7 @@ qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *
     void *ws = nullptr;
     cudaError_t e = static_scratch_address(&ws);
     if (e != cudaSuccess) return cuda_status(e, "nf4_quantize_static_ws: cudaGetSymbolAddress");
-    return cuda_status(launch_quantize(static_cast<const uint16_t *>(W), out->n_out, out->k_in, out->codes,
-                                       out->absmax_q, out->group_scale, out->absmax_mean, ws,
-                                       static_cast<cudaStream_t>(stream)),
-                       "nf4_quantize_static_ws");
+    return launch_quantize_into(W, out, ws, static_cast<cudaStream_t>(stream));
 }
 
 qn_status nf4_dequantize(const qn_nf4_weight *w, void *W_out, void *stream) {

@@ -19,16 +19,31 @@ constexpr int kGroup = 256;  // blocks per double-quantisation group
      0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f, \
      0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f}
 
-static __constant__ float c_nf4_table[16] = QN_NF4_VALUES;
+// The other quant type, the 4-bit float E2M1 (sign, two exponent bits with bias 1, one
+// mantissa bit): codes 0-7 are the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by the
+// largest, 6, each the nearest fp32 value; codes 8-15 are their negatives (8 is -0, which the
+// quantiser never produces). The quant-type knob: "Quantized LoRA (QLoRA) and 4-bit training"
+// (apxml.com), the four configuration knobs; "QLoRA paper notes" (tqpw.cn), Experiments.
+#define QN_FP4_VALUES                                                                                 \
+    {0.0f,   0x1.555556p-4f,  0x1.555556p-3f,  0x1p-2f,  0x1.555556p-2f,  0x1p-1f,  0x1.555556p-1f,  1.0f, \
+     -0.0f, -0x1.555556p-4f, -0x1.555556p-3f, -0x1p-2f, -0x1.555556p-2f, -0x1p-1f, -0x1.555556p-1f, -1.0f}
 
-__host__ __device__ inline float nf4_value(int i) {
+constexpr int kQuantNF4 = 0;
+constexpr int kQuantFP4 = 1;
+
+static __constant__ float c_tables[2][16] = {QN_NF4_VALUES, QN_FP4_VALUES};
+
+// Value of code i (0..15) of quant type qtype (kQuantNF4 or kQuantFP4).
+__host__ __device__ inline float table_value(int qtype, int i) {
 #ifdef __CUDA_ARCH__
-    return c_nf4_table[i];
+    return c_tables[qtype][i];
 #else
-    constexpr float T[16] = QN_NF4_VALUES;
-    return T[i];
+    constexpr float T[2][16] = {QN_NF4_VALUES, QN_FP4_VALUES};
+    return T[qtype][i];
 #endif
 }
+
+__host__ __device__ inline float nf4_value(int i) { return table_value(kQuantNF4, i); }
 
 // ---------------------------------------------------------------- loads
 
@@ -77,6 +92,15 @@ __device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float v) {
 __device__ __forceinline__ float block_constant(uint8_t q, float sigma, float mu) {
     return __fmaf_rn(e4m3_to_f32(q), sigma, mu);
 }
+
+// Block constant b read from global memory: c'_b with double quantisation (mu already loaded),
+// else the stored fp32 absmax (absmax != nullptr).
+__device__ __forceinline__ float load_block_constant(const uint8_t *q, const float *sigma, float mu,
+                                                     const float *absmax, int64_t b) {
+    return absmax ? __ldg(absmax + b) : block_constant(__ldg(q + b), __ldg(sigma + b / kGroup), mu);
+}
+// mu of a weight with double-quantised constants (0 when they are fp32).
+__device__ __forceinline__ float load_mu(const float *mu, const float *absmax) { return absmax ? 0.0f : __ldg(mu); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -110,7 +110,7 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
     }
     cp_async_commit();
 
-    const float mu = __ldg(p.mu);
+    const float mu = load_mu(p.mu, p.absmax);
     const int M = p.M;
 
     // Lane (gq, t) reads, per step st, the 4 code bytes [4 gq, 4 gq + 4) of block column kb of
@@ -139,8 +139,13 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
             }
             const bool ok = sv && st * 16 + 4 * t + (gq & 3) < N;
             const uint64_t bi = static_cast<uint64_t>(erow + st * 16 * nbr);
-            G.q[j] = ok ? __ldg(p.q + bi) : 0u;
-            G.s[j] = ok ? __ldg(p.sigma + bi / kGroup) : 0.0f;
+            if (p.absmax) {  // the fp32 constant itself, in G.s
+                G.q[j] = 0u;
+                G.s[j] = ok ? __ldg(p.absmax + bi) : 0.0f;
+            } else {
+                G.q[j] = ok ? __ldg(p.q + bi) : 0u;
+                G.s[j] = ok ? __ldg(p.sigma + bi / kGroup) : 0.0f;
+            }
         }
     };
 
@@ -194,7 +199,7 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
     };
 
     // The pair table is built while the first codes are in flight.
-    build_pair_lut(lut);
+    build_pair_lut(lut, p.qtype);
     __syncthreads();
 
     // ---- base: block column kb, group gi holds steps s_lo + 2 gi, + 1.
@@ -204,7 +209,7 @@ __device__ __forceinline__ void decode_bwd_body(const DecodeParams &p, uint8_t *
             if (2 * gi + j >= nst) break;
             const int64_t n0 = (s_lo + 2 * gi + j) * 16 + 4 * t;  // this lane's 4 reduction rows
             // constant of row n0 + (gq & 3), shared with the lanes of the same t
-            const float mine = block_constant(static_cast<uint8_t>(G.q[j]), G.s[j], mu);
+            const float mine = p.absmax ? G.s[j] : block_constant(static_cast<uint8_t>(G.q[j]), G.s[j], mu);
             float cp[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) cp[i] = __shfl_sync(0xffffffffu, mine, (i << 2) | t);
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kDecThreads) k_decode_bwd(const DecodeParams p
 cudaError_t launch_decode_bwd(const WeightView &w, const uint16_t *gh, int M, const uint16_t *A, const uint16_t *B,
                               int r, float s, uint16_t *gx, cudaStream_t st) {
     if (M <= 0 || w.k == 0) return cudaSuccess;
-    DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, gh, M, A, B, r, s, gx};
+    DecodeParams p{w.codes, w.q, w.sigma, w.mu, w.absmax, w.qtype, w.n, w.k, gh, M, A, B, r, s, gx};
     const int NG = pick_groups(M);
     const int rpad = (r + 15) & ~15;
     // table (later the warps' sums) | recv | upart | warp-sum scratch | staged adapter columns

@@ -61,6 +61,8 @@ struct BwdArgs {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
+    const float *absmax;  // fp32 block constants (no double quantisation), else nullptr
+    int qtype;            // table of the code nibbles
     uint16_t *gx;  // M x k
     int *err;
     uint16_t *u_ws;     // [MP][rk16] bf16 u, published by the adapter cluster
@@ -75,7 +77,8 @@ struct BwdArgs {
     DropoutArgs drop;  // mask of the forward's adapter input (thr == 0: none); offset of token 0
     int C, stages;
     int q_tma;  // FP8 codes by a TMA box (rows of FP8 codes 16-byte aligned), else per-row copies
-    uint32_t slot_bytes, g_off, q_off, s_off;  // chunk slot: codes, grad_h, FP8 codes, group scales
+    uint32_t slot_bytes, g_off, q_off, s_off;  // chunk slot: codes, grad_h, FP8 codes (or fp32 constants),
+                                               // group scales
     uint32_t b_off;                            // adapter slot: grad_h at 0, B at b_off
     uint32_t ring_off, ut_off, at_off, recv_off, bar_off, post_off;
     uint32_t codes_bytes, g_bytes, q_bytes, gb_bytes;  // transaction bytes
@@ -326,6 +329,19 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             if (p.q_tma)
                 tma_load_2d_saddr(sl + p.q_off, tm_q, &bb.full[slot], (4 * col) & ~15, static_cast<int32_t>(n0));
         }
+        if (p.absmax) {
+            // fp32 constants: per row the two 16-byte chunks from the one that holds block 4 col
+            for (int i = lane; i < 2 * kSR; i += 32) {
+                const int ri = i >> 1, h = i & 1;
+                const int64_t row = n0 + ri;
+                const int64_t cb = ((row < p.n ? row * p.nbr + 4 * col : 0) >> 2) + h;
+                const int64_t avail = row < p.n ? 4 * (nbq - 4 * cb) : 0;
+                const uint32_t bytes = avail >= 16 ? 16u : (avail > 0 ? static_cast<uint32_t>(avail) : 0u);
+                cp_async16_zfill(sl + p.q_off + 32u * ri + 16u * h, p.absmax + (bytes ? 4 * cb : 0), bytes);
+            }
+            cp_async_arrive_noinc(&bb.full[slot]);
+            return;
+        }
         if (!p.q_tma) {
             // per row the 16-byte chunk that holds its four FP8 codes of this column
             for (int i = lane; i < kSR; i += 32) {
@@ -369,7 +385,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         const uint64_t pol = l2_policy_evict_first();
         for (int s = 0; s < npre; ++s) stage_weights(s, pol);
     }
-    build_pair_lut(lut, threadIdx.x, kThreads);
+    build_pair_lut(lut, threadIdx.x, kThreads, p.qtype);
     __syncthreads();
     if (C > 1) cluster_arrive_relaxed();
     grid_dependents_launch();
@@ -456,7 +472,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // ------------------------------------------------------------------ consumers
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
-        const float mu = __ldg(p.mu);
+        const float mu = load_mu(p.mu, p.absmax);
         // source lanes of rows 2t, 2t+1, 2t+8, 2t+9 (row rho of a 16-row tile is computed by lane
         // 4 (rho & 7) + (rho >> 3))
         const int src0 = 4 * ((2 * t) & 7) + 0, src1 = 4 * ((2 * t + 1) & 7) + 0;
@@ -483,10 +499,16 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                     const int64_t row = n0 + ri;
                     if (row < p.n && blk_ok) {
                         const int64_t e = row * p.nbr + 4 * col + kg;
-                        const uint32_t qb = lds8(sl + p.q_off + 16u * ri + static_cast<uint32_t>((e - kg) & 15) + kg);
-                        const float sg =
-                            __uint_as_float(lds32(sl + p.s_off + 4u * static_cast<uint32_t>((e >> 8) - sg0)));
-                        cmine = block_constant(static_cast<uint8_t>(qb), sg, mu);
+                        if (p.absmax) {
+                            cmine = __uint_as_float(
+                                lds32(sl + p.q_off + 32u * ri + 4u * static_cast<uint32_t>(((e - kg) & 3) + kg)));
+                        } else {
+                            const uint32_t qb =
+                                lds8(sl + p.q_off + 16u * ri + static_cast<uint32_t>((e - kg) & 15) + kg);
+                            const float sg =
+                                __uint_as_float(lds32(sl + p.s_off + 4u * static_cast<uint32_t>((e >> 8) - sg0)));
+                            cmine = block_constant(static_cast<uint8_t>(qb), sg, mu);
+                        }
                     }
                 }
                 const float c0 = __shfl_sync(0xffffffffu, cmine, src0), c1 = __shfl_sync(0xffffffffu, cmine, src1);
@@ -718,10 +740,11 @@ uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 bool layout(BwdArgs &a, int MP) {
     const uint32_t codes = kSR * 128u;
     const uint32_t gb = 2u * MP * 128u;  // two 64-row boxes
-    const uint32_t qb = kSR * 16u;
+    // FP8 codes: one 16-byte chunk per row; fp32 constants: two
+    const uint32_t qb = kSR * (a.absmax ? 32u : 16u);
     // a stage's scales: from an aligned index <= 3 below the first to the last, at most
-    // (127 nbr + 3) / 256 + 1 apart, in whole 16-byte chunks
-    a.s_cap = static_cast<int>(static_cast<int64_t>(kSR) * a.nbr / 256 + 12);
+    // (127 nbr + 3) / 256 + 1 apart, in whole 16-byte chunks (none with fp32 constants)
+    a.s_cap = a.absmax ? 0 : static_cast<int>(static_cast<int64_t>(kSR) * a.nbr / 256 + 12);
     const uint32_t sb = align_up(static_cast<uint32_t>(a.s_cap) * 4u, 128);
     const uint32_t bb = a.r > 0 ? kSR * 2u * a.rpad : 0u;
     a.g_off = codes;
@@ -794,6 +817,8 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *gh, int M, const uint
     a.q = w.q;
     a.sigma = w.sigma;
     a.mu = w.mu;
+    a.absmax = w.absmax;
+    a.qtype = w.qtype;
     a.gx = gx;
     a.err = err;
     char *wsb = reinterpret_cast<char *>(err);
@@ -811,7 +836,7 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *gh, int M, const uint
     a.rk16 = (a.rpad + 15) & ~15;
     a.s = s;
     a.drop = drop;
-    a.q_tma = (a.nbr % 16) == 0 ? 1 : 0;
+    a.q_tma = (a.nbr % 16) == 0 && !w.absmax ? 1 : 0;
     const int extra = r > 0 ? 1 : 0;
     // cluster size: the largest C <= 8 with (chunks + 1) x C <= SMs, every cluster resident and
     // at least one row stage per CTA

@@ -31,6 +31,8 @@ struct DecodeParams {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
+    const float *absmax;  // fp32 block constants (no double quantisation), else nullptr
+    int qtype;            // table of the code nibbles (kQuantNF4 or kQuantFP4)
     int64_t n, k;         // W is n x k
     const uint16_t *act;  // fwd: x (M x k); bwd: grad_h (M x n)
     int M;
@@ -47,13 +49,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-// Pair table: row e (a code byte) holds bf16x2(NF4[e & 15], NF4[e >> 4]) in its first 32
-// words, one copy per lane. One row per thread; the eight 16-byte stores of a row start at a
-// column rotated by the row so that the lanes of a warp hit different banks.
-__device__ __forceinline__ void build_pair_lut(uint8_t *lut) {
+// Pair table: row e (a code byte) holds bf16x2(T[e & 15], T[e >> 4]) in its first 32 words, one
+// copy per lane (T: the table of quant type qtype). One row per thread; the eight 16-byte stores
+// of a row start at a column rotated by the row so that the lanes of a warp hit different banks.
+__device__ __forceinline__ void build_pair_lut(uint8_t *lut, int qtype) {
     uint4 *l4 = reinterpret_cast<uint4 *>(lut);
     for (int e = threadIdx.x; e < 256; e += blockDim.x) {
-        const uint32_t v = pack_bf16x2(nf4_value(e & 15), nf4_value(e >> 4));
+        const uint32_t v = pack_bf16x2(table_value(qtype, e & 15), table_value(qtype, e >> 4));
 #pragma unroll
         for (int c = 0; c < 8; ++c) l4[e * 16 + ((c + e) & 7)] = make_uint4(v, v, v, v);
     }

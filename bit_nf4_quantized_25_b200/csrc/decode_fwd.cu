@@ -102,6 +102,8 @@ struct FwdArgs {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
+    const float *absmax;  // fp32 block constants (no double quantisation), else nullptr
+    int qtype;            // table of the code nibbles
     const uint16_t *B;  // n x r
     const uint16_t *x;  // M x k (the chunk CTAs' stage copies)
     uint16_t *h;        // M x n
@@ -127,7 +129,7 @@ struct FwdArgs {
     uint32_t xs_off, xs_stage;   // ... at xs_off, xs_stage bytes per stage ([4][M][128 B])
     uint32_t a_off;              // adapter CTAs: x [4][MP][128 B] at 0, A [4][rpad][128 B] at a_off
     uint32_t ring_off, qs_off, ss_off, tb_off, bs_off, recv_off, bar_off, post_off;
-    uint32_t qs_stride;  // bytes per chunk row of the staged FP8 codes
+    uint32_t qs_stride;  // bytes per chunk row of the staged FP8 codes (or fp32 constants)
     uint32_t bs_stride;  // bytes per staged row of B
     uint32_t codes_bytes, x_bytes, xa_bytes;  // transaction bytes: codes box; x box; adapter x + A boxes
 #ifdef QN_TIMELINE
@@ -428,9 +430,21 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // FP8 codes of the slice: chunk row i holds the 16-byte aligned chunks from the one that
         // contains block 4 col_lo of that row on; the group scales of every block of the chunk
         // rows from the slice's first to its last, in whole 16-byte chunks. Bytes past the arrays
-        // read as zero.
+        // read as zero. With fp32 constants, chunk row i holds them (4 per chunk) instead.
         const int ct = threadIdx.x - 32;
-        {
+        if (p.absmax) {
+            const int64_t nbq = p.n * p.nbr;
+            const int nch = static_cast<int>(p.qs_stride >> 4);
+            for (int it = ct; it < p.R * nch; it += kConsumers * 32) {
+                const int i = it / nch, c = it - (it / nch) * nch;
+                const int64_t row = row0 + i;
+                const int64_t cb = (((row < nrow ? row : row0) * p.nbr + 4 * col_lo) >> 2) + c;  // 16-byte chunk
+                const int64_t avail = row < nrow ? 4 * (nbq - 4 * cb) : 0;
+                const uint32_t bytes = avail >= 16 ? 16u : (avail > 0 ? static_cast<uint32_t>(avail) : 0u);
+                cp_async16_zfill(s_qs + static_cast<uint32_t>(i) * p.qs_stride + 16u * c,
+                                 p.absmax + (bytes ? 4 * cb : 0), bytes);
+            }
+        } else {
             const int64_t nbq = p.n * p.nbr;
             const int nch = static_cast<int>(p.qs_stride >> 4);
             const int items = p.R * nch;
@@ -457,7 +471,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         cp_async_arrive_noinc(bb.consts);
         QN_TL(8, ct == 0);
-        build_pair_lut(lut, ct, kConsumers * 32);
+        build_pair_lut(lut, ct, kConsumers * 32, p.qtype);
         named_sync(1, kConsumers * 32);  // the table is complete
         QN_TL(23, ct == 0);
     }
@@ -633,7 +647,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
-        const float mu = __ldg(p.mu);
+        const float mu = load_mu(p.mu, p.absmax);
         // x rows of this lane's tokens (tokens beyond M read token tok % M; their columns of the
         // result are never stored): row kg M + tok of the x box, 16-byte chunks 2 t and 2 t + 1
         // of it, stored at chunk ^ (row & 7)
@@ -661,7 +675,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             const int i = 16 * mt + g + 8 * (t & 1);
             const int64_t e0 = (row0 + i) * p.nbr + 4 * col_lo;
             c_ok[pass] = mt < p.m && row0 + i < nrow;
-            c_q[pass] = s_qs + static_cast<uint32_t>(i) * p.qs_stride + static_cast<uint32_t>(e0 & 15) + kg;
+            c_q[pass] = s_qs + static_cast<uint32_t>(i) * p.qs_stride +
+                        (p.absmax ? 4u * static_cast<uint32_t>((e0 & 3) + kg) : static_cast<uint32_t>(e0 & 15) + kg);
             c_e[pass] = e0 + kg - ((s_lo & ~int64_t(3)) << 8);  // staged scales start at s_lo & ~3
         }
         int nsc = ns;
@@ -689,10 +704,14 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             for (int pass = 0; pass < NP; ++pass) {
                 float c = 0.0f;
                 if (c_ok[pass] && blk_ok) {
-                    const uint32_t qb = lds8(c_q[pass] + 4u * s);
-                    const int64_t si = (c_e[pass] + 4 * s) >> 8;
-                    const float sg = __uint_as_float(lds32(s_ss + 4u * static_cast<uint32_t>(si)));
-                    c = block_constant(static_cast<uint8_t>(qb), sg, mu);
+                    if (p.absmax) {
+                        c = __uint_as_float(lds32(c_q[pass] + 16u * s));
+                    } else {
+                        const uint32_t qb = lds8(c_q[pass] + 4u * s);
+                        const int64_t si = (c_e[pass] + 4 * s) >> 8;
+                        const float sg = __uint_as_float(lds32(s_ss + 4u * static_cast<uint32_t>(si)));
+                        c = block_constant(static_cast<uint8_t>(qb), sg, mu);
+                    }
                 }
                 cmine[pass] = c;
             }
@@ -989,12 +1008,13 @@ bool layout_mode(FwdArgs &a, int MP, bool x_once) {
     a.x_bytes = xb;
     a.xa_bytes = xpb + ab;
     const uint32_t xs = x_once ? align_up(static_cast<uint32_t>(nsmax) * xb, 128) : 0u;
-    // staged FP8 codes: 16-byte chunks per chunk row, an odd count so that rows fall on
-    // distinct bank groups
-    const int nch = (15 + 4 * nsmax + 15) / 16;
+    // staged FP8 codes (or fp32 constants): 16-byte chunks per chunk row, an odd count so that
+    // rows fall on distinct bank groups
+    const int nch = a.absmax ? (12 + 16 * nsmax + 15) / 16 : (15 + 4 * nsmax + 15) / 16;
     a.qs_stride = 16u * static_cast<uint32_t>(nch | 1);
-    // staged group scales: at most R nbr / 256 + 2 of them, in whole 16-byte chunks
-    const int64_t s_max = static_cast<int64_t>(a.R) * a.nbr / 256 + 8;
+    // staged group scales: at most R nbr / 256 + 2 of them, in whole 16-byte chunks (none with
+    // fp32 constants)
+    const int64_t s_max = a.absmax ? 0 : static_cast<int64_t>(a.R) * a.nbr / 256 + 8;
     if (s_max > (int64_t(1) << 20)) return false;
     const uint32_t qs = align_up(static_cast<uint32_t>(a.R) * a.qs_stride, 128);
     const uint32_t ss = align_up(static_cast<uint32_t>(s_max) * 4u, 128);
@@ -1124,6 +1144,8 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
     a.q = w.q;
     a.sigma = w.sigma;
     a.mu = w.mu;
+    a.absmax = w.absmax;
+    a.qtype = w.qtype;
     a.B = B;
     a.x = x;
     a.h = h;

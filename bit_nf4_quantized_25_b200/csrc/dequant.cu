@@ -1,6 +1,7 @@
-// dequant.cu -- nf4_dequantize on sm_100a: codes + double-quantised constants -> bf16 W.
+// dequant.cu -- nf4_dequantize on sm_100a: codes + block constants -> bf16 W.
 //
-// W'[e] = bf16_rn(fl32(NF4[code_e] * c'_b)), c'_b = fma(e4m3(q_b), sigma_g, mu).
+// W'[e] = bf16_rn(fl32(T[code_e] * c'_b)), T the quant type's table (NF4 or the 4-bit float),
+// c'_b = fma(e4m3(q_b), sigma_g, mu) with double quantisation, else the fp32 absmax c_b.
 // "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com): the 4-bit weights are
 // dequantised to the bf16 compute type for the matmul.
 //
@@ -20,17 +21,18 @@ constexpr int kDeqThreads = 256;
 
 __global__ void __launch_bounds__(kDeqThreads)
 k_dequant(const uint32_t *__restrict__ codes, const uint8_t *__restrict__ q, const float *__restrict__ sigma,
-          const float *__restrict__ mu_p, int64_t n_words, uint4 *__restrict__ out) {
+          const float *__restrict__ mu_p, const float *__restrict__ absmax, int qtype, int64_t n_words,
+          uint4 *__restrict__ out) {
     __shared__ float s_t[16];
-    if (threadIdx.x < 16) s_t[threadIdx.x] = nf4_value(threadIdx.x);
+    if (threadIdx.x < 16) s_t[threadIdx.x] = table_value(qtype, threadIdx.x);
     __syncthreads();
-    const float mu = __ldg(mu_p);
+    const float mu = load_mu(mu_p, absmax);
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     // A thread expands one 32-bit code word (8 weights, 16 bytes of bf16) per step, so a warp
     // reads 128 contiguous bytes and writes 512; two steps are loaded before either is expanded.
     auto expand = [&](uint32_t w, int64_t word) {
         const int64_t b = word >> 3;  // 8 words = 64 weights = one block
-        const float cp = block_constant(__ldg(q + b), __ldg(sigma + b / kGroup), mu);
+        const float cp = load_block_constant(q, sigma, mu, absmax, b);
         uint4 o;
         uint32_t *op = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
@@ -63,7 +65,8 @@ cudaError_t launch_dequant(const WeightView &w, uint16_t *out, cudaStream_t s) {
     const int64_t cap = static_cast<int64_t>(sms) * occ;  // one wave
     if (grid > cap) grid = cap;
     k_dequant<<<static_cast<unsigned>(grid), kDeqThreads, 0, s>>>(reinterpret_cast<const uint32_t *>(w.codes), w.q,
-                                                                   w.sigma, w.mu, n_words, reinterpret_cast<uint4 *>(out));
+                                                                   w.sigma, w.mu, w.absmax, w.qtype, n_words,
+                                                                   reinterpret_cast<uint4 *>(out));
     count_launch();
     return cudaGetLastError();
 }

@@ -62,6 +62,7 @@ struct GemmParams {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
+    const float *absmax;    // fp32 block constants (no double quantisation), else nullptr
     int64_t n, k;           // W is n x k
     int64_t M;              // tokens
     const uint16_t *lora;   // fwd: B (n x r); bwd: A (r x k)
@@ -76,16 +77,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-// 16 scaled table values bf16(NF4[i] * cp), split into low-byte planes L0..L3 and
-// high-byte planes H0..H3 (4 entries per register) for byte-permute lookups.
+// 16 scaled table values bf16(T[i] * cp) of quant type kQT, split into low-byte planes L0..L3
+// and high-byte planes H0..H3 (4 entries per register) for byte-permute lookups.
 struct Planes {
     uint32_t L0, L1, L2, L3, H0, H1, H2, H3;
 };
 
+template <int kQT>
 __device__ __forceinline__ Planes make_planes(float cp) {
     uint32_t E[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) E[i] = pack_bf16x2(__fmul_rn(nf4_value(2 * i), cp), __fmul_rn(nf4_value(2 * i + 1), cp));
+    for (int i = 0; i < 8; ++i)
+        E[i] = pack_bf16x2(__fmul_rn(table_value(kQT, 2 * i), cp), __fmul_rn(table_value(kQT, 2 * i + 1), cp));
     Planes P;
     P.L0 = prmt(E[0], E[1], 0x6420);
     P.H0 = prmt(E[0], E[1], 0x7531);
@@ -128,7 +131,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 // 64-element MN chunk of an MN-major tile whose K rows are 128 bytes apart.
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t j) { return row * 128u + ((j ^ (row & 7u)) << 4); }
 
-template <bool kBwd>
+template <bool kBwd, int kQT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lora,
            const __grid_constant__ CUtensorMap tm_codes, const GemmParams p) {
@@ -307,7 +310,7 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int dw = warp - 2;
         const int grp = dw >> 2;                  // stages i with i % kDqGroups == grp
         const int tid = (dw & 3) * 32 + lane;     // 0..127 within the group
-        const float mu = __ldg(p.mu);
+        const float mu = load_mu(p.mu, p.absmax);
         // fwd: thread = A row (weight row row0 + tid), 64 k per stage.
         // bwd: thread = (reduction row tid/2 of the stage, feature half tid%2).
         const uint32_t arow = kBwd ? static_cast<uint32_t>(tid >> 1) : static_cast<uint32_t>(tid);
@@ -315,8 +318,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
         const int64_t kf = row0 + 64 * half;  // bwd: first feature of this thread's block
         const bool bwd_kvalid = !kBwd || kf < K;
 
-        // The block's codes arrive by TMA into sC; its constant inputs (one byte and one float)
-        // are loaded one of this group's stages ahead.
+        // The block's codes arrive by TMA into sC; its constant inputs (one byte and one float, or
+        // the fp32 constant itself in sg) are loaded one of this group's stages ahead.
         auto load_const = [&](int i, uint32_t &qb, float &sg, bool &valid) {
             valid = false;
             qb = 0u;
@@ -332,8 +335,12 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
                 if (wrow >= N) return;
                 blk = wrow * nbr + i;
             }
-            qb = __ldg(p.q + blk);
-            sg = __ldg(p.sigma + blk / kGroup);
+            if (p.absmax) {
+                sg = __ldg(p.absmax + blk);
+            } else {
+                qb = __ldg(p.q + blk);
+                sg = __ldg(p.sigma + blk / kGroup);
+            }
             valid = true;
         };
         const uint32_t c_off = kBwd ? arow * 64u + half * 32u : arow * 32u;  // this thread's block in sC
@@ -378,7 +385,8 @@ k_gemm_nf4(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ C
             };
             if (i < nred) {
                 if (cv) {
-                    const Planes P = make_planes(block_constant(static_cast<uint8_t>(cq), cs, mu));
+                    const Planes P =
+                        make_planes<kQT>(p.absmax ? cs : block_constant(static_cast<uint8_t>(cq), cs, mu));
                     const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                     for (int j = 0; j < 8; ++j) sts128(dst(j), expand8(P, w[j]));
@@ -522,7 +530,7 @@ bool make_codes_map(CUtensorMap *m, const void *codes, int64_t n, int64_t k, boo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kBwd>
+template <bool kBwd, int kQT>
 cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M, const uint16_t *lora_rows, int r,
                              const uint16_t *lora_act, int RT, uint16_t *out, int *err, cudaStream_t st) {
     CUtensorMap tm_act, tm_lora, tm_codes;
@@ -541,12 +549,12 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
     if (ge != cudaSuccess) return ge;
     const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
     if (bit == 0 || !(configured & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_nf4<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_nf4<kBwd, kQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kGemmSmem));
         if (e != cudaSuccess) return e;
         configured |= bit;
     }
-    GemmParams p{w.codes, w.q, w.sigma, w.mu, w.n, w.k, M, lora_rows, r, out, err};
+    GemmParams p{w.codes, w.q, w.sigma, w.mu, w.absmax, w.n, w.k, M, lora_rows, r, out, err};
     const int64_t tiles_m = ((kBwd ? w.k : w.n) + kTileM - 1) / kTileM;
     const int64_t tiles_n = (M + kTileN * kHalves - 1) / (kTileN * kHalves);
     cudaLaunchConfig_t cfg = {};
@@ -559,7 +567,7 @@ cudaError_t launch_gemm_impl(const WeightView &w, const uint16_t *act, int64_t M
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_nf4<kBwd>, tm_act, tm_lora, tm_codes, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_nf4<kBwd, kQT>, tm_act, tm_lora, tm_codes, p);
     count_launch();
     return e;
 }
@@ -587,7 +595,8 @@ cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, c
         cudaError_t e = launch_lora_down(x, M, w.k, A, w.k, 1, r, s, t, RT, st, drop);
         if (e != cudaSuccess) return e;
     }
-    return launch_gemm_impl<false>(w, x, M, B, r, t, RT, h, err, st);
+    return w.qtype == kQuantFP4 ? launch_gemm_impl<false, kQuantFP4>(w, x, M, B, r, t, RT, h, err, st)
+                                : launch_gemm_impl<false, kQuantNF4>(w, x, M, B, r, t, RT, h, err, st);
 }
 
 cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, const uint16_t *A, const uint16_t *B,
@@ -599,7 +608,8 @@ cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, 
         cudaError_t e = launch_lora_down(gh, M, w.n, B, 1, r, r, s, u, RT, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_gemm_impl<true>(w, gh, M, A, r, u, RT, gx, err, st);
+    return w.qtype == kQuantFP4 ? launch_gemm_impl<true, kQuantFP4>(w, gh, M, A, r, u, RT, gx, err, st)
+                                : launch_gemm_impl<true, kQuantNF4>(w, gh, M, A, r, u, RT, gx, err, st);
 }
 
 }  // namespace qn

@@ -9,9 +9,11 @@ namespace qn {
 struct WeightView {
     int64_t n, k;  // W is n x k, k % 64 == 0
     const uint8_t *codes;
-    const uint8_t *q;
+    const uint8_t *q;      // double-quantised constants (absmax == nullptr)
     const float *sigma;
     const float *mu;
+    int qtype;             // kQuantNF4 or kQuantFP4: the table of the code nibbles
+    const float *absmax;   // fp32 block constants (no double quantisation), else nullptr
 };
 
 // LoRA dropout of the adapter's input (dropout.cuh): element e = offset + m k_in + k of the
@@ -24,20 +26,24 @@ struct DropoutArgs {
 };
 
 // Lookup used by the quantiser: the interval [-1, 1] split into 64 cells of
-// width 1/32 plus the point 1.0; for cell j, `base[j]` is the number of code
-// thresholds below the cell and `thr[j]` the single threshold inside the cell
-// (or 2.0 when there is none).
+// width 1/32 plus the point 1.0; for cell j, `thr[j]` is the single decision
+// threshold inside the cell (or 2.0 when there is none) and `codes[j]` the codes
+// below and above it (low byte: x <= thr, second byte: x > thr). `zero_word`: eight
+// copies of the code of an all-zero block.
 struct QuantCells {
     float thr[65];
-    int base[65];
+    int codes[65];
+    uint32_t zero_word;
 };
 
 // Launch counter (per host thread).
 void count_launch(int n = 1);
 
 // nf4_quantize: two kernels plus a memset of the exponent bins.
-cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
-                            float *mu, void *ws, cudaStream_t s);
+// With absmax != nullptr the block absmaxes are stored there as fp32 (no double quantisation;
+// q, sigma and mu are not written). qtype: kQuantNF4 or kQuantFP4.
+cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, int qtype, uint8_t *codes, uint8_t *q,
+                            float *sigma, float *mu, float *absmax, void *ws, cudaStream_t s);
 size_t quantize_workspace_bytes(int64_t n, int64_t k);
 // Static scratch of the allocation-free quantiser entry point: size, and its device address on
 // the current device (resolved once per device).

@@ -1,6 +1,6 @@
 // merge.cu -- fold the adapter into a 16-bit weight on sm_100a:
 //
-//   W_merged[n, k] = bf16_rn( fl32(NF4[code] * c'_b) + s * sum_j B[n,j] A[j,k] )
+//   W_merged[n, k] = bf16_rn( fl32(T[code] * c'_b) + s * sum_j B[n,j] A[j,k] )   (T: NF4 or the 4-bit float)
 //
 // ("QLoRA & PEFT family" (ai-reference-codex), 3.6 merge_and_unload; "QLoRA paper notes"
 // (tqpw.cn), Introduction: the merged weight cannot stay NF4, so it is written as bf16.)
@@ -30,6 +30,8 @@ struct MergeArgs {
     const uint8_t *q;
     const float *sigma;
     const float *mu;
+    const float *absmax;  // fp32 block constants (no double quantisation), else nullptr
+    int qtype;
     const uint16_t *A;  // r x k
     const uint16_t *B;  // n x r
     int64_t n, k;
@@ -53,9 +55,9 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(const MergeArgs p) {
     float *Dp = reinterpret_cast<float *>(smem);                                   // [128][kDPad]
     uint16_t *At = reinterpret_cast<uint16_t *>(smem + kTileRows * kDPad * 4);      // [64][rk] transposed A
     __shared__ float s_t[16];
-    if (threadIdx.x < 16) s_t[threadIdx.x] = nf4_value(threadIdx.x);
+    if (threadIdx.x < 16) s_t[threadIdx.x] = table_value(p.qtype, threadIdx.x);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const float mu = __ldg(p.mu);
+    const float mu = load_mu(p.mu, p.absmax);
     const int64_t nbr = p.k / kBlock;
     const int64_t row_tiles = (p.n + kTileRows - 1) / kTileRows;
     const int64_t tiles = row_tiles * nbr;
@@ -108,7 +110,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(const MergeArgs p) {
             if (row >= p.n) continue;
             const int64_t blk = row * nbr + col;
             const uint32_t w = __ldcs(p.codes + blk * 8 + wd);
-            const float cp = block_constant(__ldg(p.q + blk), __ldg(p.sigma + blk / kGroup), mu);
+            const float cp = load_block_constant(p.q, p.sigma, mu, p.absmax, blk);
             const float *dv = Dp + rl * kDPad + 8 * wd;
             uint4 o;
             uint32_t *op = reinterpret_cast<uint32_t *>(&o);
@@ -132,8 +134,8 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge(const MergeArgs p) {
 cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int r, float s, uint16_t *out,
                          cudaStream_t st) {
     if (w.n == 0 || w.k == 0) return cudaSuccess;
-    MergeArgs p{reinterpret_cast<const uint32_t *>(w.codes), w.q, w.sigma, w.mu, A, B, w.n, w.k, r,
-                (r + 15) / 16 * 16, s, out};
+    MergeArgs p{reinterpret_cast<const uint32_t *>(w.codes), w.q, w.sigma, w.mu, w.absmax, w.qtype, A, B, w.n, w.k,
+                r, (r + 15) / 16 * 16, s, out};
     const size_t smem = static_cast<size_t>(kTileRows) * kDPad * 4 + static_cast<size_t>(kTileCols) * p.rk * 2;
     const void *kern = reinterpret_cast<const void *>(k_merge);
     cudaError_t e = ensure_smem_limit(kern, smem);

@@ -1,14 +1,15 @@
-// quantize.cu -- nf4_quantize on sm_100a: NF4 codes with blockwise absmax (64 weights) and
-// double quantisation of the block absmaxes (tensor mean, FP8 E4M3 in groups of 256).
+// quantize.cu -- nf4_quantize on sm_100a: 4-bit codes (NF4, or the 4-bit float E2M1) with
+// blockwise absmax (64 weights) and double quantisation of the block absmaxes (tensor mean,
+// FP8 E4M3 in groups of 256), or the absmaxes kept as fp32.
 //
 // "QLoRA paper notes" (tqpw.cn), sections "NormalFloat Quantization (NF4)" and
 // "Double Quantization"; "How does QLoRA work for training?" (aivaro.ru), section 5.
 //
 // Kernel 1 (HBM-bound, one pass over W): each 8-lane group owns one 64-weight block
 // (16-byte coalesced loads), takes the absmax with three shuffles, forms x = w / absmax,
-// picks the code through a 65-cell lookup of the 15 decision thresholds (the cell index
+// picks the code through a 65-cell lookup of the decision thresholds (the cell index
 // floor(32 x + 32) is the low bits of one fma rounded toward -inf against 2^23 + 32, and the
-// cell's threshold and base code are one 8-byte shared load), packs 8 codes per
+// cell's threshold and its two codes are one 8-byte shared load), packs 8 codes per
 // 32-bit word, writes the fp32 absmax to the workspace and adds it to 256 exponent bins
 // (integer sums, so the tensor sum is exact and independent of scheduling).
 // The codes are defined by the IEEE quotient fl32(w / c). The kernel multiplies by the
@@ -16,7 +17,8 @@
 // redoes the IEEE division, for the lane's eight weights, only when a product lies within
 // 2^-21 of its cell's threshold -- the only case where the two can fall on different sides
 // of it. Near a cell edge the two may pick neighbouring cells; both give the same code there
-// because no threshold lies within 2^-19 of a cell edge (checked on the host).
+// because no threshold lies within 2^-19 of a cell edge (checked on the host; the 4-bit float
+// has a threshold on a cell edge, 1/8, so it always takes the IEEE quotient).
 // The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include <mutex>
@@ -47,10 +49,10 @@ __global__ void __launch_bounds__(kQuantThreads)
 k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ codes, float *__restrict__ cblk,
                unsigned long long *__restrict__ bins, unsigned *__restrict__ done, float *__restrict__ mu_out,
                QuantCells cells, int fast_ok_flag) {
-    __shared__ int2 s_cell[65];  // {threshold bits, base code} of each cell
+    __shared__ int2 s_cell[65];  // {threshold bits, code below | code above << 8} of each cell
     const bool fast_ok = fast_ok_flag != 0;  // reciprocal path allowed (checked on the host)
     __shared__ unsigned s_bins[256];
-    for (int i = threadIdx.x; i < 65; i += blockDim.x) s_cell[i] = make_int2(__float_as_int(cells.thr[i]), cells.base[i]);
+    for (int i = threadIdx.x; i < 65; i += blockDim.x) s_cell[i] = make_int2(__float_as_int(cells.thr[i]), cells.codes[i]);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0u;
     __syncthreads();
 
@@ -76,7 +78,7 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
         const float c = __uint_as_float(m << 16);  // block absmax, exact (a bf16 value)
-        uint32_t word = 0x77777777u;               // all-zero block: code 7 everywhere
+        uint32_t word = cells.zero_word;           // all-zero block: the code of 0 everywhere
         if (c != 0.0f) {
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
             auto weight = [&](int i) {
@@ -91,7 +93,7 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
                     min(max(static_cast<int>(__float_as_uint(__fmaf_rd(x, 32.0f, 8388640.0f)) - 0x4B000000u), 0), 64);
                 const int2 cell = s_cell[j];
                 dist = x - __int_as_float(cell.x);
-                return cell.y + (dist > 0.0f ? 1 : 0);
+                return dist > 0.0f ? (cell.y >> 8) : (cell.y & 0xff);
             };
             // c is a bf16 value, so c >= 2^-126 exactly when its exponent field is non-zero
             const bool fast = fast_ok && (m >> 7) != 0u;
@@ -256,40 +258,81 @@ k_double_quant(const float *__restrict__ cblk, int64_t nb, uint8_t *__restrict__
     }
 }
 
-// Decision thresholds t_i = largest fp32 not above the midpoint of table values i and
-// i+1; for an fp32 x, "x > t_i" equals "x is nearer to value i+1 than to value i, or
-// at equal distance goes to the lower index".
-// The reciprocal path needs every decision threshold farther than 2^-19 from every cell edge.
-int reciprocal_path_ok() {
-    for (int i = 0; i < 15; ++i) {
-        const double m = (static_cast<double>(nf4_value(i)) + static_cast<double>(nf4_value(i + 1))) * 0.5;
-        for (int j = 0; j <= 64; ++j)
-            if (fabs(m - (-1.0 + j / 32.0)) <= 0x1p-19) return 0;
+// Decision thresholds of a quant type: its distinct values ascending, each with the lowest code
+// of that value (+0 before -0), and between neighbours v_j < v_j+1 with midpoint m_j (exact in
+// fp64) a threshold t_j such that, for an fp32 x, "x > t_j" picks the upper neighbour exactly
+// when x is nearer to it, or at equal distance and its code is the lower one: t_j = the largest
+// fp32 not above m_j, one step lower still when m_j is an fp32 value and a tie goes up.
+struct Thresholds {
+    int nv;          // distinct values
+    int code[16];    // their codes, ascending by value
+    double mid[15];  // midpoints
+    float t[15];
+};
+
+Thresholds make_thresholds(int qtype) {
+    Thresholds th{};
+    double v[16];
+    for (int c = 0; c < 16; ++c) {
+        const double val = table_value(qtype, c);
+        bool seen = false;
+        for (int j = 0; j < th.nv; ++j) seen = seen || v[j] == val;
+        if (seen) continue;
+        int j = th.nv++;
+        for (; j > 0 && v[j - 1] > val; --j) {
+            v[j] = v[j - 1];
+            th.code[j] = th.code[j - 1];
+        }
+        v[j] = val;
+        th.code[j] = c;
     }
+    for (int j = 0; j + 1 < th.nv; ++j) {
+        const double m = (v[j] + v[j + 1]) * 0.5;
+        float f = static_cast<float>(m);
+        if (static_cast<double>(f) > m) f = nextafterf(f, -2.0f);
+        if (th.code[j + 1] < th.code[j] && static_cast<double>(f) == m) f = nextafterf(f, -2.0f);
+        th.mid[j] = m;
+        th.t[j] = f;
+    }
+    return th;
+}
+
+// The reciprocal path needs every decision threshold farther than 2^-19 from every cell edge.
+int reciprocal_path_ok(int qtype) {
+    const Thresholds th = make_thresholds(qtype);
+    for (int i = 0; i + 1 < th.nv; ++i)
+        for (int j = 0; j <= 64; ++j)
+            if (fabs(th.mid[i] - (-1.0 + j / 32.0)) <= 0x1p-19) return 0;
     return 1;
 }
 
-QuantCells make_cells() {
-    QuantCells c;
-    double t[15];
-    for (int i = 0; i < 15; ++i) {
-        const double m = (static_cast<double>(nf4_value(i)) + static_cast<double>(nf4_value(i + 1))) * 0.5;
-        float f = static_cast<float>(m);
-        if (static_cast<double>(f) > m) f = nextafterf(f, -2.0f);
-        t[i] = f;
-    }
+// Cells of a quant type; false if two thresholds fall into one cell.
+bool make_cells(int qtype, QuantCells *out) {
+    const Thresholds th = make_thresholds(qtype);
+    QuantCells c{};
     for (int j = 0; j <= 64; ++j) {
         const double lo = -1.0 + j / 32.0, hi = (j == 64) ? 1.0 : -1.0 + (j + 1) / 32.0;
-        int base = 0;
+        int base = 0, inside = 0;
         float thr = 2.0f;
-        for (int i = 0; i < 15; ++i) {
-            if (t[i] < lo) ++base;
-            else if (t[i] < hi || (j == 64 && t[i] <= hi)) thr = static_cast<float>(t[i]);
+        for (int i = 0; i + 1 < th.nv; ++i) {
+            if (th.t[i] < lo) {
+                ++base;
+            } else if (th.t[i] < hi || (j == 64 && th.t[i] <= hi)) {
+                thr = th.t[i];
+                ++inside;
+            }
         }
-        c.base[j] = base;
+        if (inside > 1) return false;
+        const int below = th.code[base], above = inside ? th.code[base + 1] : below;
         c.thr[j] = thr;
+        c.codes[j] = below | (above << 8);
     }
-    return c;
+    int zero = 7;
+    for (int j = 0; j < th.nv; ++j)
+        if (table_value(qtype, th.code[j]) == 0.0f) zero = th.code[j];
+    c.zero_word = 0x11111111u * static_cast<uint32_t>(zero);
+    *out = c;
+    return true;
 }
 
 // Scratch for callers that cannot allocate device memory (nf4_quantize_static_ws): a
@@ -338,15 +381,29 @@ size_t quantize_workspace_bytes(int64_t n, int64_t k) {
     return kHeaderBytes + ((static_cast<size_t>(nb) * sizeof(float) + 255) & ~size_t(255));
 }
 
-cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *q, float *sigma,
-                            float *mu, void *ws, cudaStream_t s) {
-    static const QuantCells cells = make_cells();
-    static const int fast_ok = reciprocal_path_ok();
+cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, int qtype, uint8_t *codes, uint8_t *q,
+                            float *sigma, float *mu, float *absmax, void *ws, cudaStream_t s) {
+    struct Tables {
+        QuantCells cells[2];
+        int fast_ok[2];
+        bool ok;
+    };
+    static const Tables tables = [] {
+        Tables t{};
+        t.ok = make_cells(kQuantNF4, &t.cells[0]) && make_cells(kQuantFP4, &t.cells[1]);
+        t.fast_ok[0] = reciprocal_path_ok(kQuantNF4);
+        t.fast_ok[1] = reciprocal_path_ok(kQuantFP4);
+        return t;
+    }();
+    if (!tables.ok || qtype < 0 || qtype > 1) return cudaErrorInvalidValue;
     const int64_t nb = n * k / kBlock;
     if (nb == 0) return cudaSuccess;
     auto *bins = static_cast<unsigned long long *>(ws);
     auto *done = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + kBinsBytes);
-    auto *cblk = reinterpret_cast<float *>(static_cast<char *>(ws) + kHeaderBytes);
+    // without double quantisation the absmaxes go straight to the output and the mean (unused)
+    // to the header
+    auto *cblk = absmax ? absmax : reinterpret_cast<float *>(static_cast<char *>(ws) + kHeaderBytes);
+    float *mu_out = absmax ? reinterpret_cast<float *>(static_cast<char *>(ws) + kBinsBytes + 128) : mu;
     cudaError_t e = cudaMemsetAsync(bins, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return e;
     int sms = 148, occ = 4;
@@ -361,11 +418,11 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, uint8_t *co
     const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
     if (grid < min_grid) grid = min_grid;
     k_quant_blocks<<<static_cast<unsigned>(grid), kQuantThreads, 0, s>>>(
-        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, done, mu, cells,
-        fast_ok);
+        reinterpret_cast<const uint4 *>(W), nb, reinterpret_cast<uint32_t *>(codes), cblk, bins, done, mu_out,
+        tables.cells[qtype], tables.fast_ok[qtype]);
     count_launch();
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || absmax) return e;
     const int64_t ng = (nb + kGroup - 1) / kGroup;
     int64_t grid2 = (ng + (kDqThreads / 32) - 1) / (kDqThreads / 32);
     grid2 = grid2 < static_cast<int64_t>(sms) * 4 ? grid2 : static_cast<int64_t>(sms) * 4;

@@ -2,8 +2,8 @@
 // decode_fwd.cu, input gradient in decode_bwd.cu): the bf16-pair table, shared-memory loads,
 // cluster barriers, the launch-shape planner and the error word.
 //
-// The pair table: a code byte (two nibbles) maps to a bf16 pair of NF4 values,
-// bf16x2(NF4[byte & 15], NF4[byte >> 4]). It is stored once per lane in 256-byte rows, so the
+// The pair table: a code byte (two nibbles) maps to a bf16 pair of table values (NF4 or the
+// 4-bit float), bf16x2(T[byte & 15], T[byte >> 4]). It is stored once per lane in 256-byte rows, so the
 // byte permute that extracts a byte also forms the conflict-free address (byte << 8 | lane << 2);
 // 64 KB per CTA, of which the second half of every row is unused (a packed 32 KB table needs one
 // more shift per lookup and measured slower). NF4 values: "QLoRA paper notes" (tqpw.cn),
@@ -60,14 +60,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     return v;
 }
 
-// Row e of the pair table (a code byte) holds bf16x2(NF4[e & 15], NF4[e >> 4]) in its first
-// 32 words, one copy per lane. The eight 16-byte stores of a row start at a column rotated by
-// the row so that the lanes of a warp hit different banks.
-__device__ __forceinline__ void build_pair_lut(uint8_t *lut, int tid, int nthreads) {
+// Row e of the pair table (a code byte) holds bf16x2(T[e & 15], T[e >> 4]) in its first 32
+// words, one copy per lane (T: the table of quant type qtype). The eight 16-byte stores of a row
+// start at a column rotated by the row so that the lanes of a warp hit different banks.
+__device__ __forceinline__ void build_pair_lut(uint8_t *lut, int tid, int nthreads, int qtype) {
     uint4 *l4 = reinterpret_cast<uint4 *>(lut);
     for (int i = tid; i < 256 * 8; i += nthreads) {
         const int e = i >> 3, c = i & 7;
-        const uint32_t v = pack_bf16x2(nf4_value(e & 15), nf4_value(e >> 4));
+        const uint32_t v = pack_bf16x2(table_value(qtype, e & 15), table_value(qtype, e >> 4));
         l4[e * 16 + ((c + e) & 7)] = make_uint4(v, v, v, v);
     }
 }

@@ -67,13 +67,33 @@ typedef enum {
 /* Largest supported LoRA rank. */
 #define QN_MAX_RANK 256
 
-/* A quantised weight. The struct is host memory; the four buffers are device
- * memory owned by the caller, with the sizes qn_nf4_sizes() returns; codes,
- * absmax_q and group_scale start on 16-byte boundaries (QN_EALIGN otherwise).
+/* The two other settings of the 4-bit load ("Quantized LoRA (QLoRA) and 4-bit
+ * training" (apxml.com), the four configuration knobs; "How does QLoRA work for
+ * training?" (aivaro.ru) 6, bnb_4bit_quant_type and bnb_4bit_use_double_quant):
+ *   quant type  : the table the code nibbles index. QN_QUANT_NF4 (the default):
+ *                 NormalFloat4 as printed in "QLoRA paper notes" (tqpw.cn). QN_QUANT_FP4:
+ *                 the standard 4-bit float, read as E2M1 (sign, two exponent bits with
+ *                 bias 1, one mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) divided
+ *                 by 6 onto [-1, 1] and rounded to fp32; code = sign (bit 3) | magnitude
+ *                 index (bits 0-2). "QLoRA paper notes", Experiments: NF4 does better.
+ *   block constants: QN_CONST_DQ (the default): double quantised (absmax_q,
+ *                 group_scale, absmax_mean). QN_CONST_F32: the exact fp32 block absmax
+ *                 in `absmax` (0.5 bit per weight instead of 0.127; "QLoRA & PEFT family"
+ *                 (ai-reference-codex) 3.3). */
+#define QN_QUANT_NF4 0
+#define QN_QUANT_FP4 1
+#define QN_CONST_DQ 0
+#define QN_CONST_F32 1
+
+/* A quantised weight. The struct is host memory; the buffers are device memory
+ * owned by the caller, with the sizes qn_weight_sizes() returns; codes,
+ * absmax_q, group_scale and absmax start on 16-byte boundaries (QN_EALIGN
+ * otherwise). A zero-initialised struct tail (quant_type, const_format, absmax)
+ * is NF4 with double quantisation.
  *   codes        : n_out*k_in/2 bytes. Weight e = n*k_in + k (row-major) is the
  *                  low nibble of byte e/2 when e is even, the high nibble when e
- *                  is odd. A nibble is an index 0..15 into the NF4 table
- *                  (ascending values, index 7 is 0.0).
+ *                  is odd. A nibble is an index 0..15 into the quant type's table
+ *                  (NF4: ascending values, index 7 is 0.0; FP4: see above).
  *   absmax_q     : nb = n_out*k_in/64 bytes, the FP8 E4M3 (finite variant,
  *                  max 448) code of d_b = absmax_b - mean, divided by the
  *                  group scale.
@@ -82,8 +102,13 @@ typedef enum {
  *                  straddle rows).
  *   absmax_mean  : 1 float, the exact mean of all nb block absmaxes, rounded
  *                  once to fp32.
+ *   (absmax_q, group_scale and absmax_mean: QN_CONST_DQ only; NULL otherwise.)
+ *   quant_type   : QN_QUANT_NF4 or QN_QUANT_FP4.
+ *   const_format : QN_CONST_DQ or QN_CONST_F32.
+ *   absmax       : QN_CONST_F32 only: nb floats, the block absmaxes c_b.
  * Block constant: c'_b = fma(e4m3_decode(absmax_q[b]), group_scale[b/256],
- * absmax_mean) in fp32; dequantised weight: NF4[code] * c'_b. */
+ * absmax_mean) in fp32 (QN_CONST_DQ), or c_b itself (QN_CONST_F32); dequantised
+ * weight: T[code] * c'_b with T the quant type's table. */
 typedef struct {
     int64_t n_out;
     int64_t k_in;
@@ -91,6 +116,9 @@ typedef struct {
     uint8_t *absmax_q;
     float *group_scale;
     float *absmax_mean;
+    int32_t quant_type;
+    int32_t const_format;
+    float *absmax;
 } qn_nf4_weight;
 
 /* Byte sizes of the four buffers of a quantised n_out x k_in weight.
@@ -99,13 +127,23 @@ typedef struct {
 qn_status qn_nf4_sizes(int64_t n_out, int64_t k_in, size_t *codes_bytes, size_t *absmax_bytes,
                        size_t *scale_bytes, size_t *mean_bytes);
 
+/* Byte sizes of the buffers of a quantised n_out x k_in weight with block
+ * constants const_format: QN_CONST_DQ gives qn_nf4_sizes()'s four sizes and
+ * absmax_f32_bytes = 0; QN_CONST_F32 gives codes_bytes, absmax_f32_bytes = 4 nb
+ * and zero for the three double-quantisation buffers.
+ * Errors: as qn_nf4_sizes, QN_EINVAL for an unknown const_format. */
+qn_status qn_weight_sizes(int64_t n_out, int64_t k_in, int const_format, size_t *codes_bytes, size_t *absmax_bytes,
+                          size_t *scale_bytes, size_t *mean_bytes, size_t *absmax_f32_bytes);
+
 /* Workspace bytes nf4_quantize needs for an n_out x k_in weight. Host-only. */
 qn_status qn_quantize_workspace_size(int64_t n_out, int64_t k_in, size_t *ws_bytes);
 
-/* nf4_quantize -- W (n_out x k_in bf16, device) -> the quantised weight `out`.
+/* nf4_quantize -- W (n_out x k_in bf16, device) -> the quantised weight `out`,
+ * in out's quant type and constant format.
  * Per block of 64: absmax c_b, code = index of the table value nearest to
- * fl32(w / c_b) (ties to the lower index; c_b == 0 gives code 7), two codes per
- * byte. Then mean mu of all c_b (exact, rounded once), d_b = fl32(c_b - mu),
+ * fl32(w / c_b) (ties to the lower index; c_b == 0 gives the lowest code of the
+ * value 0: 7 for NF4, 0 for FP4), two codes per byte. QN_CONST_F32: absmax[b] =
+ * c_b. QN_CONST_DQ: mean mu of all c_b (exact, rounded once), d_b = fl32(c_b - mu),
  * group scale sigma_g = fl32(max_b |d_b| / 448), absmax_q[b] =
  * e4m3_rn_satfinite(fl32(d_b / sigma_g)) (0 when sigma_g == 0).
  * Source: "QLoRA paper notes" (tqpw.cn), "NormalFloat Quantization (NF4)" and
@@ -137,7 +175,7 @@ qn_status nf4_quantize(const void *W, const qn_nf4_weight *out, void *ws, size_t
 qn_status nf4_quantize_static_ws(const void *W, const qn_nf4_weight *out, void *stream);
 
 /* nf4_dequantize -- quantised weight -> W_out (n_out x k_in bf16, device):
- * W_out[e] = bf16_rn(fl32(NF4[code_e] * c'_b)).
+ * W_out[e] = bf16_rn(fl32(T[code_e] * c'_b)).
  * Source: "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), the
  * dequantisation step to bf16 before the matmul.
  * Errors: QN_EINVAL, QN_ESHAPE, QN_EALIGN (codes or W_out not 16-byte

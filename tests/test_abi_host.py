@@ -190,3 +190,43 @@ def test_workspace_check_rejects_null(lib):
 
 def test_timeout_status_has_a_description(lib):
     assert lib.qn_status_string(6).decode() == "a kernel gave up a bounded wait"
+
+
+# ------------------------------------------- quant type and constant format (host checks)
+# "Quantized LoRA (QLoRA) and 4-bit training" (apxml.com), the four configuration knobs: the
+# quant type and double quantisation are settings of the weight; the struct carries them.
+
+def test_weight_sizes_per_constant_format(lib):
+    from bit_nf4_quantized_25_b200.binding import CONST_DQ, CONST_F32
+    v = [ctypes.c_size_t() for _ in range(5)]
+    n, k = 4096, 4096
+    nb = n * k // 64
+    assert lib.qn_weight_sizes(n, k, CONST_DQ, *(ctypes.byref(x) for x in v)) == 0
+    assert [x.value for x in v] == [n * k // 2, nb, 4 * (nb // 256), 4, 0]
+    assert lib.qn_weight_sizes(n, k, CONST_F32, *(ctypes.byref(x) for x in v)) == 0
+    assert [x.value for x in v] == [n * k // 2, 0, 0, 0, 4 * nb]
+    # 0.5 bit per weight of fp32 constants ("QLoRA & PEFT family" 3.3)
+    assert 8 * v[4].value / (n * k) == 0.5
+    assert lib.qn_weight_sizes(n, k, 7, *(ctypes.byref(x) for x in v)) == 1
+
+
+def test_format_argument_errors_before_launch(lib):
+    from bit_nf4_quantized_25_b200.binding import CONST_F32, CWeight, QN_EALIGN, QN_EINVAL
+    P = ctypes.c_void_p
+    d = lib.nf4_dequantize
+    out = P(0x900000)
+    w = _weight()
+    w.quant_type = 5
+    assert d(ctypes.byref(w), out, None) == QN_EINVAL
+    w = _weight()
+    w.const_format = 9
+    assert d(ctypes.byref(w), out, None) == QN_EINVAL
+    f32 = CWeight(128, 128, 0x100000, None, None, None, 1, CONST_F32, None)
+    assert d(ctypes.byref(f32), out, None) == QN_EINVAL  # fp32 constants without absmax
+    f32.absmax = 0x200004
+    assert d(ctypes.byref(f32), out, None) == QN_EALIGN
+    # fp32 constants need none of the double-quantisation buffers: argument checks pass and
+    # only the missing W stops the quantiser
+    f32.absmax = 0x200000
+    assert lib.nf4_quantize(None, ctypes.byref(f32), P(0x700000), 1 << 20, None) == QN_EINVAL
+    assert "W" in lib.qn_last_error().decode()

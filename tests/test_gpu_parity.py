@@ -63,8 +63,13 @@ def assert_quant_equal(w, ref, what=""):
 
 
 def to_host_weight(w):
-    return dict(codes=w.codes.cpu().numpy(), q=w.absmax_q.cpu().numpy(), sigma=w.group_scale.cpu().numpy(),
-                mu=np.float32(w.absmax_mean.cpu().numpy()[0]))
+    d = dict(codes=w.codes.cpu().numpy(), qtype=w.quant_type, dq=w.double_quant)
+    if w.double_quant:
+        d.update(q=w.absmax_q.cpu().numpy(), sigma=w.group_scale.cpu().numpy(),
+                 mu=np.float32(w.absmax_mean.cpu().numpy()[0]))
+    else:
+        d.update(absmax=w.absmax.cpu().numpy())
+    return d
 
 
 # ------------------------------------------------------------------ quantiser
@@ -165,9 +170,9 @@ def test_bulk_quantize_roundtrip(oracle):
 
 # --------------------------------------------------------------- linear layer
 
-def run_case(oracle, case: synth.LayerCase, rows=None, check_bwd=True):
+def run_case(oracle, case: synth.LayerCase, rows=None, check_bwd=True, quant_type="nf4", double_quant=True):
     W, A, B, x, gh = synth.layer_inputs(case, DEV, need_grad=check_bwd)
-    w = qb.nf4_quantize(W)
+    w = qb.nf4_quantize(W, quant_type=quant_type, double_quant=double_quant)
     r = case.r
     Ad, Bd = (A, B) if r > 0 else (None, None)
     h = qb.qlora_linear_fwd(w, x, Ad, Bd, case.alpha)
@@ -487,3 +492,105 @@ def test_dropout_rate_zero_is_the_plain_call():
     d = qb.qlora_linear_bwd_x(w, gh, A, B, 32.0, dropout=(0.0, 11, 13))
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(c, d)
+
+
+# ------------------------------------------- quant type and constant format
+# The other settings of the 4-bit load ("Quantized LoRA (QLoRA) and 4-bit training", the four
+# configuration knobs): the 4-bit float (E2M1 / 6) instead of NF4, and fp32 block constants
+# instead of double quantisation. Codes and constants bit-exact, the layer within tolerance, on
+# every kernel path: few-token forward and input gradient (streamed and per-slice), the
+# tensor-core GEMM and the merge.
+
+FORMATS = [("fp4", True), ("fp4", False), ("nf4", False)]
+
+
+def _fmt_id(f):
+    return f"{f[0]}-{'dq' if f[1] else 'f32'}"
+
+
+def assert_format_equal(w, ref, what):
+    codes = w.codes.cpu().numpy()
+    nbad = int(np.sum(codes != ref["codes"]))
+    assert nbad == 0, f"{what}: {nbad} code bytes differ"
+    if w.double_quant:
+        assert_quant_equal(w, ref, what)
+    else:
+        got = w.absmax.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), ref["absmax"].view(np.uint32)), f"{what}: fp32 constants differ"
+
+
+@pytest.mark.parametrize("fmt", FORMATS, ids=_fmt_id)
+@pytest.mark.parametrize("n,k", [(1, 64), (200, 448), (5, 64 * 172), (4096, 4096), (11008, 4096)])
+def test_format_quantize_bit_exact(oracle, fmt, n, k):
+    W = synth.student_t_bf16((n, k), 0.02, seed=n + 3 * k, device=DEV)
+    w = qb.nf4_quantize(W, quant_type=fmt[0], double_quant=fmt[1])
+    torch.cuda.synchronize()
+    ref = oracle.quantize4(bits(W), n, k, fmt[0], fmt[1])
+    assert_format_equal(w, ref, f"{_fmt_id(fmt)} {n}x{k}")
+
+
+@pytest.mark.parametrize("dq", [True, False])
+def test_fp4_every_finite_bf16_pattern(oracle, dq):
+    # exhaustive for the 4-bit float's code decision (its ties and the IEEE-quotient path)
+    u = np.arange(65536, dtype=np.uint32)
+    pats = u[((u >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    pats = np.random.default_rng(2).permutation(pats)
+    pats = np.concatenate([pats, np.zeros((-pats.size) % 256, np.uint16)])
+    n, k = pats.size // 256, 256
+    W = torch.from_numpy(pats.view(np.int16).reshape(n, k).copy()).view(torch.bfloat16).to(DEV)
+    w = qb.nf4_quantize(W, quant_type="fp4", double_quant=dq)
+    torch.cuda.synchronize()
+    assert_format_equal(w, oracle.quantize4(bits(W), n, k, "fp4", dq), "fp4 all bf16")
+
+
+def test_fp4_special_blocks(oracle):
+    # all-zero blocks (code 0), exact ties at representable midpoints, +-absmax
+    W = torch.zeros(4, 1024, dtype=torch.bfloat16)
+    W[1, ::64] = 1.0
+    W[1, 1::64] = 0.125   # 1/8 of the absmax: a midpoint between 1/12 and 1/6
+    W[1, 2::64] = -0.125
+    W[2, 7] = -3.0e-3
+    W[3, :] = -2.0
+    for dq in (True, False):
+        w = qb.nf4_quantize(W.to(DEV), quant_type="fp4", double_quant=dq)
+        torch.cuda.synchronize()
+        assert_format_equal(w, oracle.quantize4(bits(W), 4, 1024, "fp4", dq), f"fp4 special dq={dq}")
+
+
+@pytest.mark.parametrize("fmt", FORMATS, ids=_fmt_id)
+def test_format_dequant_bit_exact(oracle, fmt):
+    for n, k, seed in [(256, 256, 0), (3, 64 * 172, 5), (4096, 4096, 7)]:
+        W = synth.student_t_bf16((n, k), 0.02, seed, device=DEV)
+        w = qb.nf4_quantize(W, quant_type=fmt[0], double_quant=fmt[1])
+        deq = qb.nf4_dequantize(w)
+        torch.cuda.synchronize()
+        ref = oracle.nf4_dequant_bf16(to_host_weight(w), n, k)
+        got = bits(deq).reshape(n, k)
+        assert np.array_equal(got, ref), f"{n}x{k}: {int(np.sum(got != ref))} dequantised weights differ"
+
+
+@pytest.mark.parametrize("fmt", FORMATS, ids=_fmt_id)
+@pytest.mark.parametrize("n,k,M,r", [(4096, 4096, 1, 16), (11008, 4096, 16, 16), (4096, 11008, 5, 16),
+                                     (200, 448, 7, 5), (136, 1024, 3, 0), (256, 256, 300, 4),
+                                     (200, 448, 129, 64)])
+def test_format_layer_matches_oracle(oracle, fmt, n, k, M, r):
+    # M <= 16: streamed few-token kernels (r = 5 and n = 200 take the per-slice input gradient);
+    # M > 64: the tensor-core GEMM
+    case = synth.LayerCase(f"{_fmt_id(fmt)}{n}x{k}M{M}r{r}", n, k, M, r, 2.0 * max(r, 1), 0.02, n + k + M + r)
+    run_case(oracle, case, quant_type=fmt[0], double_quant=fmt[1])
+
+
+@pytest.mark.parametrize("fmt", FORMATS, ids=_fmt_id)
+def test_format_merge_matches_oracle(oracle, fmt):
+    n, k, r, alpha = 200, 448, 5, 10.0
+    W = synth.normal_bf16((n, k), 0.02, 4, DEV)
+    A = synth.normal_bf16((r, k), 0.01, 5, DEV)
+    B = synth.normal_bf16((n, r), 0.01, 6, DEV)
+    w = qb.nf4_quantize(W, quant_type=fmt[0], double_quant=fmt[1])
+    got = qb.qlora_merge_bf16(w, A, B, alpha)
+    torch.cuda.synchronize()
+    ref = oracle.merge_bf16(to_host_weight(w), n, k, bits(A), bits(B), r, alpha)
+    g = bits(got).reshape(n, k)
+    assert_close(torch.from_numpy(g.view(np.int16)).view(torch.bfloat16), bf16_to_f64(ref), "merge")
+    d = _ulp_diff_bf16(g, ref)
+    assert float(np.mean(d <= 1)) > 0.999, f"{int((d > 1).sum())} merged weights more than one bf16 unit off"
