@@ -36,6 +36,8 @@ SHAPES_7B = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096
              ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
 DECODE_M = (1, 4, 16)
 RANK_7B, ALPHA_7B = 16, 32.0
+TRAIN_M = 4096
+TRAIN_LAYERS = 8  # weights of 8 layers (0.8 GB) stream from HBM every training step
 
 
 def weight_bytes(n, k):
@@ -237,6 +239,69 @@ def decode_step_fn(stack, xs, outs, ws):
     return step
 
 
+def decode_bwd_step_fn(stack, ghs, gxs, ws):
+    from bit_nf4_quantized_25_b200 import binding as qb
+
+    def step():
+        for M in DECODE_M:
+            for (name, n, k, w, A, B) in stack:
+                qb.qlora_linear_bwd_x(w, ghs[(M, n)], A, B, ALPHA_7B, out=gxs[(M, k)], workspace=ws)
+    return step
+
+
+def train_step_fn(stack, acts, ws):
+    """Forward and input gradient of every linear of the stack at M = TRAIN_M tokens."""
+    from bit_nf4_quantized_25_b200 import binding as qb
+
+    def step():
+        for (name, n, k, w, A, B) in stack:
+            qb.qlora_linear_fwd(w, acts[("x", k)], A, B, ALPHA_7B, out=acts[("h", n)], workspace=ws)
+            qb.qlora_linear_bwd_x(w, acts[("g", n)], A, B, ALPHA_7B, out=acts[("gx", k)], workspace=ws)
+    return step
+
+
+def capture(step, warmup):
+    """Eager warm-up, then one step captured into a CUDA graph; returns (graph, launches per step)."""
+    import torch
+
+    from bit_nf4_quantized_25_b200 import binding as qb
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        qb.launch_count(reset=True)
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        launches = qb.launch_count(reset=True)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    return graph, launches
+
+
+def profile_traffic(name):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None when the kernel's
+    sources have changed since the counters were taken."""
+    prof = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(prof):
+        return None
+    try:
+        import hashlib
+        with open(prof) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
+    except Exception:
+        return None
+
+
 def time_graph(graph, steps, stream):
     import torch
     start = torch.cuda.Event(enable_timing=True)
@@ -271,8 +336,9 @@ def time_fn(fn, reps=10, warm=3, flush=None):
     return statistics.median(ts)
 
 
-def detail_measurements(hbm_peak, tc_peak):
-    """Other workloads of the hot path, each timed with CUDA events (L2 flushed between reps)."""
+def detail_measurements(hbm_peak, tc_peak, only=None):
+    """Other workloads of the hot path, each timed with CUDA events (L2 flushed between reps);
+    `only`: run just the entries whose name contains it."""
     import torch
 
     from bit_nf4_quantized_25_b200 import binding as qb
@@ -282,6 +348,8 @@ def detail_measurements(hbm_peak, tc_peak):
     out = {}
     # quantise and dequantise (HBM-bound)
     for (n, k) in [(4096, 4096), (11008, 4096), (28672, 8192)]:
+        if only and only not in f"quantize_{n}x{k}" and only not in f"dequant_{n}x{k}":
+            continue
         W = synth.normal_bf16((n, k), 0.02, 7, dev)
         w = qb.nf4_quantize(W)
         ws = torch.empty(qb.quantize_workspace_size(n, k), dtype=torch.uint8, device=dev)
@@ -299,6 +367,8 @@ def detail_measurements(hbm_peak, tc_peak):
             [("l70b", n, k, M, 64, 16.0, 0.015) for (n, k) in [(8192, 8192), (28672, 8192), (8192, 28672)]
              for M in (1, 16, 4096)]
     for (tag, n, k, M, r, alpha, std) in cases:
+        if only and only not in f"{tag}_{n}x{k}_M{M}":
+            continue
         W = synth.normal_bf16((n, k), std, 11, dev)
         w = qb.nf4_quantize(W)
         del W
@@ -392,21 +462,7 @@ def run_ours(args):
     per_step_flops = sum(linear_flops(n, k, M, RANK_7B) for M in DECODE_M for (_, n, k, *_r) in stack)
 
     # warm-up (eager), then capture one step into a CUDA graph
-    for _ in range(max(args.warmup, 1)):
-        step()
-    torch.cuda.synchronize()
-    stream = torch.cuda.Stream()
-    stream.wait_stream(torch.cuda.current_stream())
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        qb.launch_count(reset=True)
-        with torch.cuda.graph(graph, stream=stream):
-            step()
-        launches_per_step = qb.launch_count(reset=True)
-    torch.cuda.synchronize()
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
+    graph, launches_per_step = capture(step, args.warmup)
 
     barrier(world)
     torch.cuda.synchronize()
@@ -425,21 +481,7 @@ def run_ours(args):
     avg_launch_s = t / (args.steps * launches_per_step)
     bytes_per_launch = per_step_bytes / launches_per_step
     achieved = bytes_per_launch / avg_launch_s / 1e9
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "decode_fwd_traffic.json")
-    if os.path.exists(prof):
-        # the ncu counters count only while the kernel source they were taken on is unchanged
-        try:
-            import hashlib
-            with open(prof) as f:
-                rec = json.load(f)
-            h = hashlib.sha256()
-            for src in rec["sources"]:
-                with open(os.path.join(ROOT, src), "rb") as f:
-                    h.update(f.read())
-            traffic = rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
-        except Exception:
-            traffic = None
+    traffic = profile_traffic("decode_fwd_traffic.json")
 
     # end to end through the public API: pinned H2D of the step's inputs, the step, D2H of outputs
     pinned_in = {key: v.cpu().pin_memory() for key, v in xs.items()}
@@ -467,12 +509,41 @@ def run_ours(args):
     torch.cuda.synchronize()
     te = barrier_max(a.elapsed_time(b) * 1e-3, world)
     e2e_value = job_rate(per_step_bytes, args.steps, world, te) / 1e9
+    del graph
+
+    # the few-token input gradient over the same stack (grad_h of M = 1, 4, 16 tokens)
+    ghs = {(M, n): synth.normal_bf16((M, n), 1.0, 7100 + M + n, dev) for M in DECODE_M for n in (4096, 11008)}
+    gxs = {(M, k): torch.empty(M, k, dtype=torch.bfloat16, device=dev) for M in DECODE_M for k in (4096, 11008)}
+    graph_b, launches_b = capture(decode_bwd_step_fn(stack, ghs, gxs, ws), args.warmup)
+    barrier(world)
+    tb = barrier_max(time_graph(graph_b, args.steps, torch.cuda.current_stream()), world)
+    del graph_b
+    bwd_avg_s = tb / (args.steps * launches_b)
+    bwd_rate = per_step_bytes / launches_b / bwd_avg_s / 1e9
+
+    # the training-step shapes: forward and input gradient of TRAIN_LAYERS 7B layers at M = 4096
+    tstack = stack[:7 * min(TRAIN_LAYERS, args.layers)]
+    acts = {}
+    for k in (4096, 11008):
+        acts[("x", k)] = synth.normal_bf16((TRAIN_M, k), 1.0, 7200 + k, dev)
+        acts[("gx", k)] = torch.empty(TRAIN_M, k, dtype=torch.bfloat16, device=dev)
+    for n in (4096, 11008):
+        acts[("g", n)] = synth.normal_bf16((TRAIN_M, n), 1.0, 7300 + n, dev)
+        acts[("h", n)] = torch.empty(TRAIN_M, n, dtype=torch.bfloat16, device=dev)
+    ws_t = qb.new_workspace(max(qb.linear_workspace_size(TRAIN_M, n, k, RANK_7B) for (_, n, k) in SHAPES_7B))
+    graph_t, launches_t = capture(train_step_fn(tstack, acts, ws_t), args.warmup)
+    barrier(world)
+    tt = barrier_max(time_graph(graph_t, args.steps, torch.cuda.current_stream()), world)
+    del graph_t
+    train_flops = 2 * sum(linear_flops(n, k, TRAIN_M, RANK_7B) for (_, n, k, *_r) in tstack)
+    train_tflops = train_flops * args.steps / tt / 1e12
+    del acts, ws_t, ghs, gxs
+    torch.cuda.empty_cache()
 
     detail = None
     cpu = None
     if rank == 0 and not args.no_detail:
-        del graph
-        detail = detail_measurements(hbm_peak, tc_burst)
+        detail = detail_measurements(hbm_peak, tc_burst, args.detail_only)
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline_sample(args.cpu_budget)
 
@@ -489,6 +560,23 @@ def run_ours(args):
                          "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind, "traffic": traffic,
                          "bytes_per_launch": round(bytes_per_launch), "avg_launch_us": round(avg_launch_s * 1e6, 3)},
+            "rooflines": [
+                {"bound": "hbm", "kernel": "k_decode_bwd (few-token NF4+LoRA input gradient)",
+                 "workload": "the same stack, grad_x at M in {1,4,16}, graph-replayed",
+                 "achieved": round(bwd_rate, 1), "peak": hbm_peak, "unit": "GB/s",
+                 "frac": round(bwd_rate / hbm_peak, 4), "peak_kind": peak_kind,
+                 "traffic": profile_traffic("decode_bwd_traffic.json"),
+                 "bytes_per_launch": round(per_step_bytes / launches_b),
+                 "avg_launch_us": round(bwd_avg_s * 1e6, 3), "ms_per_step": round(tb / args.steps * 1e3, 4)},
+                {"bound": "tensor", "kernel": "k_gemm_nf4 with k_lora_down_tiled (many-token path)",
+                 "workload": f"{len(tstack) // 7} Llama-7B layers x 7 linears, forward + input gradient, "
+                             f"M={TRAIN_M}, r=16, graph-replayed (whole-step rate, adapter kernel included)",
+                 "achieved": round(train_tflops, 1), "peak": tc_sust, "unit": "TFLOP/s",
+                 "frac": round(train_tflops / tc_sust, 4),
+                 "peak_kind": f"{peak_kind} sustained (timed inside a long step); burst {tc_burst}",
+                 "frac_of_burst": round(train_tflops / tc_burst, 4), "traffic": None,
+                 "launches_per_step": launches_t, "ms_per_step": round(tt / args.steps * 1e3, 4)},
+            ],
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks,
             "cpu_baseline": cpu,
@@ -539,6 +627,7 @@ def main():
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--detail-only", default=None, help="run only the detail entries whose name contains this")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

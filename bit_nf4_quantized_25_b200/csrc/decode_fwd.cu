@@ -128,7 +128,7 @@ struct FwdArgs {
     int x_once;                  // chunk CTAs stage the x of every stage once, after the dependency wait
     uint32_t xs_off, xs_stage;   // ... at xs_off, xs_stage bytes per stage ([4][M][128 B])
     uint32_t a_off;              // adapter CTAs: x [4][MP][128 B] at 0, A [4][rpad][128 B] at a_off
-    uint32_t ring_off, qs_off, ss_off, tb_off, bs_off, recv_off, bar_off, post_off;
+    uint32_t ring_off, qs_off, ss_off, tb_off, bs_off, recv_off, bt_off, bar_off, post_off;
     uint32_t qs_stride;  // bytes per chunk row of the staged FP8 codes (or fp32 constants)
     uint32_t bs_stride;  // bytes per staged row of B
     uint32_t codes_bytes, x_bytes, xa_bytes;  // transaction bytes: codes box; x box; adapter x + A boxes
@@ -341,7 +341,7 @@ template <int NG, bool kFixedBase>
 __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CUtensorMap *tm_x, const FwdArgs &p,
                                            uint8_t *smem) {
     constexpr int MP = 8 * NG;  // padded tokens
-    constexpr int MW = 4 / NG;  // m-tiles per warp at most (m <= 4 MW)
+    constexpr int MW = 4;  // m-tiles per warp at most (m <= 4 MW)
 #ifdef QN_TIMELINE
     const long long tl_c0 = clock64();
 #endif
@@ -409,6 +409,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         fence_barrier_init();
     }
     __syncthreads();  // barriers initialised
+    float mu_pre = 0.0f;  // the weight's mean (consumers), read before the dependency wait
     if (warp == 0) {
         // ------------------------------------------ producer, before the dependency wait: weights
         if (lane == 0) {
@@ -432,6 +433,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // rows from the slice's first to its last, in whole 16-byte chunks. Bytes past the arrays
         // read as zero. With fp32 constants, chunk row i holds them (4 per chunk) instead.
         const int ct = threadIdx.x - 32;
+        mu_pre = load_mu(p.mu, p.absmax);
         if (p.absmax) {
             const int64_t nbq = p.n * p.nbr;
             const int nch = static_cast<int>(p.qs_stride >> 4);
@@ -622,6 +624,36 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         cp_async_wait_all();  // the B rows
         __syncwarp();
+        if (C > 1 && p.r > 0 && !*bb.abort_flag) {
+            // B t of the rows this CTA finalises, [nrmax][MP] fp32, while the consumers reduce:
+            // 16-row tiles of the staged B rows times t on the tensor cores
+            float *btf = reinterpret_cast<float *>(smem + p.bt_off);
+            for (int rt = 0; rt < nr; rt += 16) {
+                const int rA = min(rt + g, nr - 1), rB = min(rt + g + 8, nr - 1);
+                float d[NG][4];
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) d[tg][0] = d[tg][1] = d[tg][2] = d[tg][3] = 0.0f;
+                for (int kc = 0; kc < p.rk16 / 16; ++kc) {
+                    const uint32_t j2 = static_cast<uint32_t>(16 * kc + 2 * t) * 2u;
+                    const uint32_t ba = bs + static_cast<uint32_t>(rA) * p.bs_stride + j2;
+                    const uint32_t bb2 = bs + static_cast<uint32_t>(rB) * p.bs_stride + j2;
+                    const uint32_t a0 = lds32(ba), a2 = lds32(ba + 16), a1 = lds32(bb2), a3 = lds32(bb2 + 16);
+#pragma unroll
+                    for (int tg = 0; tg < NG; ++tg) {
+                        const uint32_t tr = tb + static_cast<uint32_t>((tg * 8 + g) * p.rk16) * 2u + j2;
+                        mma_16816(d[tg], a0, a1, a2, a3, lds32(tr), lds32(tr + 16));
+                    }
+                }
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int row = rt + g + 8 * (e >> 1), tok = tg * 8 + 2 * t + (e & 1);
+                        if (row < nr) btf[row * MP + tok] = d[tg][e];
+                    }
+            }
+            __syncwarp();
+        }
         if (lane == 0) mbar_arrive(bb.tready);
         if (C > 1) cluster_wait();  // phase 1 (every thread waits once)
     } else {
@@ -647,7 +679,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
-        const float mu = load_mu(p.mu, p.absmax);
+        const float mu = mu_pre;
         // x rows of this lane's tokens (tokens beyond M read token tok % M; their columns of the
         // result are never stored): row kg M + tok of the x box, 16-byte chunks 2 t and 2 t + 1
         // of it, stored at chunk ^ (row & 7)
@@ -896,17 +928,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 if (row >= nrow) continue;
                 float sum = 0.0f;
                 for (int src = 0; src < C; ++src) sum += recvf[(src * nrmax + rr) * MP + tok];
-                if (p.r > 0) {
-                    const uint32_t brow = bs + static_cast<uint32_t>(rr) * p.bs_stride;
-                    const uint32_t trow = tb + static_cast<uint32_t>(tok * p.rk16) * 2u;
-                    float bt = 0.0f;
-                    for (int j = 0; j < p.rpad; j += 2) {
-                        const uint32_t bv = lds32(brow + 2u * j), tv = lds32(trow + 2u * j);
-                        bt = __fmaf_rn(bf16_lo(bv), bf16_lo(tv), bt);
-                        bt = __fmaf_rn(bf16_hi(bv), bf16_hi(tv), bt);
-                    }
-                    sum += bt;
-                }
+                if (p.r > 0) sum += reinterpret_cast<const float *>(smem + p.bt_off)[rr * MP + tok];
                 p.h[static_cast<int64_t>(tok) * p.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
             }
         }
@@ -1029,8 +1051,10 @@ bool layout_mode(FwdArgs &a, int MP, bool x_once) {
     const uint32_t recv_chunk = a.C > 1 ? static_cast<uint32_t>(a.C * ((a.R + a.C - 1) / a.C) * MP * 4) : 0u;
     const uint32_t recv_adapter = a.r > 0 ? static_cast<uint32_t>(a.C * MP * a.rpad * 4) : 0u;
     const uint32_t recv = align_up(recv_chunk > recv_adapter ? recv_chunk : recv_adapter, 128);
+    // B t of the finalised rows (C > 1): [ceil(R / C)][MP] fp32
+    const uint32_t bt = a.C > 1 && a.r > 0 ? align_up(static_cast<uint32_t>((a.R + a.C - 1) / a.C * MP * 4), 128) : 0u;
     const uint32_t bars = 256;
-    const uint64_t fixed = static_cast<uint64_t>(kLutBytes) + qs + ss + tbb + bsb + xs + recv + bars;
+    const uint64_t fixed = static_cast<uint64_t>(kLutBytes) + qs + ss + tbb + bsb + xs + recv + bt + bars;
     if (fixed + a.slot_bytes > kSmemLimit) return false;
     int stages = static_cast<int>((kSmemLimit - fixed) / a.slot_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -1067,6 +1091,8 @@ bool layout_mode(FwdArgs &a, int MP, bool x_once) {
     off += xs;
     a.recv_off = off;
     off += recv;
+    a.bt_off = off;
+    off += bt;
     a.bar_off = off;
     return static_cast<uint64_t>(off) + bars <= kSmemLimit;
 }
@@ -1101,7 +1127,7 @@ cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
     found = false;
     // m is a multiple of 4 (every consumer warp holds the same number of m-tiles) unless the
     // weight has fewer than 64 rows
-    const int m_max = 16 / NG;  // four m-tile rows of warps, 4 / NG m-tiles each
+    const int m_max = 16;  // four m-tile rows of warps, up to 4 m-tiles each
     const int m_min = rows < 64 ? static_cast<int>((rows + 15) / 16) : 4;
     const int m_step = rows < 64 ? 1 : 4;
     for (int C = 1; C <= kMaxCluster && C <= a.ncol; ++C) {
