@@ -365,28 +365,30 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         cp_async_arrive_noinc(&bb.full[slot]);
     };
 
-    if (warp == 0) {
-        if (lane == 0) {
-            for (int s = 0; s < S; ++s) {
-                mbar_init(&bb.full[s], 33);  // lane 0's arrive.expect_tx + 32 cp.async arrivals
-                mbar_init(&bb.empty[s], kConsumers);
-            }
-            mbar_init(bb.recv, 1);
-            if (C > 1) mbar_arrive_expect_tx(bb.recv, static_cast<uint32_t>(C * nf * MP * 4));
-            mbar_init(bb.atile, 1);
-            *bb.abort_flag = 0u;
-            fence_barrier_init();
-            tma_prefetch_desc(tm_codes);
-            tma_prefetch_desc(tm_g);
-            if (p.q_tma) tma_prefetch_desc(tm_q);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bb.full[s], 33);  // lane 0's arrive.expect_tx + 32 cp.async arrivals
+            mbar_init(&bb.empty[s], kConsumers);
         }
-        __syncwarp();
-        // weights of the first stages before the dependency wait
+        mbar_init(bb.recv, 1);
+        if (C > 1) mbar_arrive_expect_tx(bb.recv, static_cast<uint32_t>(C * nf * MP * 4));
+        mbar_init(bb.atile, 1);
+        *bb.abort_flag = 0u;
+        fence_barrier_init();
+        tma_prefetch_desc(tm_codes);
+        tma_prefetch_desc(tm_g);
+        if (p.q_tma) tma_prefetch_desc(tm_q);
+    }
+    __syncthreads();  // barriers initialised
+    if (warp == 0) {
+        // weights of the first stages before the dependency wait; the producer then goes on to
+        // the dependency wait and the grad_h requests while the consumers build the table
         const uint64_t pol = l2_policy_evict_first();
         for (int s = 0; s < npre; ++s) stage_weights(s, pol);
+    } else {
+        build_pair_lut(lut, threadIdx.x - 32, kThreads - 32, p.qtype);
+        named_sync(1, kConsumers * 32);  // the table is complete
     }
-    build_pair_lut(lut, threadIdx.x, kThreads, p.qtype);
-    __syncthreads();
     if (C > 1) cluster_arrive_relaxed();
     grid_dependents_launch();
     grid_dependency_wait();  // grad_h, A and B may come from the preceding kernel; grad_x may be read by it

@@ -473,9 +473,6 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         }
         cp_async_arrive_noinc(bb.consts);
         QN_TL(8, ct == 0);
-        build_pair_lut(lut, ct, kConsumers * 32, p.qtype);
-        named_sync(1, kConsumers * 32);  // the table is complete
-        QN_TL(23, ct == 0);
     }
     if (C > 1) cluster_arrive_relaxed();  // phase 1: this CTA runs (its shared memory may be written)
     grid_dependents_launch();
@@ -658,10 +655,12 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         if (C > 1) cluster_wait();  // phase 1 (every thread waits once)
     } else {
         // ------------------------------------------------------------------ consumers
+        // Right after the dependency wait the x copies are issued; the pair table is built while
+        // they are in flight.
+        const int ct = threadIdx.x - 32;
         if (p.x_once) {
             // x of every stage of the slice, [stage][block][token][64 values] with 16-byte chunk c
             // of row b M + tok at c ^ (row & 7); blocks past the row read as zero
-            const int ct = threadIdx.x - 32;
             const int per = kStageBlocks * p.M * 8;  // 16-byte chunks per stage
             for (int i = ct; i < ns * per; i += kConsumers * 32) {
                 const int sx = i / per, j = i - sx * per;
@@ -673,10 +672,11 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                                      static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
                                  v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
             }
-            cp_async_wait_all();
-            named_sync(5, kConsumers * 32);  // every consumer's copies have landed
-            QN_TL(22, ct == 0);
         }
+        build_pair_lut(lut, ct, kConsumers * 32, p.qtype);
+        if (p.x_once) cp_async_wait_all();
+        named_sync(1, kConsumers * 32);  // the table is complete and every consumer's x copies have landed
+        QN_TL(22, ct == 0);
         const uint32_t lane_op = lut_lane_operand<kFixedBase>(lut, lane);
         const uint32_t lut_base = s_base;
         const float mu = mu_pre;
