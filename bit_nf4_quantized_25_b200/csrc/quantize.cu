@@ -5,8 +5,8 @@
 // "QLoRA paper notes" (tqpw.cn), sections "NormalFloat Quantization (NF4)" and
 // "Double Quantization"; "How does QLoRA work for training?" (aivaro.ru), section 5.
 //
-// Kernel 1 (HBM-bound, one pass over W): each 8-lane group owns one 64-weight block
-// (16-byte coalesced loads), takes the absmax with three shuffles, forms x = w / absmax,
+// Kernel 1 (HBM-bound, one pass over W): each 4-lane group owns one 64-weight block (two 16-byte
+// loads a lane, the warp's loads contiguous), takes the absmax with two shuffles, forms x = w / absmax,
 // picks the code through a 65-cell lookup of the decision thresholds (the cell index
 // floor(32 x + 32) is the low bits of one fma rounded toward -inf against 2^23 + 32, and the
 // cell's threshold and its two codes are one 8-byte shared load), packs 8 codes per
@@ -14,12 +14,13 @@
 // (integer sums, so the tensor sum is exact and independent of scheduling).
 // The codes are defined by the IEEE quotient fl32(w / c). The kernel multiplies by the
 // correctly rounded reciprocal instead (|w*r - w/c| < 2^-22 for |w| <= c, c normal) and
-// redoes the IEEE division, for the lane's eight weights, only when a product lies within
+// redoes the IEEE division, for the lane's sixteen weights, only when a product lies within
 // 2^-21 of its cell's threshold -- the only case where the two can fall on different sides
 // of it. Near a cell edge the two may pick neighbouring cells; both give the same code there
 // because no threshold lies within 2^-19 of a cell edge (checked on the host; the 4-bit float
 // has a threshold on a cell edge, 1/8, so it always takes the IEEE quotient).
-// The last CTA of kernel 1 rebuilds the exact mean from the bins (once).
+// The last CTA of kernel 1 rebuilds the exact mean from the bins (once): one warp forms the exact
+// 384-bit sum, one thread rounds the quotient.
 // Kernel 2 (1/64 of the data): each warp double-quantises one group of 256 block absmaxes.
 #include <mutex>
 #include <vector>
@@ -41,7 +42,8 @@ __device__ __forceinline__ uint32_t mag_max2(uint32_t u) {
     return max(u & 0x7fffu, (u >> 16) & 0x7fffu);
 }
 
-__device__ float mean_from_bins(const unsigned long long *bins, int64_t nb);
+__device__ float mean_from_sum(const uint64_t (&S)[6], int64_t nb);
+__device__ void bins_sum_warp(const unsigned long long *bins, int lane, uint64_t (&S)[6]);
 
 // The last CTA to finish (counted with an atomic, no waiting) rebuilds the exact mean from
 // the completed bins and stores it.
@@ -57,30 +59,36 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
-    const int sub = lane >> 3;  // which of the warp's 4 blocks
-    const int l8 = lane & 7;    // 8 weights of that block
+    const int sub = lane >> 2;  // which of the warp's 8 blocks
+    const int l4 = lane & 3;    // 16-byte chunks l4 and l4 + 4 of that block (8 weights each)
     const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     uint32_t cached_e = 0u, cached_sum = 0u;
 
-    // software-pipelined: the next pass's 16 bytes are requested before this pass is processed
-    auto load = [&](int64_t bb) {
-        return bb < nb ? ld_nc_v4(W + bb * 8 + l8) : make_uint4(0u, 0u, 0u, 0u);
+    // software-pipelined: the next pass's 32 bytes are requested before this pass is processed
+    auto load = [&](int64_t bb, uint4 &a, uint4 &bv) {
+        if (bb < nb) {
+            a = ld_nc_v4(W + bb * 8 + l4);
+            bv = ld_nc_v4(W + bb * 8 + 4 + l4);
+        } else {
+            a = bv = make_uint4(0u, 0u, 0u, 0u);
+        }
     };
-    uint4 v_next = load(warp_global * 4 + sub);
-    for (int64_t b0 = warp_global * 4; b0 < nb; b0 += nwarps * 4) {
+    uint4 na, nbv;
+    load(warp_global * 8 + sub, na, nbv);
+    for (int64_t b0 = warp_global * 8; b0 < nb; b0 += nwarps * 8) {
         const int64_t b = b0 + sub;
         const bool valid = b < nb;
-        const uint4 v = v_next;
-        v_next = load(b + nwarps * 4);
-        uint32_t m = max(max(mag_max2(v.x), mag_max2(v.y)), max(mag_max2(v.z), mag_max2(v.w)));
+        const uint4 va = na, vb = nbv;
+        load(b + nwarps * 8, na, nbv);
+        uint32_t m = max(max(max(mag_max2(va.x), mag_max2(va.y)), max(mag_max2(va.z), mag_max2(va.w))),
+                         max(max(mag_max2(vb.x), mag_max2(vb.y)), max(mag_max2(vb.z), mag_max2(vb.w))));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
         const float c = __uint_as_float(m << 16);  // block absmax, exact (a bf16 value)
-        uint32_t word = cells.zero_word;           // all-zero block: the code of 0 everywhere
+        uint32_t word_a = cells.zero_word, word_b = cells.zero_word;  // all-zero block: the code of 0
         if (c != 0.0f) {
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
             auto weight = [&](int i) {
                 return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
             };
@@ -98,27 +106,34 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
             // c is a bf16 value, so c >= 2^-126 exactly when its exponent field is non-zero
             const bool fast = fast_ok && (m >> 7) != 0u;
             const float r = __frcp_rn(c);
-            word = 0u;
+            word_a = word_b = 0u;
             bool redo = !fast;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 16; ++i) {
                 float dist;
                 const int code = code_of(__fmul_rn(weight(i), r), dist);
-                word |= static_cast<uint32_t>(code) << (4 * i);
+                if (i < 8)
+                    word_a |= static_cast<uint32_t>(code) << (4 * i);
+                else
+                    word_b |= static_cast<uint32_t>(code) << (4 * (i - 8));
                 redo |= fabsf(dist) <= 0x1p-21f;
             }
-            if (redo) {  // rare: all eight weights of this lane again, by the IEEE quotient
-                word = 0u;
-                for (int i = 0; i < 8; ++i) {
+            if (redo) {  // rare: all sixteen weights of this lane again, by the IEEE quotient
+                word_a = word_b = 0u;
+                for (int i = 0; i < 16; ++i) {
                     float dist;
                     const int code = code_of(__fdiv_rn(weight(i), c), dist);
-                    word |= static_cast<uint32_t>(code) << (4 * i);
+                    if (i < 8)
+                        word_a |= static_cast<uint32_t>(code) << (4 * i);
+                    else
+                        word_b |= static_cast<uint32_t>(code) << (4 * (i - 8));
                 }
             }
         }
         if (valid) {
-            codes[b * 8 + l8] = word;
-            if (l8 == 0) {
+            codes[b * 8 + l4] = word_a;
+            codes[b * 8 + 4 + l4] = word_b;
+            if (l4 == 0) {
                 cblk[b] = c;
                 const uint32_t e = m >> 7;
                 const uint32_t sig = (e == 0u) ? (m & 0x7fu) : (0x80u | (m & 0x7fu));
@@ -141,38 +156,63 @@ k_quant_blocks(const uint4 *__restrict__ W, int64_t nb, uint32_t *__restrict__ c
     __shared__ bool s_last;
     if (threadIdx.x == 0) s_last = atomicAdd(done, 1u) == gridDim.x - 1;
     __syncthreads();
-    if (s_last) {
+    if (s_last && mu_out) {
         __threadfence();
         __shared__ unsigned long long s_all[256];
         for (int i = threadIdx.x; i < 256; i += blockDim.x) s_all[i] = __ldcg(bins + i);
         __syncthreads();
-        if (threadIdx.x == 0) *mu_out = mean_from_bins(s_all, nb);
+        if (threadIdx.x < 32) {
+            uint64_t S[6];
+            bins_sum_warp(s_all, threadIdx.x, S);
+            if (threadIdx.x == 0) *mu_out = mean_from_sum(S, nb);
+        }
     }
 }
 
-// Exact mean of the block absmaxes from the exponent bins, rounded once to fp32.
-// bins[e] = sum of the 8-bit significands of the absmaxes with exponent field e;
-// such an absmax equals significand * 2^(p - 133) with p = max(e - 1, 0). Run by
-// one thread.
-__device__ float mean_from_bins(const unsigned long long *bins, int64_t nb) {
-    uint64_t S[6] = {0, 0, 0, 0, 0, 0};  // S * 2^-133 is the exact sum
-    for (int e = 0; e < 256; ++e) {
+// a += b on 384-bit integers (six 64-bit limbs, least significant first).
+__device__ __forceinline__ void add384(uint64_t (&a)[6], const uint64_t (&b)[6]) {
+    uint64_t carry = 0;
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+        const uint64_t t = a[i] + b[i];
+        const uint64_t c1 = t < b[i];
+        const uint64_t t2 = t + carry;
+        const uint64_t c2 = t2 < carry;
+        a[i] = t2;
+        carry = c1 + c2;
+    }
+}
+
+// S (every lane of a warp) = sum over e of bins[e] * 2^p(e), p(e) = max(e - 1, 0): lane l adds the
+// bins l, l + 32, ... into its own 384-bit sum (limb positions chosen by selects, so the limbs
+// stay in registers), then five butterfly steps add the lanes' sums. The exact sum times 2^-133
+// is the sum of the absmaxes.
+__device__ void bins_sum_warp(const unsigned long long *bins, int lane, uint64_t (&S)[6]) {
+#pragma unroll
+    for (int i = 0; i < 6; ++i) S[i] = 0;
+    for (int e = lane; e < 256; e += 32) {
         const uint64_t v = bins[e];
         if (v == 0) continue;
         const int p = e ? e - 1 : 0;
         const int li = p >> 6, sh = p & 63;
-        uint64_t add[2] = {v << sh, sh ? (v >> (64 - sh)) : 0ull};
-        uint64_t carry = 0;
-        for (int i = li; i < 6; ++i) {
-            const uint64_t a = (i - li < 2) ? add[i - li] : 0ull;
-            const uint64_t t = S[i] + a;
-            const uint64_t c1 = t < a;
-            const uint64_t t2 = t + carry;
-            const uint64_t c2 = t2 < carry;
-            S[i] = t2;
-            carry = c1 + c2;
-        }
+        const uint64_t lo = v << sh, hi = sh ? (v >> (64 - sh)) : 0ull;
+        uint64_t add[6];
+#pragma unroll
+        for (int i = 0; i < 6; ++i) add[i] = (i == li) ? lo : ((i == li + 1) ? hi : 0ull);
+        add384(S, add);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        uint64_t other[6];
+#pragma unroll
+        for (int i = 0; i < 6; ++i) other[i] = __shfl_xor_sync(0xffffffffu, S[i], o);
+        add384(S, other);
+    }
+}
+
+// Exact mean of the block absmaxes, rounded once to fp32, from their exact sum S * 2^-133
+// (bins_sum_warp). Run by one thread.
+__device__ float mean_from_sum(const uint64_t (&S)[6], int64_t nb) {
     int top = 5;
     while (top >= 0 && S[top] == 0) --top;
     if (top < 0 || nb <= 0) return 0.0f;
@@ -400,10 +440,9 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, int qtype, 
     if (nb == 0) return cudaSuccess;
     auto *bins = static_cast<unsigned long long *>(ws);
     auto *done = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + kBinsBytes);
-    // without double quantisation the absmaxes go straight to the output and the mean (unused)
-    // to the header
+    // without double quantisation the absmaxes go straight to the output and no mean is formed
     auto *cblk = absmax ? absmax : reinterpret_cast<float *>(static_cast<char *>(ws) + kHeaderBytes);
-    float *mu_out = absmax ? reinterpret_cast<float *>(static_cast<char *>(ws) + kBinsBytes + 128) : mu;
+    float *mu_out = absmax ? nullptr : mu;
     cudaError_t e = cudaMemsetAsync(bins, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return e;
     int sms = 148, occ = 4;
@@ -411,9 +450,9 @@ cudaError_t launch_quantize(const uint16_t *W, int64_t n, int64_t k, int qtype, 
     if (e != cudaSuccess) return e;
     e = resident_ctas(reinterpret_cast<const void *>(k_quant_blocks), kQuantThreads, 0, &occ);
     if (e != cudaSuccess) return e;
-    // 32 blocks per CTA per pass; exactly one wave of resident CTAs, never more than needed,
-    // and few enough passes per thread that the 32-bit smem bins cannot overflow.
-    int64_t grid = (nb + 31) / 32;
+    // 64 blocks per CTA per pass; exactly one wave of resident CTAs, never more than needed,
+    // and few enough blocks per CTA that the 32-bit smem bins cannot overflow.
+    int64_t grid = (nb + 63) / 64;
     grid = grid < static_cast<int64_t>(sms) * occ ? grid : static_cast<int64_t>(sms) * occ;
     const int64_t min_grid = (nb + (1ll << 22) - 1) >> 22;
     if (grid < min_grid) grid = min_grid;
