@@ -25,7 +25,7 @@ EXPORTED = ("qn_nf4_sizes", "qn_weight_sizes", "qn_quantize_workspace_size", "nf
             "qlora_workspace_size", "qlora_workspace_check", "qlora_linear_fwd", "qlora_linear_bwd_x",
             "qlora_merge_bf16", "qlora_lora_grads_workspace_size", "qlora_lora_grads", "qlora_linear_fwd_dropout",
             "qlora_linear_bwd_x_dropout", "qlora_lora_grads_dropout", "qn_status_string",
-            "qn_last_error", "qn_launch_count")
+            "qn_last_error", "qn_launch_count", "qn_selftest_wait_timeout")
 
 
 class QNError(RuntimeError):
@@ -77,6 +77,7 @@ def load(path: str | None = None):
         lib.nf4_quantize_static_ws.argtypes = [P, W, P]
         lib.qlora_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, sz]
         lib.qlora_workspace_check.argtypes = [P, P]
+        lib.qn_selftest_wait_timeout.argtypes = [P, ctypes.c_size_t, P]
         lib.qlora_linear_fwd.argtypes = [W, P, i64, P, P, ctypes.c_int, ctypes.c_float, P, P, ctypes.c_size_t, P]
         lib.qlora_linear_bwd_x.argtypes = lib.qlora_linear_fwd.argtypes
         lib.qlora_merge_bf16.argtypes = [W, P, P, ctypes.c_int, ctypes.c_float, P, P]
@@ -162,6 +163,15 @@ def workspace_check(ws: torch.Tensor, stream=None):
     """Raise QNError(QN_ETIMEOUT) if a kernel that used `ws` gave up a bounded wait since the last
     check (the error word is then cleared); synchronises the stream."""
     _check(load().qlora_workspace_check(_ptr(ws), _stream(stream)), "qlora_workspace_check")
+
+
+def selftest_wait_timeout(ws: torch.Tensor, stream=None):
+    """Enqueue the library's bounded-wait self-test on a zeroed workspace: its wait runs out and
+    sets the error word (see qn_selftest_wait_timeout in the header)."""
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check(load().qn_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "qn_selftest_wait_timeout")
 
 
 def _workspace(ws: torch.Tensor | None, need: int, device) -> tuple[torch.Tensor, int]:

@@ -331,6 +331,11 @@ qn_status qlora_workspace_check(void *ws, void *stream) {
                 word == 2 ? "dynamic shared memory not 1024-byte aligned" : "a bounded wait ran out");
 }
 
+qn_status qn_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < 256) return fail(QN_EWORKSPACE, "the self-test needs a zeroed workspace of 256 bytes");
+    return cuda_status(launch_wait_timeout_selftest(ws, static_cast<cudaStream_t>(stream)), "qn_selftest_wait_timeout");
+}
+
 qn_status qlora_linear_fwd(const qn_nf4_weight *w, const void *x, int64_t M, const void *A, const void *B, int r,
                            float alpha, void *h, void *ws, size_t ws_bytes, void *stream) {
     return qlora_linear_fwd_dropout(w, x, M, A, B, r, alpha, nullptr, h, ws, ws_bytes, stream);

@@ -112,4 +112,8 @@ cudaError_t launch_gemm_fwd(const WeightView &w, const uint16_t *x, int64_t M, c
 cudaError_t launch_gemm_bwd(const WeightView &w, const uint16_t *gh, int64_t M, const uint16_t *A, const uint16_t *B,
                             int r, float s, uint16_t *gx, void *ws, cudaStream_t st);
 
+// One kernel whose bounded wait on a workspace word that nothing sets runs out and records the
+// timeout in the workspace error word (the shared error path, checked by a test).
+cudaError_t launch_wait_timeout_selftest(void *ws, cudaStream_t st);
+
 }  // namespace qn

@@ -222,6 +222,15 @@ qn_status qlora_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r, si
  * Errors: QN_EINVAL (null ws), QN_ECUDA, QN_ETIMEOUT. */
 qn_status qlora_workspace_check(void *ws, void *stream);
 
+/* qn_selftest_wait_timeout -- a check of the error path above: enqueues one kernel that waits, with
+ * the same bounded wait the library's kernels use, on a word of the (zeroed) linear workspace that
+ * nothing ever sets. The wait runs out after its poll limit (about a second) and the kernel
+ * records the timeout in the error word, so a following qlora_workspace_check returns
+ * QN_ETIMEOUT and clears it. Nothing faults or hangs. No counterpart on the pages: it exists to
+ * test the failure path of the hot-path kernels without breaking them.
+ * ws: a linear workspace of at least 256 bytes, zeroed. Errors: QN_EWORKSPACE, QN_ECUDA. */
+qn_status qn_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream);
+
 /* qlora_linear_fwd -- h = dequant(W) x + (alpha/r) B (A x), per token row:
  *   h[m, n] = sum_k W'[n,k] x[m,k] + s * sum_j B[n,j] sum_k A[j,k] x[m,k].
  *   x : M x k_in bf16 (tokens x features); A : r x k_in bf16; B : n_out x r bf16;

@@ -212,6 +212,25 @@ def test_error_word_stays_clear(oracle, M):
     qb.workspace_check(ws)
 
 
+def test_bounded_wait_runs_out_and_is_reported():
+    # The shared failure path of the kernels, exercised without a fault: a kernel's bounded wait on a
+    # workspace word that nothing sets runs out, the kernel records the timeout in the error word,
+    # the check reports QN_ETIMEOUT and clears it, and the device stays usable.
+    ws = qb.new_workspace(4096)
+    qb.selftest_wait_timeout(ws)
+    with pytest.raises(qb.QNError) as e:
+        qb.workspace_check(ws)
+    assert e.value.status == qb.QN_ETIMEOUT
+    qb.workspace_check(ws)  # cleared
+    W = synth.normal_bf16((256, 256), 0.02, 3, DEV)
+    w = qb.nf4_quantize(W)
+    x = synth.normal_bf16((4, 256), 1.0, 4, DEV)
+    h = qb.qlora_linear_fwd(w, x, None, None, 0.0, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(h.float()).all()
+    qb.workspace_check(ws)
+
+
 def test_error_word_is_reported_and_cleared():
     # a set error word (what a kernel writes when a bounded wait runs out) is reported as
     # QN_ETIMEOUT by the check, which clears it
