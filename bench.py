@@ -354,8 +354,12 @@ def detail_measurements(hbm_peak, tc_peak, only=None):
         w = qb.nf4_quantize(W)
         ws = torch.empty(qb.quantize_workspace_size(n, k), dtype=torch.uint8, device=dev)
         deq = torch.empty_like(W)
+        torch.cuda.nvtx.range_push(f"quantize_{n}x{k}")
         tq = time_fn(lambda: qb.nf4_quantize(W, w, ws), flush=flush)
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.nvtx.range_push(f"dequant_{n}x{k}")
         td = time_fn(lambda: qb.nf4_dequantize(w, deq), flush=flush)
+        torch.cuda.nvtx.range_pop()
         by = 2 * n * k + weight_bytes(n, k)
         out[f"quantize_{n}x{k}"] = {"us": round(tq * 1e6, 2), "GB/s": round(by / tq / 1e9, 1),
                                     "hbm_frac": round(by / tq / 1e9 / hbm_peak, 3)}
@@ -379,8 +383,13 @@ def detail_measurements(hbm_peak, tc_peak, only=None):
         h = torch.empty(M, n, dtype=torch.bfloat16, device=dev)
         gx = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
         ws = qb.new_workspace(qb.linear_workspace_size(M, n, k, r))  # zeroed once, as the header asks
+        # NVTX ranges name the case, so a profiler can select one (ncu --nvtx --nvtx-include "<name>/")
+        torch.cuda.nvtx.range_push(f"{tag}_{n}x{k}_M{M}_fwd")
         tf = time_fn(lambda: qb.qlora_linear_fwd(w, x, A, B, alpha, out=h, workspace=ws), reps=5, flush=flush)
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.nvtx.range_push(f"{tag}_{n}x{k}_M{M}_bwd")
         tb = time_fn(lambda: qb.qlora_linear_bwd_x(w, g, A, B, alpha, out=gx, workspace=ws), reps=5, flush=flush)
+        torch.cuda.nvtx.range_pop()
         fl = linear_flops(n, k, M, r)
         by = fwd_bytes(n, k, M, r)
         rec = {"fwd_us": round(tf * 1e6, 2), "bwd_us": round(tb * 1e6, 2),
