@@ -557,37 +557,56 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 
     // ---------------------------------------------------------------------- reduction
     __syncthreads();
-    const uint32_t red = s_base + p.post_off;  // [3][4 blocks][4 f][32 lanes][NG][4] f32, in the idle ring
-    if (warp > 0 && rg > 0) {
+    // Sub-tile f of block kg is summed, given its adapter term and stored or pushed by warp
+    // (kg, rg = f), so that this work spreads over all the consumer warps.
+    const uint32_t red = s_base + p.post_off;  // [4 rg][4 blocks][4 f][32 lanes][NG][4] f32, in the idle ring
+    if (warp > 0) {
 #pragma unroll
-        for (int f = 0; f < 4; ++f)
+        for (int f = 0; f < 4; ++f) {
+            if (f == rg) continue;
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) {
-                const uint32_t o = red + static_cast<uint32_t>(((((rg - 1) * 4 + kg) * 4 + f) * 32 + lane) * NG + tg) * 16;
+                const uint32_t o = red + static_cast<uint32_t>((((rg * 4 + kg) * 4 + f) * 32 + lane) * NG + tg) * 16;
                 asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(o), "f"(acc[f][tg][0]), "f"(acc[f][tg][1]),
                              "f"(acc[f][tg][2]), "f"(acc[f][tg][3])
                              : "memory");
             }
+        }
     }
     __syncthreads();
     const bool run_ok = !*bb.abort_flag;
-    // features of sub-tile f: fragment row g -> 64 kg + 8 g + 2 f, row g + 8 -> 64 kg + 8 g + 2 f + 1
-    if (warp > 0 && rg == 0) {
+    const int fo = rg;  // the sub-tile this warp sums
+    // features of sub-tile fo: fragment row g -> 64 kg + 8 g + 2 fo, row g + 8 -> 64 kg + 8 g + 2 fo + 1
+    float sum[NG][4];
+    if (warp > 0) {
+        float own[NG][4];
 #pragma unroll
-        for (int q = 0; q < 3; ++q)
+        for (int f = 0; f < 4; ++f)
+            if (f == fo)
 #pragma unroll
-            for (int f = 0; f < 4; ++f)
+                for (int tg = 0; tg < NG; ++tg)
 #pragma unroll
-                for (int tg = 0; tg < NG; ++tg) {
-                    const uint4 v = lds128(red + static_cast<uint32_t>((((q * 4 + kg) * 4 + f) * 32 + lane) * NG + tg) * 16);
-                    acc[f][tg][0] += __uint_as_float(v.x);
-                    acc[f][tg][1] += __uint_as_float(v.y);
-                    acc[f][tg][2] += __uint_as_float(v.z);
-                    acc[f][tg][3] += __uint_as_float(v.w);
+                    for (int e = 0; e < 4; ++e) own[tg][e] = acc[f][tg][e];
+        // the four row-group warps' partials in rg order
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                float v[4];
+                if (q == rg) {
+                    v[0] = own[tg][0], v[1] = own[tg][1], v[2] = own[tg][2], v[3] = own[tg][3];
+                } else {
+                    const uint4 w4 = lds128(red + static_cast<uint32_t>((((q * 4 + kg) * 4 + fo) * 32 + lane) * NG + tg) * 16);
+                    v[0] = __uint_as_float(w4.x), v[1] = __uint_as_float(w4.y);
+                    v[2] = __uint_as_float(w4.z), v[3] = __uint_as_float(w4.w);
                 }
-        // adapter term of block kg (this CTA's when kg = crank mod C): A^T u from the staged tile
-        // [rpad ranks][64 features] (128-byte swizzle: chunk c of rank row j at c ^ (j & 7)); under
-        // dropout only the elements whose input survived the forward's mask receive it
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sum[tg][e] = q == 0 ? v[e] : sum[tg][e] + v[e];
+            }
+        // adapter term of block kg (this CTA's when kg = crank mod C), sub-tile fo: A^T u from the
+        // staged tile [rpad ranks][64 features] (128-byte swizzle: chunk c of rank row j at
+        // c ^ (j & 7)); under dropout only the elements whose input survived the forward's mask
+        // receive it
         if (p.r > 0 && kg % C == crank) {
             const uint32_t ab = at + static_cast<uint32_t>((kg / C) * p.rpad * 128);
             auto a_el = [&](int j, int feat) -> uint32_t {  // A[j][64 kg + feat] (bf16 bits)
@@ -600,74 +619,67 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 if (jj >= p.rpad) return 0u;
                 return a_el(jj, feat) | (a_el(jj + 1, feat) << 16);
             };
+            const int fa = 8 * g + 2 * fo, fb = fa + 1;
+            float ad[NG][4];
 #pragma unroll
-            for (int f = 0; f < 4; ++f) {
-                const int fa = 8 * g + 2 * f, fb = fa + 1;
-                float ad[NG][4];
-#pragma unroll
-                for (int tg = 0; tg < NG; ++tg) ad[tg][0] = ad[tg][1] = ad[tg][2] = ad[tg][3] = 0.0f;
-                for (int kc = 0; kc < p.rk16 / 16; ++kc) {
-                    const int j = 16 * kc + 2 * t;
-                    const uint32_t a0 = pair(j, fa), a1 = pair(j, fb), a2 = pair(j + 8, fa), a3 = pair(j + 8, fb);
-#pragma unroll
-                    for (int tg = 0; tg < NG; ++tg) {
-                        const uint32_t ur = ut + static_cast<uint32_t>((tg * 8 + g) * p.rk16 + j) * 2u;
-                        mma_16816(ad[tg], a0, a1, a2, a3, lds32(ur), lds32(ur + 16));
-                    }
-                }
+            for (int tg = 0; tg < NG; ++tg) ad[tg][0] = ad[tg][1] = ad[tg][2] = ad[tg][3] = 0.0f;
+            for (int kc = 0; kc < p.rk16 / 16; ++kc) {
+                const int j = 16 * kc + 2 * t;
+                const uint32_t a0 = pair(j, fa), a1 = pair(j, fb), a2 = pair(j + 8, fa), a3 = pair(j + 8, fb);
 #pragma unroll
                 for (int tg = 0; tg < NG; ++tg) {
-                    // fragment element e: feature 64 kg + fa + (e >> 1), token tg 8 + 2 t + (e & 1)
-                    uint32_t keep = 0xfu;
-                    if (p.drop.thr != 0u) {
-                        const int64_t feat = f0 + 64 * kg + fa;
-                        const int tok = tg * 8 + 2 * t;
-                        const uint32_t k0 =
-                            dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(tok * p.k + feat), 2);
-                        const uint32_t k1 = dropout_keep_bits(
-                            p.drop, p.drop.offset + static_cast<uint64_t>((tok + 1) * p.k + feat), 2);
-                        // e = 0: (fa, tok), 1: (fa, tok + 1), 2: (fb, tok), 3: (fb, tok + 1)
-                        keep = (k0 & 1u) | ((k1 & 1u) << 1) | ((k0 & 2u) << 1) | ((k1 & 2u) << 2);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (keep & (1u << e)) acc[f][tg][e] += ad[tg][e];
+                    const uint32_t ur = ut + static_cast<uint32_t>((tg * 8 + g) * p.rk16 + j) * 2u;
+                    mma_16816(ad[tg], a0, a1, a2, a3, lds32(ur), lds32(ur + 16));
                 }
+            }
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                // fragment element e: feature 64 kg + fa + (e >> 1), token tg 8 + 2 t + (e & 1)
+                uint32_t keep = 0xfu;
+                if (p.drop.thr != 0u) {
+                    const int64_t feat = f0 + 64 * kg + fa;
+                    const int tok = tg * 8 + 2 * t;
+                    const uint32_t k0 =
+                        dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>(tok * p.k + feat), 2);
+                    const uint32_t k1 =
+                        dropout_keep_bits(p.drop, p.drop.offset + static_cast<uint64_t>((tok + 1) * p.k + feat), 2);
+                    // e = 0: (fa, tok), 1: (fa, tok + 1), 2: (fb, tok), 3: (fb, tok + 1)
+                    keep = (k0 & 1u) | ((k1 & 1u) << 1) | ((k0 & 2u) << 1) | ((k1 & 2u) << 2);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (keep & (1u << e)) sum[tg][e] += ad[tg][e];
             }
         }
         if (C == 1 && run_ok) {
 #pragma unroll
-            for (int f = 0; f < 4; ++f)
+            for (int tg = 0; tg < NG; ++tg)
 #pragma unroll
-                for (int tg = 0; tg < NG; ++tg)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int64_t feat = f0 + 64 * kg + 8 * g + 2 * f + (e >> 1);
-                        const int tok = tg * 8 + 2 * t + (e & 1);
-                        if (feat < p.k && tok < p.M)
-                            p.gx[static_cast<int64_t>(tok) * p.k + feat] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(acc[f][tg][e]));
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const int64_t feat = f0 + 64 * kg + 8 * g + 2 * fo + (e >> 1);
+                    const int tok = tg * 8 + 2 * t + (e & 1);
+                    if (feat < p.k && tok < p.M)
+                        p.gx[static_cast<int64_t>(tok) * p.k + feat] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(sum[tg][e]));
+                }
         }
     }
     if (C > 1) {
         cluster_wait();  // phase 1: every CTA of the cluster runs (its barriers are initialised)
-        if (warp > 0 && rg == 0) {
+        if (warp > 0) {
             const uint32_t recv = s_base + p.recv_off;
 #pragma unroll
-            for (int f = 0; f < 4; ++f)
+            for (int hh = 0; hh < 2; ++hh) {
+                const int fl = 64 * kg + 8 * g + 2 * fo + hh;  // feature within the chunk
+                const int owner = (fl * C + C - 1) / kChunkFeat;
+                const int rr = fl - kChunkFeat * owner / C;
+                const uint32_t dst = mapa(recv + static_cast<uint32_t>(((crank * nfmax + rr) * MP + 2 * t) * 4),
+                                          static_cast<uint32_t>(owner));
+                const uint32_t bar = mapa(saddr(bb.recv), static_cast<uint32_t>(owner));
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int fl = 64 * kg + 8 * g + 2 * f + hh;  // feature within the chunk
-                    const int owner = (fl * C + C - 1) / kChunkFeat;
-                    const int rr = fl - kChunkFeat * owner / C;
-                    const uint32_t dst = mapa(recv + static_cast<uint32_t>(((crank * nfmax + rr) * MP + 2 * t) * 4),
-                                              static_cast<uint32_t>(owner));
-                    const uint32_t bar = mapa(saddr(bb.recv), static_cast<uint32_t>(owner));
-#pragma unroll
-                    for (int tg = 0; tg < NG; ++tg)
-                        st_async_v2(dst + 32u * tg, acc[f][tg][2 * hh], acc[f][tg][2 * hh + 1], bar);
-                }
+                for (int tg = 0; tg < NG; ++tg)
+                    st_async_v2(dst + 32u * tg, sum[tg][2 * hh], sum[tg][2 * hh + 1], bar);
+            }
         }
         const bool ok = mbar_wait(bb.recv, 0);
         if (!ok && threadIdx.x == 0) record_error(p.err, kErrTimeout);
@@ -677,9 +689,9 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 const int rr = it % nf, tok = it / nf;
                 const int64_t feat = f0 + f_lo + rr;
                 if (feat >= p.k) continue;
-                float sum = 0.0f;
-                for (int src = 0; src < C; ++src) sum += recvf[(src * nfmax + rr) * MP + tok];
-                p.gx[static_cast<int64_t>(tok) * p.k + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+                float tot = 0.0f;
+                for (int src = 0; src < C; ++src) tot += recvf[(src * nfmax + rr) * MP + tok];
+                p.gx[static_cast<int64_t>(tok) * p.k + feat] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
             }
         }
     }
@@ -763,7 +775,7 @@ bool layout(BwdArgs &a, int MP) {
     const uint32_t utb = a.r > 0 ? align_up(static_cast<uint32_t>(MP * a.rk16 * 2), 128) : 0u;
     const int nablk_max = a.r > 0 ? (4 + a.C - 1) / a.C : 0;
     const uint32_t atb = static_cast<uint32_t>(nablk_max * a.rpad * 128);
-    const uint32_t post_chunk = 3 * 4 * 4 * 32 * 16 * (MP / 8);
+    const uint32_t post_chunk = 4 * 4 * 4 * 32 * 16 * (MP / 8);
     const uint32_t post_adapter = 64 * 32 * 16;
     const uint32_t post = post_chunk > post_adapter ? post_chunk : post_adapter;
     const uint32_t recv_chunk = a.C > 1 ? static_cast<uint32_t>(a.C * ((kChunkFeat + a.C - 1) / a.C) * MP * 4) : 0u;

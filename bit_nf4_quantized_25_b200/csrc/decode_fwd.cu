@@ -337,11 +337,14 @@ __device__ __forceinline__ void adapter_body(const CUtensorMap *tm_xp, const CUt
 }
 
 // ------------------------------------------------------------------------------ chunk clusters
-template <int NG, bool kFixedBase>
+// kMT: the m-tiles of every consumer warp (m = 4 kMT), fixed at compile time so that the tile
+// loop has no branches (2: chunks of 128 rows); 0: up to MW, each checked against m.
+template <int NG, bool kFixedBase, int kMT>
 __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CUtensorMap *tm_x, const FwdArgs &p,
                                            uint8_t *smem) {
     constexpr int MP = 8 * NG;  // padded tokens
     constexpr int MW = 4;  // m-tiles per warp at most (m <= 4 MW)
+    constexpr int MWL = kMT > 0 ? kMT : MW;  // m-tiles the stage loop visits
 #ifdef QN_TIMELINE
     const long long tl_c0 = clock64();
 #endif
@@ -697,7 +700,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // rows the quad needs and share them with shuffles (MW = 4: a second pass for m-tiles
         // rg + 8, rg + 12). c_q: staged FP8 code of block kg of the first stage; c_e: its block
         // index relative to the first staged group scale (its scale is staged at c_e >> 8).
-        constexpr int NP = (MW + 1) / 2;
+        constexpr int NP = (MWL + 1) / 2;
         bool c_ok[NP];
         uint32_t c_q[NP];
         int64_t c_e[NP];
@@ -757,13 +760,58 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             // codes of row (16 mt + g), bytes 32 kg + 8 t .. + 8: 16-byte chunk 2 kg + (t >> 1) of
             // the 128-byte row, stored at chunk index ^ (row & 7) = ^ g
             const uint32_t cchunk = static_cast<uint32_t>(((2 * kg + (t >> 1)) ^ g) << 4) + 8u * (t & 1);
+            if constexpr (kMT == 2 && NG == 1) {
+                // both m-tiles of the warp at once: their table loads issue back to back and
+                // their two MMA chains interleave (constants: quad lanes 0, 1 for m-tile rg,
+                // 2, 3 for m-tile rg + 4)
+                const float cA0 = __shfl_sync(0xffffffffu, cmine[0], (lane & ~3));
+                const float cB0 = __shfl_sync(0xffffffffu, cmine[0], (lane & ~3) | 1);
+                const float cA1 = __shfl_sync(0xffffffffu, cmine[0], (lane & ~3) | 2);
+                const float cB1 = __shfl_sync(0xffffffffu, cmine[0], (lane & ~3) | 3);
+                const uint32_t cr0 = sl + static_cast<uint32_t>(16 * rg + g) * 128u + cchunk;
+                const uint32_t cr1 = cr0 + 64u * 128u;
+                const uint2 ca0 = lds64(cr0), cb0 = lds64(cr0 + 8 * 128);
+                const uint2 ca1 = lds64(cr1), cb1 = lds64(cr1 + 8 * 128);
+                uint32_t af0[4][4], af1[4][4];
 #pragma unroll
-            for (int i = 0; i < MW; ++i) {
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int i0 = (2 * kk) & 3;
+                    const uint32_t wa0 = kk < 2 ? ca0.x : ca0.y, wb0 = kk < 2 ? cb0.x : cb0.y;
+                    const uint32_t wa1 = kk < 2 ? ca1.x : ca1.y, wb1 = kk < 2 ? cb1.x : cb1.y;
+                    af0[kk][0] = lut_pair<kFixedBase>(lut_base, wa0, lane_op, i0);
+                    af0[kk][2] = lut_pair<kFixedBase>(lut_base, wa0, lane_op, i0 + 1);
+                    af0[kk][1] = lut_pair<kFixedBase>(lut_base, wb0, lane_op, i0);
+                    af0[kk][3] = lut_pair<kFixedBase>(lut_base, wb0, lane_op, i0 + 1);
+                    af1[kk][0] = lut_pair<kFixedBase>(lut_base, wa1, lane_op, i0);
+                    af1[kk][2] = lut_pair<kFixedBase>(lut_base, wa1, lane_op, i0 + 1);
+                    af1[kk][1] = lut_pair<kFixedBase>(lut_base, wb1, lane_op, i0);
+                    af1[kk][3] = lut_pair<kFixedBase>(lut_base, wb1, lane_op, i0 + 1);
+                }
+                float d0[4], d1[4];
+                mma_16816_z(d0, af0[0][0], af0[0][1], af0[0][2], af0[0][3], x0[0].x, x0[0].y);
+                mma_16816_z(d1, af1[0][0], af1[0][1], af1[0][2], af1[0][3], x0[0].x, x0[0].y);
+                mma_16816(d0, af0[1][0], af0[1][1], af0[1][2], af0[1][3], x0[0].z, x0[0].w);
+                mma_16816(d1, af1[1][0], af1[1][1], af1[1][2], af1[1][3], x0[0].z, x0[0].w);
+                mma_16816(d0, af0[2][0], af0[2][1], af0[2][2], af0[2][3], x1[0].x, x1[0].y);
+                mma_16816(d1, af1[2][0], af1[2][1], af1[2][2], af1[2][3], x1[0].x, x1[0].y);
+                mma_16816(d0, af0[3][0], af0[3][1], af0[3][2], af0[3][3], x1[0].z, x1[0].w);
+                mma_16816(d1, af1[3][0], af1[3][1], af1[3][2], af1[3][3], x1[0].z, x1[0].w);
+                acc[0][0][0] = __fmaf_rn(cA0, d0[0], acc[0][0][0]);
+                acc[0][0][1] = __fmaf_rn(cA0, d0[1], acc[0][0][1]);
+                acc[0][0][2] = __fmaf_rn(cB0, d0[2], acc[0][0][2]);
+                acc[0][0][3] = __fmaf_rn(cB0, d0[3], acc[0][0][3]);
+                acc[1][0][0] = __fmaf_rn(cA1, d1[0], acc[1][0][0]);
+                acc[1][0][1] = __fmaf_rn(cA1, d1[1], acc[1][0][1]);
+                acc[1][0][2] = __fmaf_rn(cB1, d1[2], acc[1][0][2]);
+                acc[1][0][3] = __fmaf_rn(cB1, d1[3], acc[1][0][3]);
+            } else
+#pragma unroll
+            for (int i = 0; i < MWL; ++i) {
                 const int mt = rg + 4 * i;
                 // constants of m-tile i: rows g and g + 8, held by quad lanes 2 (i & 1) and 2 (i & 1) + 1
                 const float cA = __shfl_sync(0xffffffffu, cmine[i >> 1], (lane & ~3) | (2 * (i & 1)));
                 const float cB = __shfl_sync(0xffffffffu, cmine[i >> 1], (lane & ~3) | (2 * (i & 1) + 1));
-                if (mt < p.m) {
+                if (kMT > 0 || mt < p.m) {
                     const uint32_t cr = sl + static_cast<uint32_t>(16 * mt + g) * 128u + cchunk;
                     const uint2 ca = lds64(cr), cb = lds64(cr + 8 * 128);
                     uint32_t af[4][4];
@@ -801,7 +849,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     // every box has landed): its space holds the exchange buffer of the four block-warps. The
     // consumers sum the block-warps of each m-tile in a fixed order (kg = 0, 1, 2, 3).
     QN_TL(5, threadIdx.x == 32);
-    const uint32_t red = s_base + p.post_off;  // [3][16 m-tiles][32 lanes][NG*4] f32
+    // [kg][m m-tiles][32 lanes][NG*4] f32 (kg 1..3 in slots 0..2 when C == 1, kg 0..3 otherwise)
+    const uint32_t red = s_base + p.post_off;
     auto store_partials = [&]() {
 #pragma unroll
         for (int i = 0; i < MW; ++i) {
@@ -809,7 +858,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
             if (mt < p.m) {
 #pragma unroll
                 for (int tg = 0; tg < NG; ++tg) {
-                    const uint32_t o = red + static_cast<uint32_t>((((kg - 1) * kMaxM + mt) * 32 + lane) * NG + tg) * 16;
+                    const uint32_t o = red + static_cast<uint32_t>((((kg - 1) * p.m + mt) * 32 + lane) * NG + tg) * 16;
                     asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(o), "f"(acc[i][tg][0]),
                                  "f"(acc[i][tg][1]), "f"(acc[i][tg][2]), "f"(acc[i][tg][3])
                                  : "memory");
@@ -823,7 +872,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         for (int q = 0; q < 3; ++q) {
 #pragma unroll
             for (int tg = 0; tg < NG; ++tg) {
-                const uint4 v = lds128(red + static_cast<uint32_t>(((q * kMaxM + mt) * 32 + lane) * NG + tg) * 16);
+                const uint4 v = lds128(red + static_cast<uint32_t>(((q * p.m + mt) * 32 + lane) * NG + tg) * 16);
                 acc[i][tg][0] += __uint_as_float(v.x);
                 acc[i][tg][1] += __uint_as_float(v.y);
                 acc[i][tg][2] += __uint_as_float(v.z);
@@ -882,39 +931,70 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         // Cluster: the consumers reduce among themselves and push each row's partial sums (all MP
         // token columns) to the row's owner [src][row][MP] f32 right away; the owner adds B t while
         // it sums the C partials, so t from the adapter cluster is needed only there.
+        // M-tile rg + 4 i is summed and pushed by warp (kg = i, rg), so that the sums and the
+        // pushes of the chunk's m-tiles spread over all the consumer warps.
         named_sync(2, kConsumers * 32);  // every consumer has left its loop: the ring is idle
         QN_TL(6, threadIdx.x == 32);
-        if (kg > 0) store_partials();
+#pragma unroll
+        for (int i = 0; i < MW; ++i) {
+            const int mt = rg + 4 * i;
+            if (i == kg || mt >= p.m) continue;
+#pragma unroll
+            for (int tg = 0; tg < NG; ++tg) {
+                const uint32_t o = red + static_cast<uint32_t>(((kg * p.m + mt) * 32 + lane) * NG + tg) * 16;
+                asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(o), "f"(acc[i][tg][0]), "f"(acc[i][tg][1]),
+                             "f"(acc[i][tg][2]), "f"(acc[i][tg][3])
+                             : "memory");
+            }
+        }
         named_sync(3, kConsumers * 32);
         QN_TL(9, threadIdx.x == 32);
-        if (kg == 0) {
+        const int mo = rg + 4 * kg;  // the m-tile this warp sums
+        float own[NG][4], sum[NG][4];
 #pragma unroll
-            for (int i = 0; i < MW; ++i)
-                if (rg + 4 * i < p.m) sum_partials(i);
-            QN_TL(10, threadIdx.x == 32);
+        for (int i = 0; i < MW; ++i)
+            if (i == kg)
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) own[tg][e] = acc[i][tg][e];
+        if (mo < p.m) {
+            // the four block-warps' partials in kg order
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int tg = 0; tg < NG; ++tg) {
+                    float v[4];
+                    if (q == kg) {
+                        v[0] = own[tg][0], v[1] = own[tg][1], v[2] = own[tg][2], v[3] = own[tg][3];
+                    } else {
+                        const uint4 w4 =
+                            lds128(red + static_cast<uint32_t>(((q * p.m + mo) * 32 + lane) * NG + tg) * 16);
+                        v[0] = __uint_as_float(w4.x), v[1] = __uint_as_float(w4.y);
+                        v[2] = __uint_as_float(w4.z), v[3] = __uint_as_float(w4.w);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sum[tg][e] = q == 0 ? v[e] : sum[tg][e] + v[e];
+                }
         }
+        QN_TL(10, threadIdx.x == 32);
         cluster_wait();  // phase 1: every CTA of the cluster runs (its barriers are initialised)
-        if (kg == 0) {
+        if (mo < p.m) {
             const uint32_t recv = s_base + p.recv_off;
 #pragma unroll
-            for (int i = 0; i < MW; ++i) {
-                const int mt = rg + 4 * i;
-                if (mt >= p.m) continue;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int rl = 16 * mo + g + 8 * hh;
+                const int owner = (rl * C + C - 1) / p.R;
+                const int rr = rl - p.R * owner / C;
+                const uint32_t dst = mapa(recv + static_cast<uint32_t>(((crank * nrmax + rr) * MP + 2 * t) * 4),
+                                          static_cast<uint32_t>(owner));
+                const uint32_t bar = mapa(saddr(bb.recv), static_cast<uint32_t>(owner));
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int rl = 16 * mt + g + 8 * hh;
-                    const int owner = (rl * C + C - 1) / p.R;
-                    const int rr = rl - p.R * owner / C;
-                    const uint32_t dst = mapa(recv + static_cast<uint32_t>(((crank * nrmax + rr) * MP + 2 * t) * 4),
-                                              static_cast<uint32_t>(owner));
-                    const uint32_t bar = mapa(saddr(bb.recv), static_cast<uint32_t>(owner));
-#pragma unroll
-                    for (int tg = 0; tg < NG; ++tg)
-                        st_async_v2(dst + 32u * tg, acc[i][tg][2 * hh], acc[i][tg][2 * hh + 1], bar);
-                }
+                for (int tg = 0; tg < NG; ++tg)
+                    st_async_v2(dst + 32u * tg, sum[tg][2 * hh], sum[tg][2 * hh + 1], bar);
             }
-            QN_TL(11, threadIdx.x == 32);
         }
+        QN_TL(11, threadIdx.x == 32);
         // rows [r_lo, r_hi): the C partials in rank order, plus B t
         bool ok = mbar_wait(bb.recv, 0);
         if (ok && !mbar_wait(bb.tready, 0)) ok = false;
@@ -926,10 +1006,10 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                 const int rr = it % nr, tok = it / nr;
                 const int64_t row = row0 + r_lo + rr;
                 if (row >= nrow) continue;
-                float sum = 0.0f;
-                for (int src = 0; src < C; ++src) sum += recvf[(src * nrmax + rr) * MP + tok];
-                if (p.r > 0) sum += reinterpret_cast<const float *>(smem + p.bt_off)[rr * MP + tok];
-                p.h[static_cast<int64_t>(tok) * p.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+                float tot = 0.0f;
+                for (int src = 0; src < C; ++src) tot += recvf[(src * nrmax + rr) * MP + tok];
+                if (p.r > 0) tot += reinterpret_cast<const float *>(smem + p.bt_off)[rr * MP + tok];
+                p.h[static_cast<int64_t>(tok) * p.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(tot));
             }
         }
         QN_TL(20, threadIdx.x == 32);
@@ -945,7 +1025,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
 #endif
 }
 
-template <int NG>
+// kMT: 2 for chunks of 128 rows (m = 8), whose tile loop is specialised; 0 for every other m.
+template <int NG, int kMT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_decode_fwd(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
              const __grid_constant__ CUtensorMap tm_xp, const __grid_constant__ CUtensorMap tm_a, const FwdArgs p) {
@@ -959,9 +1040,9 @@ k_decode_fwd(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant
     if (p.r > 0 && blockIdx.y == 0) {
         adapter_body<NG>(&tm_xp, &tm_a, p, smem);
     } else if ((saddr(smem) & 0x00ffffffu) == kDynSmemBase) {
-        chunk_body<NG, true>(&tm_codes, &tm_x, p, smem);
+        chunk_body<NG, true, kMT>(&tm_codes, &tm_x, p, smem);
     } else {
-        chunk_body<NG, false>(&tm_codes, &tm_x, p, smem);
+        chunk_body<NG, false, kMT>(&tm_codes, &tm_x, p, smem);
     }
 }
 
@@ -1045,7 +1126,7 @@ bool layout_mode(FwdArgs &a, int MP, bool x_once) {
     // fragment rows fall on distinct bank groups
     a.bs_stride = static_cast<uint32_t>(2 * a.rk16 + 16);
     const uint32_t bsb = a.r > 0 ? align_up(static_cast<uint32_t>((a.R + a.C - 1) / a.C) * a.bs_stride, 128) : 0u;
-    const uint32_t post_chunk = 3 * kMaxM * 32 * 16 * (MP / 8);
+    const uint32_t post_chunk = static_cast<uint32_t>((a.C > 1 ? 4 : 3) * a.m * 32 * 16 * (MP / 8));
     const uint32_t post_adapter = kConsumers * 32 * 16;
     const uint32_t post = post_chunk > post_adapter ? post_chunk : post_adapter;
     const uint32_t recv_chunk = a.C > 1 ? static_cast<uint32_t>(a.C * ((a.R + a.C - 1) / a.C) * MP * 4) : 0u;
@@ -1114,13 +1195,19 @@ double cta_bytes(const FwdArgs &a) {
     return chunk > adapter ? chunk : adapter;
 }
 
+// The kernel that runs chunks of m m-tiles.
+template <int NG>
+const void *fwd_kernel(int m) {
+    return m == 8 ? reinterpret_cast<const void *>(k_decode_fwd<NG, 2>)
+                  : reinterpret_cast<const void *>(k_decode_fwd<NG, 0>);
+}
+
 // Launch shape for `rows` weight rows: R = 16 m rows per chunk and C K-slices per cluster with
 // (chunks + 1) x C <= SMs and every cluster resident at once; the shape whose busiest CTA moves
 // the fewest bytes (ties: the first found, i.e. smaller clusters, then shorter chunks).
 template <int NG>
 cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
     constexpr int MP = 8 * NG;
-    const void *kern = reinterpret_cast<const void *>(k_decode_fwd<NG>);
     const int extra = a.r > 0 ? 1 : 0;  // the adapter cluster
     double best_cost = 0.0;
     FwdArgs best = a;
@@ -1144,7 +1231,7 @@ cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
             if (found && cost >= best_cost * (1.0 - 1e-9)) continue;
             if (C > 1) {
                 int nc = 0;
-                const cudaError_t e = resident_clusters(kern, kThreads, C, smem_bytes(c), &nc);
+                const cudaError_t e = resident_clusters(fwd_kernel<NG>(m), kThreads, C, smem_bytes(c), &nc);
                 if (e != cudaSuccess) return e;
                 if (nc < c.chunks + extra) continue;
             }
@@ -1161,7 +1248,6 @@ template <int NG>
 cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint16_t *A, const uint16_t *B, int r,
                       float s, const DropoutArgs &drop, uint16_t *h, int *err, cudaStream_t st) {
     constexpr int MP = 8 * NG;
-    const void *kern = reinterpret_cast<const void *>(k_decode_fwd<NG>);
     int sms = 148;
     cudaError_t e = device_sm_count(&sms);
     if (e != cudaSuccess) return e;
@@ -1228,7 +1314,7 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
         tm_xp = tm_x;  // never read
         tm_a = tm_x;
     }
-    e = ensure_smem_limit(kern, smem);
+    e = ensure_smem_limit(fwd_kernel<NG>(a.m), smem);
     if (e != cudaSuccess) return e;
 
     for (int64_t lo = 0; lo < w.n; lo += part) {
@@ -1253,7 +1339,10 @@ cudaError_t launch_ng(const WeightView &w, const uint16_t *x, int M, const uint1
         attr[1].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = b.C > 1 ? 2 : 1;
-        e = cudaLaunchKernelEx(&cfg, k_decode_fwd<NG>, tm_codes, tm_x, tm_xp, tm_a, b);
+        if (b.m == 8)
+            e = cudaLaunchKernelEx(&cfg, k_decode_fwd<NG, 2>, tm_codes, tm_x, tm_xp, tm_a, b);
+        else
+            e = cudaLaunchKernelEx(&cfg, k_decode_fwd<NG, 0>, tm_codes, tm_x, tm_xp, tm_a, b);
         count_launch();
         if (e != cudaSuccess) return e;
     }
