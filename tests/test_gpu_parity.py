@@ -289,6 +289,13 @@ def test_ragged_weight_shapes(oracle, n, k):
     run_case(oracle, synth.LayerCase(f"shape{n}x{k}", n, k, 5, 4, 8.0, 0.02, n + k))
 
 
+@pytest.mark.parametrize("M", [1, 7, 12])
+def test_ragged_rows_on_128_row_chunks(oracle, M):
+    # 4160 rows: the few-token planner takes 128-row chunks here, so the last chunk holds 64 rows
+    # and the specialised two-m-tile loop runs on rows past the weight (read as zero, not stored)
+    run_case(oracle, synth.LayerCase(f"rows4160_M{M}", 4160, 4096, M, 16, 32.0, 0.02, 4160 + M), check_bwd=True)
+
+
 def test_zero_adapter_and_zero_base(oracle):
     case = synth.LayerCase("zeroB", 256, 512, 9, 16, 32.0, 0.02, 77)
     W, A, B, x, gh = synth.layer_inputs(case, DEV)
