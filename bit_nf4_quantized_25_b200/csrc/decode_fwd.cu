@@ -92,6 +92,7 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStageBlocks = 4;
 constexpr int kMaxM = 16;           // m-tiles per chunk: R <= 256 rows (TMA box limit)
 constexpr int kMaxStages = 8;
+constexpr int kPreWaitStages = 2;  // code stages requested before the dependency wait when x is staged once
 constexpr int kMaxCluster = 8;
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -139,7 +140,7 @@ struct FwdArgs {
 
 // Barrier block: full[kMaxStages], empty[kMaxStages], consts, recv, tready, abort flag.
 struct Bars {
-    uint64_t *full, *empty, *consts, *recv, *tready;
+    uint64_t *full, *empty, *consts, *recv, *tready, *xready;
     volatile uint32_t *abort_flag;
 };
 
@@ -150,7 +151,8 @@ __device__ __forceinline__ Bars bars_of(uint8_t *smem, const FwdArgs &p) {
     b.consts = b.empty + kMaxStages;
     b.recv = b.consts + 1;
     b.tready = b.recv + 1;
-    b.abort_flag = reinterpret_cast<volatile uint32_t *>(b.tready + 1);
+    b.xready = b.tready + 1;
+    b.abort_flag = reinterpret_cast<volatile uint32_t *>(b.xready + 1);
     return b;
 }
 
@@ -358,11 +360,11 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     const int col_lo = p.ncol * crank / C, col_hi = p.ncol * (crank + 1) / C;
     const int ns = col_hi - col_lo;
     const int S = p.stages;
-#ifdef QN_NPRE_MAX
-    const int npre = ns < S ? (ns < QN_NPRE_MAX ? ns : QN_NPRE_MAX) : (S < QN_NPRE_MAX ? S : QN_NPRE_MAX);
-#else
-    const int npre = ns < S ? ns : S;  // stages whose codes are requested before the dependency wait
-#endif
+    // Stages whose codes are requested before the dependency wait. With x staged once, at most
+    // kPreWaitStages: the x copies issued after the wait queue behind every request in flight, and
+    // the remaining stages are requested only once x has landed.
+    const int npre_all = ns < S ? ns : S;
+    const int npre = p.x_once && npre_all > kPreWaitStages ? kPreWaitStages : npre_all;
     // rows [r_lo, r_hi) of the chunk are finalised by this CTA (C > 1)
     const int r_lo = p.R * crank / C, r_hi = p.R * (crank + 1) / C, nr = r_hi - r_lo;
     const int nrmax = (p.R + C - 1) / C;
@@ -408,6 +410,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         mbar_init(bb.recv, 1);
         if (C > 1) mbar_arrive_expect_tx(bb.recv, static_cast<uint32_t>(C * nr * MP * 4));
         mbar_init(bb.tready, 1);  // the producer: t and the B rows are in shared memory
+        mbar_init(bb.xready, kConsumers * 32);  // one cp.async arrival per consumer thread: x has landed
         *bb.abort_flag = 0u;
         fence_barrier_init();
     }
@@ -526,12 +529,14 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
         };
         int ni = 0;  // stages armed
         if (p.x_once) {
-            // The first round was armed with its code requests; from then on lane 0 waits for a
-            // free slot and requests the next stage's codes.
+            // The stages requested before the wait were armed with their requests. Once x has
+            // landed, lane 0 requests the next stages' codes, each when its slot is free.
             stage_brows();
             ni = npre;
             if (lane == 0) {
-                for (int s = npre; s < ns; ++s) {
+                const bool xok = npre >= ns || mbar_wait(bb.xready, 0);  // x first
+                if (!xok) fail();
+                for (int s = npre; xok && s < ns; ++s) {
                     const int slot = s % S;
                     if (*bb.abort_flag) break;
                     if (!mbar_wait(&bb.empty[slot], ((s / S) & 1) ^ 1)) {
@@ -659,7 +664,8 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
     } else {
         // ------------------------------------------------------------------ consumers
         // Right after the dependency wait the x copies are issued; the pair table is built while
-        // they are in flight.
+        // they are in flight. Their landing (one cp.async arrival per thread on xready) releases the
+        // producer's requests for the code stages past the first kPreWaitStages.
         const int ct = threadIdx.x - 32;
         if (p.x_once) {
             // x of every stage of the slice, [stage][block][token][64 values] with 16-byte chunk c
@@ -675,6 +681,7 @@ __device__ __forceinline__ void chunk_body(const CUtensorMap *tm_codes, const CU
                                      static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4)),
                                  v ? p.x + tok * p.k + kk : p.x, v ? 16u : 0u);
             }
+            cp_async_arrive_noinc(bb.xready);
         }
         build_pair_lut(lut, ct, kConsumers * 32, p.qtype);
         if (p.x_once) cp_async_wait_all();
