@@ -25,9 +25,10 @@
 // The adapter product u = bf16(s B^T grad_h) is computed once per call by one more cluster (the
 // first row of the grid): its CTAs stream grad_h and B over the same row slices, reduce into
 // rank 0, which publishes u in the workspace and raises a flag (the protocol of the forward
-// kernel). After the loop the four row-warps of each block are summed in a fixed order; the CTA
-// that owns a block's adapter term (block kg = crank mod C) adds A^T u on the tensor cores from
-// the A tile it staged; the partial sums go by asynchronous DSMEM stores to the CTA that finalises
+// kernel). After the loop the four row-warps of each block are summed in a fixed order (rg =
+// 0..3), sub-tile f of block kg by warp (kg, rg = f); in the CTA that owns a block's adapter term
+// (block kg = crank mod C) the same warp adds A^T u for its sub-tile on the tensor cores from the
+// A tile it staged; the partial sums go by asynchronous DSMEM stores to the CTA that finalises
 // those features, which sums the slices in rank order and stores grad_x. Bit-reproducible.
 //
 // Programmatic launch: the packed weight is requested before the dependency wait; grad_h, A and

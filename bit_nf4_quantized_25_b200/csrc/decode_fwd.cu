@@ -13,31 +13,35 @@
 //
 // Work split. One CTA per SM. A CTA owns R = 16 m weight rows over one K-slice; the C K-slices
 // of a row chunk form a thread-block cluster (R and C are chosen on the host so that the grid
-// fills the SMs and each CTA moves the fewest bytes). The CTA streams its (R rows x K-slice)
-// tile through a ring of stages. A stage holds R rows x 4 blocks of codes (one TMA box, 128-byte
-// swizzled so that the 8-byte reads of eight rows hit eight different bank groups) and the
-// matching 4 x 64 columns of the M token rows of x (one 3-D TMA box, [block][token][64 values],
-// same swizzle). The FP8 block codes and group scales of the CTA's whole slice are staged once.
-//   warp 0      : producer (one lane issues the TMA boxes; all lanes stage the constants and
-//                 the rows of B the CTA's up-projection needs).
+// fills the SMs and each CTA moves the fewest bytes; chunks of 128 rows run the k_decode_fwd<NG, 2>
+// instantiation, every other R k_decode_fwd<NG, 0>). The CTA streams its (R rows x K-slice) codes
+// through a ring of stages: a stage is R rows x 4 blocks (one TMA box, 128-byte swizzled so that
+// the 8-byte reads of eight rows hit eight different bank groups). x of the whole K-slice
+// ([stage][block][token][64 values], same swizzle) and the FP8 block codes and group scales of
+// the slice are staged once, by the consumers' 16-byte cp.async copies.
+//   warp 0      : producer (one lane issues the code boxes; all lanes stage the rows of B the CTA
+//                 finalises, copy t, and compute B t of those rows on the tensor cores).
 //   warps 1..16 : consumers. Warp (kg, rg) takes block kg of every stage and the m-tiles
 //                 rg, rg + 4, ... of the chunk: codes -> pair table -> mma.sync with x, one fp32
 //                 fragment per block scaled by c'_b = fma(e4m3(q_b), sigma_g, mu) into the
 //                 accumulators (the four lanes of a quad compute the constants the quad needs and
-//                 share them by shuffles).
+//                 share them by shuffles). In <NG, 2> a warp runs both of its m-tiles at once.
 // The adapter down-projection t = bf16(s A x) is computed once per call by one more cluster (the
-// first row of the grid, so that it is dispatched first): its CTAs stream x and A over the same K-slices, reduce their partial
-// sums into rank 0 (DSMEM), and rank 0 publishes t in the workspace and raises a flag. The other
-// CTAs' producers wait for the flag after their last stage and copy t to shared memory; the last
-// of them to do so lowers the flag again for the next call.
-// After the loop the four block-warps of each m-tile are summed in a fixed order; one CTA per
-// m-tile adds B t on the tensor cores; the partial sums go by asynchronous DSMEM stores to the
-// CTA of the cluster that finalises those rows, which waits on its own mbarrier for the bytes,
-// sums the slices in rank order and stores h. Results are bit-reproducible.
+// first row of the grid, so that it is dispatched first): its CTAs stream x and A over the same
+// K-slices, reduce their partial sums into rank 0 (DSMEM), and rank 0 publishes t in the
+// workspace and raises a flag. The other CTAs' producers wait for the flag after their last stage
+// and copy t to shared memory; the last of them to do so lowers the flag again for the next call.
+// After the loop the four block-warps of each m-tile are summed in a fixed order (kg = 0..3), each
+// m-tile by one warp. With C > 1 the sums go by asynchronous DSMEM stores to the CTA of the
+// cluster that finalises those rows, which waits on its own mbarrier for the bytes, sums the
+// slices in rank order, adds B t and stores h; with C == 1 the summing warps add B t on the
+// tensor cores and store h. Results are bit-reproducible.
 //
 // Programmatic launch: the packed weight (codes, FP8 codes, group scales) is requested BEFORE the
 // dependency wait, so the first stages of the ring fill while the preceding kernel finishes; x,
-// A and B are read, and h written, only after it. The caller guarantees that the preceding
+// A and B are read, and h written, only after it. With x staged once, only two code stages are
+// requested before the wait and the rest once x has landed: the x copies would otherwise queue
+// behind every code request in flight. The caller guarantees that the preceding
 // kernel on the stream, if it signals its dependents early, does not write the packed weight
 // (no kernel of this library that signals early writes one). The codes are read with an L2
 // evict-first policy: they are used once, and the activations and adapters should stay cached.
