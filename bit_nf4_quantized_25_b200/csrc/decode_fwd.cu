@@ -1225,7 +1225,7 @@ cudaError_t plan(FwdArgs &a, int64_t rows, int sms, bool &found) {
     found = false;
     // m is a multiple of 4 (every consumer warp holds the same number of m-tiles) unless the
     // weight has fewer than 64 rows
-    const int m_max = 16;  // four m-tile rows of warps, up to 4 m-tiles each
+    const int m_max = kMaxM;  // four m-tile rows of warps, up to 4 m-tiles each
     const int m_min = rows < 64 ? static_cast<int>((rows + 15) / 16) : 4;
     const int m_step = rows < 64 ? 1 : 4;
     for (int C = 1; C <= kMaxCluster && C <= a.ncol; ++C) {
