@@ -145,3 +145,33 @@ def test_algorithmic_bytes_per_launch_of_the_decode_step():
     n = k = 4096
     assert bench.weight_bytes(n, k) == n * k // 2 + n * k // 64 + 4 * ((n * k // 64 + 255) // 256) + 4
     assert bench.fwd_bytes(n, k, 1, 16) == bench.weight_bytes(n, k) + 2 * k + 2 * 16 * k + 2 * n * 16 + 2 * n
+
+
+def test_traffic_record_is_reported_only_while_its_sources_are_unchanged(monkeypatch, tmp_path):
+    import hashlib
+    import json
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cu"
+    src.write_bytes(b"__global__ void k() {}\n")
+    rec = {"sources": ["k.cu"], "sources_sha256_16": hashlib.sha256(src.read_bytes()).hexdigest()[:16],
+           "bytes_per_launch": 1234}
+    (tmp_path / "profiles" / "k_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profile_traffic("k_traffic.json") == 1234
+    assert bench.profile_traffic("missing.json") is None
+    src.write_bytes(b"__global__ void k() { }\n")  # the kernel changed after the capture
+    assert bench.profile_traffic("k_traffic.json") is None
+
+
+def test_committed_traffic_records_are_consistent():
+    # the records the bench quotes: their sources exist, their algorithmic bytes are the bench's own
+    # figure for one decode layer, and the measured DRAM bytes are within 1 % of it (nothing re-read)
+    import json
+    for name, kernel in (("decode_fwd_traffic.json", "k_decode_fwd"), ("decode_bwd_traffic.json", "k_decode_bwd")):
+        with open(os.path.join(bench.ROOT, "profiles", name)) as f:
+            rec = json.load(f)
+        assert rec["kernel"] == kernel
+        assert all(os.path.exists(os.path.join(bench.ROOT, s)) for s in rec["sources"])
+        assert rec["algorithmic_bytes_per_launch"] == 15_427_259
+        assert rec["launches_averaged"] == 21
+        assert 1.0 <= rec["bytes_per_launch"] / rec["algorithmic_bytes_per_launch"] < 1.01
